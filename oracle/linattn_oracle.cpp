@@ -1,0 +1,173 @@
+// Test infrastructure only: the fp64 CPU oracle for causal linear attention.
+//
+// Only the tests, the package's smoke entry and the benchmark's CPU-baseline /
+// reference arm may load this library.  The product path (the CUDA library) never
+// calls it and shares no code with it.
+//
+// What it computes is the plain definition of causal linear attention, one token at a
+// time, in double precision:
+//
+//   phi(x)  = x + 1 for x > 0, exp(x) otherwise (ELU with alpha = 1, plus one), or the
+//             identity.  Source: "Linear Attention and Retentive Networks: How Recurrent
+//             Duals and Chunkwise Tiling Eliminate the Quadratic Bottleneck", section
+//             "The Associative Property and Linear Kernel Formulation" (the kernel
+//             feature map that makes the similarity separable).
+//   S_t     = gamma * S_{t-1} + phi(k_t) v_t^T      (dk x dv)
+//   Z_t     = gamma * Z_{t-1} + phi(k_t)            (dk)
+//   o_t     = phi(q_t) S_t / (phi(q_t) . Z_t + eps)  (normalised) or phi(q_t) S_t.
+//             Sources: the same page, "The Recurrent Dual" (undecayed state, normaliser
+//             and ratio readout) and "2. The Three Computation Paradigms / B. Recurrent
+//             Representation" (the per-head scalar decay gamma, unnormalised readout);
+//             "Log-Depth Chunked Linear-Attention Scan", "Mathematical statement" (S_t and
+//             Z_t as sums over i <= t, so token t is included in its own state) and
+//             "Implementation notes" (the ratio with "+ eps" in the denominator).
+//
+// gamma == NULL means no decay (gamma = 1).  Token t is counted in its own state
+// (inclusive sums).  The decay multiplies the previous state only; the current token
+// enters with weight gamma^0 = 1.  When both decay and normalisation are requested the
+// normaliser decays the same way as the state.
+//
+// Inputs are float32 arrays: the GPU path's bf16 inputs are widened to float32 exactly
+// before they are passed here, so both sides see identical values.  All arithmetic is
+// double precision, built without fast-math.  Work is split over (b, h) pairs only,
+// with std::thread; each pair is an independent token loop.
+//
+// Layouts (all contiguous, row-major):
+//   q, k   [B, H, T, dk]      v [B, H, T, dv]      out [B, H, T, dv]  (may be NULL)
+//   S_init, S_final [B, H, dk, dv]   (S[i][j], i = key feature, j = value feature)
+//   Z_init, Z_final [B, H, dk]
+//   gamma [H] (double) or NULL.
+// S_init / Z_init may be NULL (zero initial state); the outputs may be NULL (skipped).
+
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+#include <thread>
+#include <vector>
+
+namespace {
+
+inline double feature_map(double x, int fm) {
+  if (fm == 0) return x;                    // identity
+  return x > 0.0 ? x + 1.0 : std::exp(x);   // ELU(alpha = 1) + 1
+}
+
+struct Problem {
+  const float* q;
+  const float* k;
+  const float* v;
+  int B, H;
+  long long T;
+  int dk, dv, fm;
+  const double* gamma;
+  int normalize;
+  double eps;
+  const double* S_init;
+  const double* Z_init;
+  double* out;
+  double* S_final;
+  double* Z_final;
+};
+
+// The token loop for one (b, h) pair.
+void run_pair(const Problem& p, long long bh) {
+  const int dk = p.dk, dv = p.dv;
+  const long long T = p.T;
+  const int h = static_cast<int>(bh % p.H);
+  const double g = p.gamma ? p.gamma[h] : 1.0;
+
+  std::vector<double> S(static_cast<size_t>(dk) * dv, 0.0), Z(dk, 0.0);
+  if (p.S_init)
+    for (size_t e = 0; e < S.size(); ++e) S[e] = p.S_init[bh * dk * dv + e];
+  if (p.Z_init)
+    for (int i = 0; i < dk; ++i) Z[i] = p.Z_init[bh * dk + i];
+
+  std::vector<double> fq(dk), fk(dk), num(dv);
+  const float* q = p.q + bh * T * dk;
+  const float* k = p.k + bh * T * dk;
+  const float* v = p.v + bh * T * dv;
+  double* out = p.out ? p.out + bh * T * dv : nullptr;
+
+  for (long long t = 0; t < T; ++t) {
+    for (int i = 0; i < dk; ++i) {
+      fq[i] = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
+      fk[i] = feature_map(static_cast<double>(k[t * dk + i]), p.fm);
+    }
+    const float* vt = v + t * dv;
+    // State update: decay the past, then add the current token's outer product.
+    for (int i = 0; i < dk; ++i) {
+      double* Si = &S[static_cast<size_t>(i) * dv];
+      for (int j = 0; j < dv; ++j) Si[j] = g * Si[j] + fk[i] * static_cast<double>(vt[j]);
+      Z[i] = g * Z[i] + fk[i];
+    }
+    if (!out) continue;
+    // Readout with the inclusive state.
+    for (int j = 0; j < dv; ++j) num[j] = 0.0;
+    double den = 0.0;
+    for (int i = 0; i < dk; ++i) {
+      const double* Si = &S[static_cast<size_t>(i) * dv];
+      for (int j = 0; j < dv; ++j) num[j] += fq[i] * Si[j];
+      den += fq[i] * Z[i];
+    }
+    double* ot = out + t * dv;
+    if (p.normalize) {
+      for (int j = 0; j < dv; ++j) ot[j] = num[j] / (den + p.eps);
+    } else {
+      for (int j = 0; j < dv; ++j) ot[j] = num[j];
+    }
+  }
+
+  if (p.S_final)
+    for (size_t e = 0; e < S.size(); ++e) p.S_final[bh * dk * dv + e] = S[e];
+  if (p.Z_final)
+    for (int i = 0; i < dk; ++i) p.Z_final[bh * dk + i] = Z[i];
+}
+
+}  // namespace
+
+extern "C" {
+
+// Returns 0 on success, 1 on an invalid argument.  nthreads <= 0 means one thread per
+// hardware thread (capped at B*H).
+int la_oracle_forward(const float* q, const float* k, const float* v, int B, int H,
+                      long long T, int dk, int dv, int feature_map_id,
+                      const double* gamma, int normalize, double eps,
+                      const double* S_init, const double* Z_init, double* out,
+                      double* S_final, double* Z_final, int nthreads) {
+  if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 1;
+  if (feature_map_id != 0 && feature_map_id != 1) return 1;
+  if (T > 0 && (!q || !k || !v)) return 1;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return 0;
+
+  Problem p{q, k, v, B, H, T, dk, dv, feature_map_id, gamma, normalize, eps,
+            S_init, Z_init, out, S_final, Z_final};
+
+  long long workers = nthreads > 0 ? nthreads
+                                   : static_cast<long long>(std::thread::hardware_concurrency());
+  if (workers < 1) workers = 1;
+  if (workers > BH) workers = BH;
+
+  if (workers == 1) {
+    for (long long bh = 0; bh < BH; ++bh) run_pair(p, bh);
+    return 0;
+  }
+  std::vector<std::thread> pool;
+  pool.reserve(static_cast<size_t>(workers));
+  for (long long w = 0; w < workers; ++w) {
+    pool.emplace_back([&p, w, workers, BH]() {
+      for (long long bh = w; bh < BH; bh += workers) run_pair(p, bh);
+    });
+  }
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+// The feature map alone, element-wise, for direct checks against closed forms.
+int la_oracle_feature_map(const double* x, double* y, long long n, int feature_map_id) {
+  if (feature_map_id != 0 && feature_map_id != 1) return 1;
+  for (long long e = 0; e < n; ++e) y[e] = feature_map(x[e], feature_map_id);
+  return 0;
+}
+
+}  // extern "C"

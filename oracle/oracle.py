@@ -1,0 +1,112 @@
+"""Test infrastructure only: Python access to the fp64 CPU oracle.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference arm of
+``bench.py`` may import this module.  The CUDA library never calls it.
+
+The oracle itself is ``linattn_oracle.cpp`` (a plain token loop in double precision;
+its header states what it computes and which passages of the pages it follows).  This
+module compiles it with g++ (no fast-math) and wraps the two exported functions with
+numpy arrays.  Nothing here holds arithmetic of the method.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+HERE = Path(__file__).resolve().parent
+SRC = HERE / "linattn_oracle.cpp"
+LIB = HERE / "liblinattn_oracle.so"
+
+FEATURE_MAPS = {"identity": 0, "elu1": 1}
+
+
+def build(src: Path = SRC, out: Path = LIB, force: bool = False) -> Path:
+    """Compile the oracle into a shared library (skipped when it is up to date)."""
+    if not force and out.exists() and out.stat().st_mtime >= src.stat().st_mtime:
+        return out
+    tmp = out.with_suffix(f".{os.getpid()}.tmp.so")
+    cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread",
+           "-fno-fast-math", "-o", str(tmp), str(src)]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+class Oracle:
+    """ctypes handle on one compiled copy of the oracle."""
+
+    def __init__(self, lib_path: Path | str | None = None):
+        path = Path(lib_path) if lib_path is not None else build()
+        self.path = path
+        self._lib = ctypes.CDLL(str(path))
+        f = self._lib.la_oracle_forward
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_void_p, ctypes.c_int, ctypes.c_double,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        g = self._lib.la_oracle_feature_map
+        g.restype = ctypes.c_int
+        g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int]
+
+    def feature_map(self, x, feature_map: str = "elu1") -> np.ndarray:
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        y = np.empty_like(x)
+        rc = self._lib.la_oracle_feature_map(x.ctypes.data, y.ctypes.data, x.size,
+                                             FEATURE_MAPS[feature_map])
+        if rc != 0:
+            raise ValueError(f"la_oracle_feature_map returned {rc}")
+        return y
+
+    def forward(self, q, k, v, *, feature_map: str = "elu1", gamma=None,
+                normalize: bool = True, eps: float = 0.0, S_init=None, Z_init=None,
+                want_out: bool = True, nthreads: int = 0):
+        """Run the token loop.
+
+        q, k: [B, H, T, dk]; v: [B, H, T, dv] (any float dtype; converted to float32,
+        which is exact for bf16 and float32 inputs).  gamma: per-head decays (length H)
+        or None.  Returns (out [B,H,T,dv] float64 or None, S_final [B,H,dk,dv],
+        Z_final [B,H,dk]).
+        """
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        k = np.ascontiguousarray(k, dtype=np.float32)
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        B, H, T, dk = q.shape
+        dv = v.shape[-1]
+        if k.shape != q.shape or v.shape[:3] != (B, H, T):
+            raise ValueError("shape mismatch between q, k and v")
+        g = None
+        if gamma is not None:
+            g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(H))
+        s0 = None if S_init is None else np.ascontiguousarray(S_init, dtype=np.float64)
+        z0 = None if Z_init is None else np.ascontiguousarray(Z_init, dtype=np.float64)
+        out = np.empty((B, H, T, dv), dtype=np.float64) if want_out else None
+        S = np.empty((B, H, dk, dv), dtype=np.float64)
+        Z = np.empty((B, H, dk), dtype=np.float64)
+
+        def ptr(a):
+            return None if a is None else a.ctypes.data
+
+        rc = self._lib.la_oracle_forward(ptr(q), ptr(k), ptr(v), B, H, T, dk, dv,
+                                         FEATURE_MAPS[feature_map], ptr(g), int(bool(normalize)),
+                                         float(eps), ptr(s0), ptr(z0), ptr(out), ptr(S), ptr(Z),
+                                         int(nthreads))
+        if rc != 0:
+            raise ValueError(f"la_oracle_forward returned {rc}")
+        return out, S, Z
+
+
+_default: Oracle | None = None
+
+
+def default_oracle() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
