@@ -1,0 +1,441 @@
+"""Benchmark of the chunked causal linear-attention prefill on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one whole prefill (K1 -> K2 -> K3) of the workload through the C ABI.  The
+default workload is the 128K-token retention prefill (B1 H32 T131072 d128 C64, bf16
+inputs, identity feature map, per-head decay, unnormalised).  With N GPUs (torchrun,
+one rank per GPU) every rank runs its own independent copy (weak scaling); the value is
+the tokens*heads of all ranks over the slowest rank's device time.  Rank 0 prints one
+JSON line.
+
+Extra fields: per-kernel device times from an event-instrumented pass, the roofline of
+the dominant kernel against the measured HBM bandwidth, the end-to-end rate through the
+host-buffer entry point, the oracle's rate on the host cores, and the SM clocks sampled
+during the timed region.
+
+`--impl reference` times the fp64 CPU oracle (the only reference implementation there
+is) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import torch  # noqa: E402
+
+from chunked_causal_linear_b200 import binding as B  # noqa: E402
+from chunked_causal_linear_b200 import ranks  # noqa: E402
+from chunked_causal_linear_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "causal linear-attn prefill tokens·heads/s at H=32,d=128; % of roofline"
+UNIT = "tokens*heads/s"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+KERNEL_NAMES = {
+    "logdepth": ["k1_tc", "k2_reduce", "k2_scan_totals", "k2_downsweep", "k3_tc"],
+    "sequential": ["k1_tc", "k2_sequential", "k3_tc"],
+}
+KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce": "scan.cu",
+                  "k2_scan_totals": "scan.cu", "k2_downsweep": "scan.cu",
+                  "k2_sequential": "scan.cu"}
+
+
+# ---------------------------------------------------------------------------------------
+# Algorithmic bytes
+
+
+def layout(w):
+    NC = -(-w.T // w.C)
+    Ls = max(1, -(-NC // 32))
+    G = -(-NC // Ls)
+    R = w.dk * w.dv + (w.dk if w.normalize else 0)
+    return NC, G, R
+
+
+def kernel_bytes(w, name: str, out_elem: int) -> int:
+    """Bytes each kernel must move for its own role (one launch)."""
+    BH = w.B * w.H
+    NC, G, R = layout(w)
+    e_in = 2 if w.dtype == "bf16" else 4
+    rec = BH * NC * R * 4
+    if name.startswith("k1"):
+        return BH * w.T * (w.dk + w.dv) * e_in + rec
+    if name == "k2_reduce":
+        return rec
+    if name == "k2_scan_totals":
+        return 2 * BH * G * R * 4 + BH * R * 4
+    if name == "k2_downsweep":
+        return 2 * rec + BH * G * R * 4
+    if name == "k2_sequential":
+        return 2 * rec + BH * R * 4
+    if name.startswith("k3"):
+        return BH * w.T * (2 * w.dk + w.dv) * e_in + BH * (NC - 1) * R * 4 + BH * w.T * w.dv * out_elem
+    raise KeyError(name)
+
+
+def method_bytes(w, out_elem: int) -> int:
+    """Whole-step algorithmic bytes of the three-kernel method: inputs read once, output
+    written once, final states written once, and four passes of the chunk records (K1
+    write, K2 read and write, K3 read)."""
+    BH = w.B * w.H
+    NC, G, R = layout(w)
+    e_in = 2 if w.dtype == "bf16" else 4
+    return (BH * w.T * (2 * w.dk + w.dv) * e_in + BH * w.T * w.dv * out_elem
+            + BH * (w.dk * w.dv + (w.dk if w.normalize else 0)) * 4 + 4 * BH * NC * R * 4)
+
+
+def measured_peaks() -> tuple[float, str]:
+    p = ROOT / "MEASURED_PEAKS.json"
+    try:
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(fname: str) -> str:
+    csrc = ROOT / "chunked_causal_linear_b200" / "csrc"
+    h = hashlib.sha256()
+    for f in sorted({fname, "ptx.cuh", "common.cuh"}):
+        h.update((csrc / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's source is the
+    one those counters were taken on; otherwise None."""
+    f = ROOT / "profiles" / "traffic.txt"
+    if not f.exists():
+        return None
+    want = source_hash(KERNEL_SOURCES.get(kernel, "tc_kernels.cu"))
+    for line in f.read_text().splitlines():
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
+                and parts[1] == workload and parts[2] == want:
+            return int(float(parts[3]))
+    return None
+
+
+# ---------------------------------------------------------------------------------------
+# Clocks
+
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int, interval_ms: int = 100):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.interval_ms = interval_ms
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.interval_ms)], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        for line in Path(self.tmp.name).read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid.replace("GPU-", "") not in parts[0]:
+                continue
+            rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+def clocks_bad(c) -> bool:
+    if not c:
+        return False
+    if any(r in c["reasons"] for r in BAD_REASONS):
+        return True
+    return bool(c["sm_mhz"] and c["sm_max_mhz"] and c["sm_mhz"] < 0.6 * c["sm_max_mhz"]
+                and not c["reasons"])
+
+
+# ---------------------------------------------------------------------------------------
+# CPU side (oracle): the reported baseline and the reference arm
+
+
+class OracleTimer:
+    """Times the oracle on the first T' tokens of every (b, h) of the workload, T' sized
+    for about `target_s` seconds of host work."""
+
+    def __init__(self, w, q, k, v, target_s: float):
+        from oracle.oracle import default_oracle
+        self.orc = default_oracle()
+        self.w = w
+        self.threads = max(1, min(len(os.sched_getaffinity(0)), w.B * w.H))
+        probe_t = min(w.T, 512)
+        self.inputs = (q, k, v)
+        dt = self._run(probe_t)
+        self.tp = min(w.T, max(probe_t, int(probe_t * target_s / max(dt, 1e-6))))
+        self.host = [t[:, :, :self.tp].to("cpu", torch.float32).numpy() for t in (q, k, v)]
+
+    def _run(self, tp, host=None):
+        w = self.w
+        qs, ks, vs = host if host is not None else (
+            t[:, :, :tp].to("cpu", torch.float32).numpy() for t in self.inputs)
+        t0 = time.perf_counter()
+        self.orc.forward(qs, ks, vs, feature_map=w.feature_map, gamma=w.gammas(),
+                         normalize=w.normalize, nthreads=self.threads)
+        return time.perf_counter() - t0
+
+    def rate(self):
+        dt = self._run(self.tp, self.host)
+        self.last_s = dt
+        return self.w.B * self.w.H * self.tp / dt
+
+    def sample(self):
+        return (f"first {self.tp} of {self.w.T} tokens of all {self.w.B * self.w.H} (b,h) "
+                f"pairs, full fp64 token loop, {self.last_s:.1f} s per run on "
+                f"{self.threads} threads")
+
+
+def reference_arm(args, w, info):
+    if not info.is_root:
+        return
+    # The oracle's cost per token does not depend on the values; draw the sample's inputs
+    # on the CPU with the workload's recipe.
+    probe = w.with_(T=min(w.T, 1 << 15))
+    q, k, v = make_inputs(probe, seed=0, device="cpu")
+    timer = OracleTimer(w.with_(T=probe.T), q, k, v, target_s=args.reference_step_s)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        r = timer.rate()
+        if i >= args.warmup:
+            per_step.append(r)
+    value = statistics.median(per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * w.B * w.H * w.T / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": timer.threads, "kind": "oracle",
+                         "sample": timer.sample()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+            "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
+            "gamma": "1 - 2^(-5-3h/31) per head" if w.decay else None,
+            "normalize": w.normalize, "scan": args.scan, "out_dtype": args.out_dtype,
+            "kernel_path": "tensor_core", "l2": "inputs larger than L2, no flush",
+            "parallelism": "replicas (one independent problem per GPU)"}
+
+
+# ---------------------------------------------------------------------------------------
+# GPU side
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="retention_128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--scan", default="logdepth", choices=["logdepth", "sequential"])
+    ap.add_argument("--out-dtype", default="f32", choices=["f32", "as_input"])
+    ap.add_argument("--kernel-timing-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-baseline-s", type=float, default=15.0)
+    ap.add_argument("--reference-step-s", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        info = ranks.rank_info()
+        reference_arm(args, w, info)
+        return
+
+    info = ranks.init("nccl")
+    dev = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(dev)
+    B.load_library()
+
+    q, k, v = make_inputs(w, seed=info.rank, device=dev)
+    out_dtype = torch.float32 if args.out_dtype == "f32" else q.dtype
+    out_elem = 4 if args.out_dtype == "f32" else 2
+    out = torch.empty((w.B, w.H, w.T, w.dv), dtype=out_dtype, device=dev)
+    S = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    Z = torch.empty((w.B, w.H, w.dk), dtype=torch.float32, device=dev) if w.normalize else None
+    ws = torch.empty(B.lin_attn_prefill_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.C,
+                                                        w.normalize),
+                     dtype=torch.uint8, device=dev)
+    gam = w.gammas()
+    kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
+              scan=args.scan, kernel_path="tensor_core", workspace=ws, out_dtype=args.out_dtype)
+
+    def step():
+        B.lin_attn_prefill(q, k, v, out, S, Z, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def timed_region():
+        sampler = None if args.no_clocks else ClockSampler(info.local_rank)
+        if sampler:
+            sampler.start()
+        ranks.barrier(info)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ranks.barrier(info)
+        clocks = sampler.stop() if sampler else None
+        return e0.elapsed_time(e1) / args.steps, clocks
+
+    ms, clocks = timed_region()
+    remeasured = False
+    if ranks.any_over_ranks(clocks_bad(clocks), info, dev):
+        ms, clocks = timed_region()
+        remeasured = True
+    ms_max = ranks.max_over_ranks(ms, info, dev)
+    n_kern = len(KERNEL_NAMES[args.scan])
+    value = info.world * w.tokens_heads / (ms_max / 1000.0)
+
+    # Per-kernel device times (events between the library's own launches, same stream).
+    names = KERNEL_NAMES[args.scan]
+    per = [[] for _ in names]
+    for _ in range(max(1, args.kernel_timing_steps)):
+        t = B.lin_attn_prefill_timed(q, k, v, out, S, Z, **kw)
+        for i, x in enumerate(t[:len(names)]):
+            per[i].append(x)
+    kern_ms = {n: statistics.mean(x) for n, x in zip(names, per)}
+    dom = max(kern_ms, key=kern_ms.get)
+    peak, peak_kind = measured_peaks()
+    dom_bytes = kernel_bytes(w, dom, out_elem)
+    achieved = dom_bytes / (kern_ms[dom] / 1000.0) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak,
+                "traffic": recorded_traffic(dom, w.name),
+                "algorithmic_bytes": dom_bytes, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    mb = method_bytes(w, out_elem)
+    step_roof = {"bytes_method": mb, "achieved_gbs": mb / (ms_max / 1000.0) / 1e9,
+                 "frac_of_measured": mb / (ms_max / 1000.0) / 1e9 / peak,
+                 "frac_of_nominal_8tbs": mb / (ms_max / 1000.0) / 1e9 / NOMINAL_HBM_GBS}
+
+    # End to end through the host-buffer entry point (pinned host memory).
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        Sh = torch.empty(S.shape, dtype=torch.float32).pin_memory()
+        Zh = torch.empty(Z.shape, dtype=torch.float32).pin_memory() if Z is not None else None
+        hkw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
+                   scan=args.scan, kernel_path="tensor_core", out_dtype=args.out_dtype)
+        dbuf = torch.empty(B.lin_attn_prefill_host_buffer_bytes(qh, vh, chunk=w.C,
+                                                                normalize=w.normalize,
+                                                                out_dtype=args.out_dtype),
+                           dtype=torch.uint8, device=dev)
+        B.lin_attn_prefill_host(qh, kh, vh, oh, Sh, Zh, device_buffer=dbuf, **hkw)
+        ranks.barrier(info)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            B.lin_attn_prefill_host(qh, kh, vh, oh, Sh, Zh, device_buffer=dbuf, **hkw)
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, info, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        d2h = oh.numel() * oh.element_size() + Sh.numel() * 4 + (Zh.numel() * 4 if Zh is not None else 0)
+        e2e = {"value": info.world * w.tokens_heads / (e_ms / 1000.0), "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "lin_attn_prefill_host (pinned host buffers, synchronous)"}
+        del qh, kh, vh, oh, Sh, Zh, dbuf
+
+    cpu = None
+    if info.is_root and info.world == 1 and not args.no_cpu_baseline:
+        timer = OracleTimer(w, q, k, v, target_s=args.cpu_baseline_s)
+        rate = timer.rate()
+        cpu = {"value": rate, "unit": UNIT, "cores": timer.threads, "kind": "oracle",
+               "sample": timer.sample()}
+
+    err = B.lin_attn_device_error()
+    if info.is_root:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w, args), "roofline": roofline,
+            "step_roofline": step_roof, "kernels_ms": kern_ms, "cpu_baseline": cpu,
+            "e2e": e2e, "clocks": clocks, "remeasured": remeasured,
+            "gpu_launches": n_kern * args.steps, "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+    ranks.finish(info)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,247 @@
+"""ctypes binding of ``liblinattn.so`` (include/linattn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA library.
+Tensors are torch CUDA tensors (PyTorch provides device memory and streams); the
+functions keep the C entry points' names.  If the shared library is missing, every call
+raises -- there is no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+LIB_PATH = Path(__file__).resolve().parent / "liblinattn.so"
+
+LA_OK = 0
+STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARGUMENT", 2: "LA_ERR_UNSUPPORTED",
+                3: "LA_ERR_OUT_OF_MEMORY", 4: "LA_ERR_CUDA", 5: "LA_ERR_INTERNAL"}
+FEATURE_MAPS = {"identity": 0, "elu1": 1}
+SCAN_MODES = {"logdepth": 0, "sequential": 1}
+KERNEL_PATHS = {"auto": 0, "tensor_core": 1, "fma": 2}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+OUT_DTYPES = {"as_input": 0, "f32": 1}
+
+EXPORTED_SYMBOLS = (
+    "lin_attn_prefill", "lin_attn_prefill_f32", "lin_attn_prefill_workspace_bytes",
+    "lin_attn_prefill_ex", "lin_attn_prefill_timed", "lin_attn_prefill_host",
+    "lin_attn_prefill_host_buffer_bytes",
+    "lin_attn_decode_step", "lin_attn_decode_step_f32", "lin_attn_device_error",
+    "lin_attn_status_string", "lin_attn_version",
+)
+
+
+class LinAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class PrefillArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("S_final", ctypes.c_void_p), ("Z_final", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_longlong),
+        ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
+        ("feature_map", ctypes.c_int), ("gamma", ctypes.c_void_p), ("normalize", ctypes.c_int),
+        ("eps", ctypes.c_float), ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("scan_mode", ctypes.c_int),
+        ("kernel_path", ctypes.c_int), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: Path | str | None = None) -> ctypes.CDLL:
+    """Loads the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = Path(path) if path is not None else LIB_PATH
+    if not p.exists():
+        raise RuntimeError(f"{p} is missing: build it with `python -m chunked_causal_linear_b200.build`")
+    lib = ctypes.CDLL(str(p))
+    vp, i, ll, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "lin_attn_prefill": (i, [vp, vp, vp, vp, vp, vp, i, i, ll, i, i, i, i, vp, i, vp]),
+        "lin_attn_prefill_f32": (i, [vp, vp, vp, vp, vp, vp, i, i, ll, i, i, i, i, vp, i, vp]),
+        "lin_attn_prefill_workspace_bytes": (sz, [i, i, ll, i, i, i, i]),
+        "lin_attn_prefill_ex": (i, [ctypes.POINTER(PrefillArgs)]),
+        "lin_attn_prefill_timed": (i, [ctypes.POINTER(PrefillArgs), ctypes.POINTER(f), i,
+                                       ctypes.POINTER(i)]),
+        "lin_attn_prefill_host": (i, [ctypes.POINTER(PrefillArgs), vp, sz]),
+        "lin_attn_prefill_host_buffer_bytes": (sz, [ctypes.POINTER(PrefillArgs)]),
+        "lin_attn_decode_step": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "lin_attn_decode_step_f32": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "lin_attn_device_error": (i, [ctypes.POINTER(ctypes.c_int)]),
+        "lin_attn_status_string": (ctypes.c_char_p, [i]),
+        "lin_attn_version": (i, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != LA_OK:
+        raise LinAttnError(fn, status)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _gamma_array(gamma, H):
+    if gamma is None:
+        return None, None
+    vals = [float(g) for g in gamma]
+    if len(vals) != H:
+        raise ValueError(f"gamma needs {H} values, got {len(vals)}")
+    arr = (ctypes.c_float * H)(*vals)
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, normalize, eps,
+              scan, kernel_path, workspace, stream, out_dtype="as_input"):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    garr, gptr = _gamma_array(gamma, H)
+    a = PrefillArgs()
+    a.q, a.k, a.v, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(out)
+    a.S_final, a.Z_final = _ptr(S_final), _ptr(Z_final)
+    a.B, a.H, a.T, a.dk, a.dv, a.C = B, H, T, dk, dv, int(chunk)
+    a.feature_map = FEATURE_MAPS[feature_map]
+    a.gamma = gptr
+    a.normalize = int(bool(normalize))
+    a.eps = float(eps)
+    a.dtype = DTYPES[q.dtype]
+    a.out_dtype = OUT_DTYPES[out_dtype]
+    a.scan_mode = SCAN_MODES[scan]
+    a.kernel_path = KERNEL_PATHS[kernel_path]
+    a.workspace = _ptr(workspace)
+    a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.stream = stream
+    return a, garr
+
+
+def lin_attn_prefill_workspace_bytes(B, H, T, dk, dv, C, normalize) -> int:
+    return int(load_library().lin_attn_prefill_workspace_bytes(B, H, T, dk, dv, C, int(bool(normalize))))
+
+
+def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
+                     feature_map="elu1", gamma=None, normalize=True, eps=0.0, scan="logdepth",
+                     kernel_path="auto", workspace=None, stream=None, want_states=True,
+                     out_dtype="as_input"):
+    """Runs the prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (bf16 or float32).
+
+    out_dtype "f32" writes a float32 output for bf16 inputs.  Allocates out / S_final /
+    Z_final when not given.  Returns (out, S_final, Z_final).
+    """
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        odt = torch.float32 if out_dtype == "f32" else q.dtype
+        out = torch.empty((B, H, T, dv), dtype=odt, device=q.device)
+    if want_states and S_final is None:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if want_states and normalize and Z_final is None:
+        Z_final = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
+    a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
+                        gamma=gamma, normalize=normalize, eps=eps, scan=scan,
+                        kernel_path=kernel_path, workspace=workspace,
+                        stream=_stream_handle(stream), out_dtype=out_dtype)
+    _check("lin_attn_prefill_ex", load_library().lin_attn_prefill_ex(ctypes.byref(a)))
+    del keep
+    return out, S_final, Z_final
+
+
+def lin_attn_prefill_timed(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
+                           feature_map="elu1", gamma=None, normalize=True, eps=0.0,
+                           scan="logdepth", kernel_path="auto", workspace=None, stream=None,
+                           out_dtype="as_input") -> list[float]:
+    """Runs the prefill once with an event around every kernel; returns the kernels'
+    device durations in milliseconds, in launch order (synchronous)."""
+    a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
+                        gamma=gamma, normalize=normalize, eps=eps, scan=scan,
+                        kernel_path=kernel_path, workspace=workspace,
+                        stream=_stream_handle(stream), out_dtype=out_dtype)
+    ms = (ctypes.c_float * 8)()
+    n = ctypes.c_int(0)
+    _check("lin_attn_prefill_timed",
+           load_library().lin_attn_prefill_timed(ctypes.byref(a), ms, 8, ctypes.byref(n)))
+    del keep
+    return [float(ms[i]) for i in range(n.value)]
+
+
+def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
+                          feature_map="elu1", gamma=None, normalize=True, eps=0.0,
+                          scan="logdepth", kernel_path="auto", device_buffer=None, stream=None,
+                          out_dtype="as_input"):
+    """Runs the prefill on HOST tensors (pinned for full copy bandwidth); synchronous."""
+    a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
+                        gamma=gamma, normalize=normalize, eps=eps, scan=scan,
+                        kernel_path=kernel_path, workspace=None, stream=_stream_handle(stream),
+                        out_dtype=out_dtype)
+    nbytes = 0 if device_buffer is None else device_buffer.numel() * device_buffer.element_size()
+    _check("lin_attn_prefill_host",
+           load_library().lin_attn_prefill_host(ctypes.byref(a), _ptr(device_buffer), nbytes))
+    del keep
+    return out, S_final, Z_final
+
+
+def lin_attn_prefill_host_buffer_bytes(q, v, *, chunk=64, normalize=True,
+                                       out_dtype="as_input") -> int:
+    B, H, T, dk = q.shape
+    a = PrefillArgs()
+    a.B, a.H, a.T, a.dk, a.dv, a.C = B, H, T, dk, v.shape[-1], int(chunk)
+    a.normalize = int(bool(normalize))
+    a.dtype = DTYPES[q.dtype]
+    a.out_dtype = OUT_DTYPES[out_dtype]
+    return int(load_library().lin_attn_prefill_host_buffer_bytes(ctypes.byref(a)))
+
+
+def lin_attn_decode_step(q, k, v, S, Z=None, out=None, *, feature_map="elu1", gamma=None,
+                         normalize=True, stream=None):
+    """One decode step: q, k [B,H,dk], v [B,H,dv]; S [B,H,dk,dv] and Z [B,H,dk] updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    garr, gptr = _gamma_array(gamma, H)
+    lib = load_library()
+    fn = lib.lin_attn_decode_step_f32 if q.dtype == torch.float32 else lib.lin_attn_decode_step
+    _check("lin_attn_decode_step",
+           fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(S), _ptr(Z), B, H, dk, dv,
+              FEATURE_MAPS[feature_map], gptr, int(bool(normalize)), _stream_handle(stream)))
+    del garr
+    return out
+
+
+def lin_attn_device_error() -> int:
+    code = ctypes.c_int(0)
+    _check("lin_attn_device_error", load_library().lin_attn_device_error(ctypes.byref(code)))
+    return code.value
+
+
+def lin_attn_status_string(status: int) -> str:
+    return load_library().lin_attn_status_string(int(status)).decode()
+
+
+def lin_attn_version() -> int:
+    return int(load_library().lin_attn_version())

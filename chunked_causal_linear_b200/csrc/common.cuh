@@ -1,0 +1,42 @@
+// Launch parameters and index helpers shared by every kernel of the prefill path.
+#pragma once
+
+#include <cstdint>
+
+namespace la {
+
+constexpr int kMaxHeads = 1024;
+
+// Per-head decays, passed by value in the launch parameters (gamma_h = 1 when absent).
+struct GammaTable {
+  float g[kMaxHeads];
+};
+
+// One prefill problem.  The chunk summaries live in `rec`: one record of R floats per
+// (b*H + h, chunk), holding S transposed (dv x dk, row-major: element (j, i) = S[i][j]
+// at j*dk + i) followed by Z (dk floats) when the normalised form is requested
+// (R = dk*dv + dk), else S^T alone (R = dk*dv).  Storing S^T makes the prefix state a
+// K-major operand of the tensor-core product psi(Q) P in K3.
+struct PrefillParams {
+  int BH;          // B * H
+  int H;
+  long long T;
+  int dk, dv, C;
+  int NC;          // number of chunks, ceil(T / C)
+  int L_last;      // valid tokens in the last chunk
+  int R;           // floats per chunk record
+  float eps;       // added to the denominator of the normalised form
+  float* rec;      // [BH, NC, R] chunk summaries, turned into exclusive prefixes by K2
+  float* tot;      // [BH, G, R] segment totals / segment prefixes (log-depth scan only)
+  float* S_final;  // [BH, dk, dv] or nullptr
+  float* Z_final;  // [BH, dk] or nullptr
+  int Ls;          // chunks per scan segment
+  int G;           // number of scan segments, ceil(NC / Ls) (<= 32)
+  int* err;        // device error word
+};
+
+__device__ __forceinline__ int chunk_len(const PrefillParams& p, int c) {
+  return c == p.NC - 1 ? p.L_last : p.C;
+}
+
+}  // namespace la

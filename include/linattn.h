@@ -1,0 +1,223 @@
+/*
+ * linattn.h -- C ABI of the chunked causal linear-attention library for NVIDIA B200
+ * (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * For every (batch b, head h) and every token t < T:
+ *
+ *     S_t = gamma_h * S_{t-1} + psi(k_t) v_t^T        (dk x dv, float32 state)
+ *     Z_t = gamma_h * Z_{t-1} + psi(k_t)              (dk)
+ *     o_t = psi(q_t) S_t / (psi(q_t) . Z_t + eps)     (normalised form), or
+ *     o_t = psi(q_t) S_t                              (unnormalised form)
+ *
+ * with S_{-1} = 0, Z_{-1} = 0, psi = ELU+1 (x + 1 for x > 0, e^x otherwise) or the
+ * identity, and gamma_h = 1 when no decay is given.  Sources: "Log-Depth Chunked
+ * Linear-Attention Scan", sections "Mathematical statement" (inclusive state and
+ * normaliser sums) and "Implementation notes" (ratio with eps); "Linear Attention and
+ * Retentive Networks: How Recurrent Duals and Chunkwise Tiling Eliminate the Quadratic
+ * Bottleneck", sections "The Associative Property and Linear Kernel Formulation" (ELU+1
+ * feature map), "The Recurrent Dual" and "B. Recurrent Representation" (per-head decay).
+ *
+ * How the prefill computes it (the scan page's three kernels):
+ *   K1  per chunk of C tokens: psi, decay weights, and the chunk summaries
+ *       S_loc = sum_j Xi_j psi(k_j) v_j^T,  Z_loc = sum_j Xi_j psi(k_j), Xi_j = gamma^(L-1-j)
+ *       ("Formulas"; decay placement from "C. Chunkwise Recurrent Representation").
+ *   K2  exclusive associative scan of the summaries across chunks
+ *       ((a1,S1,Z1) + (a2,S2,Z2) = (a1 a2, a2 S1 + S2, a2 Z1 + Z2), a = gamma^L), either
+ *       log-depth over segments of chunks or a sequential carry (comparison mode).
+ *   K3  per chunk: the intra-chunk causal part (psi(Q) psi(K)^T masked with gamma^(i-j))
+ *       plus Theta_i psi(q_i) P_c with the chunk's exclusive prefix P_c, Theta_i =
+ *       gamma^(i+1), then the normalisation.
+ * Positions past T in a padded last chunk contribute nothing and do not advance the
+ * decay, so S_final is exactly S_{T-1}.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   Layout   q, k: [B, H, T, dk]; v, out: [B, H, T, dv]; contiguous, row-major.
+ *            S_final / S: [B, H, dk, dv] (row i = key feature, column j = value feature);
+ *            Z_final / Z: [B, H, dk].  All float32 states.
+ *   Memory   Tensor pointers are DEVICE pointers owned by the caller, except where an
+ *            entry point says HOST.  The library never frees caller memory.  Every tensor
+ *            pointer must be 16-byte aligned.
+ *   gamma    HOST array of H float32 decays in [0, 1], or NULL for no decay.  It is read
+ *            during the call and copied into the kernel launches (at most 1024 heads).
+ *   stream   A CUDA stream (cudaStream_t / CUstream), or NULL for the legacy default.
+ *   Async    Device entry points only enqueue work and return; errors raised by the
+ *            kernels surface at the caller's next synchronisation.  No host sync.
+ *   Errors   Arguments are validated before anything is enqueued; on a non-zero status
+ *            nothing has been launched.
+ *   Determinism  No atomics on the data path; results are bitwise reproducible for a
+ *            fixed configuration.
+ */
+#ifndef LINATTN_H_
+#define LINATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream, declared here so the header needs no CUDA
+ * include. */
+typedef struct CUstream_st* la_stream_t;
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARGUMENT = 1, /* NULL required pointer, negative size, gamma outside
+                                  [0,1], normalize with the identity map, out aliasing an
+                                  input, misaligned pointer, bad enum value */
+  LA_ERR_UNSUPPORTED = 2,      /* shape outside the supported set (see below) */
+  LA_ERR_OUT_OF_MEMORY = 3,    /* the library-side workspace could not be allocated */
+  LA_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
+  LA_ERR_INTERNAL = 5          /* a kernel reported a failed internal check */
+} la_status;
+
+typedef enum { LA_FM_IDENTITY = 0, LA_FM_ELU1 = 1 } la_feature_map;
+
+typedef enum {
+  LA_SCAN_LOGDEPTH = 0,   /* K2 over segments of chunks: reduce, log-depth scan, sweep */
+  LA_SCAN_SEQUENTIAL = 1  /* K2 as one sequential carry over chunks (comparison only) */
+} la_scan_mode;
+
+typedef enum { LA_DTYPE_BF16 = 0, LA_DTYPE_F32 = 1 } la_dtype;
+
+/* Element type of `out`: the input type, or float32 (exact-to-accumulator output for
+ * bf16 inputs; the normalised form's outputs shrink with t, so bf16 output rounding can
+ * dominate the error on long sequences). */
+typedef enum { LA_OUT_AS_INPUT = 0, LA_OUT_F32 = 1 } la_out_dtype;
+
+typedef enum {
+  LA_PATH_AUTO = 0,        /* tensor-core kernels where the shape allows, else FMA kernels */
+  LA_PATH_TENSOR_CORE = 1, /* tcgen05/TMEM kernels only (LA_ERR_UNSUPPORTED otherwise) */
+  LA_PATH_FMA = 2          /* CUDA-core fp32 FMA kernels for every step */
+} la_kernel_path;
+
+/*
+ * Supported shapes.
+ *   FMA path (float32 or bf16 inputs): dk, dv multiples of 4 in [4, 128], C in {16, 32, 64}.
+ *   Tensor-core path (bf16 inputs only): dk, dv in {64, 128}, C = 64.
+ * T may be any value >= 0 (a ragged last chunk is handled), B and H any value >= 0 with
+ * B*H*T*max(dk,dv) < 2^62.
+ */
+
+/*
+ * lin_attn_prefill -- bf16 inputs and output, float32 states; the whole K1 -> K2 -> K3
+ * path on `stream`.
+ *   q, k, v   DEVICE bf16, layout above; may be NULL only when B*H*T == 0.
+ *   out       DEVICE bf16 [B,H,T,dv]; must not alias q, k or v.
+ *   S_final   DEVICE float32 [B,H,dk,dv] or NULL (not written).  Final state S_{T-1}.
+ *   Z_final   DEVICE float32 [B,H,dk] or NULL.  Written only when normalize != 0.
+ *   C         chunk length.
+ *   feature_map  la_feature_map.  normalize != 0 requires LA_FM_ELU1 (the identity map
+ *             gives a denominator of indefinite sign).
+ * Uses the log-depth scan and eps = 0.  The workspace is allocated with
+ * cudaMallocAsync / cudaFreeAsync on `stream` (LA_ERR_OUT_OF_MEMORY on failure).
+ * T == 0 zero-fills S_final / Z_final.  Returns a la_status.
+ */
+int lin_attn_prefill(const void* q, const void* k, const void* v, void* out,
+                     float* S_final, float* Z_final, int B, int H, long long T, int dk,
+                     int dv, int C, int feature_map, const float* gamma, int normalize,
+                     la_stream_t stream);
+
+/* lin_attn_prefill_f32 -- the same contract with float32 q, k, v and out; runs the
+ * fp32 FMA kernels. */
+int lin_attn_prefill_f32(const float* q, const float* k, const float* v, float* out,
+                         float* S_final, float* Z_final, int B, int H, long long T, int dk,
+                         int dv, int C, int feature_map, const float* gamma, int normalize,
+                         la_stream_t stream);
+
+/* Bytes of device workspace the prefill needs for this shape (chunk summaries and scan
+ * segment totals).  Pure host computation; 0 for an empty problem. */
+size_t lin_attn_prefill_workspace_bytes(int B, int H, long long T, int dk, int dv, int C,
+                                        int normalize);
+
+/* Every option of the prefill in one struct. */
+typedef struct la_prefill_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* S_final;         /* may be NULL */
+  float* Z_final;         /* may be NULL */
+  int B, H;
+  long long T;
+  int dk, dv, C;
+  int feature_map;        /* la_feature_map */
+  const float* gamma;     /* HOST, H values, or NULL */
+  int normalize;
+  float eps;              /* added to the denominator of the normalised form (>= 0) */
+  int dtype;              /* la_dtype of q, k and v */
+  int out_dtype;          /* la_out_dtype of out */
+  int scan_mode;          /* la_scan_mode */
+  int kernel_path;        /* la_kernel_path */
+  void* workspace;        /* DEVICE, >= lin_attn_prefill_workspace_bytes(), 256-byte
+                             aligned; NULL = allocate on the stream */
+  size_t workspace_bytes;
+  la_stream_t stream;
+} la_prefill_args;
+
+/* lin_attn_prefill_ex -- the prefill with every option of la_prefill_args.  A caller
+ * workspace that is too small or misaligned gives LA_ERR_INVALID_ARGUMENT. */
+int lin_attn_prefill_ex(const la_prefill_args* args);
+
+/*
+ * lin_attn_prefill_timed -- lin_attn_prefill_ex with a CUDA event recorded on the stream
+ * before every kernel launch and after the last one; synchronises the stream and writes
+ * each kernel's device duration (milliseconds, launch order) to kernel_ms[0 ..].
+ * *n_kernels receives the number of kernels the prefill launched (K1, the scan's
+ * kernels, K3: 5 with the log-depth scan, 3 with the sequential carry).  For profiling;
+ * the results are identical to lin_attn_prefill_ex.
+ */
+int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int max_kernels,
+                           int* n_kernels);
+
+/*
+ * lin_attn_prefill_host -- the same computation with HOST buffers, for callers whose
+ * data lives in host memory.  q, k, v, out, S_final, Z_final are HOST pointers (pinned
+ * memory gives full copy bandwidth; pageable memory works).  `device_buffer` is DEVICE
+ * memory of at least lin_attn_prefill_host_buffer_bytes() bytes used to stage the
+ * tensors and the workspace, or NULL to allocate it on the stream.  Copies the inputs
+ * to the device, runs the prefill, copies the results back and synchronises `stream`
+ * before returning, so the host outputs are ready on LA_OK.
+ */
+int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
+                          size_t device_buffer_bytes);
+size_t lin_attn_prefill_host_buffer_bytes(const la_prefill_args* host_args);
+
+/*
+ * lin_attn_decode_step -- one recurrent step for every (b, h), the O(1) decode that the
+ * prefill's final states feed ("The Recurrent Dual"; "B. Recurrent Representation").
+ *   q, k      DEVICE bf16 [B,H,dk]   v DEVICE bf16 [B,H,dv]   out DEVICE bf16 [B,H,dv]
+ *   S, Z      DEVICE float32 [B,H,dk,dv] / [B,H,dk], updated IN PLACE:
+ *             S <- gamma S + psi(k) v^T, Z <- gamma Z + psi(k); then
+ *             out = psi(q) S / (psi(q) . Z) (normalize) or psi(q) S.
+ *             Z may be NULL when normalize == 0.
+ * Shapes: dk, dv in [1, 256].  One kernel launch, no workspace.
+ */
+int lin_attn_decode_step(const void* q, const void* k, const void* v, void* out, float* S,
+                         float* Z, int B, int H, int dk, int dv, int feature_map,
+                         const float* gamma, int normalize, la_stream_t stream);
+
+/* lin_attn_decode_step_f32 -- the same with float32 q, k, v and out. */
+int lin_attn_decode_step_f32(const float* q, const float* k, const float* v, float* out,
+                             float* S, float* Z, int B, int H, int dk, int dv,
+                             int feature_map, const float* gamma, int normalize,
+                             la_stream_t stream);
+
+/* Reads and clears the device-side error word that kernels set when an internal check
+ * or a bounded wait fails (0 = none).  Synchronises the current device. */
+int lin_attn_device_error(int* code);
+
+/* A static, human-readable name for a la_status value. */
+const char* lin_attn_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int lin_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LINATTN_H_ */

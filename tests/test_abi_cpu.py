@@ -1,0 +1,146 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol the header declares,
+sizes the workspace as documented, and rejects bad arguments before touching CUDA."""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "linattn.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from chunked_causal_linear_b200.build import build
+    from chunked_causal_linear_b200.binding import load_library
+    build()
+    return load_library()
+
+
+def header_functions() -> list[str]:
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(lin_attn_\w+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_header_declares_the_expected_entry_points():
+    from chunked_causal_linear_b200.binding import EXPORTED_SYMBOLS
+    assert header_functions() == sorted(EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_links_no_torch():
+    import subprocess
+    from chunked_causal_linear_b200.binding import LIB_PATH
+    out = subprocess.run(["ldd", str(LIB_PATH)], capture_output=True, text=True).stdout
+    assert "torch" not in out and "c10" not in out
+
+
+def test_status_strings_and_version(lib):
+    from chunked_causal_linear_b200 import binding as b
+    for code, name in b.STATUS_NAMES.items():
+        assert b.lin_attn_status_string(code) == name
+    assert b.lin_attn_status_string(99) == "LA_ERR_UNKNOWN"
+    assert b.lin_attn_version() == 10000
+
+
+def expected_workspace(B, H, T, dk, dv, C, normalize):
+    if B * H == 0 or T == 0:
+        return 0
+    nc = -(-T // C)
+    R = dk * dv + (dk if normalize else 0)
+    ls = max(1, -(-nc // 32))
+    G = -(-nc // ls)
+    a256 = lambda x: (x + 255) // 256 * 256
+    return a256(B * H * nc * R * 4) + a256(B * H * G * R * 4)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 256, 32, 32, 32, 1), (4, 16, 4096, 64, 64, 64, 1),
+                                   (2, 32, 15990, 128, 128, 64, 1),
+                                   (1, 32, 131072, 128, 128, 64, 0),
+                                   (1, 8, 1048576, 64, 64, 64, 1), (1, 1, 1, 16, 16, 16, 0),
+                                   (0, 4, 100, 64, 64, 64, 1), (3, 3, 0, 64, 64, 64, 1)])
+def test_workspace_bytes(lib, shape):
+    from chunked_causal_linear_b200.binding import lin_attn_prefill_workspace_bytes
+    assert lin_attn_prefill_workspace_bytes(*shape) == expected_workspace(*shape)
+
+
+def test_scan_segments_are_at_most_32():
+    for nc in (1, 2, 31, 32, 33, 64, 250, 2048, 16384, 100000):
+        ls = max(1, math.ceil(nc / 32))
+        assert math.ceil(nc / ls) <= 32
+
+
+def _args(**kw):
+    from chunked_causal_linear_b200.binding import PrefillArgs
+    a = PrefillArgs()
+    base = dict(q=0x1000, k=0x2000000, v=0x4000000, out=0x6000000, B=1, H=2, T=128, dk=64,
+                dv=64, C=64, feature_map=1, normalize=1, eps=0.0, dtype=0, scan_mode=0,
+                kernel_path=0)
+    base.update(kw)
+    for key, val in base.items():
+        setattr(a, key, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(T=-5), 1), (dict(dk=0), 1), (dict(dtype=7), 1),
+    (dict(feature_map=3), 1), (dict(scan_mode=2), 1), (dict(kernel_path=9), 1),
+    (dict(feature_map=0, normalize=1), 1), (dict(eps=-1.0), 1), (dict(eps=float("inf")), 1),
+    (dict(dk=5), 2), (dict(dv=256), 2), (dict(C=48), 2), (dict(C=128), 2),
+    (dict(kernel_path=1, C=32), 2), (dict(kernel_path=1, dk=32), 2),
+    (dict(kernel_path=1, dtype=1), 2),
+    (dict(q=0), 1), (dict(out=0), 1), (dict(q=0x1001), 1), (dict(out=0x1008), 1),
+    (dict(out=0x1000), 1), (dict(out=0x2000000 + 64), 1),
+    (dict(workspace=0x100010), 1),
+])
+def test_argument_errors_before_any_launch(lib, kw, status):
+    a = _args(**kw)
+    assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == status
+
+
+def test_empty_problems_return_ok_without_cuda(lib):
+    for kw in (dict(B=0), dict(H=0), dict(T=0, S_final=None, Z_final=None)):
+        a = _args(**kw)
+        assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == 0
+    assert lib.lin_attn_prefill_ex(None) == 1
+
+
+def test_gamma_validation(lib):
+    a = _args(B=0)
+    for bad in ([0.5, 1.5], [-0.1, 0.5], [float("nan"), 0.5]):
+        arr = (ctypes.c_float * 2)(*bad)
+        a.gamma = ctypes.cast(arr, ctypes.c_void_p)
+        assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == 1
+    arr = (ctypes.c_float * 2)(0.0, 1.0)
+    a.gamma = ctypes.cast(arr, ctypes.c_void_p)
+    assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == 0
+    big = _args(B=0, H=2000)
+    arr2 = (ctypes.c_float * 2000)(*([0.5] * 2000))
+    big.gamma = ctypes.cast(arr2, ctypes.c_void_p)
+    assert lib.lin_attn_prefill_ex(ctypes.byref(big)) == 2
+
+
+def test_decode_argument_errors(lib):
+    f = lib.lin_attn_decode_step
+    assert f(None, None, None, None, None, None, 1, 1, 64, 64, 1, None, 1, None) == 1
+    assert f(None, None, None, None, None, None, -1, 1, 64, 64, 1, None, 1, None) == 1
+    assert f(None, None, None, None, None, None, 1, 1, 512, 64, 1, None, 1, None) == 2
+    assert f(None, None, None, None, None, None, 1, 1, 64, 64, 0, None, 1, None) == 1
+    assert f(None, None, None, None, None, None, 0, 1, 64, 64, 1, None, 1, None) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from chunked_causal_linear_b200.binding import load_library
+    with pytest.raises(RuntimeError):
+        load_library(tmp_path / "missing.so")

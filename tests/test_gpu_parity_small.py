@@ -1,0 +1,121 @@
+"""GPU parity on small shapes: every mode, both kernel paths, ragged tails.
+
+Each case runs the CUDA library through the C ABI and compares with the fp64 oracle on
+the same inputs: max |err| <= 2e-2 * rms(oracle) for bf16 inputs (tensor-core and FMA
+kernels, float32 output), <= 1e-4 * rms(oracle) for float32 inputs (FMA kernels).  A
+bf16 output adds its own rounding to that bound (see ``assert_close_rounded_out``).
+Sizes span several chunks and a ragged last chunk.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from chunked_causal_linear_b200.workloads import WORKLOADS, Workload, make_inputs
+from gpu_common import (TOL_BF16, TOL_F32, assert_close, assert_close_rounded_out,
+                        gammas_for, gpu_prefill, oracle_prefill, to_np)
+
+pytestmark = pytest.mark.gpu
+
+MODES = {
+    "norm": dict(feature_map="elu1", decay=False, normalize=True),
+    "unnorm": dict(feature_map="elu1", decay=False, normalize=False),
+    "retention": dict(feature_map="identity", decay=True, normalize=False),
+    "decay_norm": dict(feature_map="elu1", decay=True, normalize=True),
+}
+
+
+def _case(T, dk, dv, C, mode, dtype="bf16", B=2, H=3, seed=0):
+    m = MODES[mode]
+    scale = 1.0 / math.sqrt(dk) if m["feature_map"] == "identity" else 0.5
+    w = Workload("case", B=B, H=H, T=T, dk=dk, dv=dv, C=C, dtype=dtype, scale=scale,
+                 feature_map=m["feature_map"], decay=m["decay"], normalize=m["normalize"])
+    q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
+    gamma = gammas_for(H, seed) if m["decay"] else None
+    return w, q, k, v, gamma
+
+
+def _check(w, q, k, v, gamma, tol, **kw):
+    out, S, Z = gpu_prefill(q, k, v, C=w.C, feature_map=w.feature_map, gamma=gamma,
+                            normalize=w.normalize, **kw)
+    o_ref, S_ref, Z_ref = oracle_prefill(q, k, v, feature_map=w.feature_map, gamma=gamma,
+                                         normalize=w.normalize)
+    assert_close(to_np(out), o_ref, tol, "out")
+    assert_close(to_np(S), S_ref, tol, "S_final")
+    if w.normalize:
+        assert_close(to_np(Z), Z_ref, tol, "Z_final")
+
+
+@pytest.mark.parametrize("mode", sorted(MODES))
+@pytest.mark.parametrize("T", [1, 33, 64, 100, 257, 1000])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+def test_tensor_core_path(dk, dv, T, mode):
+    w, q, k, v, gamma = _case(T, dk, dv, 64, mode)
+    _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core")
+
+
+@pytest.mark.parametrize("mode", sorted(MODES))
+@pytest.mark.parametrize("T", [33, 257])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (32, 64)])
+def test_fma_path_bf16(dk, dv, T, mode):
+    w, q, k, v, gamma = _case(T, dk, dv, 64 if dk >= 64 else 32, mode)
+    _check(w, q, k, v, gamma, TOL_BF16, kernel_path="fma")
+
+
+@pytest.mark.parametrize("mode", ["norm", "retention", "decay_norm"])
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 32), (64, 32), (128, 128)])
+@pytest.mark.parametrize("T", [1, 50, 300])
+def test_fma_path_f32(T, dk, dv, C, mode):
+    w, q, k, v, gamma = _case(T, dk, dv, C, mode, dtype="f32")
+    _check(w, q, k, v, gamma, TOL_F32)
+
+
+@pytest.mark.parametrize("mode", sorted(MODES))
+@pytest.mark.parametrize("path", ["tensor_core", "fma"])
+@pytest.mark.parametrize("T", [100, 1000])
+def test_bf16_output(T, path, mode):
+    w, q, k, v, gamma = _case(T, 128, 128, 64, mode)
+    out, S, Z = gpu_prefill(q, k, v, C=64, feature_map=w.feature_map, gamma=gamma,
+                            normalize=w.normalize, kernel_path=path, out_dtype="as_input")
+    assert out.dtype == torch.bfloat16
+    o_ref, S_ref, _ = oracle_prefill(q, k, v, feature_map=w.feature_map, gamma=gamma,
+                                     normalize=w.normalize)
+    assert_close_rounded_out(to_np(out), o_ref, TOL_BF16, "bf16 out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+@pytest.mark.parametrize("mode", ["norm", "retention"])
+@pytest.mark.parametrize("T", [100, 1000, 64 * 70 + 5])
+def test_scan_modes_agree_with_oracle(T, mode):
+    w, q, k, v, gamma = _case(T, 64, 64, 64, mode)
+    for scan in ("logdepth", "sequential"):
+        _check(w, q, k, v, gamma, TOL_BF16, scan=scan)
+
+
+def test_pr1_ref_fp32_against_oracle_and_golden():
+    from golden.make_golden import SAMPLE_T, load_golden
+    w = WORKLOADS["pr1_ref"]
+    q, k, v = make_inputs(w, seed=0, device="cuda", gen_device="cpu")
+    out, S, Z = gpu_prefill(q, k, v, C=w.C, feature_map=w.feature_map, gamma=None,
+                            normalize=True)
+    o_ref, S_ref, Z_ref = oracle_prefill(q, k, v, feature_map=w.feature_map, gamma=None,
+                                         normalize=True)
+    assert_close(to_np(out), o_ref, TOL_F32, "out")
+    assert_close(to_np(S), S_ref, TOL_F32, "S_final")
+    assert_close(to_np(Z), Z_ref, TOL_F32, "Z_final")
+    gold = load_golden()
+    assert_close(to_np(out)[:, :, list(SAMPLE_T)], gold["out_sampled"], TOL_F32, "golden out")
+    assert_close(to_np(S), gold["S_final"], TOL_F32, "golden S")
+    assert_close(to_np(Z), gold["Z_final"], TOL_F32, "golden Z")
+
+
+@pytest.mark.parametrize("seed", [1])
+def test_pr1_ref_fp32_second_seed(seed):
+    w = WORKLOADS["pr1_ref"]
+    q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
+    _check(w, q, k, v, None, TOL_F32)
