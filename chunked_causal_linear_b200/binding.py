@@ -27,7 +27,7 @@ OUT_DTYPES = {"as_input": 0, "f32": 1}
 EXPORTED_SYMBOLS = (
     "lin_attn_prefill", "lin_attn_prefill_f32", "lin_attn_prefill_workspace_bytes",
     "lin_attn_prefill_ex", "lin_attn_prefill_timed", "lin_attn_prefill_host",
-    "lin_attn_prefill_host_buffer_bytes",
+    "lin_attn_prefill_host_buffer_bytes", "lin_attn_prefill_noalloc",
     "lin_attn_decode_step", "lin_attn_decode_step_f32", "lin_attn_device_error",
     "lin_attn_status_string", "lin_attn_version",
 )
@@ -74,6 +74,7 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_prefill_timed": (i, [ctypes.POINTER(PrefillArgs), ctypes.POINTER(f), i,
                                        ctypes.POINTER(i)]),
         "lin_attn_prefill_host": (i, [ctypes.POINTER(PrefillArgs), vp, sz]),
+        "lin_attn_prefill_noalloc": (i, [ctypes.POINTER(PrefillArgs)]),
         "lin_attn_prefill_host_buffer_bytes": (sz, [ctypes.POINTER(PrefillArgs)]),
         "lin_attn_decode_step": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "lin_attn_decode_step_f32": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
@@ -201,6 +202,24 @@ def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
     nbytes = 0 if device_buffer is None else device_buffer.numel() * device_buffer.element_size()
     _check("lin_attn_prefill_host",
            load_library().lin_attn_prefill_host(ctypes.byref(a), _ptr(device_buffer), nbytes))
+    del keep
+    return out, S_final, Z_final
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def lin_attn_prefill_noalloc(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
+                             feature_map="elu1", gamma=None, normalize=True, eps=0.0,
+                             scan="logdepth", kernel_path="auto", stream=None,
+                             out_dtype="as_input"):
+    """The prefill with its workspace in the library's fixed device array (no device
+    allocation by the library; the caller provides every output tensor)."""
+    a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
+                        gamma=gamma, normalize=normalize, eps=eps, scan=scan,
+                        kernel_path=kernel_path, workspace=None, stream=_stream_handle(stream),
+                        out_dtype=out_dtype)
+    _check("lin_attn_prefill_noalloc", load_library().lin_attn_prefill_noalloc(ctypes.byref(a)))
     del keep
     return out, S_final, Z_final
 

@@ -350,6 +350,9 @@ HostLayout host_layout(const la_prefill_args& a) {
 }
 
 }  // namespace
+
+int prefill_with_args(const la_prefill_args& a) { return prefill(a); }
+
 }  // namespace la
 
 extern "C" {

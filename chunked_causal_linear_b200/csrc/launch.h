@@ -4,9 +4,13 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/linattn.h"
 #include "common.cuh"
 
 namespace la {
+
+// The full prefill of lin_attn_prefill_ex (validation, workspace, launches).
+int prefill_with_args(const la_prefill_args& a);
 
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
 

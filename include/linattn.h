@@ -187,6 +187,28 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
 size_t lin_attn_prefill_host_buffer_bytes(const la_prefill_args* host_args);
 
 /*
+ * lin_attn_prefill_noalloc -- lin_attn_prefill_ex without any device allocation.  (No
+ * passage of the pages corresponds to it; it exists for callers that cannot allocate.)
+ *
+ * Callers that must not allocate device memory while they run -- processes that
+ * reserve a fixed memory budget at start-up, frameworks that route every allocation
+ * through their own allocator, code that cannot recover from a failed allocation -- use
+ * this entry point: the workspace is a fixed array inside the library's device image
+ * (LA_NOALLOC_SCRATCH_BYTES bytes, held by every GPU that loads the library until the
+ * process exits) instead of cudaMalloc / cudaMallocAsync memory.  args->workspace and
+ * args->workspace_bytes are ignored; everything else is as in lin_attn_prefill_ex.
+ *   - A problem whose workspace (lin_attn_prefill_workspace_bytes) exceeds
+ *     LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_UNSUPPORTED and launches nothing.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - Every call shares the array and it keeps the last call's contents; the kernels
+ *     write all workspace bytes before reading them, so no clearing is needed.  Calls
+ *     whose work overlaps on the GPU race on the array: serialise them.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int lin_attn_prefill_noalloc(const la_prefill_args* args);
+
+/*
  * lin_attn_decode_step -- one recurrent step for every (b, h), the O(1) decode that the
  * prefill's final states feed ("The Recurrent Dual"; "B. Recurrent Representation").
  *   q, k      DEVICE bf16 [B,H,dk]   v DEVICE bf16 [B,H,dv]   out DEVICE bf16 [B,H,dv]
