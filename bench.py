@@ -304,11 +304,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads instead (smaller cases for "
+                         "profiler captures; every other size unchanged)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     w = WORKLOADS[args.workload]
+    if args.heads:
+        w = w.with_(H=args.heads, name=f"{w.name}_h{args.heads}")
     if args.impl == "reference":
         info = ranks.rank_info()
         reference_arm(args, w, info)
