@@ -47,33 +47,51 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
-KERNEL_NAMES = {
-    "logdepth": ["k1_tc", "k2_reduce", "k2_scan_totals", "k2_downsweep", "k3_tc"],
-    "sequential": ["k1_tc", "k2_sequential", "k3_tc"],
-}
+K2_NAMES = {"logdepth": ["k2_reduce", "k2_scan_totals", "k2_downsweep"],
+            "sequential": ["k2_sequential"]}
 KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce": "scan.cu",
                   "k2_scan_totals": "scan.cu", "k2_downsweep": "scan.cu",
-                  "k2_sequential": "scan.cu"}
+                  "k2_sequential": "scan.cu", "k1_seg": "seg_kernels.cu",
+                  "k3_seg": "seg_kernels.cu"}
+
+
+def effective_algorithm(w, requested: str) -> str:
+    """The algorithm the library runs for this workload on the tensor-core path."""
+    seg_ok = w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv == 128
+    if requested == "segmented" or (requested == "auto" and seg_ok):
+        return "segmented"
+    return "chunked"
+
+
+def kernel_names(algo: str, scan: str) -> list[str]:
+    k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
+    return [k1, *K2_NAMES[scan], k3]
 
 
 # ---------------------------------------------------------------------------------------
 # Algorithmic bytes
 
 
-def layout(w):
+def layout(w, algo: str = "chunked"):
+    """(scan elements per (b, h), scan segments G, floats per record) as the library lays
+    them out: chunks for the chunked algorithm, segments of chunks for the segmented one."""
     NC = -(-w.T // w.C)
-    Ls = max(1, -(-NC // 32))
-    G = -(-NC // Ls)
+    n = NC
+    if algo == "segmented":
+        lseg = max(1, min(64, (w.B * w.H * NC) // (4 * 148)))
+        n = -(-NC // lseg)
+    Ls = max(1, -(-n // 32))
+    G = -(-n // Ls)
     R = w.dk * w.dv + (w.dk if w.normalize else 0)
-    return NC, G, R
+    return n, G, R
 
 
-def kernel_bytes(w, name: str, out_elem: int) -> int:
+def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked") -> int:
     """Bytes each kernel must move for its own role (one launch)."""
     BH = w.B * w.H
-    NC, G, R = layout(w)
+    n, G, R = layout(w, algo)
     e_in = 2 if w.dtype == "bf16" else 4
-    rec = BH * NC * R * 4
+    rec = BH * n * R * 4
     if name.startswith("k1"):
         return BH * w.T * (w.dk + w.dv) * e_in + rec
     if name == "k2_reduce":
@@ -84,9 +102,31 @@ def kernel_bytes(w, name: str, out_elem: int) -> int:
         return 2 * rec + BH * G * R * 4
     if name == "k2_sequential":
         return 2 * rec + BH * R * 4
-    if name.startswith("k3"):
-        return BH * w.T * (2 * w.dk + w.dv) * e_in + BH * (NC - 1) * R * 4 + BH * w.T * w.dv * out_elem
+    if name == "k3_tc":
+        return BH * w.T * (2 * w.dk + w.dv) * e_in + BH * (n - 1) * R * 4 + BH * w.T * w.dv * out_elem
+    if name == "k3_seg":
+        return BH * w.T * (2 * w.dk + w.dv) * e_in + rec + BH * w.T * w.dv * out_elem
     raise KeyError(name)
+
+
+def algo_bytes(w, out_elem: int, algo: str) -> int:
+    """Whole-step algorithmic bytes of an algorithm: its input reads (the segmented one
+    reads k and v in K1 and again in K3), the output, the final states, and four passes of
+    its records (K1 write, K2 read and write, K3 read)."""
+    BH = w.B * w.H
+    n, G, R = layout(w, algo)
+    e_in = 2 if w.dtype == "bf16" else 4
+    kv_again = BH * w.T * (w.dk + w.dv) * e_in if algo == "segmented" else 0
+    return (BH * w.T * (2 * w.dk + w.dv) * e_in + kv_again + BH * w.T * w.dv * out_elem
+            + BH * R * 4 + 4 * BH * n * R * 4)
+
+
+def min_bytes(w, out_elem: int) -> int:
+    """Bytes any exact method must move: q, k, v read once, output and final states written."""
+    BH = w.B * w.H
+    e_in = 2 if w.dtype == "bf16" else 4
+    return (BH * w.T * (2 * w.dk + w.dv) * e_in + BH * w.T * w.dv * out_elem
+            + BH * (w.dk * w.dv + (w.dk if w.normalize else 0)) * 4)
 
 
 def method_bytes(w, out_elem: int) -> int:
@@ -275,11 +315,41 @@ def reference_arm(args, w, info):
     print(json.dumps(line), flush=True)
 
 
+def sweep_scan(args, dev):
+    """K2 device time, log-depth scan vs sequential carry, on the chunked algorithm (every
+    chunk is a scan element): B1 H8 d64 C64 with 256 .. 16384 chunks, then the two
+    long-sequence workloads at full size."""
+    cases = [WORKLOADS["scan_depth_1m"].with_(T=nc * 64, name=f"b1h8d64_nc{nc}")
+             for nc in (256, 512, 1024, 2048, 4096, 8192, 16384)]
+    cases += [WORKLOADS["retention_128k"], WORKLOADS["scan_depth_1m"]]
+    for w in cases:
+        q, k, v = make_inputs(w, seed=0, device=dev)
+        ws = torch.empty(B.lin_attn_prefill_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.C,
+                                                            w.normalize),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
+        row = {"sweep": "k2_scan", "workload": w.name, "chunks": -(-w.T // w.C),
+               "columns": w.B * w.H * (w.dk * w.dv + (w.dk if w.normalize else 0))}
+        for scan in ("logdepth", "sequential"):
+            kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=w.gammas(),
+                      normalize=w.normalize, scan=scan, kernel_path="tensor_core",
+                      workspace=ws, out_dtype="f32", algorithm="chunked")
+            for _ in range(3):
+                B.lin_attn_prefill_timed(q, k, v, out, **kw)
+            t = [B.lin_attn_prefill_timed(q, k, v, out, **kw) for _ in range(5)]
+            k2 = [sum(x[1:-1]) for x in t]
+            row[f"k2_ms_{scan}"] = statistics.median(k2)
+        row["logdepth_speedup"] = row["k2_ms_sequential"] / row["k2_ms_logdepth"]
+        print(json.dumps(row), flush=True)
+        del q, k, v, ws, out
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
             "gamma": "1 - 2^(-5-3h/31) per head" if w.decay else None,
             "normalize": w.normalize, "scan": args.scan, "out_dtype": args.out_dtype,
+            "algorithm": effective_algorithm(w, args.algorithm),
             "kernel_path": "tensor_core", "l2": "inputs larger than L2, no flush",
             "parallelism": "replicas (one independent problem per GPU)"}
 
@@ -296,6 +366,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="retention_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--scan", default="logdepth", choices=["logdepth", "sequential"])
+    ap.add_argument("--algorithm", default="auto", choices=["auto", "chunked", "segmented"])
     ap.add_argument("--out-dtype", default="f32", choices=["f32", "as_input"])
     ap.add_argument("--kernel-timing-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -304,6 +375,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep-scan", action="store_true",
+                    help="instead of the benchmark line: time K2 (log-depth vs sequential "
+                         "carry) over a range of chunk counts, one JSON line per point")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -323,6 +397,10 @@ def main():
     dev = torch.device("cuda", info.local_rank)
     torch.cuda.set_device(dev)
     B.load_library()
+    if args.sweep_scan:
+        sweep_scan(args, dev)
+        ranks.finish(info)
+        return
 
     q, k, v = make_inputs(w, seed=info.rank, device=dev)
     out_dtype = torch.float32 if args.out_dtype == "f32" else q.dtype
@@ -334,8 +412,10 @@ def main():
                                                         w.normalize),
                      dtype=torch.uint8, device=dev)
     gam = w.gammas()
+    algo = effective_algorithm(w, args.algorithm)
     kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
-              scan=args.scan, kernel_path="tensor_core", workspace=ws, out_dtype=args.out_dtype)
+              scan=args.scan, kernel_path="tensor_core", workspace=ws, out_dtype=args.out_dtype,
+              algorithm=algo)
 
     def step():
         B.lin_attn_prefill(q, k, v, out, S, Z, **kw)
@@ -366,11 +446,11 @@ def main():
         ms, clocks = timed_region()
         remeasured = True
     ms_max = ranks.max_over_ranks(ms, info, dev)
-    n_kern = len(KERNEL_NAMES[args.scan])
+    names = kernel_names(algo, args.scan)
+    n_kern = len(names)
     value = info.world * w.tokens_heads / (ms_max / 1000.0)
 
     # Per-kernel device times (events between the library's own launches, same stream).
-    names = KERNEL_NAMES[args.scan]
     per = [[] for _ in names]
     for _ in range(max(1, args.kernel_timing_steps)):
         t = B.lin_attn_prefill_timed(q, k, v, out, S, Z, **kw)
@@ -379,17 +459,22 @@ def main():
     kern_ms = {n: statistics.mean(x) for n, x in zip(names, per)}
     dom = max(kern_ms, key=kern_ms.get)
     peak, peak_kind = measured_peaks()
-    dom_bytes = kernel_bytes(w, dom, out_elem)
+    dom_bytes = kernel_bytes(w, dom, out_elem, algo)
     achieved = dom_bytes / (kern_ms[dom] / 1000.0) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak,
                 "traffic": recorded_traffic(dom, w.name),
                 "algorithmic_bytes": dom_bytes, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s"}
-    mb = method_bytes(w, out_elem)
-    step_roof = {"bytes_method": mb, "achieved_gbs": mb / (ms_max / 1000.0) / 1e9,
-                 "frac_of_measured": mb / (ms_max / 1000.0) / 1e9 / peak,
-                 "frac_of_nominal_8tbs": mb / (ms_max / 1000.0) / 1e9 / NOMINAL_HBM_GBS}
+    ab = algo_bytes(w, out_elem, algo)
+    gbs = lambda nbytes: nbytes / (ms_max / 1000.0) / 1e9
+    step_roof = {"algorithm": algo, "bytes": ab, "achieved_gbs": gbs(ab),
+                 "frac_of_measured": gbs(ab) / peak,
+                 "frac_of_nominal_8tbs": gbs(ab) / NOMINAL_HBM_GBS,
+                 "bytes_min": min_bytes(w, out_elem),
+                 "frac_min_of_measured": gbs(min_bytes(w, out_elem)) / peak,
+                 "bytes_chunked_method": method_bytes(w, out_elem),
+                 "time_at_measured_bw_ms": ab / (peak * 1e9) * 1e3}
 
     # End to end through the host-buffer entry point (pinned host memory).
     e2e = None
@@ -399,7 +484,8 @@ def main():
         Sh = torch.empty(S.shape, dtype=torch.float32).pin_memory()
         Zh = torch.empty(Z.shape, dtype=torch.float32).pin_memory() if Z is not None else None
         hkw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
-                   scan=args.scan, kernel_path="tensor_core", out_dtype=args.out_dtype)
+                   scan=args.scan, kernel_path="tensor_core", out_dtype=args.out_dtype,
+                   algorithm=algo)
         dbuf = torch.empty(B.lin_attn_prefill_host_buffer_bytes(qh, vh, chunk=w.C,
                                                                 normalize=w.normalize,
                                                                 out_dtype=args.out_dtype),

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "LA_OK", 1: "LA_ERR_INVALID_ARGUMENT", 2: "LA_ERR_UNSUPPORTED
 FEATURE_MAPS = {"identity": 0, "elu1": 1}
 SCAN_MODES = {"logdepth": 0, "sequential": 1}
 KERNEL_PATHS = {"auto": 0, "tensor_core": 1, "fma": 2}
+ALGORITHMS = {"auto": 0, "chunked": 1, "segmented": 2}
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 OUT_DTYPES = {"as_input": 0, "f32": 1}
 
@@ -48,7 +49,9 @@ class PrefillArgs(ctypes.Structure):
         ("feature_map", ctypes.c_int), ("gamma", ctypes.c_void_p), ("normalize", ctypes.c_int),
         ("eps", ctypes.c_float), ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
         ("scan_mode", ctypes.c_int),
-        ("kernel_path", ctypes.c_int), ("workspace", ctypes.c_void_p),
+        ("kernel_path", ctypes.c_int), ("algorithm", ctypes.c_int),
+        ("segment_chunks", ctypes.c_int),
+        ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
     ]
 
@@ -119,7 +122,8 @@ def _gamma_array(gamma, H):
 
 
 def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, normalize, eps,
-              scan, kernel_path, workspace, stream, out_dtype="as_input"):
+              scan, kernel_path, workspace, stream, out_dtype="as_input", algorithm="auto",
+              segment_chunks=0):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     garr, gptr = _gamma_array(gamma, H)
@@ -135,6 +139,8 @@ def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, norm
     a.out_dtype = OUT_DTYPES[out_dtype]
     a.scan_mode = SCAN_MODES[scan]
     a.kernel_path = KERNEL_PATHS[kernel_path]
+    a.algorithm = ALGORITHMS[algorithm]
+    a.segment_chunks = int(segment_chunks)
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = stream
@@ -148,7 +154,8 @@ def lin_attn_prefill_workspace_bytes(B, H, T, dk, dv, C, normalize) -> int:
 def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
                      feature_map="elu1", gamma=None, normalize=True, eps=0.0, scan="logdepth",
                      kernel_path="auto", workspace=None, stream=None, want_states=True,
-                     out_dtype="as_input"):
+                     out_dtype="as_input", algorithm="auto",
+              segment_chunks=0):
     """Runs the prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (bf16 or float32).
 
     out_dtype "f32" writes a float32 output for bf16 inputs.  Allocates out / S_final /
@@ -166,7 +173,8 @@ def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=workspace,
-                        stream=_stream_handle(stream), out_dtype=out_dtype)
+                        stream=_stream_handle(stream), out_dtype=out_dtype, algorithm=algorithm,
+                        segment_chunks=segment_chunks)
     _check("lin_attn_prefill_ex", load_library().lin_attn_prefill_ex(ctypes.byref(a)))
     del keep
     return out, S_final, Z_final
@@ -175,13 +183,14 @@ def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
 def lin_attn_prefill_timed(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
                            feature_map="elu1", gamma=None, normalize=True, eps=0.0,
                            scan="logdepth", kernel_path="auto", workspace=None, stream=None,
-                           out_dtype="as_input") -> list[float]:
+                           out_dtype="as_input", algorithm="auto", segment_chunks=0) -> list[float]:
     """Runs the prefill once with an event around every kernel; returns the kernels'
     device durations in milliseconds, in launch order (synchronous)."""
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=workspace,
-                        stream=_stream_handle(stream), out_dtype=out_dtype)
+                        stream=_stream_handle(stream), out_dtype=out_dtype, algorithm=algorithm,
+                        segment_chunks=segment_chunks)
     ms = (ctypes.c_float * 8)()
     n = ctypes.c_int(0)
     _check("lin_attn_prefill_timed",
@@ -193,12 +202,14 @@ def lin_attn_prefill_timed(q, k, v, out, S_final=None, Z_final=None, *, chunk=64
 def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
                           feature_map="elu1", gamma=None, normalize=True, eps=0.0,
                           scan="logdepth", kernel_path="auto", device_buffer=None, stream=None,
-                          out_dtype="as_input"):
+                          out_dtype="as_input", algorithm="auto",
+              segment_chunks=0):
     """Runs the prefill on HOST tensors (pinned for full copy bandwidth); synchronous."""
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=None, stream=_stream_handle(stream),
-                        out_dtype=out_dtype)
+                        out_dtype=out_dtype, algorithm=algorithm,
+                        segment_chunks=segment_chunks)
     nbytes = 0 if device_buffer is None else device_buffer.numel() * device_buffer.element_size()
     _check("lin_attn_prefill_host",
            load_library().lin_attn_prefill_host(ctypes.byref(a), _ptr(device_buffer), nbytes))
@@ -212,13 +223,15 @@ NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 def lin_attn_prefill_noalloc(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
                              feature_map="elu1", gamma=None, normalize=True, eps=0.0,
                              scan="logdepth", kernel_path="auto", stream=None,
-                             out_dtype="as_input"):
+                             out_dtype="as_input", algorithm="auto",
+              segment_chunks=0):
     """The prefill with its workspace in the library's fixed device array (no device
     allocation by the library; the caller provides every output tensor)."""
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=None, stream=_stream_handle(stream),
-                        out_dtype=out_dtype)
+                        out_dtype=out_dtype, algorithm=algorithm,
+                        segment_chunks=segment_chunks)
     _check("lin_attn_prefill_noalloc", load_library().lin_attn_prefill_noalloc(ctypes.byref(a)))
     del keep
     return out, S_final, Z_final

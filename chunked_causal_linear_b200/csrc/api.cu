@@ -133,7 +133,7 @@ int check_gamma(const float* gamma, int H, GammaTable* gt) {
   return LA_OK;
 }
 
-enum class Path { kFma, kTensorCore };
+enum class Path { kFma, kTensorCore, kSegmented };
 
 // Validates `a` and picks the kernel path.  Touches no CUDA state except the device
 // capability query, which happens only for non-empty problems.
@@ -146,6 +146,8 @@ int validate(const la_prefill_args& a, Path* path) {
     return LA_ERR_INVALID_ARGUMENT;
   if (a.kernel_path < LA_PATH_AUTO || a.kernel_path > LA_PATH_FMA) return LA_ERR_INVALID_ARGUMENT;
   if (a.out_dtype != LA_OUT_AS_INPUT && a.out_dtype != LA_OUT_F32) return LA_ERR_INVALID_ARGUMENT;
+  if (a.algorithm < LA_ALGO_AUTO || a.algorithm > LA_ALGO_SEGMENTED) return LA_ERR_INVALID_ARGUMENT;
+  if (a.segment_chunks < 0 || a.segment_chunks > 1024) return LA_ERR_INVALID_ARGUMENT;
   if (a.normalize && a.feature_map == LA_FM_IDENTITY) return LA_ERR_INVALID_ARGUMENT;
   if (!(a.eps >= 0.f) || !std::isfinite(a.eps)) return LA_ERR_INVALID_ARGUMENT;
   if (a.gamma && a.H > kMaxHeads) return LA_ERR_UNSUPPORTED;
@@ -160,6 +162,9 @@ int validate(const la_prefill_args& a, Path* path) {
   const bool tc_shape = a.dtype == LA_DTYPE_BF16 && dim_ok_tc(a.dk) && dim_ok_tc(a.dv) &&
                         a.C == 64 && a.T < (1LL << 31);
   if (a.kernel_path == LA_PATH_TENSOR_CORE && !tc_shape) return LA_ERR_UNSUPPORTED;
+  if (a.algorithm == LA_ALGO_SEGMENTED &&
+      (!tc_shape || a.kernel_path == LA_PATH_FMA || !seg_supported(a.dk, a.dv, a.C)))
+    return LA_ERR_UNSUPPORTED;
 
   const bool empty = BH == 0 || a.T == 0;
   if (!empty) {
@@ -183,11 +188,23 @@ int validate(const la_prefill_args& a, Path* path) {
   if (!empty && a.kernel_path != LA_PATH_FMA && tc_shape) {
     if (device_is_sm100()) {
       *path = Path::kTensorCore;
-    } else if (a.kernel_path == LA_PATH_TENSOR_CORE) {
+    } else if (a.kernel_path == LA_PATH_TENSOR_CORE || a.algorithm == LA_ALGO_SEGMENTED) {
       return LA_ERR_UNSUPPORTED;
     }
   }
+  if (*path == Path::kTensorCore && a.algorithm != LA_ALGO_CHUNKED &&
+      seg_supported(a.dk, a.dv, a.C))
+    *path = Path::kSegmented;
   return LA_OK;
+}
+
+// Chunks per segment for the segmented algorithm: enough segments to give every SM a
+// few, at most 64 chunks each.
+int segment_chunks(long long BH, int NC) {
+  long long l = BH * NC / (4LL * 148);
+  if (l < 1) l = 1;
+  if (l > 64) l = 64;
+  return static_cast<int>(l);
 }
 
 int to_status(cudaError_t e) {
@@ -255,7 +272,60 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
   Flags f{a.feature_map, a.gamma != nullptr, a.normalize != 0, out_f32};
 
   cudaError_t e = cudaSuccess;
-  if (path == Path::kTensorCore) {
+  if (path == Path::kSegmented) {
+    // Segments of Lseg chunks; one record per segment at the start of the workspace,
+    // then the scan's totals over segments.
+    const int Lseg = a.segment_chunks > 0 ? a.segment_chunks : segment_chunks(BH, l.NC);
+    const int NS = (l.NC + Lseg - 1) / Lseg;
+    SegParams sp;
+    sp.BH = p.BH;
+    sp.H = p.H;
+    sp.T = p.T;
+    sp.dk = p.dk;
+    sp.dv = p.dv;
+    sp.C = p.C;
+    sp.NC = l.NC;
+    sp.L_last = l.L_last;
+    sp.Lseg = Lseg;
+    sp.NS = NS;
+    sp.R = l.R;
+    sp.eps = a.eps;
+    sp.srec = reinterpret_cast<float*>(ws);
+    sp.err = p.err;
+    const size_t srec_bytes = align256(static_cast<size_t>(BH) * NS * l.R * sizeof(float));
+    PrefillParams ps = p;  // the scan over segments: one scan element per segment
+    ps.NC = NS;
+    ps.C = Lseg * a.C;
+    ps.L_last = static_cast<int>(a.T - static_cast<long long>(NS - 1) * Lseg * a.C);
+    ps.rec = sp.srec;
+    ps.tot = reinterpret_cast<float*>(ws + srec_bytes);
+    ps.Ls = (NS + kMaxSegments - 1) / kMaxSegments;
+    ps.G = (NS + ps.Ls - 1) / ps.Ls;
+    TcMaps m;
+    const uint64_t T = static_cast<uint64_t>(a.T);
+    bool ok = make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, a.dk, T, BH, a.dk * 2ull,
+                       T * a.dk * 2ull, 64, 64) &&
+              make_map(&m.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.k, a.dk, T, BH, a.dk * 2ull,
+                       T * a.dk * 2ull, 64, 64) &&
+              make_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, a.dv, T, BH, a.dv * 2ull,
+                       T * a.dv * 2ull, 64, 64) &&
+              (out_f32 ? make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, a.dv, T, BH,
+                                  a.dv * 4ull, T * a.dv * 4ull, 32, 64)
+                       : make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.dv, T, BH,
+                                  a.dv * 2ull, T * a.dv * 2ull, 64, 64)) &&
+              make_map(&m.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.srec, a.dk, a.dv,
+                       static_cast<uint64_t>(BH) * NS, a.dk * 4ull, l.R * 4ull, 32,
+                       static_cast<uint32_t>(a.dv));
+    if (!ok) {
+      e = cudaErrorInvalidValue;
+    } else {
+      if (rec) rec->mark(s);
+      e = launch_k1_seg(sp, gt, m, f, s);
+      if (e == cudaSuccess) e = launch_k2(ps, gt, a.scan_mode, f, s, rec);
+      if (rec) rec->mark(s);
+      if (e == cudaSuccess) e = launch_k3_seg(sp, gt, m, f, s);
+    }
+  } else if (path == Path::kTensorCore) {
     TcMaps m;
     const uint64_t T = static_cast<uint64_t>(a.T);
     bool ok = make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, a.dk, T, BH, a.dk * 2ull,

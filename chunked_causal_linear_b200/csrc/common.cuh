@@ -39,4 +39,25 @@ __device__ __forceinline__ int chunk_len(const PrefillParams& p, int c) {
   return c == p.NC - 1 ? p.L_last : p.C;
 }
 
+// The segmented variant: chunks grouped into segments of Lseg chunks; one record per
+// segment (same record layout as the chunk records).
+struct SegParams {
+  int BH;
+  int H;
+  long long T;
+  int dk, dv, C;
+  int NC;          // chunks
+  int L_last;      // valid tokens in the last chunk
+  int Lseg;        // chunks per segment
+  int NS;          // segments per (b, h)
+  int R;           // floats per record
+  float eps;
+  float* srec;     // [BH, NS, R] segment totals, turned into exclusive prefixes by K2
+  int* err;
+};
+
+__device__ __forceinline__ int chunk_len(const SegParams& p, int c) {
+  return c == p.NC - 1 ? p.L_last : p.C;
+}
+
 }  // namespace la

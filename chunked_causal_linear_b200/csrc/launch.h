@@ -52,6 +52,15 @@ cudaError_t launch_k1_tc(const PrefillParams& p, const GammaTable& gt, const TcM
 cudaError_t launch_k3_tc(const PrefillParams& p, const GammaTable& gt, const TcMaps& m,
                          Flags f, cudaStream_t s);
 
+// Segmented variant (seg_kernels.cu): K1s writes one record per segment, K3s walks a
+// segment's chunks carrying the prefix in TMEM.  bf16 inputs, C = 64, dk in {64, 128},
+// dv = 128.
+bool seg_supported(int dk, int dv, int C);
+cudaError_t launch_k1_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
+                          cudaStream_t s);
+cudaError_t launch_k3_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
+                          cudaStream_t s);
+
 // One recurrent decode step for every (b, h).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* out, float* S,
                           float* Z, int BH, int H, int dk, int dv, int dtype, Flags f,

@@ -88,6 +88,20 @@ typedef enum { LA_DTYPE_BF16 = 0, LA_DTYPE_F32 = 1 } la_dtype;
  * dominate the error on long sequences). */
 typedef enum { LA_OUT_AS_INPUT = 0, LA_OUT_F32 = 1 } la_out_dtype;
 
+/*
+ * How the chunk summaries are combined.
+ *   LA_ALGO_CHUNKED    the scan page's three kernels as stated: K1 writes every chunk's
+ *                      summary, K2 scans all of them, K3 reads each chunk's prefix once.
+ *   LA_ALGO_SEGMENTED  the hierarchical form of the same scan: chunks are grouped into
+ *                      segments; K1 writes one summary per segment, K2 scans segments,
+ *                      and K3 walks each segment's chunks in order, carrying the prefix
+ *                      on chip and advancing it with the chunk's own summary.  Same
+ *                      results, about a quarter of the HBM traffic.  Tensor-core path
+ *                      only: bf16 inputs, C = 64, dk in {64, 128}, dv = 128.
+ *   LA_ALGO_AUTO       segmented where supported, else chunked.
+ */
+typedef enum { LA_ALGO_AUTO = 0, LA_ALGO_CHUNKED = 1, LA_ALGO_SEGMENTED = 2 } la_algorithm;
+
 typedef enum {
   LA_PATH_AUTO = 0,        /* tensor-core kernels where the shape allows, else FMA kernels */
   LA_PATH_TENSOR_CORE = 1, /* tcgen05/TMEM kernels only (LA_ERR_UNSUPPORTED otherwise) */
@@ -112,7 +126,7 @@ typedef enum {
  *   C         chunk length.
  *   feature_map  la_feature_map.  normalize != 0 requires LA_FM_ELU1 (the identity map
  *             gives a denominator of indefinite sign).
- * Uses the log-depth scan and eps = 0.  The workspace is allocated with
+ * Uses the log-depth scan, LA_ALGO_AUTO and eps = 0.  The workspace is allocated with
  * cudaMallocAsync / cudaFreeAsync on `stream` (LA_ERR_OUT_OF_MEMORY on failure).
  * T == 0 zero-fills S_final / Z_final.  Returns a la_status.
  */
@@ -129,7 +143,8 @@ int lin_attn_prefill_f32(const float* q, const float* k, const float* v, float* 
                          la_stream_t stream);
 
 /* Bytes of device workspace the prefill needs for this shape (chunk summaries and scan
- * segment totals).  Pure host computation; 0 for an empty problem. */
+ * segment totals), enough for either algorithm.  Pure host computation; 0 for an empty
+ * problem. */
 size_t lin_attn_prefill_workspace_bytes(int B, int H, long long T, int dk, int dv, int C,
                                         int normalize);
 
@@ -152,6 +167,9 @@ typedef struct la_prefill_args {
   int out_dtype;          /* la_out_dtype of out */
   int scan_mode;          /* la_scan_mode */
   int kernel_path;        /* la_kernel_path */
+  int algorithm;          /* la_algorithm */
+  int segment_chunks;     /* chunks per segment for LA_ALGO_SEGMENTED (1..1024), or 0 to
+                             choose automatically (a few segments per SM, at most 64) */
   void* workspace;        /* DEVICE, >= lin_attn_prefill_workspace_bytes(), 256-byte
                              aligned; NULL = allocate on the stream */
   size_t workspace_bytes;
@@ -167,7 +185,8 @@ int lin_attn_prefill_ex(const la_prefill_args* args);
  * before every kernel launch and after the last one; synchronises the stream and writes
  * each kernel's device duration (milliseconds, launch order) to kernel_ms[0 ..].
  * *n_kernels receives the number of kernels the prefill launched (K1, the scan's
- * kernels, K3: 5 with the log-depth scan, 3 with the sequential carry).  For profiling;
+ * kernels, K3: 5 with the log-depth scan, 3 with the sequential carry; the segmented
+ * algorithm launches the same count).  For profiling;
  * the results are identical to lin_attn_prefill_ex.
  */
 int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int max_kernels,

@@ -103,6 +103,10 @@ def _args(**kw):
     (dict(q=0), 1), (dict(out=0), 1), (dict(q=0x1001), 1), (dict(out=0x1008), 1),
     (dict(out=0x1000), 1), (dict(out=0x2000000 + 64), 1),
     (dict(workspace=0x100010), 1),
+    (dict(algorithm=3), 1), (dict(algorithm=-1), 1), (dict(segment_chunks=-1), 1),
+    (dict(segment_chunks=2000), 1),
+    (dict(algorithm=2, dv=64), 2), (dict(algorithm=2, C=32), 2), (dict(algorithm=2, dtype=1), 2),
+    (dict(algorithm=2, kernel_path=2), 2),
 ])
 def test_argument_errors_before_any_launch(lib, kw, status):
     a = _args(**kw)

@@ -41,8 +41,9 @@ def test_empty_batch_is_a_no_op():
     assert out.numel() == 0
 
 
+@pytest.mark.parametrize("algorithm", ["chunked", "segmented"])
 @pytest.mark.parametrize("fm", ["elu1", "identity"])
-def test_padding_does_not_leak_from_the_next_head(fm):
+def test_padding_does_not_leak_from_the_next_head(fm, algorithm):
     # T = 100: the last chunk holds 36 tokens; a naive load of the full 64-row tile would
     # read the next head's first 28 tokens.  Make those huge.
     w, q, k, v = _inputs(100, fm=fm)
@@ -51,7 +52,7 @@ def test_padding_does_not_leak_from_the_next_head(fm):
     gamma = [0.97, 0.9] if w.decay else None
     out, S, Z = B.lin_attn_prefill(q, k, v, chunk=64, feature_map=fm, gamma=gamma,
                                    normalize=w.normalize, kernel_path="tensor_core",
-                                   out_dtype="f32")
+                                   out_dtype="f32", algorithm=algorithm)
     torch.cuda.synchronize()
     o_ref, S_ref, Z_ref = oracle_prefill(q, k, v, feature_map=fm, gamma=gamma,
                                          normalize=w.normalize, heads=[(0, 0)])
@@ -59,23 +60,26 @@ def test_padding_does_not_leak_from_the_next_head(fm):
     assert_close(to_np(S[0, 0])[None], S_ref, TOL_BF16, "S head 0")
 
 
+@pytest.mark.parametrize("algorithm", ["chunked", "segmented"])
 @pytest.mark.parametrize("t0", [0, 1, 63, 64, 100, 200])
-def test_causality_bitwise(t0):
+def test_causality_bitwise(t0, algorithm):
     w, q, k, v = _inputs(256)
-    out1, _, _ = B.lin_attn_prefill(q, k, v, kernel_path="tensor_core")
+    kw = dict(kernel_path="tensor_core", algorithm=algorithm, segment_chunks=2)
+    out1, _, _ = B.lin_attn_prefill(q, k, v, **kw)
     q2, k2, v2 = q.clone(), k.clone(), v.clone()
     for t in (q2, k2, v2):
         t[:, :, t0:] = 100.0
-    out2, _, _ = B.lin_attn_prefill(q2, k2, v2, kernel_path="tensor_core")
+    out2, _, _ = B.lin_attn_prefill(q2, k2, v2, **kw)
     torch.cuda.synchronize()
     assert torch.equal(out1[:, :, :t0], out2[:, :, :t0])
 
 
-@pytest.mark.parametrize("path", ["tensor_core", "fma"])
-def test_deterministic(path):
+@pytest.mark.parametrize("path,algorithm", [("tensor_core", "chunked"),
+                                            ("tensor_core", "segmented"), ("fma", "chunked")])
+def test_deterministic(path, algorithm):
     w, q, k, v = _inputs(1000)
-    a = B.lin_attn_prefill(q, k, v, kernel_path=path)
-    b = B.lin_attn_prefill(q, k, v, kernel_path=path)
+    a = B.lin_attn_prefill(q, k, v, kernel_path=path, algorithm=algorithm)
+    b = B.lin_attn_prefill(q, k, v, kernel_path=path, algorithm=algorithm)
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)

@@ -55,7 +55,19 @@ def _check(w, q, k, v, gamma, tol, **kw):
 @pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
 def test_tensor_core_path(dk, dv, T, mode):
     w, q, k, v, gamma = _case(T, dk, dv, 64, mode)
-    _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core")
+    _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core", algorithm="chunked")
+
+
+@pytest.mark.parametrize("mode", sorted(MODES))
+@pytest.mark.parametrize("T,seg", [(1, 0), (64, 1), (100, 1), (257, 2), (1000, 3), (1000, 7),
+                                   (1000, 16), (4485, 0), (4485, 5)])
+@pytest.mark.parametrize("dk", [64, 128])
+def test_segmented_path(dk, T, seg, mode):
+    """Segments of `seg` chunks (0 = automatic): the prefix carried through several chunks
+    inside a segment, segment prefixes from the scan, a ragged last chunk."""
+    w, q, k, v, gamma = _case(T, dk, 128, 64, mode)
+    _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core", algorithm="segmented",
+           segment_chunks=seg)
 
 
 @pytest.mark.parametrize("mode", sorted(MODES))
@@ -78,10 +90,14 @@ def test_fma_path_f32(T, dk, dv, C, mode):
 @pytest.mark.parametrize("mode", sorted(MODES))
 @pytest.mark.parametrize("path", ["tensor_core", "fma"])
 @pytest.mark.parametrize("T", [100, 1000])
-def test_bf16_output(T, path, mode):
+@pytest.mark.parametrize("algorithm", ["chunked", "segmented"])
+def test_bf16_output(T, path, mode, algorithm):
+    if path == "fma" and algorithm == "segmented":
+        pytest.skip("the segmented algorithm runs on the tensor-core kernels only")
     w, q, k, v, gamma = _case(T, 128, 128, 64, mode)
     out, S, Z = gpu_prefill(q, k, v, C=64, feature_map=w.feature_map, gamma=gamma,
-                            normalize=w.normalize, kernel_path=path, out_dtype="as_input")
+                            normalize=w.normalize, kernel_path=path, out_dtype="as_input",
+                            algorithm=algorithm, segment_chunks=3)
     assert out.dtype == torch.bfloat16
     o_ref, S_ref, _ = oracle_prefill(q, k, v, feature_map=w.feature_map, gamma=gamma,
                                      normalize=w.normalize)
@@ -91,10 +107,12 @@ def test_bf16_output(T, path, mode):
 
 @pytest.mark.parametrize("mode", ["norm", "retention"])
 @pytest.mark.parametrize("T", [100, 1000, 64 * 70 + 5])
-def test_scan_modes_agree_with_oracle(T, mode):
-    w, q, k, v, gamma = _case(T, 64, 64, 64, mode)
+@pytest.mark.parametrize("dv,algorithm", [(64, "chunked"), (128, "segmented")])
+def test_scan_modes_agree_with_oracle(T, mode, dv, algorithm):
+    w, q, k, v, gamma = _case(T, 64, dv, 64, mode)
     for scan in ("logdepth", "sequential"):
-        _check(w, q, k, v, gamma, TOL_BF16, scan=scan)
+        _check(w, q, k, v, gamma, TOL_BF16, scan=scan, algorithm=algorithm,
+               segment_chunks=2 if algorithm == "segmented" else 0)
 
 
 def test_pr1_ref_fp32_against_oracle_and_golden():

@@ -27,22 +27,27 @@ SAMPLES = {
 }
 
 
-def run_bench_config(w, q, k, v, scan="logdepth"):
+def run_bench_config(w, q, k, v, scan="logdepth", algorithm="auto"):
     ws = torch.empty(B.lin_attn_prefill_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.C,
                                                         w.normalize),
                      dtype=torch.uint8, device="cuda")
     out, S, Z = B.lin_attn_prefill(q, k, v, chunk=w.C, feature_map=w.feature_map,
                                    gamma=w.gammas(), normalize=w.normalize, scan=scan,
-                                   kernel_path="tensor_core", workspace=ws, out_dtype="f32")
+                                   kernel_path="tensor_core", workspace=ws, out_dtype="f32",
+                                   algorithm=algorithm)
     torch.cuda.synchronize()
     return out, S, Z
 
 
+@pytest.mark.parametrize("algorithm", ["auto", "chunked"])
 @pytest.mark.parametrize("name", sorted(SAMPLES))
-def test_workload_full_size(name):
+def test_workload_full_size(name, algorithm):
+    """`auto` is the benchmark's configuration (segmented where dv = 128)."""
     w = WORKLOADS[name]
+    if algorithm == "chunked" and w.dv != 128:
+        pytest.skip("auto already runs the chunked algorithm at dv = 64")
     q, k, v = make_inputs(w, seed=0, device="cuda")
-    out, S, Z = run_bench_config(w, q, k, v)
+    out, S, Z = run_bench_config(w, q, k, v, algorithm=algorithm)
     heads = SAMPLES[name]
     o_ref, S_ref, Z_ref = oracle_prefill(q, k, v, feature_map=w.feature_map, gamma=w.gammas(),
                                          normalize=w.normalize, heads=heads)
