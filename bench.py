@@ -63,9 +63,11 @@ def effective_algorithm(w, requested: str) -> str:
     return "chunked"
 
 
-def kernel_names(algo: str, scan: str) -> list[str]:
+def kernel_names(w, algo: str, scan: str) -> list[str]:
     k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
-    return [k1, *K2_NAMES[scan], k3]
+    n, _, _ = layout(w, algo)
+    k2 = ["k2_scan_totals"] if scan == "logdepth" and n <= 32 else K2_NAMES[scan]
+    return [k1, *k2, k3]
 
 
 # ---------------------------------------------------------------------------------------
@@ -446,7 +448,7 @@ def main():
         ms, clocks = timed_region()
         remeasured = True
     ms_max = ranks.max_over_ranks(ms, info, dev)
-    names = kernel_names(algo, args.scan)
+    names = kernel_names(w, algo, args.scan)
     n_kern = len(names)
     value = info.world * w.tokens_heads / (ms_max / 1000.0)
 

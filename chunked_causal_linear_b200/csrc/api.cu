@@ -162,8 +162,8 @@ int validate(const la_prefill_args& a, Path* path) {
   const bool tc_shape = a.dtype == LA_DTYPE_BF16 && dim_ok_tc(a.dk) && dim_ok_tc(a.dv) &&
                         a.C == 64 && a.T < (1LL << 31);
   if (a.kernel_path == LA_PATH_TENSOR_CORE && !tc_shape) return LA_ERR_UNSUPPORTED;
-  if (a.algorithm == LA_ALGO_SEGMENTED &&
-      (!tc_shape || a.kernel_path == LA_PATH_FMA || !seg_supported(a.dk, a.dv, a.C)))
+  const bool seg_ok = seg_supported(a.dk, a.dv, a.C, a.feature_map, a.gamma != nullptr);
+  if (a.algorithm == LA_ALGO_SEGMENTED && (!tc_shape || a.kernel_path == LA_PATH_FMA || !seg_ok))
     return LA_ERR_UNSUPPORTED;
 
   const bool empty = BH == 0 || a.T == 0;
@@ -192,8 +192,7 @@ int validate(const la_prefill_args& a, Path* path) {
       return LA_ERR_UNSUPPORTED;
     }
   }
-  if (*path == Path::kTensorCore && a.algorithm != LA_ALGO_CHUNKED &&
-      seg_supported(a.dk, a.dv, a.C))
+  if (*path == Path::kTensorCore && a.algorithm != LA_ALGO_CHUNKED && seg_ok)
     *path = Path::kSegmented;
   return LA_OK;
 }

@@ -54,8 +54,8 @@ cudaError_t launch_k3_tc(const PrefillParams& p, const GammaTable& gt, const TcM
 
 // Segmented variant (seg_kernels.cu): K1s writes one record per segment, K3s walks a
 // segment's chunks carrying the prefix in TMEM.  bf16 inputs, C = 64, dk in {64, 128},
-// dv = 128.
-bool seg_supported(int dk, int dv, int C);
+// dv = 128, and not the ELU+1 map together with decay.
+bool seg_supported(int dk, int dv, int C, int fm, bool decay);
 cudaError_t launch_k1_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                           cudaStream_t s);
 cudaError_t launch_k3_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,

@@ -50,6 +50,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Default bound on any wait: about two seconds of wall time.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 
+// One arrival (release semantics) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier among `nthreads` threads (a multiple of 32) using hardware barrier `id` (1..15;
+// 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Waits until the phase with the given parity has completed.  Gives up and returns
 // false once `timeout_ns` of wall time (or 2^30 polls) have passed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,

@@ -11,7 +11,8 @@
 // total (the state after the last token) goes to S_final / Z_final.
 //
 // Log-depth mode ("Implementation notes": a Blelloch or Hillis-Steele scan) splits the
-// chunk axis into G <= 32 segments of Ls chunks:
+// chunk axis into G <= 32 segments of Ls chunks (when Ls = 1, i.e. at most 32 elements,
+// k2_scan_totals alone scans the records in place):
 //   k2_reduce       one pass over the records: each segment's aggregate (parallel over
 //                   segments and columns);
 //   k2_scan_totals  Hillis-Steele scan of the G segment aggregates, ceil(log2 G) rounds
@@ -56,11 +57,34 @@ __device__ __forceinline__ void write_final(const PrefillParams& p, int bh, int 
   write_final1(p, bh, col + 3, v.w);
 }
 
-// Decay factor of chunk c: gamma^(L_c).
+// In-place exclusive carry over chunks [cbeg, cend) of one float4 column: record c
+// receives the carry before chunk c, then carry <- a_c carry + x_c.  The next batch of
+// loads is issued before the current batch is stored, so a thread always has loads in
+// flight (in-place read-then-write streams reach copy bandwidth only this way).
 template <bool DECAY>
-__device__ __forceinline__ float chunk_decay(const PrefillParams& p, float g, float gC, int c) {
-  if (!DECAY) return 1.f;
-  return c == p.NC - 1 ? powf(g, static_cast<float>(p.L_last)) : gC;
+__device__ __forceinline__ float4 carry_in_place(float4* base, long long stride, int cbeg,
+                                                 int cend, int last, float gC, float aL,
+                                                 float4 carry) {
+  float4 x[kUnroll], y[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u)
+    if (cbeg + u < cend) x[u] = base[static_cast<long long>(cbeg + u) * stride];
+  for (int c0 = cbeg; c0 < cend; c0 += kUnroll) {
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (c0 + kUnroll + u < cend) y[u] = base[static_cast<long long>(c0 + kUnroll + u) * stride];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (c0 + u < cend) {
+        base[static_cast<long long>(c0 + u) * stride] = carry;
+        const float a = DECAY ? (c0 + u == last ? aL : gC) : 1.f;
+        carry = axpy4(a, carry, x[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) x[u] = y[u];
+  }
+  return carry;
 }
 
 // Sequential carry: one thread per float4 column, loop over all chunks.
@@ -73,21 +97,10 @@ __global__ void __launch_bounds__(kScanThreads) k2_sequential(PrefillParams p, G
   if (col4 >= R4) return;
   const float g = DECAY ? gt.g[bh % p.H] : 1.f;
   const float gC = DECAY ? powf(g, static_cast<float>(p.C)) : 1.f;
+  const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
   float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) + col4;
-  float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < p.NC; c0 += kUnroll) {
-    float4 x[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (c0 + u < p.NC) x[u] = base[static_cast<long long>(c0 + u) * R4];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (c0 + u < p.NC) {
-        base[static_cast<long long>(c0 + u) * R4] = carry;
-        carry = axpy4(chunk_decay<DECAY>(p, g, gC, c0 + u), carry, x[u]);
-      }
-    }
-  }
+  const float4 carry = carry_in_place<DECAY>(base, R4, 0, p.NC, p.NC - 1, gC, aL,
+                                             make_float4(0.f, 0.f, 0.f, 0.f));
   write_final(p, bh, col4 * 4, carry);
 }
 
@@ -103,6 +116,7 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
   if (col4 >= R4) return;
   const float g = DECAY ? gt.g[bh % p.H] : 1.f;
   const float gC = DECAY ? powf(g, static_cast<float>(p.C)) : 1.f;
+  const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
   const int cbeg = s * p.Ls;
   const int cend = min(p.NC, cbeg + p.Ls);
   const float4* base =
@@ -115,21 +129,23 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
       if (c0 + u < cend) x[u] = base[static_cast<long long>(c0 + u) * R4];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
-      if (c0 + u < cend) agg = axpy4(chunk_decay<DECAY>(p, g, gC, c0 + u), agg, x[u]);
+      if (c0 + u < cend) agg = axpy4(DECAY ? (c0 + u == p.NC - 1 ? aL : gC) : 1.f, agg, x[u]);
   }
   reinterpret_cast<float4*>(p.tot + (static_cast<long long>(bh) * p.G + s) * p.R)[col4] = agg;
 }
 
-// Hillis-Steele scan of the segment aggregates.  Block (32 columns) x (32 segments).
+// Hillis-Steele scan of the segment aggregates.  Block (32 float4 columns) x (32
+// segments); ceil(log2 G) rounds in shared memory.
 template <bool DECAY>
 __global__ void __launch_bounds__(1024) k2_scan_totals(PrefillParams p, GammaTable gt) {
-  __shared__ float sX[32][33];
-  __shared__ float sA[32][33];
-  const int ncb = (p.R + 31) / 32;
+  __shared__ float4 sX[32][33];
+  __shared__ float sA[32];
+  const int R4 = p.R / 4;
+  const int ncb = (R4 + 31) / 32;
   const int bh = blockIdx.x / ncb;
-  const int col = (blockIdx.x % ncb) * 32 + threadIdx.x;
+  const int col4 = (blockIdx.x % ncb) * 32 + threadIdx.x;
   const int s = threadIdx.y;
-  const bool live = s < p.G && col < p.R;
+  const bool live = s < p.G && col4 < R4;
   const float g = DECAY ? gt.g[bh % p.H] : 1.f;
 
   // Segment decay: product of its chunks' decays.
@@ -142,18 +158,16 @@ __global__ void __launch_bounds__(1024) k2_scan_totals(PrefillParams p, GammaTab
                                                 : static_cast<long long>(cend - cbeg) * p.C);
     a = powf(g, tokens);
   }
-  float* tot = p.tot + static_cast<long long>(bh) * p.G * p.R;
-  float x = live ? tot[static_cast<long long>(s) * p.R + col] : 0.f;
+  float4* tot = reinterpret_cast<float4*>(p.tot + static_cast<long long>(bh) * p.G * p.R);
+  float4 x = live ? tot[static_cast<long long>(s) * R4 + col4] : make_float4(0.f, 0.f, 0.f, 0.f);
 
   for (int d = 1; d < p.G; d <<= 1) {
     sX[s][threadIdx.x] = x;
-    sA[s][threadIdx.x] = a;
+    if (threadIdx.x == 0) sA[s] = a;
     __syncthreads();
     if (s >= d) {
-      const float xp = sX[s - d][threadIdx.x];
-      const float ap = sA[s - d][threadIdx.x];
-      x = fmaf(a, xp, x);
-      a = ap * a;
+      x = axpy4(a, sX[s - d][threadIdx.x], x);
+      a = sA[s - d] * a;
     }
     __syncthreads();
   }
@@ -161,8 +175,9 @@ __global__ void __launch_bounds__(1024) k2_scan_totals(PrefillParams p, GammaTab
   sX[s][threadIdx.x] = x;
   __syncthreads();
   if (live) {
-    tot[static_cast<long long>(s) * p.R + col] = s > 0 ? sX[s - 1][threadIdx.x] : 0.f;
-    if (s == p.G - 1) write_final1(p, bh, col, x);
+    tot[static_cast<long long>(s) * R4 + col4] = s > 0 ? sX[s - 1][threadIdx.x]
+                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s == p.G - 1) write_final(p, bh, col4 * 4, x);
   }
 }
 
@@ -178,24 +193,13 @@ __global__ void __launch_bounds__(kScanThreads) k2_downsweep(PrefillParams p, Ga
   if (col4 >= R4) return;
   const float g = DECAY ? gt.g[bh % p.H] : 1.f;
   const float gC = DECAY ? powf(g, static_cast<float>(p.C)) : 1.f;
+  const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
   const int cbeg = s * p.Ls;
   const int cend = min(p.NC, cbeg + p.Ls);
   float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) + col4;
-  float4 carry =
+  const float4 carry =
       reinterpret_cast<const float4*>(p.tot + (static_cast<long long>(bh) * p.G + s) * p.R)[col4];
-  for (int c0 = cbeg; c0 < cend; c0 += kUnroll) {
-    float4 x[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (c0 + u < cend) x[u] = base[static_cast<long long>(c0 + u) * R4];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (c0 + u < cend) {
-        base[static_cast<long long>(c0 + u) * R4] = carry;
-        carry = axpy4(chunk_decay<DECAY>(p, g, gC, c0 + u), carry, x[u]);
-      }
-    }
-  }
+  carry_in_place<DECAY>(base, R4, cbeg, cend, p.NC - 1, gC, aL, carry);
 }
 
 template <bool DECAY>
@@ -209,11 +213,19 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
     return cudaGetLastError();
   }
   const long long grid = nblk * p.G * p.BH;
+  const long long ncb = (R4 + 31) / 32;
+  if (p.Ls == 1) {
+    // Every segment is one element: the Hillis-Steele scan alone, in place on the records.
+    PrefillParams q = p;
+    q.tot = p.rec;
+    if (rec) rec->mark(s);
+    k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(q, gt);
+    return cudaGetLastError();
+  }
   if (rec) rec->mark(s);
   k2_reduce<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long ncb = (p.R + 31) / 32;
   if (rec) rec->mark(s);
   k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(p, gt);
   e = cudaGetLastError();

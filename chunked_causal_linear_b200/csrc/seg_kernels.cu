@@ -36,7 +36,8 @@ namespace la {
 namespace {
 
 constexpr int kC = 64;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // 8 warps: two warps per TMEM lane quarter share its columns
+constexpr int kWarps = kThreads / 32;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -98,7 +99,7 @@ struct K1sSmem {
   static constexpr uint32_t kIn = 2 * kStage + kK;  // two stages + the lo tile of K'
   static constexpr uint32_t kS = DK * DV * 4;       // staging of T_s^T, aliases the inputs
   static constexpr uint32_t kRegion = kIn > kS ? kIn : kS;
-  static constexpr uint32_t kTotal = kRegion + 4 * DK * 4 + 64 + 1024;
+  static constexpr uint32_t kTotal = kRegion + kWarps * DK * 4 + 64 + 1024;
 };
 
 template <int DK, int DV, int FM, bool DECAY, bool NORM>
@@ -113,7 +114,7 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
   uint8_t* sKl = base + 2 * L_::kStage;
   uint8_t* sS = base;
   float* sZ = reinterpret_cast<float*>(base + L_::kRegion);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + 4 * DK);  // tma[2], mma
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + kWarps * DK);  // tma[2], mma
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
 
   if (error_pending(sp.err)) return;
@@ -225,14 +226,21 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
 #pragma unroll
       for (int e = 0; e < 8; ++e) sZ[warp * DK + cc * 8 + e] = zacc[e];
     __syncthreads();
-    if (tid < DK) srec[DK * DV + tid] = sZ[tid] + sZ[DK + tid] + sZ[2 * DK + tid] + sZ[3 * DK + tid];
+    if (tid < DK) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) z += sZ[w * DK + tid];
+      srec[DK * DV + tid] = z;
+    }
   }
 
-  const int row = DV == 128 ? warp * 32 + lane : warp * 16 + lane;
+  // Epilogue: warps w and w + 4 read the same TMEM lanes, each half of the columns.
+  const int quarter = warp & 3, half = warp >> 2;
+  const int row = DV == 128 ? quarter * 32 + lane : quarter * 16 + lane;
   const bool valid = DV == 128 || lane < 16;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
 #pragma unroll
-  for (int q4 = 0; q4 < DK / 32; ++q4) {
+  for (int q4 = half * (DK / 64); q4 < (half + 1) * (DK / 64); ++q4) {
     float r[32];
     tmem_ld32(tmem + lane_base + q4 * 32, r);
     tmem_ld_wait();
@@ -259,57 +267,83 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
 }
 
 // ---------------------------------------------------------------------------------------
-// K3s (dv = 128)
+// K3s (dv = 128), warp-specialised.
+//
+// 416 threads in three roles that hand work over through mbarriers, so that the
+// transform of chunk i + 1 overlaps the MMAs and epilogues of chunk i:
+//   warps 0-3  transform: psi on the staged Q, K (bf16 hi / lo operand tiles, double
+//              buffered), Xi .* psi(K), psi(q).ZP and the Z update; then the prefix
+//              operand: P^T from TMEM -> bf16 hi / lo into TMEM, and P scaled by gamma^L.
+//   warps 4-11 epilogue (two warps per TMEM lane quarter, each half of the columns):
+//              masks and decays the scores into A (hi / lo), then combines
+//              o = Theta X + N (/ den) and stores the chunk's output tile with TMA.
+//   warp 12    control (one thread): TMA loads two chunks ahead and every tcgen05.mma;
+//              the next chunk's scores are issued before the current chunk's local
+//              product has finished.
+// Warp w reads TMEM lanes 32 (w % 4) .. + 31.  Accumulators (TMEM columns): scores
+// [0, 64), X (two buffers) [64, 128) and [448, 512), N [128, 192), P [192, 192 + dk),
+// P hi / lo after it.  Each is released by an mbarrier once its readers are done.
 
-template <int DK, bool OUTF32>
+constexpr int kThreads3 = 416;
+
+template <int DK, int FM, bool DECAY, bool OUTF32>
 struct K3sSmem {
   static constexpr int DV = 128;
   static constexpr uint32_t kQ = DK * kC * 2;
   static constexpr uint32_t kK = DK * kC * 2;
   static constexpr uint32_t kV = DV * kC * 2;
   static constexpr uint32_t kStage = kQ + kK + kV;
+  static constexpr uint32_t kLo = FM == 1 ? kQ + kK : 0;  // lo tiles of psi(Q), psi(K)
+  static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
   static constexpr uint32_t kO = kC * DV * (OUTF32 ? 4 : 2);
-  static constexpr uint32_t kSmall = (DK + 6 * kC) * 4 + 4 * DK * 4 + 64;
-  // two stages, lo tiles of psi(Q) and psi(K), K'' hi + lo, A hi + lo, output staging
-  static constexpr uint32_t kTotal = 2 * kStage + kQ + kK + 2 * kK + 2 * kA + kO + kSmall + 1024;
+  static constexpr uint32_t kSmallFloats = 5 * DK + 10 * kC;
+  static constexpr uint32_t kTotal =
+      2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kO + kSmallFloats * 4 + 16 * 8 + 1024;
 };
 
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads3, 1)
 k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
        SegParams sp, GammaTable gt) {
   constexpr int DV = 128;
-  using L_ = K3sSmem<DK, OUTF32>;
+  using L_ = K3sSmem<DK, FM, DECAY, OUTF32>;
   constexpr bool kSplitQK = FM == 1;
   constexpr uint32_t kTmemCols = 512;
-  constexpr uint32_t kColS = 0;             // scores, M = 64
-  constexpr uint32_t kColX = 64;            // X^T = P^T psi(Q)^T, M = 128, N = 64
-  constexpr uint32_t kColN = 128;           // N^T = V^T A^T
-  constexpr uint32_t kColP = 192;           // carried prefix P^T, float32, DK columns
-  constexpr uint32_t kColPH = kColP + DK;   // bf16 hi of P^T, packed, DK/2 columns
-  constexpr uint32_t kColPL = kColPH + DK / 2;
-  static_assert(kColPL + DK / 2 <= kTmemCols, "TMEM budget");
+  constexpr uint32_t kColS = 0, kColN = 128, kColP = 192;
+  constexpr uint32_t kColPH = kColP + DK, kColPL = kColPH + DK / 2;
+  constexpr uint32_t kColX[2] = {64, 448};
+  static_assert(kColPL + DK / 2 <= 448, "TMEM budget");
+  static_assert(L_::kTotal <= 232448, "shared memory budget");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
-  uint8_t* sQl = base + 2 * L_::kStage;
-  uint8_t* sKl = sQl + L_::kQ;
-  uint8_t* sKph = sKl + L_::kK;   // Xi .* psi(K), hi
-  uint8_t* sKpl = sKph + L_::kK;  // Xi .* psi(K), lo
-  uint8_t* sAh = sKpl + L_::kK;
+  uint8_t* sLo = base + 2 * L_::kStage;      // [2] x (Q lo, K lo)
+  uint8_t* sKpp = sLo + 2 * L_::kLo;         // [2] x (hi, lo)
+  uint8_t* sAh = sKpp + 2 * L_::kKpp;
   uint8_t* sAl = sAh + L_::kA;
   uint8_t* sO = sAl + L_::kA;
-  float* sZP = reinterpret_cast<float*>(sO + L_::kO);  // carried Z prefix
-  float* sDenX = sZP + DK;
-  float* sDen = sDenX + kC;
+  float* sZP = reinterpret_cast<float*>(sO + L_::kO);
+  float* sZpart = sZP + DK;        // [4][DK]
+  float* sDenX = sZpart + 4 * DK;  // [2][kC]
+  float* sDen = sDenX + 2 * kC;
   float* sTh = sDen + kC;
   float* sPow = sTh + kC;
-  float* sXi = sPow + kC;
-  float* sZpart = sXi + 2 * kC;  // [4][DK]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sZpart + 4 * DK);  // tma[2], mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  float* sXi = sPow + kC;          // [2][kC]
+  float* sDenPart = sXi + 2 * kC;  // [2][kC]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDenPart + 2 * kC);
+  uint64_t* full = bars;           // [2]
+  uint64_t* ops = bars + 2;        // [2]
+  uint64_t* pready = bars + 4;
+  uint64_t* sfree = bars + 5;
+  uint64_t* xfree = bars + 6;      // [2]
+  uint64_t* aready = bars + 8;
+  uint64_t* sdone = bars + 9;
+  uint64_t* statedone = bars + 10;
+  uint64_t* ndone = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
 
   if (error_pending(sp.err)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -322,9 +356,19 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   const float* srec = sp.srec + (static_cast<long long>(bh) * sp.NS + seg) * sp.R;
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&full[b], 1);
+      mbar_init(&ops[b], 128);
+    }
+    mbar_init(pready, 128);
+    mbar_init(sfree, 256);
+    mbar_init(&xfree[0], 256);
+    mbar_init(&xfree[1], 256);
+    mbar_init(aready, 256);
+    mbar_init(sdone, 1);
+    mbar_init(statedone, 1);
+    mbar_init(ndone, 1);
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -346,67 +390,62 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  bool failed = false;
 
-  // The segment's exclusive prefix (P^T row j) into TMEM.
-  {
-    const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(tid) * DK);
-#pragma unroll
-    for (int q4 = 0; q4 < DK / 32; ++q4) {
-      uint32_t u[32];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float4 f = src[q4 * 8 + e];
-        u[4 * e] = __float_as_uint(f.x);
-        u[4 * e + 1] = __float_as_uint(f.y);
-        u[4 * e + 2] = __float_as_uint(f.z);
-        u[4 * e + 3] = __float_as_uint(f.w);
-      }
-      tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
-    }
-    tmem_st_wait();
-  }
-
-  auto issue_load = [&](int i) {
-    uint8_t* sQ = base + (i & 1) * L_::kStage;
-    uint8_t* sK = sQ + L_::kQ;
-    uint8_t* sV = sK + L_::kK;
-    const int t0 = (cb + i) * kC;
-    mbar_arrive_expect_tx(&bars[i & 1], L_::kStage);
-#pragma unroll
-    for (int b = 0; b < DK / 64; ++b) {
-      tma_load_3d(sQ + b * kC * 128, &tm_q, &bars[i & 1], b * 64, t0, bh);
-      tma_load_3d(sK + b * kC * 128, &tm_k, &bars[i & 1], b * 64, t0, bh);
-    }
-#pragma unroll
-    for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &bars[i & 1], b * 64, t0, bh);
+  // A wait that runs out marks its thread failed, and a failed thread waits no more:
+  // the transform and epilogue roles still walk through their named barriers (on
+  // meaningless data, stored only in bounds) so that no thread of a role is left behind,
+  // and the control thread drains what it has issued before TMEM is freed.
+  auto wait = [&](uint64_t* bar, uint32_t parity, int code) -> bool {
+    if (failed) return false;
+    if (mbar_wait(bar, parity)) return true;
+    report_error(sp.err, code);
+    failed = true;
+    return false;
   };
-  if (tid == 0) issue_load(0);
 
-  constexpr int NCC = DK / 8;
-  constexpr int RG = kThreads / NCC;
-  const int cc = tid % NCC, rg = tid / NCC;
-
-  for (int i = 0; i < n; ++i) {
-    const int c = cb + i;
-    const int L = chunk_len(sp, c);
-    const int t0 = c * kC;
-    const bool last = i == n - 1;
-    const bool has_prefix = !(seg == 0 && i == 0);
-    uint8_t* sQ = base + (i & 1) * L_::kStage;
-    uint8_t* sK = sQ + L_::kQ;
-    uint8_t* sV = sK + L_::kK;
-    // The other stage was last read by chunk i - 1's MMAs, all complete by now.
-    if (tid == 0 && i + 1 < n) issue_load(i + 1);
-    if (tid < kC) sXi[tid] = tid < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tid)) : 1.f) : 0.f;
-    LA_WAIT_OR_LEAVE(&bars[i & 1], (i >> 1) & 1, kErrTmaTimeout, tmem, kTmemCols);
-
-    // psi on Q and K (hi in place + lo), Xi .* psi(K) (hi + lo) for the prefix update,
-    // psi(q) . ZP for the denominator, column sums of Xi .* psi(K) for Z.
-    float zacc[8];
+  if (warp < 4) {
+    // ------------------------------------------------------------------ transform
+    const int tw = tid;
+    {  // the segment's exclusive prefix, P^T row tw, into TMEM
+      const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(tw) * DK);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
-    {
+      for (int q4 = 0; q4 < DK / 32; ++q4) {
+        uint32_t u[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 f = src[q4 * 8 + e];
+          u[4 * e] = __float_as_uint(f.x);
+          u[4 * e + 1] = __float_as_uint(f.y);
+          u[4 * e + 2] = __float_as_uint(f.z);
+          u[4 * e + 3] = __float_as_uint(f.w);
+        }
+        tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
+      }
+      tmem_st_wait();
+    }
+    constexpr int NCC = DK / 8;
+    constexpr int RG = 128 / NCC;
+    const int cc = tw % NCC, rg = tw / NCC;
+    for (int i = 0; i < n; ++i) {
+      const int s = i & 1;
+      const int L = chunk_len(sp, cb + i);
+      const bool last = i == n - 1;
+      uint8_t* sQ = base + s * L_::kStage;
+      uint8_t* sK = sQ + L_::kQ;
+      uint8_t* sQl = sLo + s * L_::kLo;
+      uint8_t* sKl = sQl + L_::kQ;
+      uint8_t* sKph = sKpp + s * L_::kKpp;
+      uint8_t* sKpl = sKph + L_::kK;
+      float* xi = sXi + s * kC;
+      if (tw < kC) xi[tw] = tw < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tw)) : 1.f) : 0.f;
+      wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
+      named_barrier(1, 128);
+
+      float zacc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
       const uint32_t boff = (cc / 8) * (kC * 128);
       float zp[8];
 #pragma unroll
@@ -424,7 +463,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
             *reinterpret_cast<uint4*>(sK + off) = hi;
             *reinterpret_cast<uint4*>(sKl + off) = lo;
           }
-          const float w = sXi[r];
+          const float w = xi[r];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             x[e] *= w;
@@ -454,63 +493,168 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
             for (int e = 0; e < 8; ++e) part = fmaf(x[e], zp[e], part);
 #pragma unroll
             for (int o = NCC / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (cc == 0) sDenX[r] = part;
+            if (cc == 0) sDenX[s * kC + r] = part;
           }
         }
       }
-    }
-    if constexpr (NORM) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-#pragma unroll
-        for (int o = NCC; o < 32; o <<= 1) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], o);
-      if (lane < NCC)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sZpart[warp * DK + cc * 8 + e] = zacc[e];
-    }
+      fence_async_smem();
+      mbar_arrive(&ops[s]);
 
-    // Prefix operand: P^T (float32, TMEM) -> bf16 hi + lo packed into TMEM; then the
-    // carried state is scaled by gamma^L ahead of this chunk's update.
-    const float a_c = DECAY ? powf(g, static_cast<float>(L)) : 1.f;
+      const float a_c = DECAY ? powf(g, static_cast<float>(L)) : 1.f;
+      if constexpr (NORM) {
 #pragma unroll
-    for (int q4 = 0; q4 < DK / 32; ++q4) {
-      float r[32];
-      tmem_ld32(tmem + lane_base + kColP + q4 * 32, r);
-      tmem_ld_wait();
-      uint32_t hi[16], lo[16];
+        for (int e = 0; e < 8; ++e)
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(r[2 * e], r[2 * e + 1]);
-        const float2 hf = __bfloat1622float2(h);
-        hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-        lo[e] = pack2(r[2 * e] - hf.x, r[2 * e + 1] - hf.y);
+          for (int o = NCC; o < 32; o <<= 1) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], o);
+        if (lane < NCC)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sZpart[warp * DK + cc * 8 + e] = zacc[e];
+        named_barrier(1, 128);
+        if (tw < DK)
+          sZP[tw] = fmaf(a_c, sZP[tw],
+                         sZpart[tw] + sZpart[DK + tw] + sZpart[2 * DK + tw] + sZpart[3 * DK + tw]);
       }
-      tmem_st16(tmem + lane_base + kColPH + q4 * 16, hi);
-      tmem_st16(tmem + lane_base + kColPL + q4 * 16, lo);
-      if constexpr (DECAY) {
-        if (!last) {
-          uint32_t u[32];
+
+      // Prefix operand for chunk i (the state after chunk i - 1).
+      if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
+      tc_fence_after();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(r[e] * a_c);
-          tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
+      for (int q4 = 0; q4 < DK / 32; ++q4) {
+        float rr[32];
+        tmem_ld32(tmem + lane_base + kColP + q4 * 32, rr);
+        tmem_ld_wait();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(rr[2 * e], rr[2 * e + 1]);
+          const float2 hf = __bfloat1622float2(h);
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
+        }
+        tmem_st16(tmem + lane_base + kColPH + q4 * 16, hi);
+        tmem_st16(tmem + lane_base + kColPL + q4 * 16, lo);
+        if constexpr (DECAY) {
+          if (!last) {
+            uint32_t u[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * a_c);
+            tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
+          }
         }
       }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(pready);
     }
-    tmem_st_wait();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if constexpr (NORM) {
-      if (tid < DK)
-        sZP[tid] = fmaf(a_c, sZP[tid], sZpart[tid] + sZpart[DK + tid] + sZpart[2 * DK + tid] +
-                                           sZpart[3 * DK + tid]);
-    }
-
-    const uint32_t aQ = smem_u32(sQ), aQl = smem_u32(sQl), aK = smem_u32(sK), aKl = smem_u32(sKl);
-    const uint32_t aV = smem_u32(sV);
-    if (tid == 0) {
+  } else if (warp < 12) {
+    // ------------------------------------------------------------------ epilogue
+    const int tw = tid - 128;
+    const int quarter = warp & 3, half = (warp - 4) >> 2;
+    for (int i = 0; i < n; ++i) {
+      const int s = i & 1;
+      const int t0 = (cb + i) * kC;
+      const bool has_prefix = !(seg == 0 && i == 0);
+      wait(sdone, i & 1, kErrMmaTimeout);
+      wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout);
       tc_fence_after();
-      // Scores D_S = psi(Q) psi(K)^T, M = 64, N = 64.
+      {
+        // Rows 16 quarter .. + 15 (lanes 0-15), keys 32 half .. + 31.
+        const int row = quarter * 16 + lane;
+        float sc[32];
+        tmem_ld32(tmem + lane_base + kColS + 32 * half, sc);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(sfree);
+        if (lane < 16) {
+          float den_loc = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float a[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int j = 32 * half + q * 8 + e;
+              a[e] = j <= row ? sc[q * 8 + e] * sPow[row - j] : 0.f;
+              den_loc += a[e];
+            }
+            uint4 hi, lo;
+            split8(a, hi, lo);
+            *reinterpret_cast<uint4*>(sAh + sw128_offset(row, 4 * half + q)) = hi;
+            *reinterpret_cast<uint4*>(sAl + sw128_offset(row, 4 * half + q)) = lo;
+          }
+          if constexpr (NORM) sDenPart[half * kC + row] = den_loc;
+        }
+      }
+      // psi(q).ZP of this chunk is read before A is handed over: once N(i) is done the
+      // stage (and its sDenX slot) is refilled with chunk i + 2.
+      const float denx = NORM && has_prefix && tw < kC ? sDenX[s * kC + tw] : 0.f;
+      fence_async_smem();
+      mbar_arrive(aready);
+      if constexpr (NORM) {
+        named_barrier(2, 256);
+        if (tw < kC) sDen[tw] = fmaf(sTh[tw], denx, sDenPart[tw] + sDenPart[kC + tw]) + sp.eps;
+      }
+
+      wait(ndone, i & 1, kErrMmaTimeout);
+      tc_fence_after();
+      // Column j (value feature), tokens 32 half .. + 31.
+      float xo[32], no[32];
+      if (has_prefix) tmem_ld32(tmem + lane_base + kColX[s] + 32 * half, xo);
+      tmem_ld32(tmem + lane_base + kColN + 32 * half, no);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&xfree[s]);
+      if (tw == 0) bulk_wait_read_all();  // the previous tile has left the staging buffer
+      named_barrier(2, 256);
+      const int j = quarter * 32 + lane;
+#pragma unroll
+      for (int tt = 0; tt < kC / 2; ++tt) {
+        const int t = 32 * half + tt;
+        float o = has_prefix ? fmaf(sTh[t], xo[tt], no[tt]) : no[tt];
+        if constexpr (NORM) o = o / sDen[t];
+        if constexpr (OUTF32) {
+          *reinterpret_cast<float*>(sO + (j / 32) * (kC * 128) + sw128_offset(t, (j % 32) / 4) +
+                                    (j % 4) * 4) = o;
+        } else {
+          *reinterpret_cast<__nv_bfloat16*>(sO + (j / 64) * (kC * 128) +
+                                            sw128_offset(t, (j % 64) / 8) + (j % 8) * 2) =
+              __float2bfloat16_rn(o);
+        }
+      }
+      fence_async_smem();
+      named_barrier(2, 256);
+      if (tw == 0) {
+        constexpr int kOutCols = OUTF32 ? 32 : 64;
+#pragma unroll
+        for (int b = 0; b < DV / kOutCols; ++b)
+          tma_store_3d(&tm_out, sO + b * (kC * 128), b * kOutCols, t0, bh);
+        bulk_commit();
+      }
+    }
+    if (tw == 0) bulk_wait_read_all();
+  } else if (lane == 0) {
+    // ------------------------------------------------------------------ control
+    auto issue_load = [&](int i) {
+      uint8_t* sQ = base + (i & 1) * L_::kStage;
+      uint8_t* sK = sQ + L_::kQ;
+      uint8_t* sV = sK + L_::kK;
+      const int t0 = (cb + i) * kC;
+      mbar_arrive_expect_tx(&full[i & 1], L_::kStage);
+#pragma unroll
+      for (int b = 0; b < DK / 64; ++b) {
+        tma_load_3d(sQ + b * kC * 128, &tm_q, &full[i & 1], b * 64, t0, bh);
+        tma_load_3d(sK + b * kC * 128, &tm_k, &full[i & 1], b * 64, t0, bh);
+      }
+#pragma unroll
+      for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &full[i & 1], b * 64, t0, bh);
+    };
+    auto issue_scores = [&](int i) -> bool {
+      const int s = i & 1;
+      uint8_t* sQ = base + s * L_::kStage;
+      const uint32_t aQ = smem_u32(sQ), aK = aQ + L_::kQ;
+      const uint32_t aQl = smem_u32(sLo + s * L_::kLo), aKl = aQl + L_::kQ;
+      if (!wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout)) return false;
+      if (i > 0 && !wait(sfree, (i - 1) & 1, kErrMmaTimeout)) return false;
+      tc_fence_after();
       constexpr uint32_t ids = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 64, 64);
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk) {
@@ -523,26 +667,43 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           mma_bf16_ss(tmem + kColS, smem_desc_sw128(aQl + off, 16, 1024), kh, ids, 1u);
         }
       }
-      mma_commit(&bars[2]);
-      // X^T = P^T psi(Q)^T: A = P^T (TMEM, hi / lo), B = psi(Q) rows (K-major), M = 128.
+      mma_commit(sdone);
+      return true;
+    };
+    int loads = 0;
+    issue_load(loads++);
+    if (n > 1) issue_load(loads++);
+    issue_scores(0);
+    for (int i = 0; i < n && !failed; ++i) {
+      const int s = i & 1;
+      const bool last = i == n - 1;
+      const bool has_prefix = !(seg == 0 && i == 0);
+      uint8_t* sQ = base + s * L_::kStage;
+      const uint32_t aQ = smem_u32(sQ), aK = aQ + L_::kQ, aV = aK + L_::kK;
+      const uint32_t aQl = smem_u32(sLo + s * L_::kLo), aKl = aQl + L_::kQ;
+      const uint32_t aKph = smem_u32(sKpp + s * L_::kKpp), aKpl = aKph + L_::kK;
+
+      // X(i) = P^T psi(Q)^T and the prefix update with chunk i.
+      if (!wait(pready, i & 1, kErrMmaTimeout)) break;
+      if (i > 1 && !wait(&xfree[s], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
+      tc_fence_after();
       if (has_prefix) {
         constexpr uint32_t idx = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 128, 64);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
           const uint64_t qh = smem_desc_sw128(aQ + off, 16, 1024);
-          mma_bf16_ts(tmem + kColX, tmem + kColPH + kk * 8, qh, idx, kk > 0 ? 1u : 0u);
-          mma_bf16_ts(tmem + kColX, tmem + kColPL + kk * 8, qh, idx, 1u);
+          mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, qh, idx, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + kColX[s], tmem + kColPL + kk * 8, qh, idx, 1u);
           if constexpr (kSplitQK)
-            mma_bf16_ts(tmem + kColX, tmem + kColPH + kk * 8, smem_desc_sw128(aQl + off, 16, 1024),
-                        idx, 1u);
+            mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8,
+                        smem_desc_sw128(aQl + off, 16, 1024), idx, 1u);
         }
       }
-      // Prefix update P^T += V^T (Xi .* psi(K)), M = 128, N = DK, K = tokens.
       if (!last) {
         constexpr uint32_t idp = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kMNMajor, 128, DK);
-        const uint32_t bh_ = DECAY ? smem_u32(sKph) : aK;
-        const uint32_t bl_ = DECAY ? smem_u32(sKpl) : aKl;
+        const uint32_t bh_ = DECAY ? aKph : aK;
+        const uint32_t bl_ = DECAY ? aKpl : aKl;
 #pragma unroll
         for (int kk = 0; kk < kC / 16; ++kk) {
           const uint64_t da = smem_desc_sw128(aV + kk * 2048, kC * 128, 1024);
@@ -551,43 +712,11 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
             mma_bf16_ss(tmem + kColP, da, smem_desc_sw128(bl_ + kk * 2048, kC * 128, 1024), idp, 1u);
         }
       }
-    }
-    LA_WAIT_OR_LEAVE(&bars[2], 0, kErrMmaTimeout, tmem, kTmemCols);
-    tc_fence_after();
+      mma_commit(statedone);
 
-    // Mask and decay on the scores -> A (hi + lo); denominators.
-    {
-      const int row = warp * 16 + lane;
-      float s[64];
-      tmem_ld32(tmem + lane_base + kColS, *reinterpret_cast<float(*)[32]>(&s[0]));
-      tmem_ld32(tmem + lane_base + kColS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
-      tmem_ld_wait();
-      if (lane < 16) {
-        float den_loc = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float a[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j = q * 8 + e;
-            a[e] = j <= row ? s[j] * sPow[row - j] : 0.f;
-            den_loc += a[e];
-          }
-          uint4 hi, lo;
-          split8(a, hi, lo);
-          *reinterpret_cast<uint4*>(sAh + sw128_offset(row, q)) = hi;
-          *reinterpret_cast<uint4*>(sAl + sw128_offset(row, q)) = lo;
-        }
-        if constexpr (NORM)
-          sDen[row] = (has_prefix ? fmaf(sTh[row], sDenX[row], den_loc) : den_loc) + sp.eps;
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+      // N(i) = V^T A^T.
+      if (!wait(aready, i & 1, kErrMmaTimeout)) break;
       tc_fence_after();
-      // N^T = V^T A^T: A = V^T (MN-major), B = A rows (queries) K-major over keys.
       constexpr uint32_t idn = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kKMajor, 128, 64);
       const uint32_t aAh = smem_u32(sAh), aAl = smem_u32(sAl);
 #pragma unroll
@@ -597,49 +726,25 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
                     kk > 0 ? 1u : 0u);
         mma_bf16_ss(tmem + kColN, da, smem_desc_sw128(aAl + kk * 32, 16, 1024), idn, 1u);
       }
-      mma_commit(&bars[2]);
-      bulk_wait_read_all();  // the previous chunk's output store has left the staging
-    }
-    LA_WAIT_OR_LEAVE(&bars[2], 1, kErrMmaTimeout, tmem, kTmemCols);
-    tc_fence_after();
+      mma_commit(ndone);
 
-    // Output column j (this lane's value feature) for the chunk's 64 tokens.
-    {
-      const int j = tid;
-      float xo[64], no[64];
-      if (has_prefix) {
-        tmem_ld32(tmem + lane_base + kColX, *reinterpret_cast<float(*)[32]>(&xo[0]));
-        tmem_ld32(tmem + lane_base + kColX + 32, *reinterpret_cast<float(*)[32]>(&xo[32]));
-      }
-      tmem_ld32(tmem + lane_base + kColN, *reinterpret_cast<float(*)[32]>(&no[0]));
-      tmem_ld32(tmem + lane_base + kColN + 32, *reinterpret_cast<float(*)[32]>(&no[32]));
-      tmem_ld_wait();
-#pragma unroll
-      for (int t = 0; t < kC; ++t) {
-        float o = has_prefix ? fmaf(sTh[t], xo[t], no[t]) : no[t];
-        if constexpr (NORM) o = o / sDen[t];
-        if constexpr (OUTF32) {
-          *reinterpret_cast<float*>(sO + (j / 32) * (kC * 128) + sw128_offset(t, (j % 32) / 4) +
-                                    (j % 4) * 4) = o;
-        } else {
-          *reinterpret_cast<__nv_bfloat16*>(sO + (j / 64) * (kC * 128) +
-                                            sw128_offset(t, (j % 64) / 8) + (j % 8) * 2) =
-              __float2bfloat16_rn(o);
-        }
+      // The next chunk's scores go in behind N(i); the stage of chunk i is refilled with
+      // chunk i + 2 once all of chunk i's MMAs are done.
+      if (i + 1 < n && !issue_scores(i + 1)) break;
+      if (i + 2 < n) {
+        if (!wait(ndone, i & 1, kErrMmaTimeout)) break;
+        issue_load(loads++);
       }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      constexpr int kOutCols = OUTF32 ? 32 : 64;
-#pragma unroll
-      for (int b = 0; b < DV / kOutCols; ++b)
-        tma_store_3d(&tm_out, sO + b * (kC * 128), b * kOutCols, t0, bh);
-      bulk_commit();
+    if (failed) {
+      // Let the issued MMAs finish and the last two loads land before TMEM and shared
+      // memory are given up; both waits are bounded.
+      mma_commit(drain);
+      mbar_wait(drain, 0);
+      for (int j = max(0, loads - 2); j < loads; ++j) mbar_wait(&full[j & 1], (j >> 1) & 1);
     }
   }
-  if (tid == 0) bulk_wait_read_all();
+  tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
@@ -668,11 +773,11 @@ cudaError_t k1s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
 cudaError_t k3s_go_o(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
   auto kern = k3_seg<DK, FM, DECAY, NORM, OUTF32>;
-  const uint32_t sm = K3sSmem<DK, OUTF32>::kTotal;
+  const uint32_t sm = K3sSmem<DK, FM, DECAY, OUTF32>::kTotal;
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(sp.BH) * sp.NS;
-  kern<<<static_cast<unsigned>(grid), kThreads, sm, s>>>(m.q, m.k, m.v, m.out, sp, gt);
+  kern<<<static_cast<unsigned>(grid), kThreads3, sm, s>>>(m.q, m.k, m.v, m.out, sp, gt);
   return cudaGetLastError();
 }
 
@@ -680,8 +785,12 @@ template <int DK, int DV, int FM, bool DECAY, bool NORM>
 cudaError_t k3s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                    cudaStream_t s) {
   static_assert(DV == 128, "the segmented combine needs dv = 128");
-  return f.out_f32 ? k3s_go_o<DK, FM, DECAY, NORM, true>(sp, gt, m, s)
-                   : k3s_go_o<DK, FM, DECAY, NORM, false>(sp, gt, m, s);
+  if constexpr (FM == 1 && DECAY) {
+    return cudaErrorInvalidValue;  // excluded by seg_supported (shared memory budget)
+  } else {
+    return f.out_f32 ? k3s_go_o<DK, FM, DECAY, NORM, true>(sp, gt, m, s)
+                     : k3s_go_o<DK, FM, DECAY, NORM, false>(sp, gt, m, s);
+  }
 }
 
 #define LA_SEG_FLAGS(DK, DV, GO)                                          \
@@ -700,8 +809,10 @@ cudaError_t k3s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
 
 }  // namespace
 
-bool seg_supported(int dk, int dv, int C) {
-  return C == kC && (dk == 64 || dk == 128) && dv == 128;
+bool seg_supported(int dk, int dv, int C, int fm, bool decay) {
+  // ELU+1 with decay needs both the psi lo tiles and the decayed key tiles double
+  // buffered, which does not fit in shared memory next to the two stages.
+  return C == kC && (dk == 64 || dk == 128) && dv == 128 && !(fm == 1 && decay);
 }
 
 cudaError_t launch_k1_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,

@@ -96,8 +96,9 @@ typedef enum { LA_OUT_AS_INPUT = 0, LA_OUT_F32 = 1 } la_out_dtype;
  *                      segments; K1 writes one summary per segment, K2 scans segments,
  *                      and K3 walks each segment's chunks in order, carrying the prefix
  *                      on chip and advancing it with the chunk's own summary.  Same
- *                      results, about a quarter of the HBM traffic.  Tensor-core path
- *                      only: bf16 inputs, C = 64, dk in {64, 128}, dv = 128.
+ *                      results, about a third of the HBM traffic.  Tensor-core path
+ *                      only: bf16 inputs, C = 64, dk in {64, 128}, dv = 128, and not the
+ *                      ELU+1 map together with a decay.
  *   LA_ALGO_AUTO       segmented where supported, else chunked.
  */
 typedef enum { LA_ALGO_AUTO = 0, LA_ALGO_CHUNKED = 1, LA_ALGO_SEGMENTED = 2 } la_algorithm;
@@ -184,9 +185,9 @@ int lin_attn_prefill_ex(const la_prefill_args* args);
  * lin_attn_prefill_timed -- lin_attn_prefill_ex with a CUDA event recorded on the stream
  * before every kernel launch and after the last one; synchronises the stream and writes
  * each kernel's device duration (milliseconds, launch order) to kernel_ms[0 ..].
- * *n_kernels receives the number of kernels the prefill launched (K1, the scan's
- * kernels, K3: 5 with the log-depth scan, 3 with the sequential carry; the segmented
- * algorithm launches the same count).  For profiling;
+ * *n_kernels receives the number of kernels the prefill launched: K1, the scan's kernels
+ * (3 for the log-depth scan over more than 32 elements, 1 for at most 32 elements or for
+ * the sequential carry), K3.  For profiling;
  * the results are identical to lin_attn_prefill_ex.
  */
 int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int max_kernels,

@@ -16,6 +16,7 @@ import pytest
 import torch
 
 from chunked_causal_linear_b200.workloads import WORKLOADS, Workload, make_inputs
+from chunked_causal_linear_b200 import binding as B
 from gpu_common import (TOL_BF16, TOL_F32, assert_close, assert_close_rounded_out,
                         gammas_for, gpu_prefill, oracle_prefill, to_np)
 
@@ -66,6 +67,15 @@ def test_segmented_path(dk, T, seg, mode):
     """Segments of `seg` chunks (0 = automatic): the prefix carried through several chunks
     inside a segment, segment prefixes from the scan, a ragged last chunk."""
     w, q, k, v, gamma = _case(T, dk, 128, 64, mode)
+    if mode == "decay_norm":
+        # ELU+1 with decay is not offered by the segmented kernels (shared memory); an
+        # explicit request is refused and `auto` runs the chunked algorithm.
+        with pytest.raises(B.LinAttnError) as e:
+            gpu_prefill(q, k, v, C=64, feature_map=w.feature_map, gamma=gamma,
+                        normalize=w.normalize, kernel_path="tensor_core", algorithm="segmented")
+        assert e.value.status == 2
+        _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core", algorithm="auto")
+        return
     _check(w, q, k, v, gamma, TOL_BF16, kernel_path="tensor_core", algorithm="segmented",
            segment_chunks=seg)
 
@@ -94,6 +104,8 @@ def test_fma_path_f32(T, dk, dv, C, mode):
 def test_bf16_output(T, path, mode, algorithm):
     if path == "fma" and algorithm == "segmented":
         pytest.skip("the segmented algorithm runs on the tensor-core kernels only")
+    if mode == "decay_norm" and algorithm == "segmented":
+        pytest.skip("ELU+1 with decay runs on the chunked algorithm only")
     w, q, k, v, gamma = _case(T, 128, 128, 64, mode)
     out, S, Z = gpu_prefill(q, k, v, C=64, feature_map=w.feature_map, gamma=gamma,
                             normalize=w.normalize, kernel_path=path, out_dtype="as_input",
