@@ -63,9 +63,9 @@ def effective_algorithm(w, requested: str) -> str:
     return "chunked"
 
 
-def kernel_names(w, algo: str, scan: str) -> list[str]:
+def kernel_names(w, algo: str, scan: str, lseg: int = 0) -> list[str]:
     k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
-    n, _, _ = layout(w, algo)
+    n, _, _ = layout(w, algo, lseg)
     k2 = ["k2_scan_totals"] if scan == "logdepth" and n <= 32 else K2_NAMES[scan]
     return [k1, *k2, k3]
 
@@ -74,24 +74,32 @@ def kernel_names(w, algo: str, scan: str) -> list[str]:
 # Algorithmic bytes
 
 
-def layout(w, algo: str = "chunked"):
+def segment_length(w, lseg: int = 0) -> int:
+    """Chunks per segment of the segmented algorithm: the requested count, else the
+    library's automatic choice (about four segments per SM, at most 64 chunks)."""
+    NC = -(-w.T // w.C)
+    if lseg > 0:
+        return min(lseg, NC)
+    return max(1, min(64, (w.B * w.H * NC) // (4 * 148)))
+
+
+def layout(w, algo: str = "chunked", lseg: int = 0):
     """(scan elements per (b, h), scan segments G, floats per record) as the library lays
     them out: chunks for the chunked algorithm, segments of chunks for the segmented one."""
     NC = -(-w.T // w.C)
     n = NC
     if algo == "segmented":
-        lseg = max(1, min(64, (w.B * w.H * NC) // (4 * 148)))
-        n = -(-NC // lseg)
+        n = -(-NC // segment_length(w, lseg))
     Ls = max(1, -(-n // 32))
     G = -(-n // Ls)
     R = w.dk * w.dv + (w.dk if w.normalize else 0)
     return n, G, R
 
 
-def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked") -> int:
+def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked", lseg: int = 0) -> int:
     """Bytes each kernel must move for its own role (one launch)."""
     BH = w.B * w.H
-    n, G, R = layout(w, algo)
+    n, G, R = layout(w, algo, lseg)
     e_in = 2 if w.dtype == "bf16" else 4
     rec = BH * n * R * 4
     if name.startswith("k1"):
@@ -111,12 +119,12 @@ def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked") -> int:
     raise KeyError(name)
 
 
-def algo_bytes(w, out_elem: int, algo: str) -> int:
+def algo_bytes(w, out_elem: int, algo: str, lseg: int = 0) -> int:
     """Whole-step algorithmic bytes of an algorithm: its input reads (the segmented one
     reads k and v in K1 and again in K3), the output, the final states, and four passes of
     its records (K1 write, K2 read and write, K3 read)."""
     BH = w.B * w.H
-    n, G, R = layout(w, algo)
+    n, G, R = layout(w, algo, lseg)
     e_in = 2 if w.dtype == "bf16" else 4
     kv_again = BH * w.T * (w.dk + w.dv) * e_in if algo == "segmented" else 0
     return (BH * w.T * (2 * w.dk + w.dv) * e_in + kv_again + BH * w.T * w.dv * out_elem
@@ -352,6 +360,8 @@ def config_of(w, args):
             "gamma": "1 - 2^(-5-3h/31) per head" if w.decay else None,
             "normalize": w.normalize, "scan": args.scan, "out_dtype": args.out_dtype,
             "algorithm": effective_algorithm(w, args.algorithm),
+            **({"segment_chunks": segment_length(w, getattr(args, "segment_chunks", 0))}
+               if effective_algorithm(w, args.algorithm) == "segmented" else {}),
             "kernel_path": "tensor_core", "l2": "inputs larger than L2, no flush",
             "parallelism": "replicas (one independent problem per GPU)"}
 
@@ -380,6 +390,8 @@ def main():
     ap.add_argument("--sweep-scan", action="store_true",
                     help="instead of the benchmark line: time K2 (log-depth vs sequential "
                          "carry) over a range of chunk counts, one JSON line per point")
+    ap.add_argument("--segment-chunks", type=int, default=0,
+                    help="chunks per segment of the segmented algorithm (0: automatic)")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -417,7 +429,7 @@ def main():
     algo = effective_algorithm(w, args.algorithm)
     kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
               scan=args.scan, kernel_path="tensor_core", workspace=ws, out_dtype=args.out_dtype,
-              algorithm=algo)
+              algorithm=algo, segment_chunks=args.segment_chunks)
 
     def step():
         B.lin_attn_prefill(q, k, v, out, S, Z, **kw)
@@ -448,7 +460,7 @@ def main():
         ms, clocks = timed_region()
         remeasured = True
     ms_max = ranks.max_over_ranks(ms, info, dev)
-    names = kernel_names(w, algo, args.scan)
+    names = kernel_names(w, algo, args.scan, args.segment_chunks)
     n_kern = len(names)
     value = info.world * w.tokens_heads / (ms_max / 1000.0)
 
@@ -461,14 +473,14 @@ def main():
     kern_ms = {n: statistics.mean(x) for n, x in zip(names, per)}
     dom = max(kern_ms, key=kern_ms.get)
     peak, peak_kind = measured_peaks()
-    dom_bytes = kernel_bytes(w, dom, out_elem, algo)
+    dom_bytes = kernel_bytes(w, dom, out_elem, algo, args.segment_chunks)
     achieved = dom_bytes / (kern_ms[dom] / 1000.0) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak,
                 "traffic": recorded_traffic(dom, w.name),
                 "algorithmic_bytes": dom_bytes, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s"}
-    ab = algo_bytes(w, out_elem, algo)
+    ab = algo_bytes(w, out_elem, algo, args.segment_chunks)
     gbs = lambda nbytes: nbytes / (ms_max / 1000.0) / 1e9
     step_roof = {"algorithm": algo, "bytes": ab, "achieved_gbs": gbs(ab),
                  "frac_of_measured": gbs(ab) / peak,

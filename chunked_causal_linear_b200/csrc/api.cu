@@ -290,6 +290,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     sp.R = l.R;
     sp.eps = a.eps;
     sp.srec = reinterpret_cast<float*>(ws);
+    sp.out = a.out;
     sp.err = p.err;
     const size_t srec_bytes = align256(static_cast<size_t>(BH) * NS * l.R * sizeof(float));
     PrefillParams ps = p;  // the scan over segments: one scan element per segment
@@ -308,10 +309,6 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
                        T * a.dk * 2ull, 64, 64) &&
               make_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, a.dv, T, BH, a.dv * 2ull,
                        T * a.dv * 2ull, 64, 64) &&
-              (out_f32 ? make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, a.dv, T, BH,
-                                  a.dv * 4ull, T * a.dv * 4ull, 32, 64)
-                       : make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.dv, T, BH,
-                                  a.dv * 2ull, T * a.dv * 2ull, 64, 64)) &&
               make_map(&m.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.srec, a.dk, a.dv,
                        static_cast<uint64_t>(BH) * NS, a.dk * 4ull, l.R * 4ull, 32,
                        static_cast<uint32_t>(a.dv));

@@ -53,6 +53,7 @@ struct SegParams {
   int R;           // floats per record
   float eps;
   float* srec;     // [BH, NS, R] segment totals, turned into exclusive prefixes by K2
+  void* out;       // [BH, T, dv] output, bf16 or fp32
   int* err;
 };
 

@@ -269,22 +269,28 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
 // ---------------------------------------------------------------------------------------
 // K3s (dv = 128), warp-specialised.
 //
-// 416 threads in three roles that hand work over through mbarriers, so that the
+// 576 threads in four roles that hand work over through mbarriers, so that the
 // transform of chunk i + 1 overlaps the MMAs and epilogues of chunk i:
-//   warps 0-3  transform: psi on the staged Q, K (bf16 hi / lo operand tiles, double
-//              buffered), Xi .* psi(K), psi(q).ZP and the Z update; then the prefix
-//              operand: P^T from TMEM -> bf16 hi / lo into TMEM, and P scaled by gamma^L.
-//   warps 4-11 epilogue (two warps per TMEM lane quarter, each half of the columns):
-//              masks and decays the scores into A (hi / lo), then combines
-//              o = Theta X + N (/ den) and stores the chunk's output tile with TMA.
-//   warp 12    control (one thread): TMA loads two chunks ahead and every tcgen05.mma;
-//              the next chunk's scores are issued before the current chunk's local
-//              product has finished.
+//   warps 0-7   transform (two warps per TMEM lane quarter, each half of the key features):
+//               psi on the staged Q, K (bf16 hi / lo operand tiles, double buffered),
+//               Xi .* psi(K), psi(q).ZP and the Z update; then the prefix operand: P^T
+//               from TMEM -> bf16 hi / lo into TMEM, and P scaled by gamma^L.
+//   warps 8-15  epilogue (two warps per TMEM lane quarter, each half of the columns):
+//               masks and decays the scores into A (hi / lo), then combines
+//               o = Theta X + N (/ den) and writes it straight to global memory (a warp
+//               stores 32 consecutive value features of one token per instruction).
+//   warp 16     producer (one thread): TMA loads of Q, K, V into a two-stage ring; a
+//               stage is refilled as soon as the last MMA reading it (N of its chunk) is done.
+//   warp 17     MMA issuer (one thread): every tcgen05.mma.  Shared-memory descriptors are
+//               built once per stage; each k-step only adds a constant offset, so the
+//               tensor pipe, not the issuing thread, sets the pace.
 // Warp w reads TMEM lanes 32 (w % 4) .. + 31.  Accumulators (TMEM columns): scores
 // [0, 64), X (two buffers) [64, 128) and [448, 512), N [128, 192), P [192, 192 + dk),
 // P hi / lo after it.  Each is released by an mbarrier once its readers are done.
 
-constexpr int kThreads3 = 416;
+constexpr int kThreads3 = 576;
+constexpr int kXfThreads = 256;  // transform warps 0-7
+constexpr int kEpThreads = 256;  // epilogue warps 8-15
 
 template <int DK, int FM, bool DECAY, bool OUTF32>
 struct K3sSmem {
@@ -296,17 +302,21 @@ struct K3sSmem {
   static constexpr uint32_t kLo = FM == 1 ? kQ + kK : 0;  // lo tiles of psi(Q), psi(K)
   static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
-  static constexpr uint32_t kO = kC * DV * (OUTF32 ? 4 : 2);
-  static constexpr uint32_t kSmallFloats = 5 * DK + 10 * kC;
+  static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC;
+  static constexpr uint32_t kBars = 15;
   static constexpr uint32_t kTotal =
-      2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kO + kSmallFloats * 4 + 16 * 8 + 1024;
+      2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
 };
+
+// A shared-memory descriptor advanced by a byte offset: the start address field holds
+// address >> 4 in its low 14 bits and every operand of this kernel lies below 256 KB, so
+// the addition never carries out of the field.
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
 __global__ void __launch_bounds__(kThreads3, 1)
 k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-       SegParams sp, GammaTable gt) {
+       const __grid_constant__ CUtensorMap tm_v, SegParams sp, GammaTable gt) {
   constexpr int DV = 128;
   using L_ = K3sSmem<DK, FM, DECAY, OUTF32>;
   constexpr bool kSplitQK = FM == 1;
@@ -323,10 +333,9 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   uint8_t* sKpp = sLo + 2 * L_::kLo;         // [2] x (hi, lo)
   uint8_t* sAh = sKpp + 2 * L_::kKpp;
   uint8_t* sAl = sAh + L_::kA;
-  uint8_t* sO = sAl + L_::kA;
-  float* sZP = reinterpret_cast<float*>(sO + L_::kO);
-  float* sZpart = sZP + DK;        // [4][DK]
-  float* sDenX = sZpart + 4 * DK;  // [2][kC]
+  float* sZP = reinterpret_cast<float*>(sAl + L_::kA);
+  float* sZpart = sZP + DK;        // [8][DK]
+  float* sDenX = sZpart + 8 * DK;  // [2][kC]
   float* sDen = sDenX + 2 * kC;
   float* sTh = sDen + kC;
   float* sPow = sTh + kC;
@@ -343,7 +352,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   uint64_t* statedone = bars + 10;
   uint64_t* ndone = bars + 11;
   uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* empty = bars + 13;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L_::kBars);
 
   if (error_pending(sp.err)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -358,13 +368,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&full[b], 1);
-      mbar_init(&ops[b], 128);
+      mbar_init(&ops[b], kXfThreads);
+      mbar_init(&xfree[b], kEpThreads);
+      mbar_init(&empty[b], 1);
     }
-    mbar_init(pready, 128);
-    mbar_init(sfree, 256);
-    mbar_init(&xfree[0], 256);
-    mbar_init(&xfree[1], 256);
-    mbar_init(aready, 256);
+    mbar_init(pready, kXfThreads);
+    mbar_init(sfree, kEpThreads);
+    mbar_init(aready, kEpThreads);
     mbar_init(sdone, 1);
     mbar_init(statedone, 1);
     mbar_init(ndone, 1);
@@ -373,7 +383,6 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_out);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -396,7 +405,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   // A wait that runs out marks its thread failed, and a failed thread waits no more:
   // the transform and epilogue roles still walk through their named barriers (on
   // meaningless data, stored only in bounds) so that no thread of a role is left behind,
-  // and the control thread drains what it has issued before TMEM is freed.
+  // and the MMA issuer drains what it has issued before TMEM is freed.
   auto wait = [&](uint64_t* bar, uint32_t parity, int code) -> bool {
     if (failed) return false;
     if (mbar_wait(bar, parity)) return true;
@@ -405,13 +414,16 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     return false;
   };
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------------ transform
     const int tw = tid;
-    {  // the segment's exclusive prefix, P^T row tw, into TMEM
-      const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(tw) * DK);
+    constexpr int kHalf = DK / 2;  // key features of P handled by this thread
+    const uint32_t pcol = static_cast<uint32_t>(warp >> 2) * kHalf;
+    {  // the segment's exclusive prefix: row (lane) of P^T, this thread's half
+      const int row = (warp & 3) * 32 + lane;
+      const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
 #pragma unroll
-      for (int q4 = 0; q4 < DK / 32; ++q4) {
+      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
         uint32_t u[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -421,12 +433,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           u[4 * e + 2] = __float_as_uint(f.z);
           u[4 * e + 3] = __float_as_uint(f.w);
         }
-        tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
+        tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
       }
       tmem_st_wait();
     }
     constexpr int NCC = DK / 8;
-    constexpr int RG = 128 / NCC;
+    constexpr int RG = kXfThreads / NCC;
+    constexpr int kRows = kC / RG;
     const int cc = tw % NCC, rg = tw / NCC;
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
@@ -441,7 +454,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       float* xi = sXi + s * kC;
       if (tw < kC) xi[tw] = tw < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tw)) : 1.f) : 0.f;
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
-      named_barrier(1, 128);
+      named_barrier(1, kXfThreads);
 
       float zacc[8];
 #pragma unroll
@@ -450,11 +463,27 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       float zp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) zp[e] = NORM ? sZP[cc * 8 + e] : 0.f;
-      for (int r = rg; r < kC; r += RG) {
+      // Every shared load of this thread's rows first, then the arithmetic and stores
+      // (a load issued after a store to shared memory waits for it).
+      uint4 kraw[kRows], qraw[kRows];
+      float wr[kRows];
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        const int r = rg + k * RG;
+        const uint32_t off = boff + sw128_offset(r, cc % 8);
+        if constexpr (kSplitQK || DECAY || NORM) {
+          kraw[k] = *reinterpret_cast<const uint4*>(sK + off);
+          wr[k] = xi[r];
+        }
+        if constexpr (kSplitQK || NORM) qraw[k] = *reinterpret_cast<const uint4*>(sQ + off);
+      }
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        const int r = rg + k * RG;
         const uint32_t off = boff + sw128_offset(r, cc % 8);
         if constexpr (kSplitQK || DECAY || NORM) {
           float x[8];
-          unpack8(*reinterpret_cast<const uint4*>(sK + off), x);
+          unpack8(kraw[k], x);
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = r < L ? feature<FM>(x[e]) : 0.f;
           if constexpr (kSplitQK) {
@@ -463,10 +492,9 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
             *reinterpret_cast<uint4*>(sK + off) = hi;
             *reinterpret_cast<uint4*>(sKl + off) = lo;
           }
-          const float w = xi[r];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            x[e] *= w;
+            x[e] *= wr[k];
             zacc[e] += x[e];
           }
           if constexpr (DECAY) {
@@ -478,7 +506,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         }
         if constexpr (kSplitQK || NORM) {
           float x[8];
-          unpack8(*reinterpret_cast<const uint4*>(sQ + off), x);
+          unpack8(qraw[k], x);
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = feature<FM>(x[e]);
           if constexpr (kSplitQK) {
@@ -500,7 +528,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       fence_async_smem();
       mbar_arrive(&ops[s]);
 
-      const float a_c = DECAY ? powf(g, static_cast<float>(L)) : 1.f;
+      // gamma^L: Theta of the chunk's last token for a full chunk.
+      const float a_c = DECAY ? (L == kC ? sTh[kC - 1] : powf(g, static_cast<float>(L))) : 1.f;
       if constexpr (NORM) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -509,19 +538,24 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         if (lane < NCC)
 #pragma unroll
           for (int e = 0; e < 8; ++e) sZpart[warp * DK + cc * 8 + e] = zacc[e];
-        named_barrier(1, 128);
-        if (tw < DK)
-          sZP[tw] = fmaf(a_c, sZP[tw],
-                         sZpart[tw] + sZpart[DK + tw] + sZpart[2 * DK + tw] + sZpart[3 * DK + tw]);
+        named_barrier(1, kXfThreads);
+        if (tw < DK) {
+          float zs = 0.f;
+#pragma unroll
+          for (int w = 0; w < 8; ++w) zs += sZpart[w * DK + tw];
+          sZP[tw] = fmaf(a_c, sZP[tw], zs);
+        }
       }
 
-      // Prefix operand for chunk i (the state after chunk i - 1).
+      // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of
+      // the key features.
       if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
       tc_fence_after();
 #pragma unroll
-      for (int q4 = 0; q4 < DK / 32; ++q4) {
+      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
+        const uint32_t col = pcol + q4 * 32;
         float rr[32];
-        tmem_ld32(tmem + lane_base + kColP + q4 * 32, rr);
+        tmem_ld32(tmem + lane_base + kColP + col, rr);
         tmem_ld_wait();
         uint32_t hi[16], lo[16];
 #pragma unroll
@@ -531,14 +565,14 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           hi[e] = *reinterpret_cast<const uint32_t*>(&h);
           lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
         }
-        tmem_st16(tmem + lane_base + kColPH + q4 * 16, hi);
-        tmem_st16(tmem + lane_base + kColPL + q4 * 16, lo);
+        tmem_st16(tmem + lane_base + kColPH + col / 2, hi);
+        tmem_st16(tmem + lane_base + kColPL + col / 2, lo);
         if constexpr (DECAY) {
           if (!last) {
             uint32_t u[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * a_c);
-            tmem_st32(tmem + lane_base + kColP + q4 * 32, u);
+            tmem_st32(tmem + lane_base + kColP + col, u);
           }
         }
       }
@@ -546,13 +580,15 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       tc_fence_before();
       mbar_arrive(pready);
     }
-  } else if (warp < 12) {
+  } else if (warp < 16) {
     // ------------------------------------------------------------------ epilogue
-    const int tw = tid - 128;
-    const int quarter = warp & 3, half = (warp - 4) >> 2;
+    const int tw = tid - kXfThreads;
+    const int quarter = warp & 3, half = (warp - 8) >> 2;
+    const int j = quarter * 32 + lane;  // value feature of this thread's output column
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      const int t0 = (cb + i) * kC;
+      const long long t0 = static_cast<long long>(cb + i) * kC;
+      const int L = chunk_len(sp, cb + i);
       const bool has_prefix = !(seg == 0 && i == 0);
       wait(sdone, i & 1, kErrMmaTimeout);
       wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout);
@@ -566,33 +602,39 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         tc_fence_before();
         mbar_arrive(sfree);
         if (lane < 16) {
+          // gamma^(row - key), zero above the diagonal; all loads before the stores.
           float den_loc = 0.f;
+          uint4 hi[4], lo[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float a[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const int j = 32 * half + q * 8 + e;
-              a[e] = j <= row ? sc[q * 8 + e] * sPow[row - j] : 0.f;
+              const int d = row - 32 * half - q * 8 - e;
+              a[e] = d >= 0 ? sc[q * 8 + e] * sPow[d] : 0.f;
               den_loc += a[e];
             }
-            uint4 hi, lo;
-            split8(a, hi, lo);
-            *reinterpret_cast<uint4*>(sAh + sw128_offset(row, 4 * half + q)) = hi;
-            *reinterpret_cast<uint4*>(sAl + sw128_offset(row, 4 * half + q)) = lo;
+            split8(a, hi[q], lo[q]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<uint4*>(sAh + sw128_offset(row, 4 * half + q)) = hi[q];
+            *reinterpret_cast<uint4*>(sAl + sw128_offset(row, 4 * half + q)) = lo[q];
           }
           if constexpr (NORM) sDenPart[half * kC + row] = den_loc;
         }
       }
-      // psi(q).ZP of this chunk is read before A is handed over: once N(i) is done the
-      // stage (and its sDenX slot) is refilled with chunk i + 2.
-      const float denx = NORM && has_prefix && tw < kC ? sDenX[s * kC + tw] : 0.f;
       fence_async_smem();
-      mbar_arrive(aready);
       if constexpr (NORM) {
-        named_barrier(2, 256);
-        if (tw < kC) sDen[tw] = fmaf(sTh[tw], denx, sDenPart[tw] + sDenPart[kC + tw]) + sp.eps;
+        // psi(q).ZP of this chunk is read before A is handed over: once N(i) is done
+        // the stage (and its sDenX slot) is refilled with chunk i + 2.
+        named_barrier(2, kEpThreads);
+        if (tw < kC) {
+          const float den_loc = sDenPart[tw] + sDenPart[kC + tw];
+          sDen[tw] = (has_prefix ? fmaf(sTh[tw], sDenX[s * kC + tw], den_loc) : den_loc) + sp.eps;
+        }
       }
+      mbar_arrive(aready);
 
       wait(ndone, i & 1, kErrMmaTimeout);
       tc_fence_after();
@@ -603,55 +645,91 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&xfree[s]);
-      if (tw == 0) bulk_wait_read_all();  // the previous tile has left the staging buffer
-      named_barrier(2, 256);
-      const int j = quarter * 32 + lane;
+      if constexpr (NORM) named_barrier(2, kEpThreads);  // sDen of this chunk
+      // Theta (and den) of this warp's 32 tokens as float4 broadcasts, all before the
+      // first global store.
+      if (has_prefix) {
 #pragma unroll
-      for (int tt = 0; tt < kC / 2; ++tt) {
-        const int t = 32 * half + tt;
-        float o = has_prefix ? fmaf(sTh[t], xo[tt], no[tt]) : no[tt];
-        if constexpr (NORM) o = o / sDen[t];
-        if constexpr (OUTF32) {
-          *reinterpret_cast<float*>(sO + (j / 32) * (kC * 128) + sw128_offset(t, (j % 32) / 4) +
-                                    (j % 4) * 4) = o;
-        } else {
-          *reinterpret_cast<__nv_bfloat16*>(sO + (j / 64) * (kC * 128) +
-                                            sw128_offset(t, (j % 64) / 8) + (j % 8) * 2) =
-              __float2bfloat16_rn(o);
+        for (int q = 0; q < 8; ++q) {
+          const float4 th = *reinterpret_cast<const float4*>(sTh + 32 * half + 4 * q);
+          no[4 * q] = fmaf(th.x, xo[4 * q], no[4 * q]);
+          no[4 * q + 1] = fmaf(th.y, xo[4 * q + 1], no[4 * q + 1]);
+          no[4 * q + 2] = fmaf(th.z, xo[4 * q + 2], no[4 * q + 2]);
+          no[4 * q + 3] = fmaf(th.w, xo[4 * q + 3], no[4 * q + 3]);
         }
       }
-      fence_async_smem();
-      named_barrier(2, 256);
-      if (tw == 0) {
-        constexpr int kOutCols = OUTF32 ? 32 : 64;
+      if constexpr (NORM) {
 #pragma unroll
-        for (int b = 0; b < DV / kOutCols; ++b)
-          tma_store_3d(&tm_out, sO + b * (kC * 128), b * kOutCols, t0, bh);
-        bulk_commit();
+        for (int q = 0; q < 8; ++q) {
+          const float4 dn = *reinterpret_cast<const float4*>(sDen + 32 * half + 4 * q);
+          no[4 * q] /= dn.x;
+          no[4 * q + 1] /= dn.y;
+          no[4 * q + 2] /= dn.z;
+          no[4 * q + 3] /= dn.w;
+        }
+      }
+      const long long row0 = static_cast<long long>(bh) * sp.T + t0 + 32 * half;
+      const int nt = min(32, L - 32 * half);  // tokens of this half inside the sequence
+#pragma unroll
+      for (int tt = 0; tt < 32; ++tt) {
+        if (tt < nt) {
+          const long long idx = (row0 + tt) * DV + j;
+          if constexpr (OUTF32)
+            __stcs(static_cast<float*>(sp.out) + idx, no[tt]);
+          else
+            static_cast<__nv_bfloat16*>(sp.out)[idx] = __float2bfloat16_rn(no[tt]);
+        }
       }
     }
-    if (tw == 0) bulk_wait_read_all();
-  } else if (lane == 0) {
-    // ------------------------------------------------------------------ control
-    auto issue_load = [&](int i) {
-      uint8_t* sQ = base + (i & 1) * L_::kStage;
-      uint8_t* sK = sQ + L_::kQ;
-      uint8_t* sV = sK + L_::kK;
-      const int t0 = (cb + i) * kC;
-      mbar_arrive_expect_tx(&full[i & 1], L_::kStage);
+  } else if (warp == 16) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int loads = 0;
+      for (int i = 0; i < n; ++i) {
+        // Stage i & 1 is free once N(i - 2), the last MMA reading it, is done.
+        if (i >= 2 && !wait(&empty[i & 1], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
+        uint8_t* sQ = base + (i & 1) * L_::kStage;
+        uint8_t* sK = sQ + L_::kQ;
+        uint8_t* sV = sK + L_::kK;
+        const int t0 = (cb + i) * kC;
+        mbar_arrive_expect_tx(&full[i & 1], L_::kStage);
 #pragma unroll
-      for (int b = 0; b < DK / 64; ++b) {
-        tma_load_3d(sQ + b * kC * 128, &tm_q, &full[i & 1], b * 64, t0, bh);
-        tma_load_3d(sK + b * kC * 128, &tm_k, &full[i & 1], b * 64, t0, bh);
+        for (int b = 0; b < DK / 64; ++b) {
+          tma_load_3d(sQ + b * kC * 128, &tm_q, &full[i & 1], b * 64, t0, bh);
+          tma_load_3d(sK + b * kC * 128, &tm_k, &full[i & 1], b * 64, t0, bh);
+        }
+#pragma unroll
+        for (int b = 0; b < DV / 64; ++b)
+          tma_load_3d(sV + b * kC * 128, &tm_v, &full[i & 1], b * 64, t0, bh);
+        ++loads;
       }
-#pragma unroll
-      for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &full[i & 1], b * 64, t0, bh);
-    };
+      // The last two loads have landed before shared memory is given up (in a run
+      // without failures they were consumed already; the waits are bounded).
+      for (int jl = max(0, loads - 2); jl < loads; ++jl) mbar_wait(&full[jl & 1], (jl >> 1) & 1);
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer
+    // Descriptors of stage 0 (K-major: 128-byte rows, 1024-byte groups of eight; MN-major:
+    // 128-byte atoms, kC * 128 bytes apart); stage 1 is kStage bytes further on.
+    const uint32_t a0 = smem_u32(base);
+    const uint64_t dQk = smem_desc_sw128(a0, 16, 1024);                       // Q, K-major
+    const uint64_t dKk = smem_desc_sw128(a0 + L_::kQ, 16, 1024);              // K, K-major
+    const uint64_t dKm = smem_desc_sw128(a0 + L_::kQ, kC * 128, 1024);        // K, MN-major
+    const uint64_t dVm = smem_desc_sw128(a0 + L_::kQ + L_::kK, kC * 128, 1024);  // V, MN-major
+    const uint32_t lo0 = smem_u32(sLo), kp0 = smem_u32(sKpp);
+    const uint64_t dQlk = smem_desc_sw128(lo0, 16, 1024);
+    const uint64_t dKlk = smem_desc_sw128(lo0 + L_::kQ, 16, 1024);
+    const uint64_t dKlm = smem_desc_sw128(lo0 + L_::kQ, kC * 128, 1024);
+    const uint64_t dKhm = smem_desc_sw128(kp0, kC * 128, 1024);
+    const uint64_t dKpm = smem_desc_sw128(kp0 + L_::kK, kC * 128, 1024);
+    const uint64_t dAh = smem_desc_sw128(smem_u32(sAh), 16, 1024);
+    const uint64_t dAl = smem_desc_sw128(smem_u32(sAl), 16, 1024);
+    constexpr uint32_t kStageD = L_::kStage >> 4, kLoD = L_::kLo >> 4, kKppD = L_::kKpp >> 4;
+
     auto issue_scores = [&](int i) -> bool {
       const int s = i & 1;
-      uint8_t* sQ = base + s * L_::kStage;
-      const uint32_t aQ = smem_u32(sQ), aK = aQ + L_::kQ;
-      const uint32_t aQl = smem_u32(sLo + s * L_::kLo), aKl = aQl + L_::kQ;
+      const uint64_t q = dQk + s * kStageD, k = dKk + s * kStageD;
+      const uint64_t ql = dQlk + s * kLoD, kl = dKlk + s * kLoD;
       if (!wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout)) return false;
       if (i > 0 && !wait(sfree, (i - 1) & 1, kErrMmaTimeout)) return false;
       tc_fence_after();
@@ -659,29 +737,22 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk) {
         const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
-        const uint64_t qh = smem_desc_sw128(aQ + off, 16, 1024);
-        const uint64_t kh = smem_desc_sw128(aK + off, 16, 1024);
-        mma_bf16_ss(tmem + kColS, qh, kh, ids, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(k, off), ids, kk > 0 ? 1u : 0u);
         if constexpr (kSplitQK) {
-          mma_bf16_ss(tmem + kColS, qh, smem_desc_sw128(aKl + off, 16, 1024), ids, 1u);
-          mma_bf16_ss(tmem + kColS, smem_desc_sw128(aQl + off, 16, 1024), kh, ids, 1u);
+          mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(kl, off), ids, 1u);
+          mma_bf16_ss(tmem + kColS, desc_at(ql, off), desc_at(k, off), ids, 1u);
         }
       }
       mma_commit(sdone);
       return true;
     };
-    int loads = 0;
-    issue_load(loads++);
-    if (n > 1) issue_load(loads++);
     issue_scores(0);
     for (int i = 0; i < n && !failed; ++i) {
       const int s = i & 1;
       const bool last = i == n - 1;
       const bool has_prefix = !(seg == 0 && i == 0);
-      uint8_t* sQ = base + s * L_::kStage;
-      const uint32_t aQ = smem_u32(sQ), aK = aQ + L_::kQ, aV = aK + L_::kK;
-      const uint32_t aQl = smem_u32(sLo + s * L_::kLo), aKl = aQl + L_::kQ;
-      const uint32_t aKph = smem_u32(sKpp + s * L_::kKpp), aKpl = aKph + L_::kK;
+      const uint64_t q = dQk + s * kStageD, ql = dQlk + s * kLoD;
+      const uint64_t v = dVm + s * kStageD;
 
       // X(i) = P^T psi(Q)^T and the prefix update with chunk i.
       if (!wait(pready, i & 1, kErrMmaTimeout)) break;
@@ -692,24 +763,22 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
-          const uint64_t qh = smem_desc_sw128(aQ + off, 16, 1024);
-          mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, qh, idx, kk > 0 ? 1u : 0u);
-          mma_bf16_ts(tmem + kColX[s], tmem + kColPL + kk * 8, qh, idx, 1u);
+          mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, desc_at(q, off), idx,
+                      kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + kColX[s], tmem + kColPL + kk * 8, desc_at(q, off), idx, 1u);
           if constexpr (kSplitQK)
-            mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8,
-                        smem_desc_sw128(aQl + off, 16, 1024), idx, 1u);
+            mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, desc_at(ql, off), idx, 1u);
         }
       }
       if (!last) {
         constexpr uint32_t idp = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kMNMajor, 128, DK);
-        const uint32_t bh_ = DECAY ? aKph : aK;
-        const uint32_t bl_ = DECAY ? aKpl : aKl;
+        const uint64_t bh_ = DECAY ? dKhm + s * kKppD : dKm + s * kStageD;
+        const uint64_t bl_ = DECAY ? dKpm + s * kKppD : dKlm + s * kLoD;
 #pragma unroll
         for (int kk = 0; kk < kC / 16; ++kk) {
-          const uint64_t da = smem_desc_sw128(aV + kk * 2048, kC * 128, 1024);
-          mma_bf16_ss(tmem + kColP, da, smem_desc_sw128(bh_ + kk * 2048, kC * 128, 1024), idp, 1u);
+          mma_bf16_ss(tmem + kColP, desc_at(v, kk * 2048), desc_at(bh_, kk * 2048), idp, 1u);
           if constexpr (kSplitQK || DECAY)
-            mma_bf16_ss(tmem + kColP, da, smem_desc_sw128(bl_ + kk * 2048, kC * 128, 1024), idp, 1u);
+            mma_bf16_ss(tmem + kColP, desc_at(v, kk * 2048), desc_at(bl_, kk * 2048), idp, 1u);
         }
       }
       mma_commit(statedone);
@@ -718,30 +787,22 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       if (!wait(aready, i & 1, kErrMmaTimeout)) break;
       tc_fence_after();
       constexpr uint32_t idn = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kKMajor, 128, 64);
-      const uint32_t aAh = smem_u32(sAh), aAl = smem_u32(sAl);
 #pragma unroll
       for (int kk = 0; kk < kC / 16; ++kk) {
-        const uint64_t da = smem_desc_sw128(aV + kk * 2048, kC * 128, 1024);
-        mma_bf16_ss(tmem + kColN, da, smem_desc_sw128(aAh + kk * 32, 16, 1024), idn,
+        mma_bf16_ss(tmem + kColN, desc_at(v, kk * 2048), desc_at(dAh, kk * 32), idn,
                     kk > 0 ? 1u : 0u);
-        mma_bf16_ss(tmem + kColN, da, smem_desc_sw128(aAl + kk * 32, 16, 1024), idn, 1u);
+        mma_bf16_ss(tmem + kColN, desc_at(v, kk * 2048), desc_at(dAl, kk * 32), idn, 1u);
       }
       mma_commit(ndone);
+      mma_commit(&empty[s]);
 
-      // The next chunk's scores go in behind N(i); the stage of chunk i is refilled with
-      // chunk i + 2 once all of chunk i's MMAs are done.
+      // The next chunk's scores go in right behind N(i).
       if (i + 1 < n && !issue_scores(i + 1)) break;
-      if (i + 2 < n) {
-        if (!wait(ndone, i & 1, kErrMmaTimeout)) break;
-        issue_load(loads++);
-      }
     }
     if (failed) {
-      // Let the issued MMAs finish and the last two loads land before TMEM and shared
-      // memory are given up; both waits are bounded.
+      // Let the issued MMAs finish before TMEM is given up (bounded).
       mma_commit(drain);
       mbar_wait(drain, 0);
-      for (int j = max(0, loads - 2); j < loads; ++j) mbar_wait(&full[j & 1], (j >> 1) & 1);
     }
   }
   tc_fence_before();
@@ -777,7 +838,7 @@ cudaError_t k3s_go_o(const SegParams& sp, const GammaTable& gt, const TcMaps& m,
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(sp.BH) * sp.NS;
-  kern<<<static_cast<unsigned>(grid), kThreads3, sm, s>>>(m.q, m.k, m.v, m.out, sp, gt);
+  kern<<<static_cast<unsigned>(grid), kThreads3, sm, s>>>(m.q, m.k, m.v, sp, gt);
   return cudaGetLastError();
 }
 
