@@ -76,46 +76,57 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Uniform bounded wait: every thread waits; if any gave up the whole CTA reports and
-// leaves (after freeing its TMEM).
-#define LA_WAIT_OR_LEAVE(bar, parity, code, tmem, ncols)          \
-  do {                                                            \
-    const bool ok_ = mbar_wait((bar), (parity));                  \
-    if (__syncthreads_or(!ok_)) {                                 \
-      if (threadIdx.x == 0) report_error(sp.err, (code));         \
-      if ((threadIdx.x >> 5) == 0) tmem_dealloc((tmem), (ncols)); \
-      return;                                                     \
-    }                                                             \
-  } while (0)
+// A shared-memory descriptor advanced by a byte offset: the start address field holds
+// address >> 4 in its low 14 bits and every operand of these kernels lies below 256 KB, so
+// the addition never carries out of the field.
+__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 
 // ---------------------------------------------------------------------------------------
-// K1s
+// K1s, warp-specialised: one CTA per (b*H + h, segment).
+//   warps 0-7  transform: psi, the segment-relative weights gamma^(len_s - 1 - tau), the
+//              hi / lo split of the weighted keys (hi in place, lo beside the stage) and the
+//              Z column sums, chunk by chunk with no CTA-wide barrier; at the end, the
+//              epilogue (TMEM -> swizzled staging -> one TMA store of the record).
+//   warp 8     producer (one thread): TMA loads of K, V into a four-stage ring, a stage
+//              refilled as soon as the MMAs reading it are done.
+//   warp 9     MMA issuer (one thread): V^T K' into one TMEM accumulator for the segment.
+// One CTA per SM (about 200 KB of shared memory at d = 128): four chunks of loads in
+// flight per SM cover the memory latency, and 1024 CTAs make nearly seven even waves.
+
+constexpr int kThreads1 = 320;
+constexpr int kStages1 = 4;
 
 template <int DK, int DV>
 struct K1sSmem {
   static constexpr uint32_t kK = DK * kC * 2;
   static constexpr uint32_t kV = DV * kC * 2;
-  static constexpr uint32_t kStage = kK + kV;
-  static constexpr uint32_t kIn = 2 * kStage + kK;  // two stages + the lo tile of K'
+  static constexpr uint32_t kStage = kK + kV + kK;  // K (hi in place), V, lo tile of K'
+  static constexpr uint32_t kIn = kStages1 * kStage;
   static constexpr uint32_t kS = DK * DV * 4;       // staging of T_s^T, aliases the inputs
   static constexpr uint32_t kRegion = kIn > kS ? kIn : kS;
-  static constexpr uint32_t kTotal = kRegion + kWarps * DK * 4 + 64 + 1024;
+  static constexpr uint32_t kBars = 3 * kStages1 + 1;
+  static constexpr uint32_t kTotal = kRegion + kWarps * DK * 4 + (kBars + 1) * 8 + 1024;
 };
 
 template <int DK, int DV, int FM, bool DECAY, bool NORM>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads1, 1)
 k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
        const __grid_constant__ CUtensorMap tm_srec, SegParams sp, GammaTable gt) {
   using L_ = K1sSmem<DK, DV>;
   constexpr bool kSplit = FM == 1 || DECAY;
   constexpr uint32_t kTmemCols = DK;
+  static_assert(L_::kTotal <= 232448, "shared memory budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
-  uint8_t* sKl = base + 2 * L_::kStage;
   uint8_t* sS = base;
-  float* sZ = reinterpret_cast<float*>(base + L_::kRegion);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + kWarps * DK);  // tma[2], mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  float* sZ = reinterpret_cast<float*>(base + L_::kRegion);           // [8][DK]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sZ + kWarps * DK);
+  uint64_t* full = bars;                  // [kStages1]
+  uint64_t* ops = bars + kStages1;        // [kStages1], 256 arrivals
+  uint64_t* empty = bars + 2 * kStages1;  // [kStages1], MMA commits
+  uint64_t* done = bars + 3 * kStages1;   // the segment's last MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L_::kBars);
 
   if (error_pending(sp.err)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -130,9 +141,12 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
   const float g = DECAY ? gt.g[bh % sp.H] : 1.f;
 
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
+    for (int b = 0; b < kStages1; ++b) {
+      mbar_init(&full[b], 1);
+      mbar_init(&ops[b], kThreads);
+      mbar_init(&empty[b], 1);
+    }
+    mbar_init(done, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -146,122 +160,175 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  auto issue_load = [&](int i) {
-    uint8_t* sK = base + (i & 1) * L_::kStage;
-    uint8_t* sV = sK + L_::kK;
-    const int t0 = (cb + i) * kC;
-    mbar_arrive_expect_tx(&bars[i & 1], L_::kK + L_::kV);
-#pragma unroll
-    for (int b = 0; b < DK / 64; ++b) tma_load_3d(sK + b * kC * 128, &tm_k, &bars[i & 1], b * 64, t0, bh);
-#pragma unroll
-    for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &bars[i & 1], b * 64, t0, bh);
+  bool failed = false;
+  // A wait that runs out marks its thread failed; a failed thread waits no more, so every
+  // role reaches the end (the transform warps walk on over meaningless data, in bounds).
+  auto wait = [&](uint64_t* bar, uint32_t parity, int code) -> bool {
+    if (failed) return false;
+    if (mbar_wait(bar, parity)) return true;
+    report_error(sp.err, code);
+    failed = true;
+    return false;
   };
-  if (tid == 0) issue_load(0);
 
   constexpr int NCC = DK / 8;
   constexpr int RG = kThreads / NCC;
-  const int cc = tid % NCC, rg = tid / NCC;
-  float zacc[8];
+  constexpr int kRows = kC / RG;
+  if (warp < kWarps) {
+    // ------------------------------------------------------------------ transform
+    const int cc = tid % NCC, rg = tid / NCC;
+    float zacc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
-
-  for (int i = 0; i < n; ++i) {
-    const int c = cb + i;
-    const int L = chunk_len(sp, c);
-    uint8_t* sK = base + (i & 1) * L_::kStage;
-    uint8_t* sV = sK + L_::kK;
-    if (i >= 1) LA_WAIT_OR_LEAVE(&bars[2], (i - 1) & 1, kErrMmaTimeout, tmem, kTmemCols);
-    if (tid == 0 && i + 1 < n) issue_load(i + 1);
-    LA_WAIT_OR_LEAVE(&bars[i & 1], (i >> 1) & 1, kErrTmaTimeout, tmem, kTmemCols);
-
-    if constexpr (kSplit || NORM) {
-      const uint32_t boff = (cc / 8) * (kC * 128);
-      for (int r = rg; r < kC; r += RG) {
-        const uint32_t off = boff + sw128_offset(r, cc % 8);
-        const int tau = i * kC + r;  // token within the segment
-        const float w = r < L ? (DECAY ? powf(g, static_cast<float>(seg_tokens - 1 - tau)) : 1.f) : 0.f;
-        float x[8];
-        unpack8(*reinterpret_cast<const uint4*>(sK + off), x);
+    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+    // The weight of row r of chunk i is gamma^(len_s - 1 - 64 i - r).  For gamma >= 1/2 it
+    // is formed as gamma^(len_s - 1 - 64 i) * gamma^(-r) (gamma^(-r) <= 2^63, one powf per
+    // chunk); smaller gamma takes one powf per row, since gamma^(-r) would overflow.
+    const bool factored = DECAY && g >= 0.5f;
+    float ginv[kRows];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] = feature<FM>(x[e]) * w;
-          zacc[e] += x[e];
+    for (int k = 0; k < kRows; ++k)
+      ginv[k] = factored ? powf(g, -static_cast<float>(rg + k * RG)) : 1.f;
+    for (int i = 0; i < n; ++i) {
+      const int st = i % kStages1;
+      const int L = chunk_len(sp, cb + i);
+      uint8_t* sK = base + st * L_::kStage;
+      uint8_t* sKl = sK + L_::kK + L_::kV;
+      wait(&full[st], (i / kStages1) & 1, kErrTmaTimeout);
+      if constexpr (kSplit || NORM) {
+        const float wb = factored ? powf(g, static_cast<float>(seg_tokens - 1 - i * kC)) : 1.f;
+        const uint32_t boff = (cc / 8) * (kC * 128);
+        uint4 raw[kRows];
+#pragma unroll
+        for (int k = 0; k < kRows; ++k)
+          raw[k] = *reinterpret_cast<const uint4*>(sK + boff + sw128_offset(rg + k * RG, cc % 8));
+#pragma unroll
+        for (int k = 0; k < kRows; ++k) {
+          const int r = rg + k * RG;
+          float w = 0.f;
+          if (r < L) {
+            if (!DECAY) w = 1.f;
+            else if (factored) w = wb * ginv[k];
+            else w = powf(g, static_cast<float>(seg_tokens - 1 - i * kC - r));
+          }
+          float x[8];
+          unpack8(raw[k], x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            x[e] = feature<FM>(x[e]) * w;
+            zacc[e] += x[e];
+          }
+          if constexpr (kSplit) {
+            uint4 hi, lo;
+            split8(x, hi, lo);
+            const uint32_t off = boff + sw128_offset(r, cc % 8);
+            *reinterpret_cast<uint4*>(sK + off) = hi;
+            *reinterpret_cast<uint4*>(sKl + off) = lo;
+          }
         }
-        if constexpr (kSplit) {
-          uint4 hi, lo;
-          split8(x, hi, lo);
-          *reinterpret_cast<uint4*>(sK + off) = hi;
-          *reinterpret_cast<uint4*>(sKl + off) = lo;
-        }
+        fence_async_smem();
+      }
+      mbar_arrive(&ops[st]);
+    }
+
+    // Z of the segment: column sums over this CTA's threads.
+    float* srec = sp.srec + (static_cast<long long>(bh) * sp.NS + seg) * sp.R;
+    if constexpr (NORM) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+#pragma unroll
+        for (int o = NCC; o < 32; o <<= 1) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], o);
+      if (lane < NCC)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sZ[warp * DK + cc * 8 + e] = zacc[e];
+      named_barrier(1, kThreads);
+      if (tid < DK) {
+        float z = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) z += sZ[w * DK + tid];
+        srec[DK * DV + tid] = z;
+      }
+    }
+
+    // Epilogue: warps w and w + 4 read the same TMEM lanes, each half of the columns.  The
+    // staging aliases the load stages: every load has been consumed and every MMA is done.
+    wait(done, 0, kErrMmaTimeout);
+    tc_fence_after();
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = DV == 128 ? quarter * 32 + lane : quarter * 16 + lane;
+    const bool valid = DV == 128 || lane < 16;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+#pragma unroll
+    for (int q4 = half * (DK / 64); q4 < (half + 1) * (DK / 64); ++q4) {
+      float r[32];
+      tmem_ld32(tmem + lane_base + q4 * 32, r);
+      tmem_ld_wait();
+      if (valid) {
+        uint8_t* box = sS + q4 * (DV * 128);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4*>(box + sw128_offset(row, q)) =
+              make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
       }
     }
     fence_async_smem();
-    __syncthreads();
+    tc_fence_before();
+    named_barrier(1, kThreads);
     if (tid == 0) {
+#pragma unroll
+      for (int q4 = 0; q4 < DK / 32; ++q4)
+        tma_store_3d(&tm_srec, sS + q4 * (DV * 128), q4 * 32, 0, bh * sp.NS + seg);
+      bulk_commit();
+      bulk_wait_read_all();
+    }
+  } else if (warp == kWarps) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int loads = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % kStages1;
+        if (i >= kStages1 && !wait(&empty[st], ((i / kStages1) - 1) & 1, kErrMmaTimeout)) break;
+        uint8_t* sK = base + st * L_::kStage;
+        uint8_t* sV = sK + L_::kK;
+        const int t0 = (cb + i) * kC;
+        mbar_arrive_expect_tx(&full[st], L_::kK + L_::kV);
+#pragma unroll
+        for (int b = 0; b < DK / 64; ++b) tma_load_3d(sK + b * kC * 128, &tm_k, &full[st], b * 64, t0, bh);
+#pragma unroll
+        for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &full[st], b * 64, t0, bh);
+        ++loads;
+      }
+      // Every issued load has landed before the stages are reused as staging (bounded).
+      for (int j = max(0, loads - kStages1); j < loads; ++j)
+        mbar_wait(&full[j % kStages1], (j / kStages1) & 1);
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------------------------ MMA issuer
+    const uint32_t a0 = smem_u32(base);
+    const uint64_t dK = smem_desc_sw128(a0, kC * 128, 1024);                  // MN-major
+    const uint64_t dV = smem_desc_sw128(a0 + L_::kK, kC * 128, 1024);
+    const uint64_t dKl = smem_desc_sw128(a0 + L_::kK + L_::kV, kC * 128, 1024);
+    constexpr uint32_t kStageD = L_::kStage >> 4;
+    constexpr uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kMNMajor, DV, DK);
+    for (int i = 0; i < n && !failed; ++i) {
+      const int st = i % kStages1;
+      if (!wait(&ops[st], (i / kStages1) & 1, kErrMmaTimeout)) break;
       tc_fence_after();
-      constexpr uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kMNMajor, DV, DK);
-      const uint32_t aK = smem_u32(sK), aKl = smem_u32(sKl), aV = smem_u32(sV);
+      const uint64_t k = dK + st * kStageD, v = dV + st * kStageD, kl = dKl + st * kStageD;
 #pragma unroll
       for (int kk = 0; kk < kC / 16; ++kk) {
-        const uint64_t da = smem_desc_sw128(aV + kk * 2048, kC * 128, 1024);
-        mma_bf16_ss(tmem, da, smem_desc_sw128(aK + kk * 2048, kC * 128, 1024), idesc,
+        mma_bf16_ss(tmem, desc_at(v, kk * 2048), desc_at(k, kk * 2048), idesc,
                     (i > 0 || kk > 0) ? 1u : 0u);
         if constexpr (kSplit)
-          mma_bf16_ss(tmem, da, smem_desc_sw128(aKl + kk * 2048, kC * 128, 1024), idesc, 1u);
+          mma_bf16_ss(tmem, desc_at(v, kk * 2048), desc_at(kl, kk * 2048), idesc, 1u);
       }
-      mma_commit(&bars[2]);
+      mma_commit(&empty[st]);
     }
+    // The transform warps read the accumulator once this lands (also after a failure,
+    // so that no MMA is in flight when TMEM is given up).
+    mma_commit(done);
+    if (failed) mbar_wait(done, 0);
   }
-  LA_WAIT_OR_LEAVE(&bars[2], (n - 1) & 1, kErrMmaTimeout, tmem, kTmemCols);
-  tc_fence_after();
-
-  float* srec = sp.srec + (static_cast<long long>(bh) * sp.NS + seg) * sp.R;
-  if constexpr (NORM) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-#pragma unroll
-      for (int o = NCC; o < 32; o <<= 1) zacc[e] += __shfl_xor_sync(0xffffffffu, zacc[e], o);
-    if (lane < NCC)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sZ[warp * DK + cc * 8 + e] = zacc[e];
-    __syncthreads();
-    if (tid < DK) {
-      float z = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) z += sZ[w * DK + tid];
-      srec[DK * DV + tid] = z;
-    }
-  }
-
-  // Epilogue: warps w and w + 4 read the same TMEM lanes, each half of the columns.
-  const int quarter = warp & 3, half = warp >> 2;
-  const int row = DV == 128 ? quarter * 32 + lane : quarter * 16 + lane;
-  const bool valid = DV == 128 || lane < 16;
-  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-#pragma unroll
-  for (int q4 = half * (DK / 64); q4 < (half + 1) * (DK / 64); ++q4) {
-    float r[32];
-    tmem_ld32(tmem + lane_base + q4 * 32, r);
-    tmem_ld_wait();
-    if (valid) {
-      uint8_t* box = sS + q4 * (DV * 128);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(box + sw128_offset(row, q)) =
-            make_float4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-    }
-  }
-  fence_async_smem();
   tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {
-#pragma unroll
-    for (int q4 = 0; q4 < DK / 32; ++q4)
-      tma_store_3d(&tm_srec, sS + q4 * (DV * 128), q4 * 32, 0, bh * sp.NS + seg);
-    bulk_commit();
-    bulk_wait_read_all();
-  }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
@@ -308,10 +375,6 @@ struct K3sSmem {
       2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
 };
 
-// A shared-memory descriptor advanced by a byte offset: the start address field holds
-// address >> 4 in its low 14 bits and every operand of this kernel lies below 256 KB, so
-// the addition never carries out of the field.
-__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
 __global__ void __launch_bounds__(kThreads3, 1)
@@ -827,7 +890,7 @@ cudaError_t k1s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(sp.BH) * sp.NS;
-  kern<<<static_cast<unsigned>(grid), kThreads, sm, s>>>(m.k, m.v, m.rec, sp, gt);
+  kern<<<static_cast<unsigned>(grid), kThreads1, sm, s>>>(m.k, m.v, m.rec, sp, gt);
   return cudaGetLastError();
 }
 
