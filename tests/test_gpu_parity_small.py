@@ -149,3 +149,27 @@ def test_pr1_ref_fp32_second_seed(seed):
     w = WORKLOADS["pr1_ref"]
     q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
     _check(w, q, k, v, None, TOL_F32)
+
+
+@pytest.mark.parametrize("algorithm", ["chunked", "segmented"])
+@pytest.mark.parametrize("T", [200, 1000])
+def test_extreme_decays(algorithm, T):
+    # gamma = 0 (each state holds only the current token), decays fast enough that the
+    # segment weights gamma^(len - 1 - tau) underflow to zero, gamma = 1/2 (where the
+    # segment-summary kernel switches how it forms its weights), and gamma = 1.  Checked
+    # per head, so that the gamma = 1 heads' larger outputs do not set the other heads'
+    # bound.
+    gam = [float(np.float32(x)) for x in (0.0, 0.05, 0.3, 0.5, 0.7, 1.0)]
+    w = Workload("extreme_decay", B=1, H=len(gam), T=T, dk=128, dv=128, C=64, dtype="bf16",
+                 scale=1.0 / math.sqrt(128), feature_map="identity", decay=True,
+                 normalize=False)
+    q, k, v = make_inputs(w, seed=7, device="cuda", gen_device="cpu")
+    out, S, _ = gpu_prefill(q, k, v, C=64, feature_map="identity", gamma=gam, normalize=False,
+                            kernel_path="tensor_core", algorithm=algorithm,
+                            segment_chunks=2 if algorithm == "segmented" else 0)
+    o_ref, S_ref, _ = oracle_prefill(q, k, v, feature_map="identity", gamma=gam,
+                                     normalize=False)
+    o, s = to_np(out), to_np(S)
+    for h, g in enumerate(gam):
+        assert_close(o[:, h], o_ref[:, h], TOL_BF16, f"out, gamma={g}")
+        assert_close(s[:, h], S_ref[:, h], TOL_BF16, f"S_final, gamma={g}")
