@@ -477,6 +477,21 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     return false;
   };
 
+  // Decayed prefix kept as P = c P~ (TMEM holds P~): within a window of W chunks the
+  // state update adds V^T (Xi .* psi(K)) / c, the epilogue scales X by c, and only the
+  // window's first chunk rescales P~ in TMEM, instead of every chunk writing gamma^L P
+  // back.  c = gamma^(64 m) m chunks into the window; W keeps 1 / c <= 2^60.  Heads with
+  // gamma < ~0.52 (and gamma = 0) keep W = 1: P itself, decayed every chunk.
+  int W = 1;
+  if constexpr (DECAY) {
+    if (g > 0.f) {
+      const float lg = -log2f(g);
+      W = lg > 0.f ? static_cast<int>(fminf(16.f, 60.f / (64.f * lg))) : 16;
+    }
+    if (W < 2) W = 1;
+  }
+  const bool renorm = W >= 2;
+
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
     const int tw = tid;
@@ -515,7 +530,10 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       uint8_t* sKph = sKpp + s * L_::kKpp;
       uint8_t* sKpl = sKph + L_::kK;
       float* xi = sXi + s * kC;
-      if (tw < kC) xi[tw] = tw < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tw)) : 1.f) : 0.f;
+      if (tw < kC)
+        xi[tw] = tw < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tw - (renorm ? kC * (i % W + 1) : 0)))
+                                 : 1.f)
+                        : 0.f;
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
       named_barrier(1, kXfThreads);
 
@@ -614,12 +632,24 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       // the key features.
       if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
       tc_fence_after();
+      // A window's first chunk turns P~ back into P (c = gamma^(64 W) since the last one).
+      const bool rescale = renorm && i > 0 && i % W == 0;
+      const float c_w = rescale ? powf(g, static_cast<float>(kC * W)) : 1.f;
 #pragma unroll
       for (int q4 = 0; q4 < kHalf / 32; ++q4) {
         const uint32_t col = pcol + q4 * 32;
         float rr[32];
         tmem_ld32(tmem + lane_base + kColP + col, rr);
         tmem_ld_wait();
+        if (rescale) {
+          uint32_t u[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            rr[e] *= c_w;
+            u[e] = __float_as_uint(rr[e]);
+          }
+          tmem_st32(tmem + lane_base + kColP + col, u);
+        }
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -631,7 +661,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         tmem_st16(tmem + lane_base + kColPH + col / 2, hi);
         tmem_st16(tmem + lane_base + kColPL + col / 2, lo);
         if constexpr (DECAY) {
-          if (!last) {
+          if (!renorm && !last) {
             uint32_t u[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * a_c);
@@ -657,34 +687,38 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout);
       tc_fence_after();
       {
-        // Rows 16 quarter .. + 15 (lanes 0-15), keys 32 half .. + 31.
-        const int row = quarter * 16 + lane;
-        float sc[32];
-        tmem_ld32(tmem + lane_base + kColS + 32 * half, sc);
+        // Row 16 quarter + (lane % 16), keys kb .. kb + 15 with kb = 32 half + 16 (lane / 16):
+        // the 64-row score tile sits in lanes 0-15 of each quarter, and the 16-lane load
+        // gives both halves of the warp a share of its columns.
+        const int row = quarter * 16 + (lane & 15);
+        const int kb = 32 * half + 16 * (lane >> 4);
+        float sc[16];
+        tmem_ld16x2_x16(tmem + lane_base + kColS + 32 * half, sc);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(sfree);
-        if (lane < 16) {
-          // gamma^(row - key), zero above the diagonal; all loads before the stores.
-          float den_loc = 0.f;
-          uint4 hi[4], lo[4];
+        // gamma^(row - key), zero above the diagonal; all loads before the stores.
+        float den_loc = 0.f;
+        uint4 hi[2], lo[2];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float a[8];
+        for (int q = 0; q < 2; ++q) {
+          float a[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int d = row - 32 * half - q * 8 - e;
-              a[e] = d >= 0 ? sc[q * 8 + e] * sPow[d] : 0.f;
-              den_loc += a[e];
-            }
-            split8(a, hi[q], lo[q]);
+          for (int e = 0; e < 8; ++e) {
+            const int d = row - kb - q * 8 - e;
+            a[e] = d >= 0 ? sc[q * 8 + e] * sPow[d] : 0.f;
+            den_loc += a[e];
           }
+          split8(a, hi[q], lo[q]);
+        }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            *reinterpret_cast<uint4*>(sAh + sw128_offset(row, 4 * half + q)) = hi[q];
-            *reinterpret_cast<uint4*>(sAl + sw128_offset(row, 4 * half + q)) = lo[q];
-          }
-          if constexpr (NORM) sDenPart[half * kC + row] = den_loc;
+        for (int q = 0; q < 2; ++q) {
+          *reinterpret_cast<uint4*>(sAh + sw128_offset(row, kb / 8 + q)) = hi[q];
+          *reinterpret_cast<uint4*>(sAl + sw128_offset(row, kb / 8 + q)) = lo[q];
+        }
+        if constexpr (NORM) {
+          den_loc += __shfl_xor_sync(0xffffffffu, den_loc, 16);
+          if (lane < 16) sDenPart[half * kC + row] = den_loc;
         }
       }
       fence_async_smem();
@@ -712,13 +746,15 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       // Theta (and den) of this warp's 32 tokens as float4 broadcasts, all before the
       // first global store.
       if (has_prefix) {
+        // X was computed from P~: the chunk's Theta carries the window factor c.
+        const float c = renorm ? powf(g, static_cast<float>(kC * (i % W))) : 1.f;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 th = *reinterpret_cast<const float4*>(sTh + 32 * half + 4 * q);
-          no[4 * q] = fmaf(th.x, xo[4 * q], no[4 * q]);
-          no[4 * q + 1] = fmaf(th.y, xo[4 * q + 1], no[4 * q + 1]);
-          no[4 * q + 2] = fmaf(th.z, xo[4 * q + 2], no[4 * q + 2]);
-          no[4 * q + 3] = fmaf(th.w, xo[4 * q + 3], no[4 * q + 3]);
+          no[4 * q] = fmaf(th.x * c, xo[4 * q], no[4 * q]);
+          no[4 * q + 1] = fmaf(th.y * c, xo[4 * q + 1], no[4 * q + 1]);
+          no[4 * q + 2] = fmaf(th.z * c, xo[4 * q + 2], no[4 * q + 2]);
+          no[4 * q + 3] = fmaf(th.w * c, xo[4 * q + 3], no[4 * q + 3]);
         }
       }
       if constexpr (NORM) {
