@@ -173,3 +173,23 @@ def test_extreme_decays(algorithm, T):
     for h, g in enumerate(gam):
         assert_close(o[:, h], o_ref[:, h], TOL_BF16, f"out, gamma={g}")
         assert_close(s[:, h], S_ref[:, h], TOL_BF16, f"S_final, gamma={g}")
+
+
+def test_segmented_decay_windows():
+    # Segments of 40 chunks with decays whose renormalisation windows are 6 (gamma 0.9)
+    # to 16 chunks (gamma >= 0.97) long, so that every head rescales its carried prefix
+    # at least twice inside a segment; 0.6 keeps the per-chunk decay.  Ragged tail.
+    gam = [float(np.float32(x)) for x in (0.6, 0.9, 0.95, 0.97, 0.99, 1.0)]
+    T = 2 * 40 * 64 + 100
+    w = Workload("decay_windows", B=1, H=len(gam), T=T, dk=128, dv=128, C=64, dtype="bf16",
+                 scale=1.0 / math.sqrt(128), feature_map="identity", decay=True,
+                 normalize=False)
+    q, k, v = make_inputs(w, seed=3, device="cuda", gen_device="cpu")
+    out, S, _ = gpu_prefill(q, k, v, C=64, feature_map="identity", gamma=gam, normalize=False,
+                            kernel_path="tensor_core", algorithm="segmented", segment_chunks=40)
+    o_ref, S_ref, _ = oracle_prefill(q, k, v, feature_map="identity", gamma=gam,
+                                     normalize=False)
+    o, s = to_np(out), to_np(S)
+    for h, g in enumerate(gam):
+        assert_close(o[:, h], o_ref[:, h], TOL_BF16, f"out, gamma={g}")
+        assert_close(s[:, h], S_ref[:, h], TOL_BF16, f"S_final, gamma={g}")
