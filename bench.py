@@ -517,7 +517,7 @@ def main():
         d2h = oh.numel() * oh.element_size() + Sh.numel() * 4 + (Zh.numel() * 4 if Zh is not None else 0)
         e2e = {"value": info.world * w.tokens_heads / (e_ms / 1000.0), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "lin_attn_prefill_host (pinned host buffers, synchronous)"}
+               "api": "lin_attn_prefill_host (pinned host buffers; copies in, kernels and copies out overlapped across groups of heads; synchronous)"}
         del qh, kh, vh, oh, Sh, Zh, dbuf
 
     cpu = None

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -513,27 +514,106 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
   const size_t e = h.dtype == LA_DTYPE_F32 ? 4 : 2;
   const size_t eo = (h.dtype == LA_DTYPE_F32 || h.out_dtype == LA_OUT_F32) ? 4 : 2;
   const size_t T = static_cast<size_t>(h.T);
-  const size_t nq = BH * T * h.dk * e, nv = BH * T * h.dv * e, no = BH * T * h.dv * eo;
+  // Per (b, h) pair: bytes of q (= k), v, out, S and Z.  Pairs are contiguous in every
+  // tensor, so a group of heads of one batch row is one byte range of each.
+  const size_t pq = T * h.dk * e, pv = T * h.dv * e, po = T * h.dv * eo;
+  const size_t pS = static_cast<size_t>(h.dk) * h.dv * 4, pZ = static_cast<size_t>(h.dk) * 4;
+  // Groups of at least 32 MB of input (at most 16 groups): group g + 1 is copied in while
+  // group g runs and group g - 1 is copied out, so the two copy directions overlap.
+  const size_t in_bytes = BH * (2 * pq + pv);
+  const int groups_target = static_cast<int>(std::min<size_t>(16, in_bytes >> 25));
+  const int hpg = groups_target > 1 && BH > 1
+                      ? std::max(1, static_cast<int>((BH + groups_target - 1) / groups_target))
+                      : h.H;
+  const int heads_per_group = std::min(hpg, h.H);
   cudaError_t err = cudaSuccess;
-  if (nq) err = cudaMemcpyAsync(buf + hl.q, h.q, nq, cudaMemcpyHostToDevice, s);
-  if (err == cudaSuccess && nq) err = cudaMemcpyAsync(buf + hl.k, h.k, nq, cudaMemcpyHostToDevice, s);
-  if (err == cudaSuccess && nv) err = cudaMemcpyAsync(buf + hl.v, h.v, nv, cudaMemcpyHostToDevice, s);
-  la_prefill_args d = h;
-  d.q = buf + hl.q;
-  d.k = buf + hl.k;
-  d.v = buf + hl.v;
-  d.out = buf + hl.out;
-  d.S_final = h.S_final ? reinterpret_cast<float*>(buf + hl.S) : nullptr;
-  d.Z_final = h.Z_final ? reinterpret_cast<float*>(buf + hl.Z) : nullptr;
-  d.workspace = buf + hl.ws;
-  d.workspace_bytes = hl.total - hl.ws;
-  if (err == cudaSuccess) st = la::prefill(d);
-  if (err == cudaSuccess && st == LA_OK) {
-    if (no) err = cudaMemcpyAsync(h.out, d.out, no, cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess && h.S_final)
-      err = cudaMemcpyAsync(h.S_final, d.S_final, BH * h.dk * h.dv * 4, cudaMemcpyDeviceToHost, s);
-    if (err == cudaSuccess && h.Z_final && h.normalize)
-      err = cudaMemcpyAsync(h.Z_final, d.Z_final, BH * h.dk * 4, cudaMemcpyDeviceToHost, s);
+  cudaStream_t sc[2] = {nullptr, nullptr};  // copy-in, copy-out (compute runs on s)
+  cudaEvent_t ev_start = nullptr;
+  const bool pipelined = groups_target > 1 && BH > 1;
+  if (pipelined && BH > 0 && T > 0) {
+    for (auto& x : sc)
+      if (err == cudaSuccess) err = cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking);
+    if (err == cudaSuccess) err = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+    if (err == cudaSuccess) err = cudaEventRecord(ev_start, s);  // caller's prior work
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(sc[0], ev_start, 0);
+    for (int b = 0; b < h.B && err == cudaSuccess && st == LA_OK; ++b) {
+      for (int h0 = 0; h0 < h.H && err == cudaSuccess && st == LA_OK; h0 += heads_per_group) {
+        const int hn = std::min(heads_per_group, h.H - h0);
+        const size_t bh0 = static_cast<size_t>(b) * h.H + h0;
+        auto src = [](const void* p, size_t off) { return static_cast<const uint8_t*>(p) + off; };
+        err = cudaMemcpyAsync(buf + hl.q + bh0 * pq, src(h.q, bh0 * pq), hn * pq,
+                              cudaMemcpyHostToDevice, sc[0]);
+        if (err == cudaSuccess)
+          err = cudaMemcpyAsync(buf + hl.k + bh0 * pq, src(h.k, bh0 * pq), hn * pq,
+                                cudaMemcpyHostToDevice, sc[0]);
+        if (err == cudaSuccess)
+          err = cudaMemcpyAsync(buf + hl.v + bh0 * pv, src(h.v, bh0 * pv), hn * pv,
+                                cudaMemcpyHostToDevice, sc[0]);
+        cudaEvent_t ev_in = nullptr, ev_done = nullptr;
+        if (err == cudaSuccess) err = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
+        if (err == cudaSuccess) err = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+        if (err == cudaSuccess) err = cudaEventRecord(ev_in, sc[0]);
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(s, ev_in, 0);
+        la_prefill_args d = h;
+        d.B = 1;
+        d.H = hn;
+        d.gamma = h.gamma ? h.gamma + h0 : nullptr;
+        d.q = buf + hl.q + bh0 * pq;
+        d.k = buf + hl.k + bh0 * pq;
+        d.v = buf + hl.v + bh0 * pv;
+        d.out = buf + hl.out + bh0 * po;
+        d.S_final = h.S_final ? reinterpret_cast<float*>(buf + hl.S + bh0 * pS) : nullptr;
+        d.Z_final = h.Z_final ? reinterpret_cast<float*>(buf + hl.Z + bh0 * pZ) : nullptr;
+        d.workspace = buf + hl.ws;  // one group at a time on the compute stream
+        d.workspace_bytes = hl.total - hl.ws;
+        d.stream = s;
+        if (err == cudaSuccess) st = la::prefill(d);
+        if (err == cudaSuccess && st == LA_OK) err = cudaEventRecord(ev_done, s);
+        if (err == cudaSuccess && st == LA_OK) err = cudaStreamWaitEvent(sc[1], ev_done, 0);
+        if (err == cudaSuccess && st == LA_OK)
+          err = cudaMemcpyAsync(static_cast<uint8_t*>(h.out) + bh0 * po, d.out, hn * po,
+                                cudaMemcpyDeviceToHost, sc[1]);
+        if (err == cudaSuccess && st == LA_OK && h.S_final)
+          err = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(h.S_final) + bh0 * pS, d.S_final,
+                                hn * pS, cudaMemcpyDeviceToHost, sc[1]);
+        if (err == cudaSuccess && st == LA_OK && h.Z_final && h.normalize)
+          err = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(h.Z_final) + bh0 * pZ, d.Z_final,
+                                hn * pZ, cudaMemcpyDeviceToHost, sc[1]);
+        // Events may be destroyed once recorded; the waits already made keep their order.
+        if (ev_in) cudaEventDestroy(ev_in);
+        if (ev_done) cudaEventDestroy(ev_done);
+      }
+    }
+    // Every copy has finished before the buffer is released and the call returns.
+    for (auto& x : sc)
+      if (x) {
+        const cudaError_t se = cudaStreamSynchronize(x);
+        if (err == cudaSuccess) err = se;
+        cudaStreamDestroy(x);
+      }
+    if (ev_start) cudaEventDestroy(ev_start);
+  } else {
+    const size_t nq = BH * pq, nv = BH * pv, no = BH * po;
+    if (nq) err = cudaMemcpyAsync(buf + hl.q, h.q, nq, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess && nq) err = cudaMemcpyAsync(buf + hl.k, h.k, nq, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess && nv) err = cudaMemcpyAsync(buf + hl.v, h.v, nv, cudaMemcpyHostToDevice, s);
+    la_prefill_args d = h;
+    d.q = buf + hl.q;
+    d.k = buf + hl.k;
+    d.v = buf + hl.v;
+    d.out = buf + hl.out;
+    d.S_final = h.S_final ? reinterpret_cast<float*>(buf + hl.S) : nullptr;
+    d.Z_final = h.Z_final ? reinterpret_cast<float*>(buf + hl.Z) : nullptr;
+    d.workspace = buf + hl.ws;
+    d.workspace_bytes = hl.total - hl.ws;
+    if (err == cudaSuccess) st = la::prefill(d);
+    if (err == cudaSuccess && st == LA_OK) {
+      if (no) err = cudaMemcpyAsync(h.out, d.out, no, cudaMemcpyDeviceToHost, s);
+      if (err == cudaSuccess && h.S_final)
+        err = cudaMemcpyAsync(h.S_final, d.S_final, BH * pS, cudaMemcpyDeviceToHost, s);
+      if (err == cudaSuccess && h.Z_final && h.normalize)
+        err = cudaMemcpyAsync(h.Z_final, d.Z_final, BH * pZ, cudaMemcpyDeviceToHost, s);
+    }
   }
   if (owned) cudaFreeAsync(buf, s);
   const cudaError_t se = cudaStreamSynchronize(s);

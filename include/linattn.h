@@ -200,7 +200,13 @@ int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int ma
  * memory of at least lin_attn_prefill_host_buffer_bytes() bytes used to stage the
  * tensors and the workspace, or NULL to allocate it on the stream.  Copies the inputs
  * to the device, runs the prefill, copies the results back and synchronises `stream`
- * before returning, so the host outputs are ready on LA_OK.
+ * before returning, so the host outputs are ready on LA_OK.  Problems of 64 MB of inputs
+ * or more are processed in groups of heads (up to 16, each at least 32 MB) on two copy
+ * streams of the library's own plus `stream`, so that the copies into the device, the
+ * kernels and the copies back overlap; the work still starts after everything queued on
+ * `stream` before the call.  Each (b, h) is computed exactly as by lin_attn_prefill_ex
+ * whenever the segmented algorithm's segment length is fixed (segment_chunks > 0) or the
+ * chunked algorithm runs.
  */
 int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
                           size_t device_buffer_bytes);

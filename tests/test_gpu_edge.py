@@ -196,3 +196,28 @@ def test_argument_errors_on_device_tensors():
 
 def test_no_device_error_reported():
     assert B.lin_attn_device_error() == 0
+
+
+@pytest.mark.parametrize("fm,norm,decay", [("identity", False, True), ("elu1", True, False)])
+def test_host_entry_point_pipelines_large_problems(fm, norm, decay):
+    # About 100 MB of inputs: the host entry point splits the heads into groups whose
+    # copies overlap the kernels.  With the segment length fixed, each (b, h) is computed
+    # exactly as by the device entry point, so the results are bitwise equal.
+    w = Workload("host_pipe", B=2, H=4, T=16384, dk=128, dv=128, C=64, dtype="bf16",
+                 scale=1.0 / math.sqrt(128) if fm == "identity" else 0.5, feature_map=fm,
+                 decay=decay, normalize=norm)
+    q, k, v = make_inputs(w, seed=9, device="cuda", gen_device="cpu")
+    gamma = gammas_for(4, 9) if decay else None
+    kw = dict(feature_map=fm, gamma=gamma, normalize=norm, out_dtype="f32", segment_chunks=16)
+    out_d, S_d, Z_d = B.lin_attn_prefill(q, k, v, **kw)
+    torch.cuda.synchronize()
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+    S_h = torch.empty(S_d.shape, dtype=torch.float32).pin_memory()
+    Z_h = torch.empty((2, 4, 128), dtype=torch.float32).pin_memory() if norm else None
+    B.lin_attn_prefill_host(qh, kh, vh, out_h, S_h, Z_h, **kw)
+    assert torch.equal(out_h, out_d.cpu())
+    assert torch.equal(S_h, S_d.cpu())
+    if norm:
+        assert torch.equal(Z_h, Z_d.cpu())
+    assert B.lin_attn_device_error() == 0
