@@ -30,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "lin_attn_prefill_ex", "lin_attn_prefill_timed", "lin_attn_prefill_host",
     "lin_attn_prefill_host_buffer_bytes", "lin_attn_prefill_noalloc",
     "lin_attn_decode_step", "lin_attn_decode_step_f32", "lin_attn_device_error",
-    "lin_attn_status_string", "lin_attn_version",
+    "lin_attn_status_string", "lin_attn_version", "lin_attn_combine_states",
 )
 
 
@@ -53,6 +53,7 @@ class PrefillArgs(ctypes.Structure):
         ("segment_chunks", ctypes.c_int),
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
+        ("S_init", ctypes.c_void_p), ("Z_init", ctypes.c_void_p), ("states_only", ctypes.c_int),
     ]
 
 
@@ -84,6 +85,8 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_device_error": (i, [ctypes.POINTER(ctypes.c_int)]),
         "lin_attn_status_string": (ctypes.c_char_p, [i]),
         "lin_attn_version": (i, []),
+        "lin_attn_combine_states": (i, [vp, vp, i, i, ctypes.POINTER(ll), i, i, i, i, vp, vp,
+                                        vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -123,7 +126,7 @@ def _gamma_array(gamma, H):
 
 def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, normalize, eps,
               scan, kernel_path, workspace, stream, out_dtype="as_input", algorithm="auto",
-              segment_chunks=0):
+              segment_chunks=0, S_init=None, Z_init=None, states_only=False):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     garr, gptr = _gamma_array(gamma, H)
@@ -144,6 +147,8 @@ def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, norm
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = stream
+    a.S_init, a.Z_init = _ptr(S_init), _ptr(Z_init)
+    a.states_only = int(bool(states_only))
     return a, garr
 
 
@@ -154,16 +159,18 @@ def lin_attn_prefill_workspace_bytes(B, H, T, dk, dv, C, normalize) -> int:
 def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
                      feature_map="elu1", gamma=None, normalize=True, eps=0.0, scan="logdepth",
                      kernel_path="auto", workspace=None, stream=None, want_states=True,
-                     out_dtype="as_input", algorithm="auto",
-              segment_chunks=0):
+                     out_dtype="as_input", algorithm="auto", segment_chunks=0, S_init=None,
+                     Z_init=None, states_only=False):
     """Runs the prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (bf16 or float32).
 
     out_dtype "f32" writes a float32 output for bf16 inputs.  Allocates out / S_final /
-    Z_final when not given.  Returns (out, S_final, Z_final).
+    Z_final when not given.  S_init / Z_init: the state before token 0 (device float32,
+    may be S_final / Z_final themselves).  states_only: compute the final states only (no
+    output; out stays None).  Returns (out, S_final, Z_final).
     """
     B, H, T, dk = q.shape
     dv = v.shape[-1]
-    if out is None:
+    if out is None and not states_only:
         odt = torch.float32 if out_dtype == "f32" else q.dtype
         out = torch.empty((B, H, T, dv), dtype=odt, device=q.device)
     if want_states and S_final is None:
@@ -174,10 +181,31 @@ def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=workspace,
                         stream=_stream_handle(stream), out_dtype=out_dtype, algorithm=algorithm,
-                        segment_chunks=segment_chunks)
+                        segment_chunks=segment_chunks, S_init=S_init, Z_init=Z_init,
+                        states_only=states_only)
     _check("lin_attn_prefill_ex", load_library().lin_attn_prefill_ex(ctypes.byref(a)))
     del keep
     return out, S_final, Z_final
+
+
+def lin_attn_combine_states(S_parts, Z_parts, upto, part_tokens, *, gamma=None, S_out=None,
+                            Z_out=None, stream=None):
+    """Incoming state of part `upto` of a sequence split into parts (see the header):
+    S_parts [parts,B,H,dk,dv], Z_parts [parts,B,H,dk] or None, part_tokens a list of
+    ints.  Returns (S_out, Z_out)."""
+    parts, B, H, dk, dv = S_parts.shape
+    if S_out is None:
+        S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=S_parts.device)
+    if Z_parts is not None and Z_out is None:
+        Z_out = torch.empty((B, H, dk), dtype=torch.float32, device=S_parts.device)
+    toks = (ctypes.c_longlong * max(1, parts))(*[int(t) for t in part_tokens])
+    garr, gptr = _gamma_array(gamma, H)
+    _check("lin_attn_combine_states",
+           load_library().lin_attn_combine_states(_ptr(S_parts), _ptr(Z_parts), parts, int(upto),
+                                                  toks, B, H, dk, dv, gptr, _ptr(S_out),
+                                                  _ptr(Z_out), _stream_handle(stream)))
+    del garr
+    return S_out, Z_out
 
 
 def lin_attn_prefill_timed(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
@@ -202,14 +230,16 @@ def lin_attn_prefill_timed(q, k, v, out, S_final=None, Z_final=None, *, chunk=64
 def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
                           feature_map="elu1", gamma=None, normalize=True, eps=0.0,
                           scan="logdepth", kernel_path="auto", device_buffer=None, stream=None,
-                          out_dtype="as_input", algorithm="auto",
-              segment_chunks=0):
-    """Runs the prefill on HOST tensors (pinned for full copy bandwidth); synchronous."""
+                          out_dtype="as_input", algorithm="auto", segment_chunks=0, S_init=None,
+                          Z_init=None, states_only=False):
+    """Runs the prefill on HOST tensors (pinned for full copy bandwidth); synchronous.
+    S_init / Z_init, when given, are host tensors too."""
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,
                         gamma=gamma, normalize=normalize, eps=eps, scan=scan,
                         kernel_path=kernel_path, workspace=None, stream=_stream_handle(stream),
                         out_dtype=out_dtype, algorithm=algorithm,
-                        segment_chunks=segment_chunks)
+                        segment_chunks=segment_chunks, S_init=S_init, Z_init=Z_init,
+                        states_only=states_only)
     nbytes = 0 if device_buffer is None else device_buffer.numel() * device_buffer.element_size()
     _check("lin_attn_prefill_host",
            load_library().lin_attn_prefill_host(ctypes.byref(a), _ptr(device_buffer), nbytes))

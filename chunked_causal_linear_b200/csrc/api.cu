@@ -149,6 +149,9 @@ int validate(const la_prefill_args& a, Path* path) {
   if (a.out_dtype != LA_OUT_AS_INPUT && a.out_dtype != LA_OUT_F32) return LA_ERR_INVALID_ARGUMENT;
   if (a.algorithm < LA_ALGO_AUTO || a.algorithm > LA_ALGO_SEGMENTED) return LA_ERR_INVALID_ARGUMENT;
   if (a.segment_chunks < 0 || a.segment_chunks > 1024) return LA_ERR_INVALID_ARGUMENT;
+  if (a.states_only != 0 && a.states_only != 1) return LA_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(a.S_init) & 3u) || (reinterpret_cast<uintptr_t>(a.Z_init) & 3u))
+    return LA_ERR_INVALID_ARGUMENT;
   if (a.normalize && a.feature_map == LA_FM_IDENTITY) return LA_ERR_INVALID_ARGUMENT;
   if (!(a.eps >= 0.f) || !std::isfinite(a.eps)) return LA_ERR_INVALID_ARGUMENT;
   if (a.gamma && a.H > kMaxHeads) return LA_ERR_UNSUPPORTED;
@@ -169,15 +172,17 @@ int validate(const la_prefill_args& a, Path* path) {
 
   const bool empty = BH == 0 || a.T == 0;
   if (!empty) {
-    if (!a.q || !a.k || !a.v || !a.out) return LA_ERR_INVALID_ARGUMENT;
-    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out))
+    const bool want_out = !a.states_only;
+    if (!a.q || !a.k || !a.v || (want_out && !a.out)) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || (a.out && !aligned16(a.out)))
       return LA_ERR_INVALID_ARGUMENT;
     const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
     const size_t eo = (a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32) ? 4 : 2;
     const size_t nq = static_cast<size_t>(BH) * a.T * a.dk * e;
     const size_t nv = static_cast<size_t>(BH) * a.T * a.dv * e;
     const size_t no = static_cast<size_t>(BH) * a.T * a.dv * eo;
-    if (overlaps(a.out, no, a.q, nq) || overlaps(a.out, no, a.k, nq) || overlaps(a.out, no, a.v, nv))
+    if (a.out && (overlaps(a.out, no, a.q, nq) || overlaps(a.out, no, a.k, nq) ||
+                  overlaps(a.out, no, a.v, nv)))
       return LA_ERR_INVALID_ARGUMENT;
   }
   if ((a.S_final && !aligned16(a.S_final)) || (a.Z_final && !aligned16(a.Z_final)))
@@ -225,14 +230,16 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
   const long long BH = static_cast<long long>(a.B) * a.H;
   if (BH == 0) return LA_OK;
   if (a.T == 0) {
-    if (a.S_final) {
-      cudaError_t e = cudaMemsetAsync(a.S_final, 0, static_cast<size_t>(BH) * a.dk * a.dv * 4, s);
-      if (e != cudaSuccess) return LA_ERR_CUDA;
-    }
-    if (a.Z_final && a.normalize) {
-      cudaError_t e = cudaMemsetAsync(a.Z_final, 0, static_cast<size_t>(BH) * a.dk * 4, s);
-      if (e != cudaSuccess) return LA_ERR_CUDA;
-    }
+    // No tokens: the final state is the initial one (or zero).
+    auto put = [&](float* dst, const float* init, size_t bytes) -> bool {
+      if (!dst) return true;
+      if (!init) return cudaMemsetAsync(dst, 0, bytes, s) == cudaSuccess;
+      if (init == dst) return true;
+      return cudaMemcpyAsync(dst, init, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    };
+    if (!put(a.S_final, a.S_init, static_cast<size_t>(BH) * a.dk * a.dv * 4)) return LA_ERR_CUDA;
+    if (a.normalize && !put(a.Z_final, a.Z_init, static_cast<size_t>(BH) * a.dk * 4))
+      return LA_ERR_CUDA;
     return LA_OK;
   }
 
@@ -265,6 +272,9 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
   p.tot = reinterpret_cast<float*>(ws + l.tot_off);
   p.S_final = a.S_final;
   p.Z_final = a.normalize ? a.Z_final : nullptr;
+  p.S_init = a.S_init;
+  p.Z_init = a.normalize ? a.Z_init : nullptr;
+  p.has_init = p.S_init != nullptr || p.Z_init != nullptr;
   p.Ls = l.Ls;
   p.G = l.G;
   p.err = error_word_ptr();
@@ -292,6 +302,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     sp.eps = a.eps;
     sp.srec = reinterpret_cast<float*>(ws);
     sp.out = a.out;
+    sp.has_init = p.has_init;
     sp.err = p.err;
     const size_t srec_bytes = align256(static_cast<size_t>(BH) * NS * l.R * sizeof(float));
     PrefillParams ps = p;  // the scan over segments: one scan element per segment
@@ -320,7 +331,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
       e = launch_k1_seg(sp, gt, m, f, s);
       if (e == cudaSuccess) e = launch_k2(ps, gt, a.scan_mode, f, s, rec);
       if (rec) rec->mark(s);
-      if (e == cudaSuccess) e = launch_k3_seg(sp, gt, m, f, s);
+      if (e == cudaSuccess && !a.states_only) e = launch_k3_seg(sp, gt, m, f, s);
     }
   } else if (path == Path::kTensorCore) {
     TcMaps m;
@@ -331,10 +342,11 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
                        T * a.dk * 2ull, 64, 64) &&
               make_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, a.dv, T, BH, a.dv * 2ull,
                        T * a.dv * 2ull, 64, 64) &&
-              (out_f32 ? make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, a.dv, T, BH,
-                                  a.dv * 4ull, T * a.dv * 4ull, 32, 64)
-                       : make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.dv, T, BH,
-                                  a.dv * 2ull, T * a.dv * 2ull, 64, 64)) &&
+              (a.states_only ||
+               (out_f32 ? make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, a.dv, T, BH,
+                                   a.dv * 4ull, T * a.dv * 4ull, 32, 64)
+                        : make_map(&m.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.dv, T, BH,
+                                   a.dv * 2ull, T * a.dv * 2ull, 64, 64))) &&
               make_map(&m.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.rec, a.dk, a.dv,
                        static_cast<uint64_t>(BH) * l.NC, a.dk * 4ull, l.R * 4ull, 32,
                        static_cast<uint32_t>(a.dv));
@@ -345,14 +357,15 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
       e = launch_k1_tc(p, gt, m, f, s);
       if (e == cudaSuccess) e = launch_k2(p, gt, a.scan_mode, f, s, rec);
       if (rec) rec->mark(s);
-      if (e == cudaSuccess) e = launch_k3_tc(p, gt, m, f, s);
+      if (e == cudaSuccess && !a.states_only) e = launch_k3_tc(p, gt, m, f, s);
     }
   } else {
     if (rec) rec->mark(s);
     e = launch_k1_fma(p, gt, a.k, a.v, a.dtype, f, s);
     if (e == cudaSuccess) e = launch_k2(p, gt, a.scan_mode, f, s, rec);
     if (rec) rec->mark(s);
-    if (e == cudaSuccess) e = launch_k3_fma(p, gt, a.q, a.k, a.v, a.out, a.dtype, f, s);
+    if (e == cudaSuccess && !a.states_only)
+      e = launch_k3_fma(p, gt, a.q, a.k, a.v, a.out, a.dtype, f, s);
   }
   if (rec) rec->mark(s);
   if (owned) {
@@ -549,6 +562,12 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
         if (err == cudaSuccess)
           err = cudaMemcpyAsync(buf + hl.v + bh0 * pv, src(h.v, bh0 * pv), hn * pv,
                                 cudaMemcpyHostToDevice, sc[0]);
+        if (err == cudaSuccess && h.S_init)
+          err = cudaMemcpyAsync(buf + hl.S + bh0 * pS, src(h.S_init, bh0 * pS), hn * pS,
+                                cudaMemcpyHostToDevice, sc[0]);
+        if (err == cudaSuccess && h.Z_init && h.normalize)
+          err = cudaMemcpyAsync(buf + hl.Z + bh0 * pZ, src(h.Z_init, bh0 * pZ), hn * pZ,
+                                cudaMemcpyHostToDevice, sc[0]);
         cudaEvent_t ev_in = nullptr, ev_done = nullptr;
         if (err == cudaSuccess) err = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
         if (err == cudaSuccess) err = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
@@ -564,13 +583,15 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
         d.out = buf + hl.out + bh0 * po;
         d.S_final = h.S_final ? reinterpret_cast<float*>(buf + hl.S + bh0 * pS) : nullptr;
         d.Z_final = h.Z_final ? reinterpret_cast<float*>(buf + hl.Z + bh0 * pZ) : nullptr;
+        d.S_init = h.S_init ? reinterpret_cast<float*>(buf + hl.S + bh0 * pS) : nullptr;
+        d.Z_init = h.Z_init ? reinterpret_cast<float*>(buf + hl.Z + bh0 * pZ) : nullptr;
         d.workspace = buf + hl.ws;  // one group at a time on the compute stream
         d.workspace_bytes = hl.total - hl.ws;
         d.stream = s;
         if (err == cudaSuccess) st = la::prefill(d);
         if (err == cudaSuccess && st == LA_OK) err = cudaEventRecord(ev_done, s);
         if (err == cudaSuccess && st == LA_OK) err = cudaStreamWaitEvent(sc[1], ev_done, 0);
-        if (err == cudaSuccess && st == LA_OK)
+        if (err == cudaSuccess && st == LA_OK && h.out && !h.states_only)
           err = cudaMemcpyAsync(static_cast<uint8_t*>(h.out) + bh0 * po, d.out, hn * po,
                                 cudaMemcpyDeviceToHost, sc[1]);
         if (err == cudaSuccess && st == LA_OK && h.S_final)
@@ -597,6 +618,10 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
     if (nq) err = cudaMemcpyAsync(buf + hl.q, h.q, nq, cudaMemcpyHostToDevice, s);
     if (err == cudaSuccess && nq) err = cudaMemcpyAsync(buf + hl.k, h.k, nq, cudaMemcpyHostToDevice, s);
     if (err == cudaSuccess && nv) err = cudaMemcpyAsync(buf + hl.v, h.v, nv, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess && h.S_init)
+      err = cudaMemcpyAsync(buf + hl.S, h.S_init, BH * pS, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess && h.Z_init && h.normalize)
+      err = cudaMemcpyAsync(buf + hl.Z, h.Z_init, BH * pZ, cudaMemcpyHostToDevice, s);
     la_prefill_args d = h;
     d.q = buf + hl.q;
     d.k = buf + hl.k;
@@ -604,11 +629,13 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
     d.out = buf + hl.out;
     d.S_final = h.S_final ? reinterpret_cast<float*>(buf + hl.S) : nullptr;
     d.Z_final = h.Z_final ? reinterpret_cast<float*>(buf + hl.Z) : nullptr;
+    d.S_init = h.S_init ? reinterpret_cast<float*>(buf + hl.S) : nullptr;
+    d.Z_init = h.Z_init ? reinterpret_cast<float*>(buf + hl.Z) : nullptr;
     d.workspace = buf + hl.ws;
     d.workspace_bytes = hl.total - hl.ws;
     if (err == cudaSuccess) st = la::prefill(d);
     if (err == cudaSuccess && st == LA_OK) {
-      if (no) err = cudaMemcpyAsync(h.out, d.out, no, cudaMemcpyDeviceToHost, s);
+      if (no && h.out && !h.states_only) err = cudaMemcpyAsync(h.out, d.out, no, cudaMemcpyDeviceToHost, s);
       if (err == cudaSuccess && h.S_final)
         err = cudaMemcpyAsync(h.S_final, d.S_final, BH * pS, cudaMemcpyDeviceToHost, s);
       if (err == cudaSuccess && h.Z_final && h.normalize)

@@ -30,6 +30,9 @@ struct PrefillParams {
   float* tot;      // [BH, G, R] segment totals / segment prefixes (log-depth scan only)
   float* S_final;  // [BH, dk, dv] or nullptr
   float* Z_final;  // [BH, dk] or nullptr
+  const float* S_init;  // [BH, dk, dv] state before token 0, or nullptr (zero)
+  const float* Z_init;  // [BH, dk] or nullptr (zero)
+  bool has_init;   // chunk 0 has a (nonzero) prefix: S_init or Z_init given
   int Ls;          // chunks per scan segment
   int G;           // number of scan segments, ceil(NC / Ls) (<= 32)
   int* err;        // device error word
@@ -54,6 +57,7 @@ struct SegParams {
   float eps;
   float* srec;     // [BH, NS, R] segment totals, turned into exclusive prefixes by K2
   void* out;       // [BH, T, dv] output, bf16 or fp32
+  bool has_init;   // segment 0 starts from a given state (its prefix is not zero)
   int* err;
 };
 

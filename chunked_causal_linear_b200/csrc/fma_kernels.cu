@@ -106,6 +106,8 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
 
   const long long item = blockIdx.x;
   const int c = static_cast<int>(item % p.NC);
+  // Chunk 0 has a prefix too when the sequence continues from an initial state.
+  const bool pre = c > 0 || p.has_init;
   const int bh = static_cast<int>(item / p.NC);
   const long long t0 = static_cast<long long>(c) * C;
   const int L = chunk_len(p, c);
@@ -121,9 +123,9 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
   }
   for (int e = threadIdx.x; e < C * dv; e += blockDim.x) sV[e] = e / dv < L ? to_f(vb[e]) : 0.f;
   const float* rec = p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R;
-  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) sP[e] = c > 0 ? rec[e] : 0.f;
+  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) sP[e] = pre ? rec[e] : 0.f;
   if (NORM)
-    for (int i = threadIdx.x; i < dk; i += blockDim.x) sZP[i] = c > 0 ? rec[dk * dv + i] : 0.f;
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) sZP[i] = pre ? rec[dk * dv + i] : 0.f;
   for (int i = threadIdx.x; i < C; i += blockDim.x)
     sTh[i] = DECAY ? powf(g, static_cast<float>(i + 1)) : 1.f;
   __syncthreads();
@@ -152,7 +154,7 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
     const int i = e / dv, j = e % dv;
     if (i >= L) continue;
     float inter = 0.f, loc = 0.f;
-    if (c > 0)
+    if (pre)
       for (int kk = 0; kk < dk; ++kk) inter = fmaf(sQ[i * dk + kk], sP[j * dk + kk], inter);
     for (int t = 0; t <= i; ++t) loc = fmaf(sA[i * C + t], sV[t * dv + j], loc);
     float o = fmaf(sTh[i], inter, loc);

@@ -22,6 +22,9 @@
 // Sequential mode (comparison only) carries the state through every chunk in order.
 // Both modes read and write float4 columns; a warp touches 512 contiguous bytes of a
 // record per step.
+// A caller-given state before token 0 (S_init, Z_init) is the scan's first element: the
+// exclusive prefix of chunk 0 is that state, and every later prefix carries it decayed by
+// gamma^(tokens before the chunk) -- the same monoid with one more element in front.
 
 #include "common.cuh"
 #include "launch.h"
@@ -55,6 +58,22 @@ __device__ __forceinline__ void write_final(const PrefillParams& p, int bh, int 
   write_final1(p, bh, col + 1, v.y);
   write_final1(p, bh, col + 2, v.z);
   write_final1(p, bh, col + 3, v.w);
+}
+
+// The initial state of record column `col` (same mapping as write_final1); zero without one.
+__device__ __forceinline__ float read_init1(const PrefillParams& p, int bh, int col) {
+  const int dkdv = p.dk * p.dv;
+  if (col < dkdv) {
+    if (!p.S_init) return 0.f;
+    const int j = col / p.dk, i = col % p.dk;
+    return p.S_init[static_cast<long long>(bh) * dkdv + static_cast<long long>(i) * p.dv + j];
+  }
+  return p.Z_init ? p.Z_init[static_cast<long long>(bh) * p.dk + (col - dkdv)] : 0.f;
+}
+
+__device__ __forceinline__ float4 read_init(const PrefillParams& p, int bh, int col) {
+  return make_float4(read_init1(p, bh, col), read_init1(p, bh, col + 1), read_init1(p, bh, col + 2),
+                     read_init1(p, bh, col + 3));
 }
 
 // In-place exclusive carry over chunks [cbeg, cend) of one float4 column: record c
@@ -100,7 +119,7 @@ __global__ void __launch_bounds__(kScanThreads) k2_sequential(PrefillParams p, G
   const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
   float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) + col4;
   const float4 carry = carry_in_place<DECAY>(base, R4, 0, p.NC, p.NC - 1, gC, aL,
-                                             make_float4(0.f, 0.f, 0.f, 0.f));
+                                             read_init(p, bh, col4 * 4));
   write_final(p, bh, col4 * 4, carry);
 }
 
@@ -171,12 +190,16 @@ __global__ void __launch_bounds__(1024) k2_scan_totals(PrefillParams p, GammaTab
     }
     __syncthreads();
   }
+  // `a` is now the product of the decays of segments 0 .. s: the initial state reaches
+  // the end of segment s scaled by it.
+  const float4 init = (p.S_init || p.Z_init) && live ? read_init(p, bh, col4 * 4)
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  x = axpy4(a, init, x);
   // Inclusive -> exclusive.
   sX[s][threadIdx.x] = x;
   __syncthreads();
   if (live) {
-    tot[static_cast<long long>(s) * R4 + col4] = s > 0 ? sX[s - 1][threadIdx.x]
-                                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    tot[static_cast<long long>(s) * R4 + col4] = s > 0 ? sX[s - 1][threadIdx.x] : init;
     if (s == p.G - 1) write_final(p, bh, col4 * 4, x);
   }
 }

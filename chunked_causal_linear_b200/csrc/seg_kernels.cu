@@ -682,7 +682,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       const int s = i & 1;
       const long long t0 = static_cast<long long>(cb + i) * kC;
       const int L = chunk_len(sp, cb + i);
-      const bool has_prefix = !(seg == 0 && i == 0);
+      const bool has_prefix = !(seg == 0 && i == 0) || sp.has_init;
       wait(sdone, i & 1, kErrMmaTimeout);
       wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout);
       tc_fence_after();
@@ -849,7 +849,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     for (int i = 0; i < n && !failed; ++i) {
       const int s = i & 1;
       const bool last = i == n - 1;
-      const bool has_prefix = !(seg == 0 && i == 0);
+      const bool has_prefix = !(seg == 0 && i == 0) || sp.has_init;
       const uint64_t q = dQk + s * kStageD, ql = dQlk + s * kLoD;
       const uint64_t v = dVm + s * kStageD;
 

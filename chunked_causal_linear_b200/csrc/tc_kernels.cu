@@ -297,6 +297,8 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
   if (error_pending(p.err)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = static_cast<int>(blockIdx.x % p.NC);
+  // Chunk 0 has a prefix too when the sequence continues from an initial state.
+  const bool pre = c > 0 || p.has_init;
   const int bh = static_cast<int>(blockIdx.x / p.NC);
   const int t0 = c * kC;
   const int L = chunk_len(p, c);
@@ -322,7 +324,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
     sPow[tid] = DECAY ? powf(g, static_cast<float>(tid)) : 1.f;
   }
   if constexpr (NORM) {
-    if (tid < DK) sZP[tid] = c > 0 ? rec[DK * DV + tid] : 0.f;
+    if (tid < DK) sZP[tid] = pre ? rec[DK * DV + tid] : 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -330,7 +332,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], L_::kQ + L_::kK + L_::kV + (c > 0 ? L_::kP : 0u));
+    mbar_arrive_expect_tx(&bars[0], L_::kQ + L_::kK + L_::kV + (pre ? L_::kP : 0u));
 #pragma unroll
     for (int b = 0; b < DK / 64; ++b) {
       tma_load_3d(sQh + b * kC * 128, &tm_q, &bars[0], b * 64, t0, bh);
@@ -338,7 +340,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
     }
 #pragma unroll
     for (int b = 0; b < DV / 64; ++b) tma_load_3d(sV + b * kC * 128, &tm_v, &bars[0], b * 64, t0, bh);
-    if (c > 0) {
+    if (pre) {
 #pragma unroll
       for (int b = 0; b < DK / 32; ++b)
         tma_load_3d(sP + b * (DV * 128), &tm_rec, &bars[0], b * 32, 0, bh * p.NC + c);
@@ -417,7 +419,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
 
   // Prefix state P_c^T: float32 -> bf16 hi + lo, in place (all values are read into
   // registers before any is overwritten).
-  if (c > 0) {
+  if (pre) {
     constexpr int NF = DK * DV / kTcThreads;  // floats per thread
     const int j = tid % DV;
     const int c0 = (tid / DV) * NF;
@@ -449,7 +451,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
   }
   __syncthreads();
 
-  if (tid == 0 && c > 0) {
+  if (tid == 0 && pre) {
     tc_fence_after();
     constexpr uint32_t idx = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 64, DV);
     const uint32_t aPh = smem_u32(sPh), aPl = smem_u32(sPl);
@@ -540,7 +542,7 @@ k3_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensor
         float o[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float num = c > 0 ? fmaf(th, xo[e], no[e]) : no[e];
+          const float num = pre ? fmaf(th, xo[e], no[e]) : no[e];
           o[e] = NORM ? num / den : num;
         }
         if constexpr (OUTF32) {

@@ -175,6 +175,17 @@ typedef struct la_prefill_args {
                              aligned; NULL = allocate on the stream */
   size_t workspace_bytes;
   la_stream_t stream;
+  /* The state before token 0, for a sequence that continues an earlier one: DEVICE
+   * float32 in the layout of S_final / Z_final, or NULL for zero.  The scan takes it as
+   * its first element (the scan page's monoid with one more element in front), so every
+   * chunk's prefix carries it decayed by gamma^(tokens before the chunk) and S_final
+   * includes gamma^T S_init.  May be the same memory as S_final / Z_final (each element
+   * is read before it is written).  Z_init is used only when normalising. */
+  const float* S_init;
+  const float* Z_init;
+  /* 1: compute only S_final / Z_final (the summaries and the scan, no output: `out` may
+   * be NULL) -- the per-part totals of a sequence split across devices.  0: full prefill. */
+  int states_only;
 } la_prefill_args;
 
 /* lin_attn_prefill_ex -- the prefill with every option of la_prefill_args.  A caller
@@ -195,7 +206,8 @@ int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int ma
 
 /*
  * lin_attn_prefill_host -- the same computation with HOST buffers, for callers whose
- * data lives in host memory.  q, k, v, out, S_final, Z_final are HOST pointers (pinned
+ * data lives in host memory.  q, k, v, out, S_final, Z_final (and S_init, Z_init when
+ * given) are HOST pointers (pinned
  * memory gives full copy bandwidth; pageable memory works).  `device_buffer` is DEVICE
  * memory of at least lin_attn_prefill_host_buffer_bytes() bytes used to stage the
  * tensors and the workspace, or NULL to allocate it on the stream.  Copies the inputs
@@ -211,6 +223,26 @@ int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int ma
 int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
                           size_t device_buffer_bytes);
 size_t lin_attn_prefill_host_buffer_bytes(const la_prefill_args* host_args);
+
+/*
+ * lin_attn_combine_states -- the incoming state of one part of a sequence that is split
+ * into consecutive parts (for example one part per device, each computing its part's
+ * final state from a zero start with states_only = 1).  The scan page's monoid applied
+ * to whole parts ("Log-Depth Chunked Linear-Attention Scan", Formulas; with the decay of
+ * "Linear Attention and Retentive Networks ...", C. Chunkwise Recurrent Representation):
+ *     P = 0;  for j < upto:  P = gamma_h^(part_tokens[j]) P + S_parts[j]
+ * and likewise for Z.  P is part `upto`'s S_init (upto = parts gives the whole
+ * sequence's final state).
+ *   S_parts   DEVICE [parts, B, H, dk, dv] float32 (each part's final state)
+ *   Z_parts   DEVICE [parts, B, H, dk] float32, or NULL (then Z_out is not written)
+ *   part_tokens HOST [parts], tokens in each part (>= 0)
+ *   gamma     HOST [H] decays in [0, 1], or NULL for none
+ *   S_out     DEVICE [B, H, dk, dv]; Z_out DEVICE [B, H, dk] or NULL
+ * 0 <= upto <= parts <= 64.  Asynchronous on `stream`.
+ */
+int lin_attn_combine_states(const float* S_parts, const float* Z_parts, int parts, int upto,
+                            const long long* part_tokens, int B, int H, int dk, int dv,
+                            const float* gamma, float* S_out, float* Z_out, la_stream_t stream);
 
 /*
  * lin_attn_prefill_noalloc -- lin_attn_prefill_ex without any device allocation.  (No

@@ -148,3 +148,34 @@ def test_binding_fails_loudly_without_library(tmp_path):
     from chunked_causal_linear_b200.binding import load_library
     with pytest.raises(RuntimeError):
         load_library(tmp_path / "missing.so")
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(states_only=2), 1), (dict(states_only=-1), 1), (dict(S_init=0x1002), 1),
+    (dict(Z_init=0x1001), 1), (dict(states_only=1, out=None, algorithm=2, dv=64), 2),
+])
+def test_initial_state_and_states_only_argument_errors(lib, kw, status):
+    a = _args(**kw)
+    assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == status
+
+
+def test_states_only_needs_no_output_for_an_empty_problem(lib):
+    a = _args(B=0, out=None, states_only=1)
+    assert lib.lin_attn_prefill_ex(ctypes.byref(a)) == 0
+
+
+def test_combine_states_argument_errors(lib):
+    f = lib.lin_attn_combine_states
+    toks = (ctypes.c_longlong * 3)(10, 20, 30)
+    g_ok = (ctypes.c_float * 2)(0.5, 1.0)
+    g_bad = (ctypes.c_float * 2)(0.5, 1.5)
+    S, O = 0x100000, 0x200000
+    assert f(S, None, 3, 4, toks, 1, 2, 64, 64, g_ok, O, None, None) == 1   # upto > parts
+    assert f(S, None, 3, -1, toks, 1, 2, 64, 64, g_ok, O, None, None) == 1
+    assert f(S, None, 65, 1, toks, 1, 2, 64, 64, g_ok, O, None, None) == 2  # > 64 parts
+    assert f(S, None, 3, 1, toks, 1, 2, 64, 64, g_bad, O, None, None) == 1  # gamma > 1
+    assert f(None, None, 3, 1, toks, 1, 2, 64, 64, g_ok, O, None, None) == 1
+    assert f(S, None, 3, 1, toks, 1, 2, 64, 64, g_ok, O, 0x300000, None) == 1  # Z_out, no Z
+    neg = (ctypes.c_longlong * 3)(10, -1, 30)
+    assert f(S, None, 3, 1, neg, 1, 2, 64, 64, g_ok, O, None, None) == 1
+    assert f(S, None, 3, 1, toks, 0, 2, 64, 64, g_ok, O, None, None) == 0   # empty
