@@ -354,6 +354,94 @@ def sweep_scan(args, dev):
         del q, k, v, ws, out
 
 
+def seq_shard_bench(args, w, info, dev):
+    """One sequence of the workload split across the ranks (seqshard.prefill_sequence_sharded):
+    every rank holds one contiguous token range.  Timed like the main benchmark (device
+    events, barriers, max over ranks); the phases of one step are timed separately."""
+    from chunked_causal_linear_b200.seqshard import part_ranges, prefill_sequence_sharded
+    rng = part_ranges(w.T, info.world, w.C)
+    toks = [n for _, n in rng]
+    s0, n = rng[info.rank]
+    wr = w.with_(T=max(n, 1), name=f"{w.name}_part{info.rank}")
+    q, k, v = make_inputs(wr, seed=info.rank, device=dev)
+    out = torch.empty((w.B, w.H, wr.T, w.dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(B.lin_attn_prefill_workspace_bytes(w.B, w.H, wr.T, w.dk, w.dv, w.C,
+                                                        w.normalize), dtype=torch.uint8, device=dev)
+    gam = w.gammas()
+    algo = effective_algorithm(wr, args.algorithm)
+    kw = dict(chunk=w.C, feature_map=w.feature_map, scan=args.scan, kernel_path="tensor_core",
+              workspace=ws, out_dtype="f32", algorithm=algo, segment_chunks=args.segment_chunks)
+
+    def step():
+        return prefill_sequence_sharded(q, k, v, out, info=info, part_tokens=toks, gamma=gam,
+                                        normalize=w.normalize, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ranks.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ranks.barrier(info)
+    ms_max = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, info, dev)
+
+    # Phases of one step, each timed on its own.
+    def timed(fn, reps=5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+    _, S_loc, Z_loc = B.lin_attn_prefill(q, k, v, None, gamma=gam, normalize=w.normalize,
+                                         states_only=True, **kw)
+    from chunked_causal_linear_b200.seqshard import _gather
+    S_parts = _gather(S_loc, info)
+    Z_parts = _gather(Z_loc, info) if w.normalize else None
+    S_in, Z_in = B.lin_attn_combine_states(S_parts, Z_parts, info.rank, toks, gamma=gam)
+    phases = {
+        "states_pass": timed(lambda: B.lin_attn_prefill(q, k, v, None, gamma=gam,
+                                                        normalize=w.normalize, states_only=True,
+                                                        **kw)),
+        "all_gather": timed(lambda: _gather(S_loc, info)),
+        "combine": timed(lambda: B.lin_attn_combine_states(S_parts, Z_parts, info.rank, toks,
+                                                           gamma=gam)),
+        "prefill": timed(lambda: B.lin_attn_prefill(q, k, v, out, gamma=gam,
+                                                    normalize=w.normalize, S_init=S_in,
+                                                    Z_init=Z_in, **kw)),
+    }
+    phases = {key: ranks.max_over_ranks(val, info, dev) for key, val in phases.items()}
+    err = B.lin_attn_device_error()
+    if info.is_root:
+        cfg = config_of(w, args)
+        cfg["parallelism"] = (f"sequence-sharded over {info.world} rank(s): ranges of "
+                              f"{toks} tokens, all_gather of B*H*(dk*dv+dk) floats per rank")
+        e_in = 2
+        extra = w.B * w.H * w.T * (w.dk + w.dv) * e_in  # the states pass reads k, v again
+        peak, _ = measured_peaks()
+        ab = algo_bytes(w, 4, algo, args.segment_chunks) + extra
+        line = {
+            "metric": METRIC, "value": w.tokens_heads / (ms_max / 1000.0), "unit": UNIT,
+            "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "mode": "seq_shard", "phases_ms": phases,
+            "step_roofline": {"bytes": ab, "achieved_gbs": ab / (ms_max / 1000.0) / 1e9 / info.world,
+                              "frac_of_measured": ab / (ms_max / 1000.0) / 1e9 / info.world / peak,
+                              "note": "per GPU; the bytes include the states pass's second read "
+                                      "of k and v"},
+            "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
@@ -392,6 +480,11 @@ def main():
                          "carry) over a range of chunk counts, one JSON line per point")
     ap.add_argument("--segment-chunks", type=int, default=0,
                     help="chunks per segment of the segmented algorithm (0: automatic)")
+    ap.add_argument("--seq-shard", action="store_true",
+                    help="instead of independent replicas: one sequence split across the ranks "
+                         "(each rank a contiguous token range; states-only pass, all_gather of "
+                         "the range states, fold, prefill from the incoming state); strong "
+                         "scaling")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -413,6 +506,10 @@ def main():
     B.load_library()
     if args.sweep_scan:
         sweep_scan(args, dev)
+        ranks.finish(info)
+        return
+    if args.seq_shard:
+        seq_shard_bench(args, w, info, dev)
         ranks.finish(info)
         return
 
