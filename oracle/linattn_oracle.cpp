@@ -38,6 +38,9 @@
 //   Z_init, Z_final [B, H, dk]
 //   gamma [H] (double) or NULL.
 // S_init / Z_init may be NULL (zero initial state); the outputs may be NULL (skipped).
+//
+// la_oracle_backward differentiates the unnormalised form by hand, token by token (the
+// chain rule through the recurrence; see backward_pair), for the backward pass.
 
 #include <cmath>
 #include <cstddef>
@@ -123,6 +126,95 @@ void run_pair(const Problem& p, long long bh) {
     for (int i = 0; i < dk; ++i) p.Z_final[bh * dk + i] = Z[i];
 }
 
+// Backward of the unnormalised form for one (b, h) pair.  With do_t = dL/do_t and
+// dS_final = dL/dS_final (or zero), differentiating the recurrence above gives
+//   dphi(q_t) = S_t do_t                                   (forward sweep, S_t as above)
+//   G_t       = phi(q_t) do_t^T + gamma G_{t+1},  G_{T-1} = phi(q_{T-1}) do_{T-1}^T + dS_final
+//   dphi(k_t) = G_t v_t,   dv_t = G_t^T phi(k_t)           (reverse sweep)
+//   dS_init   = gamma G_0
+// and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k) with phi' = 1 (identity) or
+// 1 for x > 0, exp(x) otherwise (ELU + 1).  Every sum is the plain chain rule through
+// S_t = gamma S_{t-1} + phi(k_t) v_t^T and o_t = phi(q_t) S_t, one token at a time.
+struct BackwardProblem {
+  const float* q;
+  const float* k;
+  const float* v;
+  const double* dout;
+  int H;
+  long long T;
+  int dk, dv, fm;
+  const double* gamma;
+  const double* S_init;
+  const double* dS_final;
+  double* dq;
+  double* dk_out;
+  double* dv_out;
+  double* dS_init;
+};
+
+inline double feature_map_derivative(double x, int fm) {
+  if (fm == 0) return 1.0;
+  return x > 0.0 ? 1.0 : std::exp(x);
+}
+
+void backward_pair(const BackwardProblem& p, long long bh) {
+  const int dk = p.dk, dv = p.dv;
+  const long long T = p.T;
+  const int h = static_cast<int>(bh % p.H);
+  const double g = p.gamma ? p.gamma[h] : 1.0;
+  const float* q = p.q + bh * T * dk;
+  const float* k = p.k + bh * T * dk;
+  const float* v = p.v + bh * T * dv;
+  const double* dout = p.dout + bh * T * dv;
+
+  // Forward sweep: S_t, then dphi(q_t) = S_t do_t.
+  std::vector<double> S(static_cast<size_t>(dk) * dv, 0.0);
+  if (p.S_init)
+    for (size_t e = 0; e < S.size(); ++e) S[e] = p.S_init[bh * dk * dv + e];
+  for (long long t = 0; t < T; ++t) {
+    for (int i = 0; i < dk; ++i) {
+      const double fk = feature_map(static_cast<double>(k[t * dk + i]), p.fm);
+      double* Si = &S[static_cast<size_t>(i) * dv];
+      for (int j = 0; j < dv; ++j) Si[j] = g * Si[j] + fk * static_cast<double>(v[t * dv + j]);
+    }
+    for (int i = 0; i < dk; ++i) {
+      const double* Si = &S[static_cast<size_t>(i) * dv];
+      double acc = 0.0;
+      for (int j = 0; j < dv; ++j) acc += Si[j] * dout[t * dv + j];
+      const double x = static_cast<double>(q[t * dk + i]);
+      p.dq[(bh * T + t) * dk + i] = acc * feature_map_derivative(x, p.fm);
+    }
+  }
+
+  // Reverse sweep: G accumulates phi(q_t) do_t^T and decays by gamma between tokens.
+  std::vector<double> G(static_cast<size_t>(dk) * dv, 0.0), fk(dk);
+  if (p.dS_final)
+    for (size_t e = 0; e < G.size(); ++e) G[e] = p.dS_final[bh * dk * dv + e];
+  for (long long t = T - 1; t >= 0; --t) {
+    for (int i = 0; i < dk; ++i) {
+      const double fq = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
+      double* Gi = &G[static_cast<size_t>(i) * dv];
+      for (int j = 0; j < dv; ++j) Gi[j] += fq * dout[t * dv + j];
+      fk[i] = feature_map(static_cast<double>(k[t * dk + i]), p.fm);
+    }
+    for (int i = 0; i < dk; ++i) {
+      const double* Gi = &G[static_cast<size_t>(i) * dv];
+      double acc = 0.0;
+      for (int j = 0; j < dv; ++j) acc += Gi[j] * static_cast<double>(v[t * dv + j]);
+      const double x = static_cast<double>(k[t * dk + i]);
+      p.dk_out[(bh * T + t) * dk + i] = acc * feature_map_derivative(x, p.fm);
+    }
+    for (int j = 0; j < dv; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < dk; ++i) acc += G[static_cast<size_t>(i) * dv + j] * fk[i];
+      p.dv_out[(bh * T + t) * dv + j] = acc;
+    }
+    for (double& x : G) x *= g;  // G_{t-1} receives gamma G_t
+  }
+  if (p.dS_init)
+    for (size_t e = 0; e < G.size(); ++e) p.dS_init[bh * dk * dv + e] = G[e];
+}
+
 }  // namespace
 
 extern "C" {
@@ -159,6 +251,34 @@ int la_oracle_forward(const float* q, const float* k, const float* v, int B, int
       for (long long bh = w; bh < BH; bh += workers) run_pair(p, bh);
     });
   }
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+// Backward of the unnormalised form (see backward_pair).  dout [B, H, T, dv] (double),
+// dS_final [B, H, dk, dv] or NULL, S_init as in la_oracle_forward.  Writes dq, dk
+// [B, H, T, dk], dv [B, H, T, dv] and dS_init [B, H, dk, dv] (may be NULL), all double.
+int la_oracle_backward(const float* q, const float* k, const float* v, const double* dout,
+                       int B, int H, long long T, int dk, int dv, int feature_map_id,
+                       const double* gamma, const double* S_init, const double* dS_final,
+                       double* dq, double* dk_out, double* dv_out, double* dS_init,
+                       int nthreads) {
+  if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 1;
+  if (feature_map_id != 0 && feature_map_id != 1) return 1;
+  if (T > 0 && (!q || !k || !v || !dout || !dq || !dk_out || !dv_out)) return 1;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return 0;
+  BackwardProblem p{q, k, v, dout, H, T, dk, dv, feature_map_id, gamma, S_init, dS_final,
+                    dq, dk_out, dv_out, dS_init};
+  long long workers = nthreads > 0 ? nthreads
+                                   : static_cast<long long>(std::thread::hardware_concurrency());
+  if (workers < 1) workers = 1;
+  if (workers > BH) workers = BH;
+  std::vector<std::thread> pool;
+  for (long long w = 0; w < workers; ++w)
+    pool.emplace_back([&p, w, workers, BH]() {
+      for (long long bh = w; bh < BH; bh += workers) backward_pair(p, bh);
+    });
   for (auto& th : pool) th.join();
   return 0;
 }
