@@ -42,6 +42,7 @@ from chunked_causal_linear_b200 import ranks  # noqa: E402
 from chunked_causal_linear_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "causal linear-attn prefill tokens·heads/s at H=32,d=128; % of roofline"
+METRIC_BWD = "causal linear-attn backward tokens·heads/s at H=32,d=128; % of roofline"
 UNIT = "tokens*heads/s"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
@@ -57,7 +58,8 @@ KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce
 
 def effective_algorithm(w, requested: str) -> str:
     """The algorithm the library runs for this workload on the tensor-core path."""
-    seg_ok = w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv == 128
+    seg_ok = (w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv == 128
+              and not (w.feature_map == "elu1" and w.decay))
     if requested == "segmented" or (requested == "auto" and seg_ok):
         return "segmented"
     return "chunked"
@@ -442,6 +444,204 @@ def seq_shard_bench(args, w, info, dev):
         print(json.dumps(line), flush=True)
 
 
+class BackwardOracleTimer(OracleTimer):
+    """OracleTimer for the oracle's backward (gradients of the unnormalised form)."""
+
+    def __init__(self, w, q, k, v, do, target_s: float):
+        self.do = do
+        super().__init__(w, q, k, v, target_s)
+        self.host_do = do[:, :, :self.tp].to("cpu", torch.float64).numpy()
+
+    def _run(self, tp, host=None):
+        w = self.w
+        qs, ks, vs = host if host is not None else (
+            t[:, :, :tp].to("cpu", torch.float32).numpy() for t in self.inputs)
+        dos = self.host_do if host is not None else self.do[:, :, :tp].to("cpu", torch.float64).numpy()
+        t0 = time.perf_counter()
+        self.orc.backward(qs, ks, vs, dos, feature_map=w.feature_map, gamma=w.gammas(),
+                          nthreads=self.threads)
+        return time.perf_counter() - t0
+
+    def sample(self):
+        return (f"first {self.tp} of {self.w.T} tokens of all {self.w.B * self.w.H} (b,h) "
+                f"pairs, fp64 forward sweep and reverse state-gradient sweep, "
+                f"{self.last_s:.1f} s per run on {self.threads} threads")
+
+
+def backward_bytes(w, out_elem: int, algo_of, lseg: int = 0):
+    """Algorithmic bytes per launch of every kernel of the backward, in launch order, for
+    the bench's call (no initial or final state): the reversal of the inputs, three
+    prefills -- (do, v, psi(k)), reversed (k, q, do), reversed (v, do, psi(q)); two more
+    for the lo halves of psi under ELU+1 with bf16 inputs -- and the reversal of the
+    outputs."""
+    BH = w.B * w.H
+    e = 2 if w.dtype == "bf16" else 4
+    elu = w.feature_map == "elu1"
+    split = elu and w.dtype == "bf16"
+    w_f32 = out_elem == 4 or elu
+    ew = 4 if w_f32 else 2
+    nk, nv = BH * w.T * w.dk, BH * w.T * w.dv
+    ops = []
+    n_in = 2 * nk + 2 * nv + (2 * nk if elu else 0) + (2 * nk if split else 0)
+    ops.append(("bwd_reverse_inputs", 2 * n_in * e))
+    wa = w.with_(dk=w.dv, dv=w.dk, feature_map="identity", normalize=False)
+    wb = w.with_(normalize=False)
+    passes = [(wa, 4 if elu else out_elem)] * (2 if split else 1) + [(wb, ew)] + \
+        [(wa, ew)] * (2 if split else 1)
+    for pw, oe in passes:
+        algo = algo_of(pw)
+        for name in kernel_names(pw, algo, "logdepth", lseg):
+            ops.append((name, kernel_bytes(pw, name, oe, algo, lseg)))
+    post = nv * ew + nv * out_elem + nk * ew + nk * out_elem
+    if split:
+        post += nk * 4
+    if elu:
+        post += nk * e + nk * 4 + (nk * 4 if split else 0) + nk * e + nk * out_elem
+    ops.append(("bwd_reverse_outputs", post))
+    return ops
+
+
+def backward_bench(args, w, info, dev):
+    """One backward of the unnormalised form (lin_attn_backward: grad_q, grad_k, grad_v for
+    a given grad_out) per step, timed like the prefill."""
+    if w.normalize:
+        w = w.with_(normalize=False, name=f"{w.name}_unnormalised")
+    q, k, v = make_inputs(w, seed=info.rank, device=dev)
+    g = torch.Generator(device=dev).manual_seed(1000 + info.rank)
+    do = torch.randn((w.B, w.H, w.T, w.dv), generator=g, device=dev).to(q.dtype)
+    odt = torch.float32 if args.out_dtype == "f32" else q.dtype
+    out_elem = 4 if args.out_dtype == "f32" else 2
+    gq = torch.empty(q.shape, dtype=odt, device=dev)
+    gk = torch.empty(k.shape, dtype=odt, device=dev)
+    gv = torch.empty(v.shape, dtype=odt, device=dev)
+    gam = w.gammas()
+    ws = torch.empty(B.lin_attn_backward_workspace_bytes(q, v, chunk=w.C, feature_map=w.feature_map,
+                                                        out_dtype=args.out_dtype, gamma=gam),
+                     dtype=torch.uint8, device=dev)
+    kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, out_dtype=args.out_dtype,
+              kernel_path="tensor_core", algorithm=args.algorithm, workspace=ws,
+              segment_chunks=args.segment_chunks)
+
+    def step():
+        B.lin_attn_backward(q, k, v, do, gq, gk, gv, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def timed_region():
+        sampler = None if args.no_clocks else ClockSampler(info.local_rank)
+        if sampler:
+            sampler.start()
+        ranks.barrier(info)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ranks.barrier(info)
+        return e0.elapsed_time(e1) / args.steps, (sampler.stop() if sampler else None)
+
+    ms, clocks = timed_region()
+    remeasured = False
+    if ranks.any_over_ranks(clocks_bad(clocks), info, dev):
+        ms, clocks = timed_region()
+        remeasured = True
+    ms_max = ranks.max_over_ranks(ms, info, dev)
+    value = info.world * w.tokens_heads / (ms_max / 1000.0)
+
+    # Per-kernel device times; kernels of the same name (the three passes) are pooled.
+    tot, cnt, launches = {}, {}, 0
+    reps = max(1, args.kernel_timing_steps)
+    for _ in range(reps):
+        t = B.lin_attn_backward_timed(q, k, v, do, gq, gk, gv, **kw)
+        launches = len(t)
+        for name, x in t:
+            tot[name] = tot.get(name, 0.0) + x / reps
+            cnt[name] = cnt.get(name, 0) + 1
+    per_launch = {n: tot[n] / (cnt[n] / reps) for n in tot}
+    algo_of = lambda pw: effective_algorithm(pw, args.algorithm)
+    ops = backward_bytes(w, out_elem, algo_of, args.segment_chunks)
+    bytes_of = {}
+    for name, nb in ops:
+        bytes_of.setdefault(name, []).append(nb)
+    dom = max(tot, key=tot.get)
+    peak, peak_kind = measured_peaks()
+    dom_bytes = statistics.mean(bytes_of[dom]) if dom in bytes_of else None
+    achieved = dom_bytes / (per_launch[dom] / 1000.0) / 1e9 if dom_bytes else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak if achieved else None,
+                "traffic": None, "algorithmic_bytes": dom_bytes,
+                "launches_per_step": cnt[dom] // reps,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    step_bytes = sum(nb for _, nb in ops)
+    BH = w.B * w.H
+    e_in = 2 if w.dtype == "bf16" else 4
+    min_b = BH * w.T * (2 * w.dk + 2 * w.dv) * e_in + BH * w.T * (2 * w.dk + w.dv) * out_elem
+    gbs = lambda nb: nb / (ms_max / 1000.0) / 1e9
+    step_roof = {"bytes": step_bytes, "achieved_gbs": gbs(step_bytes),
+                 "frac_of_measured": gbs(step_bytes) / peak, "bytes_min": min_b,
+                 "frac_min_of_measured": gbs(min_b) / peak,
+                 "note": "bytes = the sum of every kernel's algorithmic bytes (three prefills "
+                         "and the reversals); bytes_min = q, k, v, grad_out read once and the "
+                         "three gradients written once"}
+
+    # End to end: pinned host inputs copied in, the backward, the gradients copied out.
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (gq, gk, gv)]
+        din = [torch.empty_like(t) for t in (q, k, v, do)]
+
+        def e2e_step():
+            for d_, h_ in zip(din, hin):
+                d_.copy_(h_, non_blocking=True)
+            B.lin_attn_backward(*din, gq, gk, gv, **kw)
+            for h_, d_ in zip(hout, (gq, gk, gv)):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ranks.barrier(info)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, info, dev)
+        e2e = {"value": info.world * w.tokens_heads / (e_ms / 1000.0), "unit": UNIT,
+               "ms_per_step": e_ms,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
+               "api": "lin_attn_backward between pinned-host copies on the same stream"}
+        del hin, hout, din
+
+    cpu = None
+    if info.is_root and info.world == 1 and not args.no_cpu_baseline:
+        timer = BackwardOracleTimer(w, q, k, v, do, target_s=args.cpu_baseline_s)
+        cpu = {"value": timer.rate(), "unit": UNIT, "cores": timer.threads, "kind": "oracle",
+               "sample": timer.sample()}
+    err = B.lin_attn_device_error()
+    if info.is_root:
+        cfg = config_of(w, args)
+        cfg["algorithm"] = args.algorithm
+        cfg.pop("segment_chunks", None)
+        line = {
+            "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg, "mode": "backward", "roofline": roofline,
+            "step_roofline": step_roof, "kernels_ms": tot, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks, "remeasured": remeasured,
+            "gpu_launches": launches * args.steps, "device_error": err,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
@@ -485,6 +685,9 @@ def main():
                          "(each rank a contiguous token range; states-only pass, all_gather of "
                          "the range states, fold, prefill from the incoming state); strong "
                          "scaling")
+    ap.add_argument("--backward", action="store_true",
+                    help="instead of the prefill: the backward of the unnormalised form "
+                         "(grad_q, grad_k, grad_v for a random grad_out)")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -510,6 +713,10 @@ def main():
         return
     if args.seq_shard:
         seq_shard_bench(args, w, info, dev)
+        ranks.finish(info)
+        return
+    if args.backward:
+        backward_bench(args, w, info, dev)
         ranks.finish(info)
         return
 

@@ -31,6 +31,7 @@ EXPORTED_SYMBOLS = (
     "lin_attn_prefill_host_buffer_bytes", "lin_attn_prefill_noalloc",
     "lin_attn_decode_step", "lin_attn_decode_step_f32", "lin_attn_device_error",
     "lin_attn_status_string", "lin_attn_version", "lin_attn_combine_states",
+    "lin_attn_backward", "lin_attn_backward_workspace_bytes", "lin_attn_backward_timed",
 )
 
 
@@ -54,6 +55,22 @@ class PrefillArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
         ("S_init", ctypes.c_void_p), ("Z_init", ctypes.c_void_p), ("states_only", ctypes.c_int),
+    ]
+
+
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("grad_out", ctypes.c_void_p), ("grad_q", ctypes.c_void_p), ("grad_k", ctypes.c_void_p),
+        ("grad_v", ctypes.c_void_p), ("S_init", ctypes.c_void_p),
+        ("grad_S_final", ctypes.c_void_p), ("grad_S_init", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_longlong),
+        ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
+        ("feature_map", ctypes.c_int), ("gamma", ctypes.c_void_p), ("dtype", ctypes.c_int),
+        ("out_dtype", ctypes.c_int), ("scan_mode", ctypes.c_int), ("kernel_path", ctypes.c_int),
+        ("algorithm", ctypes.c_int), ("segment_chunks", ctypes.c_int),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("stream", ctypes.c_void_p),
     ]
 
 
@@ -87,6 +104,10 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_version": (i, []),
         "lin_attn_combine_states": (i, [vp, vp, i, i, ctypes.POINTER(ll), i, i, i, i, vp, vp,
                                         vp, vp]),
+        "lin_attn_backward": (i, [ctypes.POINTER(BackwardArgs)]),
+        "lin_attn_backward_workspace_bytes": (sz, [ctypes.POINTER(BackwardArgs)]),
+        "lin_attn_backward_timed": (i, [ctypes.POINTER(BackwardArgs), ctypes.POINTER(f),
+                                        ctypes.POINTER(ctypes.c_char_p), i, ctypes.POINTER(i)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -247,14 +268,113 @@ def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
     return out, S_final, Z_final
 
 
+def make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init=None,
+                       grad_S_final=None, grad_S_init=None, chunk=64, feature_map="identity",
+                       gamma=None, out_dtype="as_input", scan="logdepth", kernel_path="auto",
+                       algorithm="auto", segment_chunks=0, workspace=None, stream=None):
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    garr, gptr = _gamma_array(gamma, H)
+    a = BackwardArgs()
+    a.q, a.k, a.v, a.grad_out = _ptr(q), _ptr(k), _ptr(v), _ptr(grad_out)
+    a.grad_q, a.grad_k, a.grad_v = _ptr(grad_q), _ptr(grad_k), _ptr(grad_v)
+    a.S_init, a.grad_S_final, a.grad_S_init = _ptr(S_init), _ptr(grad_S_final), _ptr(grad_S_init)
+    a.B, a.H, a.T, a.dk, a.dv, a.C = B, H, T, dk, dv, int(chunk)
+    a.feature_map = FEATURE_MAPS[feature_map]
+    a.gamma = gptr
+    a.dtype = DTYPES[q.dtype]
+    a.out_dtype = OUT_DTYPES[out_dtype]
+    a.scan_mode = SCAN_MODES[scan]
+    a.kernel_path = KERNEL_PATHS[kernel_path]
+    a.algorithm = ALGORITHMS[algorithm]
+    a.segment_chunks = int(segment_chunks)
+    a.workspace = _ptr(workspace)
+    a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.stream = stream
+    return a, garr
+
+
+def lin_attn_backward(q, k, v, grad_out, grad_q=None, grad_k=None, grad_v=None, *,
+                      S_init=None, grad_S_final=None, want_grad_S_init=False, grad_S_init=None,
+                      chunk=64, feature_map="identity", gamma=None, out_dtype="as_input",
+                      scan="logdepth", kernel_path="auto", algorithm="auto", segment_chunks=0,
+                      workspace=None, stream=None):
+    """Gradients of the unnormalised form for the loss <grad_out, out> + <grad_S_final,
+    S_final> (see the header).  q, k [B,H,T,dk], v, grad_out [B,H,T,dv] on the device.
+    Allocates the gradients not given.  Returns (grad_q, grad_k, grad_v, grad_S_init);
+    grad_S_init is None unless requested (want_grad_S_init or a tensor)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    odt = torch.float32 if out_dtype == "f32" else q.dtype
+    mk = lambda d: torch.empty((B, H, T, d), dtype=odt, device=q.device)
+    grad_q = mk(dk) if grad_q is None else grad_q
+    grad_k = mk(dk) if grad_k is None else grad_k
+    grad_v = mk(dv) if grad_v is None else grad_v
+    if grad_S_init is None and want_grad_S_init:
+        grad_S_init = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    a, keep = make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, S_init=S_init,
+                                 grad_S_final=grad_S_final, grad_S_init=grad_S_init, chunk=chunk,
+                                 feature_map=feature_map, gamma=gamma, out_dtype=out_dtype,
+                                 scan=scan, kernel_path=kernel_path, algorithm=algorithm,
+                                 segment_chunks=segment_chunks, workspace=workspace,
+                                 stream=_stream_handle(stream))
+    _check("lin_attn_backward", load_library().lin_attn_backward(ctypes.byref(a)))
+    del keep
+    return grad_q, grad_k, grad_v, grad_S_init
+
+
+def lin_attn_backward_timed(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init=None,
+                            grad_S_final=None, grad_S_init=None, chunk=64, feature_map="identity",
+                            gamma=None, out_dtype="as_input", scan="logdepth", kernel_path="auto",
+                            algorithm="auto", segment_chunks=0, workspace=None,
+                            stream=None) -> list[tuple[str, float]]:
+    """Runs the backward once with an event around every kernel; returns (name,
+    milliseconds) per kernel in launch order (synchronous)."""
+    a, keep = make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, S_init=S_init,
+                                 grad_S_final=grad_S_final, grad_S_init=grad_S_init, chunk=chunk,
+                                 feature_map=feature_map, gamma=gamma, out_dtype=out_dtype,
+                                 scan=scan, kernel_path=kernel_path, algorithm=algorithm,
+                                 segment_chunks=segment_chunks, workspace=workspace,
+                                 stream=_stream_handle(stream))
+    cap = 48
+    ms = (ctypes.c_float * cap)()
+    names = (ctypes.c_char_p * cap)()
+    n = ctypes.c_int(0)
+    _check("lin_attn_backward_timed",
+           load_library().lin_attn_backward_timed(ctypes.byref(a), ms, names, cap,
+                                                  ctypes.byref(n)))
+    del keep
+    return [(names[i].decode(), float(ms[i])) for i in range(n.value)]
+
+
+def lin_attn_backward_workspace_bytes(q, v, *, chunk=64, feature_map="identity",
+                                      out_dtype="as_input", S_init=False, grad_S_final=False,
+                                      gamma=None) -> int:
+    """Workspace bytes of lin_attn_backward for these shapes and options (S_init /
+    grad_S_final: whether they will be given)."""
+    B, H, T, dk = q.shape
+    garr, gptr = _gamma_array(gamma, H)
+    a = BackwardArgs()
+    a.B, a.H, a.T, a.dk, a.dv, a.C = B, H, T, dk, v.shape[-1], int(chunk)
+    a.feature_map = FEATURE_MAPS[feature_map]
+    a.gamma = gptr
+    a.dtype = DTYPES[q.dtype]
+    a.out_dtype = OUT_DTYPES[out_dtype]
+    # Only whether the states are given matters to the size; any non-null value says so.
+    a.S_init = 16 if S_init else None
+    a.grad_S_final = 16 if grad_S_final else None
+    n = int(load_library().lin_attn_backward_workspace_bytes(ctypes.byref(a)))
+    del garr
+    return n
+
+
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 def lin_attn_prefill_noalloc(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
                              feature_map="elu1", gamma=None, normalize=True, eps=0.0,
                              scan="logdepth", kernel_path="auto", stream=None,
-                             out_dtype="as_input", algorithm="auto",
-              segment_chunks=0):
+                             out_dtype="as_input", algorithm="auto", segment_chunks=0):
     """The prefill with its workspace in the library's fixed device array (no device
     allocation by the library; the caller provides every output tensor)."""
     a, keep = make_args(q, k, v, out, S_final, Z_final, chunk=chunk, feature_map=feature_map,

@@ -327,10 +327,10 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     if (!ok) {
       e = cudaErrorInvalidValue;
     } else {
-      if (rec) rec->mark(s);
+      if (rec) rec->mark(s, "k1_seg");
       e = launch_k1_seg(sp, gt, m, f, s);
       if (e == cudaSuccess) e = launch_k2(ps, gt, a.scan_mode, f, s, rec);
-      if (rec) rec->mark(s);
+      if (rec && !a.states_only) rec->mark(s, "k3_seg");
       if (e == cudaSuccess && !a.states_only) e = launch_k3_seg(sp, gt, m, f, s);
     }
   } else if (path == Path::kTensorCore) {
@@ -353,21 +353,21 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     if (!ok) {
       e = cudaErrorInvalidValue;
     } else {
-      if (rec) rec->mark(s);
+      if (rec) rec->mark(s, "k1_tc");
       e = launch_k1_tc(p, gt, m, f, s);
       if (e == cudaSuccess) e = launch_k2(p, gt, a.scan_mode, f, s, rec);
-      if (rec) rec->mark(s);
+      if (rec && !a.states_only) rec->mark(s, "k3_tc");
       if (e == cudaSuccess && !a.states_only) e = launch_k3_tc(p, gt, m, f, s);
     }
   } else {
-    if (rec) rec->mark(s);
+    if (rec) rec->mark(s, "k1_fma");
     e = launch_k1_fma(p, gt, a.k, a.v, a.dtype, f, s);
     if (e == cudaSuccess) e = launch_k2(p, gt, a.scan_mode, f, s, rec);
-    if (rec) rec->mark(s);
+    if (rec && !a.states_only) rec->mark(s, "k3_fma");
     if (e == cudaSuccess && !a.states_only)
       e = launch_k3_fma(p, gt, a.q, a.k, a.v, a.out, a.dtype, f, s);
   }
-  if (rec) rec->mark(s);
+  if (rec) rec->mark(s);  // end of the last kernel (an unnamed mark)
   if (owned) {
     cudaError_t e2 = cudaFreeAsync(ws, s);
     if (e == cudaSuccess) e = e2;
@@ -431,7 +431,15 @@ HostLayout host_layout(const la_prefill_args& a) {
 
 }  // namespace
 
-int prefill_with_args(const la_prefill_args& a) { return prefill(a); }
+int prefill_with_args(const la_prefill_args& a, Recorder* rec) { return prefill(a, rec); }
+
+int check_prefill_args(const la_prefill_args& a) {
+  Path path;
+  const int st = validate(a, &path);
+  if (st != LA_OK) return st;
+  GammaTable gt;
+  return check_gamma(a.gamma, a.H, &gt);
+}
 
 }  // namespace la
 

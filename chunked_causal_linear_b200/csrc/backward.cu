@@ -1,0 +1,583 @@
+// Backward pass of the unnormalised form: the gradients of "Linear Attention and Retentive
+// Networks ..." (B. Recurrent Representation, with S_{-1} = S_init) written as three
+// causal linear attentions, each computed by the library's own prefill.
+//
+// With G_t = dL/dS_t (G_t = psi(q_t) do_t^T + gamma G_{t+1}, G_{T-1} holding dS_final):
+//   dpsi(q)_t = S_t do_t       = sum_{s<=t} gamma^(t-s) (do_t . v_s) psi(k_s)
+//                                + gamma^(t+1) S_init^T-readout
+//       -> the prefill of (q', k', v') = (do, v, psi(k)) with the identity map and
+//          S'_init = S_init^T;
+//   dv_s        = G_s^T psi(k_s) = sum_{t>=s} gamma^(t-s) (psi(k_s) . psi(q_t)) do_t
+//                                  + gamma^(T-1-s) dS_final^T psi(k_s)
+//       -> on the time-reversed sequence (sigma = T-1-s) the prefill of (k, q, do) with
+//          the model's map, S'_init = dS_final / gamma (its readout weight gamma^(sigma+1)
+//          then gives gamma^sigma); its final state is G_0;
+//   dpsi(k)_s   = G_s v_s      -> reversed, the prefill of (v, do, psi(q)) with the
+//          identity map and S'_init = dS_final^T / gamma;
+//   dS_init     = gamma G_0.
+// The element-wise kernels here reverse time, apply psi and psi', and fold in the
+// dS_final terms of heads whose decay is too small to divide by.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/linattn.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace la {
+namespace {
+
+// Heads with gamma below this take the dS_final terms from fix_small_decay (terms
+// gamma^sigma, sigma >= 3, are below 2^-60 of the sigma = 0 term and are dropped).
+constexpr float kSmallDecay = 0x1p-20f;
+constexpr int kSmallDecayTerms = 3;
+constexpr int kMaxJobs = 8;
+
+__device__ __forceinline__ float psi(float x, int fm) {
+  return fm == LA_FM_ELU1 ? (x > 0.f ? x + 1.f : expf(x)) : x;
+}
+__device__ __forceinline__ float psi_prime(float x, int fm) {
+  return fm == LA_FM_ELU1 ? (x > 0.f ? 1.f : expf(x)) : 1.f;
+}
+
+// Four consecutive elements of a bf16 or float32 row.
+__device__ __forceinline__ float4 load4(const void* base, long long idx, bool f32) {
+  if (f32) return __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx));
+  const uint2 u = __ldcs(reinterpret_cast<const uint2*>(
+      static_cast<const __nv_bfloat16*>(base) + idx));
+  __nv_bfloat162 a, b;
+  std::memcpy(&a, &u.x, 4);
+  std::memcpy(&b, &u.y, 4);
+  const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+__device__ __forceinline__ void store4(void* base, long long idx, float4 x, bool f32) {
+  if (f32) {
+    __stcs(reinterpret_cast<float4*>(static_cast<float*>(base) + idx), x);
+    return;
+  }
+  const __nv_bfloat162 a = __float22bfloat162_rn(make_float2(x.x, x.y));
+  const __nv_bfloat162 b = __float22bfloat162_rn(make_float2(x.z, x.w));
+  uint2 u;
+  std::memcpy(&u.x, &a, 4);
+  std::memcpy(&u.y, &b, 4);
+  __stcs(reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + idx), u);
+}
+
+// dst[bh, t'] = f(src[bh, t] + src2[bh, t]) * g(x[bh, t']) for rows of d elements, where
+// t' = T-1-t when `flip`, else t; f = psi when `fm_src` is ELU+1, g = psi' of x when `x` is
+// given.  With `lo`, dst receives the part of the value that bf16 rounding drops
+// (value - bf16(value), itself rounded to bf16): a bf16 hi + lo pair carries psi to about
+// 16 bits, like the split operands of the prefill's own kernels.
+struct RowJob {
+  const void* src;
+  const void* src2;  // added to src (same type), or nullptr
+  void* dst;
+  const void* x;     // multiplier input (same layout as dst, type of the inputs) or nullptr
+  int d;
+  int fm_src;        // la_feature_map applied to src
+  int fm_x;          // la_feature_map whose derivative multiplies by x
+  bool flip, lo;
+  bool src_f32, dst_f32, x_f32;
+};
+struct RowJobs {
+  RowJob j[kMaxJobs];
+};
+
+// One 4-element group per thread and grid-stride loop; blockIdx.y selects the job.
+__global__ void __launch_bounds__(256) row_jobs(RowJobs jobs, long long BH, long long T) {
+  const RowJob& J = jobs.j[blockIdx.y];
+  const long long gpr = J.d / 4;  // groups per row
+  const long long n = BH * T * gpr;
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = g / gpr, col = (g - row * gpr) * 4;
+    const long long bh = row / T, t = row - bh * T;
+    const long long drow = J.flip ? bh * T + (T - 1 - t) : row;
+    float4 a = load4(J.src, row * J.d + col, J.src_f32);
+    if (J.src2) {
+      const float4 b = load4(J.src2, row * J.d + col, J.src_f32);
+      a = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    }
+    if (J.fm_src == LA_FM_ELU1)
+      a = make_float4(psi(a.x, 1), psi(a.y, 1), psi(a.z, 1), psi(a.w, 1));
+    if (J.lo) {
+      auto rest = [](float v) { return v - __bfloat162float(__float2bfloat16_rn(v)); };
+      a = make_float4(rest(a.x), rest(a.y), rest(a.z), rest(a.w));
+    }
+    if (J.x && J.fm_x == LA_FM_ELU1) {
+      const float4 x = load4(J.x, drow * J.d + col, J.x_f32);
+      a = make_float4(a.x * psi_prime(x.x, 1), a.y * psi_prime(x.y, 1),
+                      a.z * psi_prime(x.z, 1), a.w * psi_prime(x.w, 1));
+    }
+    store4(J.dst, drow * J.d + col, a, J.dst_f32);
+  }
+}
+
+// dst[bh] = scale_h * (transpose ? src[bh]^T : src[bh]) for [rows x cols] float32
+// matrices (dst is rows x cols; src is cols x rows when transposing).  scale_h is 1 / gamma_h
+// (0 for heads below kSmallDecay) when `inverse_decay`, else 1.
+__global__ void prep_state(const float* __restrict__ src, float* __restrict__ dst, int rows,
+                           int cols, bool transpose, bool inverse_decay, int H, long long n,
+                           GammaTable gt) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const long long per = static_cast<long long>(rows) * cols;
+  const long long bh = idx / per;
+  const int e = static_cast<int>(idx - bh * per), r = e / cols, c = e - r * cols;
+  float s = 1.f;
+  if (inverse_decay) {
+    const float g = gt.g[bh % H];
+    s = g >= kSmallDecay ? 1.f / g : 0.f;
+  }
+  dst[idx] = s * src[bh * per + (transpose ? static_cast<long long>(c) * rows + r : e)];
+}
+
+// dS_init = gamma_h * G_0 (+ gamma_h^T dS_final for heads below kSmallDecay, whose G_0 lacks
+// the dS_final term), in place on G_0.
+__global__ void finish_state(float* __restrict__ G0, const float* __restrict__ dS_final, int per,
+                             int H, long long n, long long T, GammaTable gt) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const float g = gt.g[(idx / per) % H];
+  float x = g * G0[idx];
+  if (dS_final && g < kSmallDecay) {
+    // gamma^T with T >= 1; for gamma = 0 only T = 0 would survive, and T = 0 never runs.
+    const float gT = T == 1 ? g : (g == 0.f ? 0.f : exp2f(static_cast<float>(T) * log2f(g)));
+    x = fmaf(gT, dS_final[idx], x);
+  }
+  G0[idx] = x;
+}
+
+// For heads below kSmallDecay: the terms gamma^sigma dS_final v and gamma^sigma
+// dS_final^T psi(k) of the reversed rows sigma < 3, added to the float32 outputs of the
+// reversed passes (Wk: dpsi(k) reversed [T, dk]; Wv: dv reversed [T, dv]).  One block per
+// (b, h); threads cover the dk + dv output columns.
+__global__ void fix_small_decay(const float* __restrict__ dS_final, const void* k,
+                                const void* v, float* __restrict__ Wk, float* __restrict__ Wv,
+                                int dk, int dv, int H, long long T, int fm, bool in_f32,
+                                GammaTable gt) {
+  const long long bh = blockIdx.x;
+  const float g = gt.g[bh % H];
+  if (g >= kSmallDecay) return;
+  const float* dS = dS_final + bh * dk * dv;
+  float w = 1.f;
+  for (int sg = 0; sg < kSmallDecayTerms && sg < T; ++sg) {
+    const long long t = bh * T + (T - 1 - sg);  // the original row of reversed row sg
+    for (int c = threadIdx.x; c < dk + dv; c += blockDim.x) {
+      float acc = 0.f;
+      if (c < dk) {  // (dS v_t)_c
+        for (int j = 0; j < dv; ++j) {
+          const long long e = t * dv + j;
+          const float vj = in_f32 ? static_cast<const float*>(v)[e]
+                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(v)[e]);
+          acc = fmaf(dS[c * dv + j], vj, acc);
+        }
+        Wk[(bh * T + sg) * dk + c] += w * acc;
+      } else {  // (dS^T psi(k_t))_j
+        const int j = c - dk;
+        for (int i = 0; i < dk; ++i) {
+          const long long e = t * dk + i;
+          const float ki = in_f32 ? static_cast<const float*>(k)[e]
+                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(k)[e]);
+          acc = fmaf(dS[i * dv + j], psi(ki, fm), acc);
+        }
+        Wv[(bh * T + sg) * dv + j] += w * acc;
+      }
+    }
+    w *= g;
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  if (!a || !b || an == 0 || bn == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+bool has_small_decay(const la_backward_args& a) {
+  if (!a.gamma || !a.grad_S_final) return false;
+  for (int h = 0; h < a.H; ++h)
+    if (a.gamma[h] < kSmallDecay) return true;
+  return false;
+}
+
+// Workspace of one backward call.  Reversed copies of the inputs (type `dtype`): kr, qr
+// [T, dk], dor, vr [T, dv]; for ELU+1 also psi(q) reversed and psi(k) in order [T, dk],
+// each with its bf16 residual (the lo half) when the inputs are bf16.  The reversed passes'
+// outputs Wk [T, dk], Wv [T, dv] (float32 when they are multiplied by psi' or corrected,
+// else the output type); for ELU+1 the grad_q pass's float32 output Wq [T, dk], and the
+// float32 outputs of the lo passes.  Three [dk x dv] states per (b, h), then the prefill
+// workspace.
+struct BwdLayout {
+  size_t kr, qr, dor, vr, pqr, pk, pqr_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC, pw, total;
+  bool w_f32, elu, split;
+};
+
+BwdLayout bwd_layout(const la_backward_args& a) {
+  BwdLayout l{};
+  const size_t BH = static_cast<size_t>(a.B > 0 ? a.B : 0) * (a.H > 0 ? a.H : 0);
+  const size_t T = static_cast<size_t>(a.T > 0 ? a.T : 0);
+  const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
+  const bool out_f32 = a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32;
+  l.elu = a.feature_map == LA_FM_ELU1;
+  l.split = l.elu && a.dtype == LA_DTYPE_BF16;
+  l.w_f32 = out_f32 || l.elu || has_small_decay(a);
+  const size_t ew = l.w_f32 ? 4 : 2;
+  const size_t nk = BH * T * a.dk, nv = BH * T * a.dv, ns = BH * a.dk * a.dv * 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  l.kr = take(nk * e);
+  l.qr = take(nk * e);
+  l.dor = take(nv * e);
+  l.vr = take(nv * e);
+  l.pqr = take(l.elu ? nk * e : 0);
+  l.pk = take(l.elu ? nk * e : 0);
+  l.pqr_lo = take(l.split ? nk * e : 0);
+  l.pk_lo = take(l.split ? nk * e : 0);
+  l.Wk = take(nk * ew);
+  l.Wv = take(nv * ew);
+  l.Wq = take(l.elu ? nk * 4 : 0);
+  l.Wk_lo = take(l.split ? nk * 4 : 0);
+  l.Wq_lo = take(l.split ? nk * 4 : 0);
+  l.SA = take(a.S_init ? ns : 0);
+  l.SB = take(a.grad_S_final ? ns : 0);
+  l.SC = take(a.grad_S_final ? ns : 0);
+  l.pw = off;
+  off += lin_attn_prefill_workspace_bytes(a.B, a.H, a.T, a.dk, a.dv, a.C, 0);
+  l.total = off;
+  return l;
+}
+
+// The prefill arguments of one pass; q, k, v, out and the states are filled in by the
+// caller.
+la_prefill_args pass_args(const la_backward_args& a, int dk, int dv, int fm, int out_dtype) {
+  la_prefill_args p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = a.B;
+  p.H = a.H;
+  p.T = a.T;
+  p.dk = dk;
+  p.dv = dv;
+  p.C = a.C;
+  p.feature_map = fm;
+  p.gamma = a.gamma;
+  p.normalize = 0;
+  p.eps = 0.f;
+  p.dtype = a.dtype;
+  p.out_dtype = out_dtype;
+  p.scan_mode = a.scan_mode;
+  p.kernel_path = a.kernel_path;
+  p.algorithm = a.algorithm;
+  p.segment_chunks = a.segment_chunks;
+  p.stream = a.stream;
+  return p;
+}
+
+int validate(const la_backward_args& a) {
+  if (a.B < 0 || a.H < 0 || a.T < 0 || a.dk <= 0 || a.dv <= 0 || a.C <= 0)
+    return LA_ERR_INVALID_ARGUMENT;
+  if (a.dtype != LA_DTYPE_BF16 && a.dtype != LA_DTYPE_F32) return LA_ERR_INVALID_ARGUMENT;
+  if (a.out_dtype != LA_OUT_AS_INPUT && a.out_dtype != LA_OUT_F32) return LA_ERR_INVALID_ARGUMENT;
+  if (a.feature_map != LA_FM_IDENTITY && a.feature_map != LA_FM_ELU1) return LA_ERR_INVALID_ARGUMENT;
+  if (a.gamma && a.H > kMaxHeads) return LA_ERR_UNSUPPORTED;
+  if (a.gamma)
+    for (int h = 0; h < a.H; ++h)
+      if (!(a.gamma[h] >= 0.f && a.gamma[h] <= 1.f)) return LA_ERR_INVALID_ARGUMENT;
+  if (a.workspace && (reinterpret_cast<uintptr_t>(a.workspace) & 255u) != 0)
+    return LA_ERR_INVALID_ARGUMENT;
+  for (const void* p : {static_cast<const void*>(a.S_init), static_cast<const void*>(a.grad_S_final),
+                        static_cast<const void*>(a.grad_S_init)})
+    if (!aligned16(p)) return LA_ERR_INVALID_ARGUMENT;
+  // The three passes' shapes and options, checked as the prefill will check them (as
+  // states-only calls, so that no output buffer is needed; q stands for every input).
+  const long long BH = static_cast<long long>(a.B) * a.H;
+  const bool empty = BH == 0 || a.T == 0;
+  const int fms[3] = {LA_FM_IDENTITY, a.feature_map, LA_FM_IDENTITY};
+  const int dks[3] = {a.dv, a.dk, a.dv}, dvs[3] = {a.dk, a.dv, a.dk};
+  for (int i = 0; i < 3; ++i) {
+    la_prefill_args p = pass_args(a, dks[i], dvs[i], fms[i], LA_OUT_F32);
+    p.q = p.k = p.v = empty ? nullptr : a.q;
+    p.states_only = 1;
+    const int st = check_prefill_args(p);
+    if (st != LA_OK) return st;
+  }
+  if (!empty) {
+    const void* in[4] = {a.q, a.k, a.v, a.grad_out};
+    void* out[3] = {a.grad_q, a.grad_k, a.grad_v};
+    for (const void* p : in)
+      if (!p || !aligned16(p)) return LA_ERR_INVALID_ARGUMENT;
+    for (const void* p : out)
+      if (!p || !aligned16(p)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
+    const size_t eo = (a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32) ? 4 : 2;
+    const size_t nk = static_cast<size_t>(BH) * a.T * a.dk, nv = static_cast<size_t>(BH) * a.T * a.dv;
+    const size_t in_n[4] = {nk * e, nk * e, nv * e, nv * e};
+    const size_t out_n[3] = {nk * eo, nk * eo, nv * eo};
+    for (int o = 0; o < 3; ++o) {
+      for (int i = 0; i < 4; ++i)
+        if (overlaps(out[o], out_n[o], in[i], in_n[i])) return LA_ERR_INVALID_ARGUMENT;
+      for (int o2 = o + 1; o2 < 3; ++o2)
+        if (overlaps(out[o], out_n[o], out[o2], out_n[o2])) return LA_ERR_INVALID_ARGUMENT;
+    }
+  }
+  return LA_OK;
+}
+
+cudaError_t launch_rows(const RowJobs& jobs, int n, long long BH, long long T, cudaStream_t s,
+                        Recorder* rec, const char* name) {
+  if (n == 0) return cudaSuccess;
+  // Enough 256-thread blocks to fill every SM several times over; each thread then walks
+  // its share with a grid stride.
+  long long groups = 0;
+  for (int i = 0; i < n; ++i) groups = std::max(groups, BH * T * (jobs.j[i].d / 4));
+  long long blocks = (groups + 255) / 256;
+  blocks = std::min<long long>(blocks, 148LL * 8);
+  if (blocks < 1) blocks = 1;
+  if (rec) rec->mark(s, name);
+  row_jobs<<<dim3(static_cast<unsigned>(blocks), n), 256, 0, s>>>(jobs, BH, T);
+  return cudaGetLastError();
+}
+
+int backward(const la_backward_args& a, Recorder* rec = nullptr) {
+  int st = validate(a);
+  if (st != LA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(a.stream);
+  const long long BH = static_cast<long long>(a.B) * a.H;
+  if (BH == 0) return LA_OK;
+  const size_t state_bytes = static_cast<size_t>(BH) * a.dk * a.dv * 4;
+  if (a.T == 0) {
+    // No tokens: S_final = S_init, so dS_init = dS_final.
+    if (!a.grad_S_init) return LA_OK;
+    cudaError_t e = a.grad_S_final
+                        ? cudaMemcpyAsync(a.grad_S_init, a.grad_S_final, state_bytes,
+                                          cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(a.grad_S_init, 0, state_bytes, s);
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+
+  GammaTable gt;
+  for (int h = 0; h < kMaxHeads; ++h) gt.g[h] = 1.f;
+  if (a.gamma)
+    for (int h = 0; h < a.H; ++h) gt.g[h] = a.gamma[h];
+
+  const BwdLayout l = bwd_layout(a);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  bool owned = false;
+  if (ws) {
+    if (a.workspace_bytes < l.total) return LA_ERR_INVALID_ARGUMENT;
+  } else {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), l.total, s) != cudaSuccess) {
+      cudaGetLastError();
+      return LA_ERR_OUT_OF_MEMORY;
+    }
+    owned = true;
+  }
+  auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
+  const bool in_f32 = a.dtype == LA_DTYPE_F32;
+  const bool out_f32 = in_f32 || a.out_dtype == LA_OUT_F32;
+  const bool elu = a.feature_map == LA_FM_ELU1;
+  const int w_dtype = l.w_f32 ? LA_OUT_F32 : LA_OUT_AS_INPUT;
+  const long long T = a.T;
+
+  // Reversed inputs (psi(q) reversed and psi(k) in order for ELU+1, as hi / lo pairs for
+  // bf16 inputs).
+  auto job = [](RowJobs& J, int& n, const void* src, const void* src2, void* dst, const void* x,
+                int d, int fm_src, int fm_x, bool flip, bool lo, bool sf, bool df, bool xf) {
+    J.j[n++] = RowJob{src, src2, dst, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
+  };
+  RowJobs pre{};
+  int np = 0;
+  const bool f = in_f32;
+  job(pre, np, a.k, nullptr, at(l.kr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
+  job(pre, np, a.q, nullptr, at(l.qr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
+  job(pre, np, a.grad_out, nullptr, at(l.dor), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f,
+      f, f);
+  job(pre, np, a.v, nullptr, at(l.vr), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f, f, f);
+  if (elu) {
+    job(pre, np, a.q, nullptr, at(l.pqr), nullptr, a.dk, LA_FM_ELU1, 0, true, false, f, f, f);
+    job(pre, np, a.k, nullptr, at(l.pk), nullptr, a.dk, LA_FM_ELU1, 0, false, false, f, f, f);
+  }
+  if (l.split) {
+    job(pre, np, a.q, nullptr, at(l.pqr_lo), nullptr, a.dk, LA_FM_ELU1, 0, true, true, f, f, f);
+    job(pre, np, a.k, nullptr, at(l.pk_lo), nullptr, a.dk, LA_FM_ELU1, 0, false, true, f, f, f);
+  }
+  cudaError_t e = launch_rows(pre, np, BH, T, s, rec, "bwd_reverse_inputs");
+
+  // Initial states of the three passes.
+  float* SA = a.S_init ? static_cast<float*>(at(l.SA)) : nullptr;
+  float* SB = a.grad_S_final ? static_cast<float*>(at(l.SB)) : nullptr;
+  float* SC = a.grad_S_final ? static_cast<float*>(at(l.SC)) : nullptr;
+  const long long ns = BH * a.dk * a.dv;
+  const unsigned sblocks = static_cast<unsigned>((ns + 255) / 256);
+  if (rec && (SA || SB)) rec->mark(s, "bwd_prep_states");
+  if (e == cudaSuccess && SA) {
+    prep_state<<<sblocks, 256, 0, s>>>(a.S_init, SA, a.dv, a.dk, true, false, a.H, ns, gt);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && SB) {
+    prep_state<<<sblocks, 256, 0, s>>>(a.grad_S_final, SB, a.dk, a.dv, false, a.gamma != nullptr,
+                                       a.H, ns, gt);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && SC) {
+    prep_state<<<sblocks, 256, 0, s>>>(a.grad_S_final, SC, a.dv, a.dk, true, a.gamma != nullptr,
+                                       a.H, ns, gt);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) st = LA_ERR_CUDA;
+
+  auto run = [&](la_prefill_args p) {
+    if (st != LA_OK) return;
+    p.workspace = at(l.pw);
+    p.workspace_bytes = l.total - l.pw;
+    const int r = prefill_with_args(p, rec);
+    if (r != LA_OK) st = r == LA_ERR_INVALID_ARGUMENT || r == LA_ERR_UNSUPPORTED ? LA_ERR_INTERNAL : r;
+  };
+  // grad_q (or, for ELU+1, dpsi(q) in float32): (do, v, psi(k)) in order, identity map;
+  // linear in psi(k), so the lo half of a split psi(k) is a second pass from a zero state.
+  {
+    la_prefill_args p = pass_args(a, a.dv, a.dk, LA_FM_IDENTITY, elu ? LA_OUT_F32 : a.out_dtype);
+    p.q = a.grad_out;
+    p.k = a.v;
+    p.v = elu ? at(l.pk) : a.k;
+    p.out = elu ? at(l.Wq) : a.grad_q;
+    p.S_init = SA;
+    run(p);
+    if (l.split) {
+      p.v = at(l.pk_lo);
+      p.out = at(l.Wq_lo);
+      p.S_init = nullptr;
+      run(p);
+    }
+  }
+  // grad_v reversed: (k, q, do) reversed with the model's map; final state G_0.
+  {
+    la_prefill_args p = pass_args(a, a.dk, a.dv, a.feature_map, w_dtype);
+    p.q = at(l.kr);
+    p.k = at(l.qr);
+    p.v = at(l.dor);
+    p.out = at(l.Wv);
+    p.S_init = SB;
+    p.S_final = a.grad_S_init;
+    run(p);
+  }
+  // dpsi(k) reversed: (v, do, psi(q)) reversed, identity map (lo half as for grad_q).
+  {
+    la_prefill_args p = pass_args(a, a.dv, a.dk, LA_FM_IDENTITY, w_dtype);
+    p.q = at(l.vr);
+    p.k = at(l.dor);
+    p.v = elu ? at(l.pqr) : at(l.qr);
+    p.out = at(l.Wk);
+    p.S_init = SC;
+    run(p);
+    if (l.split) {
+      p.v = at(l.pqr_lo);
+      p.out = at(l.Wk_lo);
+      p.S_init = nullptr;
+      run(p);
+    }
+  }
+  e = cudaSuccess;
+  if (st == LA_OK && has_small_decay(a)) {
+    if (rec) rec->mark(s, "bwd_fix_small_decay");
+    fix_small_decay<<<static_cast<unsigned>(BH), 128, 0, s>>>(
+        a.grad_S_final, a.k, a.v, static_cast<float*>(at(l.Wk)), static_cast<float*>(at(l.Wv)),
+        a.dk, a.dv, a.H, T, a.feature_map, in_f32, gt);
+    e = cudaGetLastError();
+  }
+  if (st == LA_OK && e == cudaSuccess && a.grad_S_init && a.gamma) {
+    if (rec) rec->mark(s, "bwd_finish_state");
+    finish_state<<<sblocks, 256, 0, s>>>(a.grad_S_init, a.grad_S_final, a.dk * a.dv, a.H, ns, T,
+                                         gt);
+    e = cudaGetLastError();
+  }
+  // Back to forward time, with psi' where the map has one.
+  if (st == LA_OK && e == cudaSuccess) {
+    RowJobs post{};
+    int n = 0;
+    const bool wf = l.w_f32;
+    job(post, n, at(l.Wv), nullptr, a.grad_v, nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, wf,
+        out_f32, f);
+    job(post, n, at(l.Wk), l.split ? at(l.Wk_lo) : nullptr, a.grad_k, a.k, a.dk, LA_FM_IDENTITY,
+        a.feature_map, true, false, wf, out_f32, f);
+    if (elu)  // grad_q = psi'(q) .* dpsi(q)
+      job(post, n, at(l.Wq), l.split ? at(l.Wq_lo) : nullptr, a.grad_q, a.q, a.dk,
+          LA_FM_IDENTITY, a.feature_map, false, false, true, out_f32, f);
+    e = launch_rows(post, n, BH, T, s, rec, "bwd_reverse_outputs");
+  }
+  if (rec) rec->mark(s);
+  if (e != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
+  if (owned) {
+    const cudaError_t e2 = cudaFreeAsync(ws, s);
+    if (e2 != cudaSuccess && st == LA_OK) st = LA_ERR_CUDA;
+  }
+  return st;
+}
+
+}  // namespace
+}  // namespace la
+
+extern "C" int lin_attn_backward(const la_backward_args* args) {
+  if (!args) return LA_ERR_INVALID_ARGUMENT;
+  return la::backward(*args);
+}
+
+extern "C" int lin_attn_backward_timed(const la_backward_args* args, float* kernel_ms,
+                                       const char** kernel_names, int max_kernels,
+                                       int* n_kernels) {
+  if (!args || !kernel_ms || !kernel_names || !n_kernels || max_kernels < 1)
+    return LA_ERR_INVALID_ARGUMENT;
+  *n_kernels = 0;
+  constexpr int kMaxEvents = 48;
+  cudaEvent_t ev[kMaxEvents];
+  const char* label[kMaxEvents] = {nullptr};
+  int created = 0;
+  for (; created < kMaxEvents; ++created)
+    if (cudaEventCreate(&ev[created]) != cudaSuccess) break;
+  if (created < kMaxEvents) {
+    for (int i = 0; i < created; ++i) cudaEventDestroy(ev[i]);
+    return LA_ERR_CUDA;
+  }
+  la::Recorder rec;
+  rec.ev = ev;
+  rec.label = label;
+  rec.cap = kMaxEvents;
+  int st = la::backward(*args, &rec);
+  if (st == LA_OK && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(args->stream)) !=
+                         cudaSuccess)
+    st = LA_ERR_CUDA;
+  if (st == LA_OK) {
+    int nk = 0;
+    for (int i = 0; i + 1 < rec.n && nk < max_kernels; ++i) {
+      if (!label[i]) continue;  // the gap between two passes
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, ev[i], ev[i + 1]);
+      kernel_ms[nk] = ms;
+      kernel_names[nk] = label[i];
+      ++nk;
+    }
+    *n_kernels = nk;
+  }
+  for (int i = 0; i < kMaxEvents; ++i) cudaEventDestroy(ev[i]);
+  return st;
+}
+
+extern "C" size_t lin_attn_backward_workspace_bytes(const la_backward_args* args) {
+  if (!args || args->B <= 0 || args->H <= 0 || args->T <= 0) return 0;
+  return la::bwd_layout(*args).total;
+}

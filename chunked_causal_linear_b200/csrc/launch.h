@@ -9,8 +9,8 @@
 
 namespace la {
 
-// The full prefill of lin_attn_prefill_ex (validation, workspace, launches).
-int prefill_with_args(const la_prefill_args& a);
+// The argument checks of the prefill alone: LA_OK when prefill_with_args(a) would launch.
+int check_prefill_args(const la_prefill_args& a);
 
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
 
@@ -22,15 +22,25 @@ struct Flags {
 };
 
 // Optional per-kernel timing: when set, every launcher records the next event on the
-// stream just before each of its kernel launches.
+// stream just before each of its kernel launches, labelled with the kernel's name, and the
+// prefill records an unlabelled event after its last kernel.  Interval i (event i to
+// event i + 1) is the kernel `label[i]`; an unlabelled interval holds no kernel.
 struct Recorder {
   cudaEvent_t* ev = nullptr;
+  const char** label = nullptr;
   int n = 0;
   int cap = 0;
-  void mark(cudaStream_t s) {
-    if (ev && n < cap) cudaEventRecord(ev[n++], s);
+  void mark(cudaStream_t s, const char* name = nullptr) {
+    if (ev && n < cap) {
+      if (label) label[n] = name;
+      cudaEventRecord(ev[n++], s);
+    }
   }
 };
+
+// The full prefill of lin_attn_prefill_ex (validation, workspace, launches), optionally
+// recording an event before every kernel.
+int prefill_with_args(const la_prefill_args& a, Recorder* rec = nullptr);
 
 // CUDA-core fp32 FMA kernels (any supported shape, float32 or bf16 inputs).
 cudaError_t launch_k1_fma(const PrefillParams& p, const GammaTable& gt, const void* k,

@@ -231,7 +231,7 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
   const int R4 = p.R / 4;
   const long long nblk = (R4 + kScanThreads - 1) / kScanThreads;
   if (mode == 1) {
-    if (rec) rec->mark(s);
+    if (rec) rec->mark(s, "k2_sequential");
     k2_sequential<DECAY><<<static_cast<unsigned>(nblk * p.BH), kScanThreads, 0, s>>>(p, gt);
     return cudaGetLastError();
   }
@@ -241,19 +241,19 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
     // Every segment is one element: the Hillis-Steele scan alone, in place on the records.
     PrefillParams q = p;
     q.tot = p.rec;
-    if (rec) rec->mark(s);
+    if (rec) rec->mark(s, "k2_scan_totals");
     k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(q, gt);
     return cudaGetLastError();
   }
-  if (rec) rec->mark(s);
+  if (rec) rec->mark(s, "k2_reduce");
   k2_reduce<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (rec) rec->mark(s);
+  if (rec) rec->mark(s, "k2_scan_totals");
   k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(p, gt);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (rec) rec->mark(s);
+  if (rec) rec->mark(s, "k2_downsweep");
   k2_downsweep<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);
   return cudaGetLastError();
 }

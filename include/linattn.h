@@ -267,6 +267,85 @@ int lin_attn_combine_states(const float* S_parts, const float* Z_parts, int part
 int lin_attn_prefill_noalloc(const la_prefill_args* args);
 
 /*
+ * lin_attn_backward -- gradients of the unnormalised form (o_t = psi(q_t) S_t, any decay,
+ * either feature map) for the loss L = sum(grad_out . out) + sum(grad_S_final . S_final).
+ * The scan page asks for forward and backward latency ("Log-Depth Chunked
+ * Linear-Attention Scan", Implementation notes); the gradients are those of the recurrent
+ * form of "Linear Attention and Retentive Networks ..." (B. Recurrent Representation)
+ * with S_{-1} = S_init.  With G_t = dL/dS_t accumulated backwards in time,
+ *     G_t = psi(q_t) grad_out_t^T + gamma G_{t+1},  G_{T-1} includes grad_S_final,
+ *     grad_q_t = psi'(q_t) .* (S_t grad_out_t),
+ *     grad_k_t = psi'(k_t) .* (G_t v_t),   grad_v_t = G_t^T psi(k_t),
+ *     grad_S_init = gamma G_0.
+ * Each sum is itself a causal linear attention, so the library computes them with three
+ * prefills (all their kernels, on the same workspace):
+ *   grad_q  the prefill of (q, k, v) = (grad_out, v, psi(k)) under the identity map,
+ *           started from S_init^T;
+ *   grad_v  the prefill of (psi: k, q, grad_out) on the time-reversed sequence, started
+ *           from grad_S_final / gamma (its final state is G_0);
+ *   grad_k  the prefill of (v, grad_out, psi(q)) under the identity map on the
+ *           time-reversed sequence, started from grad_S_final^T / gamma;
+ * plus element-wise kernels that reverse time, apply psi and psi', and fold in the
+ * grad_S_final terms of heads whose decay is below 2^-20 (for those heads the division
+ * by gamma is replaced by the exact first three terms, the rest being below 2^-60).
+ * The normalised form's gradient is not provided.
+ *
+ *   q, k, v, grad_out  DEVICE, the forward's inputs and dL/dout, type `dtype`,
+ *                      [B,H,T,dk] / [B,H,T,dk] / [B,H,T,dv] / [B,H,T,dv].
+ *   grad_q, grad_k, grad_v  DEVICE outputs, the shapes of q, k, v, type per out_dtype;
+ *                      must not overlap any input or each other.
+ *   S_init             DEVICE float32 [B,H,dk,dv], the forward's initial state, or NULL.
+ *   grad_S_final       DEVICE float32 [B,H,dk,dv] or NULL (zero).
+ *   grad_S_init        DEVICE float32 [B,H,dk,dv] output, or NULL (not computed).
+ *   The other fields as in la_prefill_args; every pass uses `algorithm`, `kernel_path`,
+ *   `scan_mode` and `segment_chunks`.  Supported shapes: those of the prefill for both
+ *   (dk, dv) and (dv, dk).  Workspace: lin_attn_backward_workspace_bytes(), or NULL to
+ *   allocate on the stream.  Asynchronous; arguments are checked before any launch.
+ */
+typedef struct la_backward_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* grad_out;
+  void* grad_q;
+  void* grad_k;
+  void* grad_v;
+  const float* S_init;        /* may be NULL */
+  const float* grad_S_final;  /* may be NULL */
+  float* grad_S_init;         /* may be NULL */
+  int B, H;
+  long long T;
+  int dk, dv, C;
+  int feature_map;            /* la_feature_map */
+  const float* gamma;         /* HOST, H values, or NULL */
+  int dtype;                  /* la_dtype of q, k, v, grad_out */
+  int out_dtype;              /* la_out_dtype of grad_q, grad_k, grad_v */
+  int scan_mode;
+  int kernel_path;
+  int algorithm;
+  int segment_chunks;
+  void* workspace;            /* DEVICE, 256-byte aligned, or NULL */
+  size_t workspace_bytes;
+  la_stream_t stream;
+} la_backward_args;
+
+int lin_attn_backward(const la_backward_args* args);
+
+/* lin_attn_backward_timed -- lin_attn_backward with a CUDA event recorded before every
+ * kernel (or group of small kernels) and after the last; synchronises the stream and
+ * writes each one's device duration (milliseconds, launch order) to kernel_ms[0 ..] and
+ * its name to kernel_names[0 ..] (static strings owned by the library: the prefill
+ * kernels' names, "bwd_reverse_inputs", "bwd_prep_states", "bwd_fix_small_decay",
+ * "bwd_finish_state", "bwd_reverse_outputs").  *n_kernels receives the count.  For
+ * profiling; the results are identical to lin_attn_backward. */
+int lin_attn_backward_timed(const la_backward_args* args, float* kernel_ms,
+                            const char** kernel_names, int max_kernels, int* n_kernels);
+
+/* Device workspace of lin_attn_backward for these arguments (the reversed copies of the
+ * inputs, the passes' float32 outputs, the prefill workspace).  Pure host computation. */
+size_t lin_attn_backward_workspace_bytes(const la_backward_args* args);
+
+/*
  * lin_attn_decode_step -- one recurrent step for every (b, h), the O(1) decode that the
  * prefill's final states feed ("The Recurrent Dual"; "B. Recurrent Representation").
  *   q, k      DEVICE bf16 [B,H,dk]   v DEVICE bf16 [B,H,dv]   out DEVICE bf16 [B,H,dv]

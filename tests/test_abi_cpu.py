@@ -179,3 +179,70 @@ def test_combine_states_argument_errors(lib):
     neg = (ctypes.c_longlong * 3)(10, -1, 30)
     assert f(S, None, 3, 1, neg, 1, 2, 64, 64, g_ok, O, None, None) == 1
     assert f(S, None, 3, 1, toks, 0, 2, 64, 64, g_ok, O, None, None) == 0   # empty
+
+
+def _bwd_args(**kw):
+    from chunked_causal_linear_b200.binding import BackwardArgs
+    a = BackwardArgs()
+    base = dict(q=0x1000, k=0x2000000, v=0x4000000, grad_out=0x6000000, grad_q=0x8000000,
+                grad_k=0xA000000, grad_v=0xC000000, B=1, H=2, T=128, dk=64, dv=64, C=64,
+                feature_map=0, dtype=0, out_dtype=0, scan_mode=0, kernel_path=0)
+    base.update(kw)
+    for key, val in base.items():
+        setattr(a, key, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(dtype=7), 1), (dict(feature_map=3), 1), (dict(out_dtype=5), 1),
+    (dict(scan_mode=4), 1), (dict(algorithm=9), 1),
+    (dict(dk=5), 2), (dict(dv=256), 2), (dict(C=48), 2), (dict(kernel_path=1, dtype=1), 2),
+    (dict(algorithm=2), 2),  # dv = 64: no pass can take the segmented algorithm
+    (dict(q=0), 1), (dict(grad_out=0), 1), (dict(grad_q=0), 1), (dict(grad_v=0), 1),
+    (dict(q=0x1008), 1), (dict(grad_k=0x8000008), 1),
+    (dict(grad_q=0x1000), 1),                       # grad_q is q
+    (dict(grad_v=0x6000000 + 256), 1),              # grad_v inside grad_out
+    (dict(grad_k=0x8000000 + 16), 1),               # grad_k overlaps grad_q
+    (dict(S_init=0x100004), 1), (dict(grad_S_final=0x100008), 1),
+    (dict(grad_S_init=0x100002), 1), (dict(workspace=0x100010), 1),
+])
+def test_backward_argument_errors_before_any_launch(lib, kw, status):
+    a = _bwd_args(**kw)
+    assert lib.lin_attn_backward(ctypes.byref(a)) == status
+
+
+def test_backward_gamma_and_empty_problems(lib):
+    assert lib.lin_attn_backward(None) == 1
+    for kw in (dict(B=0), dict(H=0)):
+        assert lib.lin_attn_backward(ctypes.byref(_bwd_args(**kw))) == 0
+    a = _bwd_args(B=0)
+    for bad in ([0.5, 1.5], [-0.1, 0.5], [float("nan"), 0.5]):
+        arr = (ctypes.c_float * 2)(*bad)
+        a.gamma = ctypes.cast(arr, ctypes.c_void_p)
+        assert lib.lin_attn_backward(ctypes.byref(a)) == 1
+    # the ELU+1 map with a decay has no segmented pass
+    arr = (ctypes.c_float * 2)(0.5, 0.9)
+    a = _bwd_args(dk=128, dv=128, feature_map=1, algorithm=2)
+    a.gamma = ctypes.cast(arr, ctypes.c_void_p)
+    assert lib.lin_attn_backward(ctypes.byref(a)) == 2
+
+
+def test_backward_workspace_bytes(lib):
+    import torch
+    from chunked_causal_linear_b200 import binding as B
+    q = torch.empty(2, 3, 100, 64, dtype=torch.bfloat16)
+    v = torch.empty(2, 3, 100, 128, dtype=torch.bfloat16)
+    pw = B.lin_attn_prefill_workspace_bytes(2, 3, 100, 64, 128, 64, False)
+    al = lambda x: (x + 255) // 256 * 256
+    n_k, n_v = 2 * 3 * 100 * 64, 2 * 3 * 100 * 128
+    # identity map, bf16 out: four reversed inputs, two bf16 reversed outputs
+    want = 2 * al(n_k * 2) + 2 * al(n_v * 2) + al(n_k * 2) + al(n_v * 2) + pw
+    assert B.lin_attn_backward_workspace_bytes(q, v) == want
+    # ELU+1: psi(q) reversed and psi(k) with their bf16 residuals, float32 reversed
+    # outputs, the float32 grad_q precursor, the lo passes' outputs, and the two states of
+    # grad_S_final
+    ns = al(2 * 3 * 64 * 128 * 4)
+    want = (6 * al(n_k * 2) + 2 * al(n_v * 2) + al(n_k * 4) + al(n_v * 4) + al(n_k * 4)
+            + 2 * al(n_k * 4) + 2 * ns + pw)
+    assert B.lin_attn_backward_workspace_bytes(q, v, feature_map="elu1", grad_S_final=True) == want
+    assert B.lin_attn_backward_workspace_bytes(q[:, :, :0], v[:, :, :0]) == 0
