@@ -468,36 +468,50 @@ class BackwardOracleTimer(OracleTimer):
                 f"{self.last_s:.1f} s per run on {self.threads} threads")
 
 
-def backward_bytes(w, out_elem: int, algo_of, lseg: int = 0):
+def backward_native(w, algorithm: str) -> bool:
+    """Whether the library runs the backward's two reversed passes as reverse-mode
+    prefills (bf16, C = 64, dk = dv = 128, not the chunked algorithm, not ELU+1 with decay)
+    rather than on reversed copies."""
+    return (w.dtype == "bf16" and w.C == 64 and w.dk == 128 and w.dv == 128
+            and algorithm != "chunked" and not (w.feature_map == "elu1" and w.decay))
+
+
+def backward_bytes(w, out_elem: int, algorithm: str, lseg: int = 0):
     """Algorithmic bytes per launch of every kernel of the backward, in launch order, for
-    the bench's call (no initial or final state): the reversal of the inputs, three
-    prefills -- (do, v, psi(k)), reversed (k, q, do), reversed (v, do, psi(q)); two more
-    for the lo halves of psi under ELU+1 with bf16 inputs -- and the reversal of the
-    outputs."""
+    the bench's call (no initial or final state): the input preparation (reversed copies,
+    psi), three prefills -- (do, v, psi(k)), reversed (k, q, do), reversed (v, do, psi(q));
+    two more for the lo halves of psi under ELU+1 with bf16 inputs -- and the output
+    finish (reversal back, psi')."""
     BH = w.B * w.H
     e = 2 if w.dtype == "bf16" else 4
     elu = w.feature_map == "elu1"
     split = elu and w.dtype == "bf16"
-    w_f32 = out_elem == 4 or elu
+    native = backward_native(w, algorithm)
+    wk, wv = (not native) or elu, not native
+    w_f32 = native or out_elem == 4 or elu
     ew = 4 if w_f32 else 2
     nk, nv = BH * w.T * w.dk, BH * w.T * w.dv
     ops = []
-    n_in = 2 * nk + 2 * nv + (2 * nk if elu else 0) + (2 * nk if split else 0)
-    ops.append(("bwd_reverse_inputs", 2 * n_in * e))
+    n_in = (0 if native else 2 * nk + 2 * nv) + (2 * nk if elu else 0) + (2 * nk if split else 0)
+    if n_in:
+        ops.append(("bwd_reverse_inputs", 2 * n_in * e))
     wa = w.with_(dk=w.dv, dv=w.dk, feature_map="identity", normalize=False)
     wb = w.with_(normalize=False)
-    passes = [(wa, 4 if elu else out_elem)] * (2 if split else 1) + [(wb, ew)] + \
-        [(wa, ew)] * (2 if split else 1)
+    passes = [(wa, 4 if elu else out_elem)] * (2 if split else 1) + \
+        [(wb, ew if wv else out_elem)] + [(wa, ew if wk else out_elem)] * (2 if split else 1)
     for pw, oe in passes:
-        algo = algo_of(pw)
+        algo = effective_algorithm(pw, algorithm)
         for name in kernel_names(pw, algo, "logdepth", lseg):
             ops.append((name, kernel_bytes(pw, name, oe, algo, lseg)))
-    post = nv * ew + nv * out_elem + nk * ew + nk * out_elem
-    if split:
-        post += nk * 4
+    post = 0
+    if wv:
+        post += nv * ew + nv * out_elem
+    if wk:
+        post += nk * ew + nk * out_elem + (nk * 4 if split else 0) + (nk * e if elu else 0)
     if elu:
-        post += nk * e + nk * 4 + (nk * 4 if split else 0) + nk * e + nk * out_elem
-    ops.append(("bwd_reverse_outputs", post))
+        post += nk * 4 + (nk * 4 if split else 0) + nk * e + nk * out_elem
+    if post:
+        ops.append(("bwd_reverse_outputs", post))
     return ops
 
 
@@ -562,8 +576,7 @@ def backward_bench(args, w, info, dev):
             tot[name] = tot.get(name, 0.0) + x / reps
             cnt[name] = cnt.get(name, 0) + 1
     per_launch = {n: tot[n] / (cnt[n] / reps) for n in tot}
-    algo_of = lambda pw: effective_algorithm(pw, args.algorithm)
-    ops = backward_bytes(w, out_elem, algo_of, args.segment_chunks)
+    ops = backward_bytes(w, out_elem, args.algorithm, args.segment_chunks)
     bytes_of = {}
     for name, nb in ops:
         bytes_of.setdefault(name, []).append(nb)
@@ -585,9 +598,11 @@ def backward_bench(args, w, info, dev):
     step_roof = {"bytes": step_bytes, "achieved_gbs": gbs(step_bytes),
                  "frac_of_measured": gbs(step_bytes) / peak, "bytes_min": min_b,
                  "frac_min_of_measured": gbs(min_b) / peak,
+                 "reversed_passes": "reverse-mode prefills" if backward_native(w, args.algorithm)
+                 else "prefills on reversed copies",
                  "note": "bytes = the sum of every kernel's algorithmic bytes (three prefills "
-                         "and the reversals); bytes_min = q, k, v, grad_out read once and the "
-                         "three gradients written once"}
+                         "and the element-wise kernels); bytes_min = q, k, v, grad_out read once "
+                         "and the three gradients written once"}
 
     # End to end: pinned host inputs copied in, the backward, the gradients copied out.
     e2e = None

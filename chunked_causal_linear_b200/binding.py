@@ -55,6 +55,7 @@ class PrefillArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
         ("S_init", ctypes.c_void_p), ("Z_init", ctypes.c_void_p), ("states_only", ctypes.c_int),
+        ("reverse", ctypes.c_int),
     ]
 
 
@@ -147,7 +148,7 @@ def _gamma_array(gamma, H):
 
 def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, normalize, eps,
               scan, kernel_path, workspace, stream, out_dtype="as_input", algorithm="auto",
-              segment_chunks=0, S_init=None, Z_init=None, states_only=False):
+              segment_chunks=0, S_init=None, Z_init=None, states_only=False, reverse=False):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     garr, gptr = _gamma_array(gamma, H)
@@ -170,6 +171,7 @@ def make_args(q, k, v, out, S_final, Z_final, *, chunk, feature_map, gamma, norm
     a.stream = stream
     a.S_init, a.Z_init = _ptr(S_init), _ptr(Z_init)
     a.states_only = int(bool(states_only))
+    a.reverse = int(bool(reverse))
     return a, garr
 
 
@@ -181,13 +183,14 @@ def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
                      feature_map="elu1", gamma=None, normalize=True, eps=0.0, scan="logdepth",
                      kernel_path="auto", workspace=None, stream=None, want_states=True,
                      out_dtype="as_input", algorithm="auto", segment_chunks=0, S_init=None,
-                     Z_init=None, states_only=False):
+                     Z_init=None, states_only=False, reverse=False):
     """Runs the prefill on device tensors q, k [B,H,T,dk], v [B,H,T,dv] (bf16 or float32).
 
     out_dtype "f32" writes a float32 output for bf16 inputs.  Allocates out / S_final /
     Z_final when not given.  S_init / Z_init: the state before token 0 (device float32,
     may be S_final / Z_final themselves).  states_only: compute the final states only (no
-    output; out stays None).  Returns (out, S_final, Z_final).
+    output; out stays None).  reverse: the anti-causal direction (token T-1 first;
+    segmented algorithm only).  Returns (out, S_final, Z_final).
     """
     B, H, T, dk = q.shape
     dv = v.shape[-1]
@@ -203,7 +206,7 @@ def lin_attn_prefill(q, k, v, out=None, S_final=None, Z_final=None, *, chunk=64,
                         kernel_path=kernel_path, workspace=workspace,
                         stream=_stream_handle(stream), out_dtype=out_dtype, algorithm=algorithm,
                         segment_chunks=segment_chunks, S_init=S_init, Z_init=Z_init,
-                        states_only=states_only)
+                        states_only=states_only, reverse=reverse)
     _check("lin_attn_prefill_ex", load_library().lin_attn_prefill_ex(ctypes.byref(a)))
     del keep
     return out, S_final, Z_final

@@ -150,6 +150,7 @@ int validate(const la_prefill_args& a, Path* path) {
   if (a.algorithm < LA_ALGO_AUTO || a.algorithm > LA_ALGO_SEGMENTED) return LA_ERR_INVALID_ARGUMENT;
   if (a.segment_chunks < 0 || a.segment_chunks > 1024) return LA_ERR_INVALID_ARGUMENT;
   if (a.states_only != 0 && a.states_only != 1) return LA_ERR_INVALID_ARGUMENT;
+  if (a.reverse != 0 && a.reverse != 1) return LA_ERR_INVALID_ARGUMENT;
   if ((reinterpret_cast<uintptr_t>(a.S_init) & 3u) || (reinterpret_cast<uintptr_t>(a.Z_init) & 3u))
     return LA_ERR_INVALID_ARGUMENT;
   if (a.normalize && a.feature_map == LA_FM_IDENTITY) return LA_ERR_INVALID_ARGUMENT;
@@ -200,6 +201,7 @@ int validate(const la_prefill_args& a, Path* path) {
   }
   if (*path == Path::kTensorCore && a.algorithm != LA_ALGO_CHUNKED && seg_ok)
     *path = Path::kSegmented;
+  if (a.reverse && !empty && *path != Path::kSegmented) return LA_ERR_UNSUPPORTED;
   return LA_OK;
 }
 
@@ -303,6 +305,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     sp.srec = reinterpret_cast<float*>(ws);
     sp.out = a.out;
     sp.has_init = p.has_init;
+    sp.reverse = a.reverse != 0;
     sp.err = p.err;
     const size_t srec_bytes = align256(static_cast<size_t>(BH) * NS * l.R * sizeof(float));
     PrefillParams ps = p;  // the scan over segments: one scan element per segment

@@ -156,13 +156,14 @@ __global__ void finish_state(float* __restrict__ G0, const float* __restrict__ d
 }
 
 // For heads below kSmallDecay: the terms gamma^sigma dS_final v and gamma^sigma
-// dS_final^T psi(k) of the reversed rows sigma < 3, added to the float32 outputs of the
-// reversed passes (Wk: dpsi(k) reversed [T, dk]; Wv: dv reversed [T, dv]).  One block per
-// (b, h); threads cover the dk + dv output columns.
+// dS_final^T psi(k) of the reversed rows sigma < 3 (tokens T-1-sigma), added to the
+// float32 outputs of the reversed passes (Wk: dpsi(k) [T, dk]; Wv: dv [T, dv]; rows in
+// reversed order unless `in_order`).  One block per (b, h); threads cover the dk + dv
+// output columns.
 __global__ void fix_small_decay(const float* __restrict__ dS_final, const void* k,
                                 const void* v, float* __restrict__ Wk, float* __restrict__ Wv,
                                 int dk, int dv, int H, long long T, int fm, bool in_f32,
-                                GammaTable gt) {
+                                bool in_order, GammaTable gt) {
   const long long bh = blockIdx.x;
   const float g = gt.g[bh % H];
   if (g >= kSmallDecay) return;
@@ -170,6 +171,7 @@ __global__ void fix_small_decay(const float* __restrict__ dS_final, const void* 
   float w = 1.f;
   for (int sg = 0; sg < kSmallDecayTerms && sg < T; ++sg) {
     const long long t = bh * T + (T - 1 - sg);  // the original row of reversed row sg
+    const long long w_row = in_order ? t : bh * T + sg;  // its row in Wk / Wv
     for (int c = threadIdx.x; c < dk + dv; c += blockDim.x) {
       float acc = 0.f;
       if (c < dk) {  // (dS v_t)_c
@@ -179,7 +181,7 @@ __global__ void fix_small_decay(const float* __restrict__ dS_final, const void* 
                                   : __bfloat162float(static_cast<const __nv_bfloat16*>(v)[e]);
           acc = fmaf(dS[c * dv + j], vj, acc);
         }
-        Wk[(bh * T + sg) * dk + c] += w * acc;
+        Wk[w_row * dk + c] += w * acc;
       } else {  // (dS^T psi(k_t))_j
         const int j = c - dk;
         for (int i = 0; i < dk; ++i) {
@@ -188,7 +190,7 @@ __global__ void fix_small_decay(const float* __restrict__ dS_final, const void* 
                                   : __bfloat162float(static_cast<const __nv_bfloat16*>(k)[e]);
           acc = fmaf(dS[i * dv + j], psi(ki, fm), acc);
         }
-        Wv[(bh * T + sg) * dv + j] += w * acc;
+        Wv[w_row * dv + j] += w * acc;
       }
     }
     w *= g;
@@ -212,16 +214,31 @@ bool has_small_decay(const la_backward_args& a) {
   return false;
 }
 
-// Workspace of one backward call.  Reversed copies of the inputs (type `dtype`): kr, qr
-// [T, dk], dor, vr [T, dv]; for ELU+1 also psi(q) reversed and psi(k) in order [T, dk],
-// each with its bf16 residual (the lo half) when the inputs are bf16.  The reversed passes'
-// outputs Wk [T, dk], Wv [T, dv] (float32 when they are multiplied by psi' or corrected,
-// else the output type); for ELU+1 the grad_q pass's float32 output Wq [T, dk], and the
-// float32 outputs of the lo passes.  Three [dk x dv] states per (b, h), then the prefill
-// workspace.
+// Whether the two reversed passes run on the segmented kernels in reverse mode (reading
+// the inputs and writing the outputs in memory order) rather than on reversed copies.  A
+// pure function of the arguments: bf16 inputs, C = 64, dk = dv = 128, a tensor-core
+// algorithm that may be segmented, and not ELU+1 with a decay (whose model-map pass has no
+// segmented kernel).
+bool native_reverse(const la_backward_args& a) {
+  return a.dtype == LA_DTYPE_BF16 && a.C == 64 && a.dk == 128 && a.dv == 128 &&
+         a.algorithm != LA_ALGO_CHUNKED && a.kernel_path != LA_PATH_FMA &&
+         !(a.feature_map == LA_FM_ELU1 && a.gamma != nullptr) && a.T < (1LL << 31);
+}
+
+// Workspace of one backward call.
+//   Reversed copies (only without native reverse), type `dtype`: kr, qr [T, dk], dor,
+//   vr [T, dv].
+//   ELU+1: psi(q) for the dpsi(k) pass (reversed without native reverse) and psi(k) in
+//   order [T, dk], each with its bf16 residual (lo) when the inputs are bf16.
+//   Outputs of the reversed passes Wk [T, dk], Wv [T, dv] where they cannot go straight to
+//   grad_k / grad_v: always without native reverse (float32 when multiplied by psi' or
+//   corrected, else the output type); with it, float32 and only where psi' or the
+//   small-decay terms still apply.  ELU+1: the grad_q pass's float32 output Wq [T, dk] and
+//   the lo passes' float32 outputs.
+//   Three [dk x dv] states per (b, h), then the prefill workspace.
 struct BwdLayout {
-  size_t kr, qr, dor, vr, pqr, pk, pqr_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC, pw, total;
-  bool w_f32, elu, split;
+  size_t kr, qr, dor, vr, pq, pk, pq_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC, pw, total;
+  bool native, elu, split, fix, wk, wv, w_f32;
 };
 
 BwdLayout bwd_layout(const la_backward_args& a) {
@@ -230,9 +247,13 @@ BwdLayout bwd_layout(const la_backward_args& a) {
   const size_t T = static_cast<size_t>(a.T > 0 ? a.T : 0);
   const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
   const bool out_f32 = a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32;
+  l.native = native_reverse(a);
   l.elu = a.feature_map == LA_FM_ELU1;
   l.split = l.elu && a.dtype == LA_DTYPE_BF16;
-  l.w_f32 = out_f32 || l.elu || has_small_decay(a);
+  l.fix = has_small_decay(a);
+  l.wk = !l.native || l.elu || l.fix;
+  l.wv = !l.native || l.fix;
+  l.w_f32 = l.native || out_f32 || l.elu || l.fix;
   const size_t ew = l.w_f32 ? 4 : 2;
   const size_t nk = BH * T * a.dk, nv = BH * T * a.dv, ns = BH * a.dk * a.dv * 4;
   size_t off = 0;
@@ -241,16 +262,17 @@ BwdLayout bwd_layout(const la_backward_args& a) {
     off = align256(off + bytes);
     return o;
   };
-  l.kr = take(nk * e);
-  l.qr = take(nk * e);
-  l.dor = take(nv * e);
-  l.vr = take(nv * e);
-  l.pqr = take(l.elu ? nk * e : 0);
+  const bool flip = !l.native;
+  l.kr = take(flip ? nk * e : 0);
+  l.qr = take(flip ? nk * e : 0);
+  l.dor = take(flip ? nv * e : 0);
+  l.vr = take(flip ? nv * e : 0);
+  l.pq = take(l.elu ? nk * e : 0);
   l.pk = take(l.elu ? nk * e : 0);
-  l.pqr_lo = take(l.split ? nk * e : 0);
+  l.pq_lo = take(l.split ? nk * e : 0);
   l.pk_lo = take(l.split ? nk * e : 0);
-  l.Wk = take(nk * ew);
-  l.Wv = take(nv * ew);
+  l.Wk = take(l.wk ? nk * ew : 0);
+  l.Wv = take(l.wv ? nv * ew : 0);
   l.Wq = take(l.elu ? nk * 4 : 0);
   l.Wk_lo = take(l.split ? nk * 4 : 0);
   l.Wq_lo = take(l.split ? nk * 4 : 0);
@@ -309,10 +331,12 @@ int validate(const la_backward_args& a) {
   const bool empty = BH == 0 || a.T == 0;
   const int fms[3] = {LA_FM_IDENTITY, a.feature_map, LA_FM_IDENTITY};
   const int dks[3] = {a.dv, a.dk, a.dv}, dvs[3] = {a.dk, a.dv, a.dk};
+  const bool native = native_reverse(a);
   for (int i = 0; i < 3; ++i) {
     la_prefill_args p = pass_args(a, dks[i], dvs[i], fms[i], LA_OUT_F32);
     p.q = p.k = p.v = empty ? nullptr : a.q;
     p.states_only = 1;
+    p.reverse = native && i > 0;
     const int st = check_prefill_args(p);
     if (st != LA_OK) return st;
   }
@@ -391,29 +415,30 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
   const bool in_f32 = a.dtype == LA_DTYPE_F32;
   const bool out_f32 = in_f32 || a.out_dtype == LA_OUT_F32;
   const bool elu = a.feature_map == LA_FM_ELU1;
-  const int w_dtype = l.w_f32 ? LA_OUT_F32 : LA_OUT_AS_INPUT;
   const long long T = a.T;
 
-  // Reversed inputs (psi(q) reversed and psi(k) in order for ELU+1, as hi / lo pairs for
-  // bf16 inputs).
+  // Inputs of the passes: reversed copies unless the reversed passes run natively; for
+  // ELU+1, psi(q) (reversed likewise) and psi(k) in order, as hi / lo pairs for bf16.
   auto job = [](RowJobs& J, int& n, const void* src, const void* src2, void* dst, const void* x,
                 int d, int fm_src, int fm_x, bool flip, bool lo, bool sf, bool df, bool xf) {
     J.j[n++] = RowJob{src, src2, dst, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
   };
   RowJobs pre{};
   int np = 0;
-  const bool f = in_f32;
-  job(pre, np, a.k, nullptr, at(l.kr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
-  job(pre, np, a.q, nullptr, at(l.qr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
-  job(pre, np, a.grad_out, nullptr, at(l.dor), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f,
-      f, f);
-  job(pre, np, a.v, nullptr, at(l.vr), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f, f, f);
+  const bool f = in_f32, rv = !l.native;
+  if (rv) {
+    job(pre, np, a.k, nullptr, at(l.kr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
+    job(pre, np, a.q, nullptr, at(l.qr), nullptr, a.dk, LA_FM_IDENTITY, 0, true, false, f, f, f);
+    job(pre, np, a.grad_out, nullptr, at(l.dor), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false,
+        f, f, f);
+    job(pre, np, a.v, nullptr, at(l.vr), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f, f, f);
+  }
   if (elu) {
-    job(pre, np, a.q, nullptr, at(l.pqr), nullptr, a.dk, LA_FM_ELU1, 0, true, false, f, f, f);
+    job(pre, np, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f);
     job(pre, np, a.k, nullptr, at(l.pk), nullptr, a.dk, LA_FM_ELU1, 0, false, false, f, f, f);
   }
   if (l.split) {
-    job(pre, np, a.q, nullptr, at(l.pqr_lo), nullptr, a.dk, LA_FM_ELU1, 0, true, true, f, f, f);
+    job(pre, np, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f);
     job(pre, np, a.k, nullptr, at(l.pk_lo), nullptr, a.dk, LA_FM_ELU1, 0, false, true, f, f, f);
   }
   cudaError_t e = launch_rows(pre, np, BH, T, s, rec, "bwd_reverse_inputs");
@@ -465,39 +490,42 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
       run(p);
     }
   }
-  // grad_v reversed: (k, q, do) reversed with the model's map; final state G_0.
+  // grad_v: (k, q, do) in reverse time with the model's map; final state G_0.
+  const int w_dtype = l.w_f32 ? LA_OUT_F32 : LA_OUT_AS_INPUT;
   {
-    la_prefill_args p = pass_args(a, a.dk, a.dv, a.feature_map, w_dtype);
-    p.q = at(l.kr);
-    p.k = at(l.qr);
-    p.v = at(l.dor);
-    p.out = at(l.Wv);
+    la_prefill_args p = pass_args(a, a.dk, a.dv, a.feature_map, l.wv ? w_dtype : a.out_dtype);
+    p.reverse = l.native;
+    p.q = rv ? at(l.kr) : a.k;
+    p.k = rv ? at(l.qr) : a.q;
+    p.v = rv ? at(l.dor) : a.grad_out;
+    p.out = l.wv ? at(l.Wv) : a.grad_v;
     p.S_init = SB;
     p.S_final = a.grad_S_init;
     run(p);
   }
-  // dpsi(k) reversed: (v, do, psi(q)) reversed, identity map (lo half as for grad_q).
+  // dpsi(k): (v, do, psi(q)) in reverse time, identity map (lo half as for grad_q).
   {
-    la_prefill_args p = pass_args(a, a.dv, a.dk, LA_FM_IDENTITY, w_dtype);
-    p.q = at(l.vr);
-    p.k = at(l.dor);
-    p.v = elu ? at(l.pqr) : at(l.qr);
-    p.out = at(l.Wk);
+    la_prefill_args p = pass_args(a, a.dv, a.dk, LA_FM_IDENTITY, l.wk ? w_dtype : a.out_dtype);
+    p.reverse = l.native;
+    p.q = rv ? at(l.vr) : a.v;
+    p.k = rv ? at(l.dor) : a.grad_out;
+    p.v = elu ? at(l.pq) : (rv ? at(l.qr) : a.q);
+    p.out = l.wk ? at(l.Wk) : a.grad_k;
     p.S_init = SC;
     run(p);
     if (l.split) {
-      p.v = at(l.pqr_lo);
+      p.v = at(l.pq_lo);
       p.out = at(l.Wk_lo);
       p.S_init = nullptr;
       run(p);
     }
   }
   e = cudaSuccess;
-  if (st == LA_OK && has_small_decay(a)) {
+  if (st == LA_OK && l.fix) {
     if (rec) rec->mark(s, "bwd_fix_small_decay");
     fix_small_decay<<<static_cast<unsigned>(BH), 128, 0, s>>>(
         a.grad_S_final, a.k, a.v, static_cast<float*>(at(l.Wk)), static_cast<float*>(at(l.Wv)),
-        a.dk, a.dv, a.H, T, a.feature_map, in_f32, gt);
+        a.dk, a.dv, a.H, T, a.feature_map, in_f32, l.native, gt);
     e = cudaGetLastError();
   }
   if (st == LA_OK && e == cudaSuccess && a.grad_S_init && a.gamma) {
@@ -506,15 +534,18 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
                                          gt);
     e = cudaGetLastError();
   }
-  // Back to forward time, with psi' where the map has one.
+  // The gradients in forward time (reversed back unless the passes ran natively), with
+  // psi' where the map has one.
   if (st == LA_OK && e == cudaSuccess) {
     RowJobs post{};
     int n = 0;
     const bool wf = l.w_f32;
-    job(post, n, at(l.Wv), nullptr, a.grad_v, nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, wf,
-        out_f32, f);
-    job(post, n, at(l.Wk), l.split ? at(l.Wk_lo) : nullptr, a.grad_k, a.k, a.dk, LA_FM_IDENTITY,
-        a.feature_map, true, false, wf, out_f32, f);
+    if (l.wv)
+      job(post, n, at(l.Wv), nullptr, a.grad_v, nullptr, a.dv, LA_FM_IDENTITY, 0, rv, false, wf,
+          out_f32, f);
+    if (l.wk)
+      job(post, n, at(l.Wk), l.split ? at(l.Wk_lo) : nullptr, a.grad_k, a.k, a.dk,
+          LA_FM_IDENTITY, a.feature_map, rv, false, wf, out_f32, f);
     if (elu)  // grad_q = psi'(q) .* dpsi(q)
       job(post, n, at(l.Wq), l.split ? at(l.Wq_lo) : nullptr, a.grad_q, a.q, a.dk,
           LA_FM_IDENTITY, a.feature_map, false, false, true, out_f32, f);

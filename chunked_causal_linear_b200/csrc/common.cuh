@@ -58,6 +58,8 @@ struct SegParams {
   float* srec;     // [BH, NS, R] segment totals, turned into exclusive prefixes by K2
   void* out;       // [BH, T, dv] output, bf16 or fp32
   bool has_init;   // segment 0 starts from a given state (its prefix is not zero)
+  bool reverse;    // the sequence runs from token T - 1 down to token 0: chunk c covers
+                   // tokens [T - 64 (c + 1), T - 64 c), its position p is token T-64c-1-p
   int* err;
 };
 

@@ -180,14 +180,17 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
     float zacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
-    // The weight of row r of chunk i is gamma^(len_s - 1 - 64 i - r).  For gamma >= 1/2 it
-    // is formed as gamma^(len_s - 1 - 64 i) * gamma^(-r) (gamma^(-r) <= 2^63, one powf per
-    // chunk); smaller gamma takes one powf per row, since gamma^(-r) would overflow.
+    // The weight of the token at chunk position p of chunk i is gamma^(len_s - 1 - 64 i - p);
+    // tile row r holds position p = r, or p = 63 - r when the sequence runs in reverse
+    // (the tile is loaded in memory order).  For gamma >= 1/2 it is formed as a per-chunk
+    // factor times gamma^(-r) (<= 2^63) or gamma^r; smaller gamma takes one powf per row,
+    // since gamma^(-r) would overflow.
+    const bool rev = sp.reverse;
     const bool factored = DECAY && g >= 0.5f;
     float ginv[kRows];
 #pragma unroll
     for (int k = 0; k < kRows; ++k)
-      ginv[k] = factored ? powf(g, -static_cast<float>(rg + k * RG)) : 1.f;
+      ginv[k] = factored ? powf(g, (rev ? 1.f : -1.f) * static_cast<float>(rg + k * RG)) : 1.f;
     for (int i = 0; i < n; ++i) {
       const int st = i % kStages1;
       const int L = chunk_len(sp, cb + i);
@@ -195,7 +198,8 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
       uint8_t* sKl = sK + L_::kK + L_::kV;
       wait(&full[st], (i / kStages1) & 1, kErrTmaTimeout);
       if constexpr (kSplit || NORM) {
-        const float wb = factored ? powf(g, static_cast<float>(seg_tokens - 1 - i * kC)) : 1.f;
+        const int e0 = rev ? seg_tokens - kC - i * kC : seg_tokens - 1 - i * kC;
+        const float wb = factored ? powf(g, static_cast<float>(e0)) : 1.f;
         const uint32_t boff = (cc / 8) * (kC * 128);
         uint4 raw[kRows];
 #pragma unroll
@@ -205,10 +209,10 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
         for (int k = 0; k < kRows; ++k) {
           const int r = rg + k * RG;
           float w = 0.f;
-          if (r < L) {
+          if ((rev ? kC - 1 - r : r) < L) {
             if (!DECAY) w = 1.f;
             else if (factored) w = wb * ginv[k];
-            else w = powf(g, static_cast<float>(seg_tokens - 1 - i * kC - r));
+            else w = powf(g, static_cast<float>(rev ? e0 + r : e0 - r));
           }
           float x[8];
           unpack8(raw[k], x);
@@ -289,7 +293,9 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
         if (i >= kStages1 && !wait(&empty[st], ((i / kStages1) - 1) & 1, kErrMmaTimeout)) break;
         uint8_t* sK = base + st * L_::kStage;
         uint8_t* sV = sK + L_::kK;
-        const int t0 = (cb + i) * kC;
+        // In reverse the chunk's tile starts 64 (c + 1) tokens before the end; the ragged
+        // last chunk starts at a negative row, which the load fills with zeros.
+        const int t0 = sp.reverse ? static_cast<int>(sp.T) - (cb + i + 1) * kC : (cb + i) * kC;
         mbar_arrive_expect_tx(&full[st], L_::kK + L_::kV);
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) tma_load_3d(sK + b * kC * 128, &tm_k, &full[st], b * 64, t0, bh);
@@ -376,7 +382,7 @@ struct K3sSmem {
 };
 
 
-template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
+template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV>
 __global__ void __launch_bounds__(kThreads3, 1)
 k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
        const __grid_constant__ CUtensorMap tm_v, SegParams sp, GammaTable gt) {
@@ -451,10 +457,15 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // Tile row r holds chunk position p = r, or p = 63 - r in reverse (the tile is loaded in
+  // memory order); sTh is indexed by tile row, sPow by position difference.  The direction
+  // is a template parameter: the causal kernel carries no trace of the reverse one.
+  constexpr bool rev = REV;
   if (tid < kC) {
-    sTh[tid] = DECAY ? powf(g, static_cast<float>(tid + 1)) : 1.f;
+    sTh[tid] = DECAY ? powf(g, static_cast<float>((rev ? kC - 1 - tid : tid) + 1)) : 1.f;
     sPow[tid] = DECAY ? powf(g, static_cast<float>(tid)) : 1.f;
   }
+  const float g64 = DECAY ? powf(g, static_cast<float>(kC)) : 1.f;
   if constexpr (NORM) {
     if (tid < DK) sZP[tid] = srec[DK * DV + tid];
   }
@@ -530,10 +541,12 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       uint8_t* sKph = sKpp + s * L_::kKpp;
       uint8_t* sKpl = sKph + L_::kK;
       float* xi = sXi + s * kC;
-      if (tw < kC)
-        xi[tw] = tw < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - tw - (renorm ? kC * (i % W + 1) : 0)))
-                                 : 1.f)
-                        : 0.f;
+      if (tw < kC) {
+        const int p = rev ? kC - 1 - tw : tw;
+        xi[tw] = p < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - p - (renorm ? kC * (i % W + 1) : 0)))
+                                : 1.f)
+                       : 0.f;
+      }
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
       named_barrier(1, kXfThreads);
 
@@ -566,7 +579,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           float x[8];
           unpack8(kraw[k], x);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = r < L ? feature<FM>(x[e]) : 0.f;
+          for (int e = 0; e < 8; ++e) x[e] = (rev ? kC - 1 - r : r) < L ? feature<FM>(x[e]) : 0.f;
           if constexpr (kSplitQK) {
             uint4 hi, lo;
             split8(x, hi, lo);
@@ -610,7 +623,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       mbar_arrive(&ops[s]);
 
       // gamma^L: Theta of the chunk's last token for a full chunk.
-      const float a_c = DECAY ? (L == kC ? sTh[kC - 1] : powf(g, static_cast<float>(L))) : 1.f;
+      const float a_c = DECAY ? (L == kC ? g64 : powf(g, static_cast<float>(L))) : 1.f;
       if constexpr (NORM) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -680,7 +693,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     const int j = quarter * 32 + lane;  // value feature of this thread's output column
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      const long long t0 = static_cast<long long>(cb + i) * kC;
+      const long long t0 = rev ? sp.T - static_cast<long long>(cb + i + 1) * kC
+                               : static_cast<long long>(cb + i) * kC;
       const int L = chunk_len(sp, cb + i);
       const bool has_prefix = !(seg == 0 && i == 0) || sp.has_init;
       wait(sdone, i & 1, kErrMmaTimeout);
@@ -705,7 +719,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           float a[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int d = row - kb - q * 8 - e;
+            const int d = rev ? kb + q * 8 + e - row : row - kb - q * 8 - e;
             a[e] = d >= 0 ? sc[q * 8 + e] * sPow[d] : 0.f;
             den_loc += a[e];
           }
@@ -768,10 +782,12 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         }
       }
       const long long row0 = static_cast<long long>(bh) * sp.T + t0 + 32 * half;
-      const int nt = min(32, L - 32 * half);  // tokens of this half inside the sequence
+      // Tokens of this half inside the sequence: tile rows [t_lo, t_hi).
+      const int t_lo = rev ? max(0, kC - L - 32 * half) : 0;
+      const int t_hi = rev ? 32 : min(32, L - 32 * half);
 #pragma unroll
       for (int tt = 0; tt < 32; ++tt) {
-        if (tt < nt) {
+        if (tt >= t_lo && tt < t_hi) {
           const long long idx = (row0 + tt) * DV + j;
           if constexpr (OUTF32)
             __stcs(static_cast<float*>(sp.out) + idx, no[tt]);
@@ -790,7 +806,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         uint8_t* sQ = base + (i & 1) * L_::kStage;
         uint8_t* sK = sQ + L_::kQ;
         uint8_t* sV = sK + L_::kK;
-        const int t0 = (cb + i) * kC;
+        const int t0 = rev ? static_cast<int>(sp.T) - (cb + i + 1) * kC : (cb + i) * kC;
         mbar_arrive_expect_tx(&full[i & 1], L_::kStage);
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) {
@@ -930,15 +946,21 @@ cudaError_t k1s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
   return cudaGetLastError();
 }
 
-template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
-cudaError_t k3s_go_o(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
-  auto kern = k3_seg<DK, FM, DECAY, NORM, OUTF32>;
+template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV>
+cudaError_t k3s_go_r(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
+  auto kern = k3_seg<DK, FM, DECAY, NORM, OUTF32, REV>;
   const uint32_t sm = K3sSmem<DK, FM, DECAY, OUTF32>::kTotal;
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(sp.BH) * sp.NS;
   kern<<<static_cast<unsigned>(grid), kThreads3, sm, s>>>(m.q, m.k, m.v, sp, gt);
   return cudaGetLastError();
+}
+
+template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32>
+cudaError_t k3s_go_o(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
+  return sp.reverse ? k3s_go_r<DK, FM, DECAY, NORM, OUTF32, true>(sp, gt, m, s)
+                    : k3s_go_r<DK, FM, DECAY, NORM, OUTF32, false>(sp, gt, m, s);
 }
 
 template <int DK, int DV, int FM, bool DECAY, bool NORM>

@@ -186,6 +186,12 @@ typedef struct la_prefill_args {
   /* 1: compute only S_final / Z_final (the summaries and the scan, no output: `out` may
    * be NULL) -- the per-part totals of a sequence split across devices.  0: full prefill. */
   int states_only;
+  /* 1: run the recurrence from token T-1 down to token 0 (the anti-causal direction):
+   * out_t = psi(q_t) S'_t with S'_t = gamma S'_{t+1} + psi(k_t) v_t^T, S'_T = S_init, and
+   * S_final = S'_0 -- the prefill of the time-reversed sequence, with every tensor kept
+   * in its memory order.  Segmented algorithm only (LA_ERR_UNSUPPORTED otherwise).
+   * 0: causal. */
+  int reverse;
 } la_prefill_args;
 
 /* lin_attn_prefill_ex -- the prefill with every option of la_prefill_args.  A caller
@@ -285,9 +291,14 @@ int lin_attn_prefill_noalloc(const la_prefill_args* args);
  *           from grad_S_final / gamma (its final state is G_0);
  *   grad_k  the prefill of (v, grad_out, psi(q)) under the identity map on the
  *           time-reversed sequence, started from grad_S_final^T / gamma;
- * plus element-wise kernels that reverse time, apply psi and psi', and fold in the
- * grad_S_final terms of heads whose decay is below 2^-20 (for those heads the division
- * by gamma is replaced by the exact first three terms, the rest being below 2^-60).
+ * plus element-wise kernels that apply psi and psi' and fold in the grad_S_final terms
+ * of heads whose decay is below 2^-20 (for those heads the division by gamma is replaced
+ * by the exact first three terms, the rest being below 2^-60).  The two time-reversed
+ * passes run as reverse-mode prefills (la_prefill_args.reverse) when bf16 inputs, C = 64,
+ * dk = dv = 128 and not ELU+1 with a decay; otherwise on reversed copies of their inputs,
+ * their outputs reversed back.  Under ELU+1 with bf16 inputs, psi(k) and psi(q) enter
+ * two passes as the value operand; they are split into bf16 hi and lo halves and those
+ * passes run once per half, so that psi keeps about 16 bits as in the forward kernels.
  * The normalised form's gradient is not provided.
  *
  *   q, k, v, grad_out  DEVICE, the forward's inputs and dL/dout, type `dtype`,

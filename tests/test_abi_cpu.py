@@ -153,6 +153,8 @@ def test_binding_fails_loudly_without_library(tmp_path):
 @pytest.mark.parametrize("kw,status", [
     (dict(states_only=2), 1), (dict(states_only=-1), 1), (dict(S_init=0x1002), 1),
     (dict(Z_init=0x1001), 1), (dict(states_only=1, out=None, algorithm=2, dv=64), 2),
+    (dict(reverse=2), 1), (dict(reverse=-1), 1), (dict(reverse=1, algorithm=1), 2),
+    (dict(reverse=1, kernel_path=2), 2),
 ])
 def test_initial_state_and_states_only_argument_errors(lib, kw, status):
     a = _args(**kw)
@@ -246,3 +248,11 @@ def test_backward_workspace_bytes(lib):
             + 2 * al(n_k * 4) + 2 * ns + pw)
     assert B.lin_attn_backward_workspace_bytes(q, v, feature_map="elu1", grad_S_final=True) == want
     assert B.lin_attn_backward_workspace_bytes(q[:, :, :0], v[:, :, :0]) == 0
+    # dk = dv = 128: the reversed passes run as reverse-mode prefills, with no reversed
+    # copies; identity map with float32 gradients needs the prefill workspace alone
+    q2 = torch.empty(2, 3, 100, 128, dtype=torch.bfloat16)
+    pw2 = B.lin_attn_prefill_workspace_bytes(2, 3, 100, 128, 128, 64, False)
+    assert B.lin_attn_backward_workspace_bytes(q2, q2, out_dtype="f32") == pw2
+    n2 = 2 * 3 * 100 * 128
+    want = 4 * al(n2 * 2) + 4 * al(n2 * 4) + pw2  # ELU+1: psi(q), psi(k) hi / lo; Wk, Wq, lo
+    assert B.lin_attn_backward_workspace_bytes(q2, q2, feature_map="elu1", out_dtype="f32") == want
