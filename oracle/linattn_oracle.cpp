@@ -39,8 +39,8 @@
 //   gamma [H] (double) or NULL.
 // S_init / Z_init may be NULL (zero initial state); the outputs may be NULL (skipped).
 //
-// la_oracle_backward differentiates the unnormalised form by hand, token by token (the
-// chain rule through the recurrence; see backward_pair), for the backward pass.
+// la_oracle_backward differentiates both forms by hand, token by token (the chain rule
+// through the recurrence; see backward_pair), for the backward pass.
 
 #include <cmath>
 #include <cstddef>
@@ -126,15 +126,18 @@ void run_pair(const Problem& p, long long bh) {
     for (int i = 0; i < dk; ++i) p.Z_final[bh * dk + i] = Z[i];
 }
 
-// Backward of the unnormalised form for one (b, h) pair.  With do_t = dL/do_t and
-// dS_final = dL/dS_final (or zero), differentiating the recurrence above gives
-//   dphi(q_t) = S_t do_t                                   (forward sweep, S_t as above)
-//   G_t       = phi(q_t) do_t^T + gamma G_{t+1},  G_{T-1} = phi(q_{T-1}) do_{T-1}^T + dS_final
-//   dphi(k_t) = G_t v_t,   dv_t = G_t^T phi(k_t)           (reverse sweep)
-//   dS_init   = gamma G_0
+// Backward for one (b, h) pair.  With do_t = dL/do_t, dS_final = dL/dS_final and
+// dZ_final = dL/dZ_final (or zero), differentiating the recurrence above one token at a
+// time.  The output is o_t = n_t / d_t with n_t = phi(q_t) S_t and d_t = phi(q_t) . Z_t
+// + eps (normalised form), or o_t = n_t (unnormalised: d_t = 1 and no Z terms).  So
+//   dn_t = do_t / d_t,   dd_t = -(do_t . n_t) / d_t^2            (dd_t = 0 unnormalised)
+//   dphi(q_t) = S_t dn_t + Z_t dd_t                              (forward sweep)
+//   G_t = phi(q_t) dn_t^T + gamma G_{t+1},  G_{T-1} = phi(q_{T-1}) dn_{T-1}^T + dS_final
+//   g_t = phi(q_t) dd_t   + gamma g_{t+1},  g_{T-1} = phi(q_{T-1}) dd_{T-1}   + dZ_final
+//   dphi(k_t) = G_t v_t + g_t,   dv_t = G_t^T phi(k_t)           (reverse sweep)
+//   dS_init = gamma G_0,   dZ_init = gamma g_0
 // and dq = dphi(q) * phi'(q), dk = dphi(k) * phi'(k) with phi' = 1 (identity) or
-// 1 for x > 0, exp(x) otherwise (ELU + 1).  Every sum is the plain chain rule through
-// S_t = gamma S_{t-1} + phi(k_t) v_t^T and o_t = phi(q_t) S_t, one token at a time.
+// 1 for x > 0, exp(x) otherwise (ELU + 1).
 struct BackwardProblem {
   const float* q;
   const float* k;
@@ -144,12 +147,17 @@ struct BackwardProblem {
   long long T;
   int dk, dv, fm;
   const double* gamma;
+  int normalize;
+  double eps;
   const double* S_init;
+  const double* Z_init;
   const double* dS_final;
+  const double* dZ_final;
   double* dq;
   double* dk_out;
   double* dv_out;
   double* dS_init;
+  double* dZ_init;
 };
 
 inline double feature_map_derivative(double x, int fm) {
@@ -167,39 +175,64 @@ void backward_pair(const BackwardProblem& p, long long bh) {
   const float* v = p.v + bh * T * dv;
   const double* dout = p.dout + bh * T * dv;
 
-  // Forward sweep: S_t, then dphi(q_t) = S_t do_t.
-  std::vector<double> S(static_cast<size_t>(dk) * dv, 0.0);
+  // Forward sweep: S_t and Z_t, the output's numerator and denominator, the gradients
+  // that reach them (kept for the reverse sweep), and dphi(q_t).
+  std::vector<double> S(static_cast<size_t>(dk) * dv, 0.0), Z(dk, 0.0), fq(dk), n(dv);
+  std::vector<double> dn(static_cast<size_t>(T) * dv), dd(static_cast<size_t>(T), 0.0);
   if (p.S_init)
     for (size_t e = 0; e < S.size(); ++e) S[e] = p.S_init[bh * dk * dv + e];
+  if (p.normalize && p.Z_init)
+    for (int i = 0; i < dk; ++i) Z[i] = p.Z_init[bh * dk + i];
   for (long long t = 0; t < T; ++t) {
     for (int i = 0; i < dk; ++i) {
       const double fk = feature_map(static_cast<double>(k[t * dk + i]), p.fm);
       double* Si = &S[static_cast<size_t>(i) * dv];
       for (int j = 0; j < dv; ++j) Si[j] = g * Si[j] + fk * static_cast<double>(v[t * dv + j]);
+      Z[i] = g * Z[i] + fk;
+      fq[i] = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
     }
+    double den = 1.0, don = 0.0;
+    if (p.normalize) {
+      den = p.eps;
+      for (int i = 0; i < dk; ++i) den += fq[i] * Z[i];
+    }
+    for (int j = 0; j < dv; ++j) {
+      double acc = 0.0;
+      for (int i = 0; i < dk; ++i) acc += fq[i] * S[static_cast<size_t>(i) * dv + j];
+      n[j] = acc;
+      don += dout[t * dv + j] * acc;
+      dn[static_cast<size_t>(t) * dv + j] = dout[t * dv + j] / den;
+    }
+    if (p.normalize) dd[static_cast<size_t>(t)] = -don / (den * den);
     for (int i = 0; i < dk; ++i) {
       const double* Si = &S[static_cast<size_t>(i) * dv];
       double acc = 0.0;
-      for (int j = 0; j < dv; ++j) acc += Si[j] * dout[t * dv + j];
+      for (int j = 0; j < dv; ++j) acc += Si[j] * dn[static_cast<size_t>(t) * dv + j];
+      acc += Z[i] * dd[static_cast<size_t>(t)];
       const double x = static_cast<double>(q[t * dk + i]);
       p.dq[(bh * T + t) * dk + i] = acc * feature_map_derivative(x, p.fm);
     }
   }
 
-  // Reverse sweep: G accumulates phi(q_t) do_t^T and decays by gamma between tokens.
-  std::vector<double> G(static_cast<size_t>(dk) * dv, 0.0), fk(dk);
+  // Reverse sweep: G accumulates phi(q_t) dn_t^T, g accumulates phi(q_t) dd_t, and both
+  // decay by gamma between tokens.
+  std::vector<double> G(static_cast<size_t>(dk) * dv, 0.0), gz(dk, 0.0), fk(dk);
   if (p.dS_final)
     for (size_t e = 0; e < G.size(); ++e) G[e] = p.dS_final[bh * dk * dv + e];
+  if (p.normalize && p.dZ_final)
+    for (int i = 0; i < dk; ++i) gz[i] = p.dZ_final[bh * dk + i];
   for (long long t = T - 1; t >= 0; --t) {
+    const double* dnt = &dn[static_cast<size_t>(t) * dv];
     for (int i = 0; i < dk; ++i) {
-      const double fq = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
+      const double fqi = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
       double* Gi = &G[static_cast<size_t>(i) * dv];
-      for (int j = 0; j < dv; ++j) Gi[j] += fq * dout[t * dv + j];
+      for (int j = 0; j < dv; ++j) Gi[j] += fqi * dnt[j];
+      gz[i] += fqi * dd[static_cast<size_t>(t)];
       fk[i] = feature_map(static_cast<double>(k[t * dk + i]), p.fm);
     }
     for (int i = 0; i < dk; ++i) {
       const double* Gi = &G[static_cast<size_t>(i) * dv];
-      double acc = 0.0;
+      double acc = gz[i];
       for (int j = 0; j < dv; ++j) acc += Gi[j] * static_cast<double>(v[t * dv + j]);
       const double x = static_cast<double>(k[t * dk + i]);
       p.dk_out[(bh * T + t) * dk + i] = acc * feature_map_derivative(x, p.fm);
@@ -210,9 +243,12 @@ void backward_pair(const BackwardProblem& p, long long bh) {
       p.dv_out[(bh * T + t) * dv + j] = acc;
     }
     for (double& x : G) x *= g;  // G_{t-1} receives gamma G_t
+    for (double& x : gz) x *= g;
   }
   if (p.dS_init)
     for (size_t e = 0; e < G.size(); ++e) p.dS_init[bh * dk * dv + e] = G[e];
+  if (p.dZ_init)
+    for (int i = 0; i < dk; ++i) p.dZ_init[bh * dk + i] = p.normalize ? gz[i] : 0.0;
 }
 
 }  // namespace
@@ -255,21 +291,23 @@ int la_oracle_forward(const float* q, const float* k, const float* v, int B, int
   return 0;
 }
 
-// Backward of the unnormalised form (see backward_pair).  dout [B, H, T, dv] (double),
-// dS_final [B, H, dk, dv] or NULL, S_init as in la_oracle_forward.  Writes dq, dk
-// [B, H, T, dk], dv [B, H, T, dv] and dS_init [B, H, dk, dv] (may be NULL), all double.
+// Backward (see backward_pair).  dout [B, H, T, dv] (double), dS_final [B, H, dk, dv] and
+// dZ_final [B, H, dk] or NULL, S_init / Z_init as in la_oracle_forward.  Writes dq, dk
+// [B, H, T, dk], dv [B, H, T, dv], dS_init [B, H, dk, dv] and dZ_init [B, H, dk] (each
+// may be NULL; dZ_init is zero for the unnormalised form), all double.
 int la_oracle_backward(const float* q, const float* k, const float* v, const double* dout,
                        int B, int H, long long T, int dk, int dv, int feature_map_id,
-                       const double* gamma, const double* S_init, const double* dS_final,
+                       const double* gamma, int normalize, double eps, const double* S_init,
+                       const double* Z_init, const double* dS_final, const double* dZ_final,
                        double* dq, double* dk_out, double* dv_out, double* dS_init,
-                       int nthreads) {
+                       double* dZ_init, int nthreads) {
   if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 1;
   if (feature_map_id != 0 && feature_map_id != 1) return 1;
   if (T > 0 && (!q || !k || !v || !dout || !dq || !dk_out || !dv_out)) return 1;
   const long long BH = static_cast<long long>(B) * H;
   if (BH == 0) return 0;
-  BackwardProblem p{q, k, v, dout, H, T, dk, dv, feature_map_id, gamma, S_init, dS_final,
-                    dq, dk_out, dv_out, dS_init};
+  BackwardProblem p{q, k, v, dout, H, T, dk, dv, feature_map_id, gamma, normalize, eps,
+                    S_init, Z_init, dS_final, dZ_final, dq, dk_out, dv_out, dS_init, dZ_init};
   long long workers = nthreads > 0 ? nthreads
                                    : static_cast<long long>(std::thread::hardware_concurrency());
   if (workers < 1) workers = 1;

@@ -55,7 +55,7 @@ class Oracle:
         b.restype = ctypes.c_int
         b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
-            [ctypes.c_void_p] * 7 + [ctypes.c_int]
+            [ctypes.c_void_p, ctypes.c_int, ctypes.c_double] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
         g = self._lib.la_oracle_feature_map
         g.restype = ctypes.c_int
         g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int]
@@ -106,10 +106,12 @@ class Oracle:
             raise ValueError(f"la_oracle_forward returned {rc}")
         return out, S, Z
 
-    def backward(self, q, k, v, dout, *, feature_map: str = "elu1", gamma=None, S_init=None,
-                 dS_final=None, nthreads: int = 0):
-        """Gradients of the unnormalised form: given dL/dout (and dL/dS_final, or zero),
-        returns (dq, dk, dv, dS_init), float64."""
+    def backward(self, q, k, v, dout, *, feature_map: str = "elu1", gamma=None,
+                 normalize: bool = False, eps: float = 0.0, S_init=None, Z_init=None,
+                 dS_final=None, dZ_final=None, nthreads: int = 0):
+        """Gradients of L = <dout, out> + <dS_final, S_final> (+ <dZ_final, Z_final>
+        normalised) with respect to q, k, v and the initial state.  Returns (dq, dk, dv,
+        dS_init, dZ_init), float64 (dZ_init zero for the unnormalised form)."""
         q = np.ascontiguousarray(q, dtype=np.float32)
         k = np.ascontiguousarray(k, dtype=np.float32)
         v = np.ascontiguousarray(v, dtype=np.float32)
@@ -119,17 +121,19 @@ class Oracle:
         if k.shape != q.shape or v.shape[:3] != (B, H, T) or do.shape != v.shape:
             raise ValueError("shape mismatch between q, k, v and dout")
         g = None if gamma is None else np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(H))
-        s0 = None if S_init is None else np.ascontiguousarray(S_init, dtype=np.float64)
-        dsf = None if dS_final is None else np.ascontiguousarray(dS_final, dtype=np.float64)
+        f64 = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+        s0, z0, dsf, dzf = f64(S_init), f64(Z_init), f64(dS_final), f64(dZ_final)
         dq = np.empty((B, H, T, dk)); dk_ = np.empty((B, H, T, dk)); dv_ = np.empty((B, H, T, dv))
-        ds0 = np.empty((B, H, dk, dv))
+        ds0 = np.empty((B, H, dk, dv)); dz0 = np.empty((B, H, dk))
         ptr = lambda a: None if a is None else a.ctypes.data
         rc = self._lib.la_oracle_backward(ptr(q), ptr(k), ptr(v), ptr(do), B, H, T, dk, dv,
-                                          FEATURE_MAPS[feature_map], ptr(g), ptr(s0), ptr(dsf),
-                                          ptr(dq), ptr(dk_), ptr(dv_), ptr(ds0), int(nthreads))
+                                          FEATURE_MAPS[feature_map], ptr(g), int(bool(normalize)),
+                                          float(eps), ptr(s0), ptr(z0), ptr(dsf), ptr(dzf),
+                                          ptr(dq), ptr(dk_), ptr(dv_), ptr(ds0), ptr(dz0),
+                                          int(nthreads))
         if rc != 0:
             raise ValueError(f"la_oracle_backward returned {rc}")
-        return dq, dk_, dv_, ds0
+        return dq, dk_, dv_, ds0, dz0
 
 
 _default: Oracle | None = None
