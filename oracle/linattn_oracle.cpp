@@ -189,12 +189,13 @@ void backward_pair(const BackwardProblem& p, long long bh) {
       double* Si = &S[static_cast<size_t>(i) * dv];
       for (int j = 0; j < dv; ++j) Si[j] = g * Si[j] + fk * static_cast<double>(v[t * dv + j]);
       Z[i] = g * Z[i] + fk;
-      fq[i] = feature_map(static_cast<double>(q[t * dk + i]), p.fm);
+      const double xq = q[t * dk + i];
+      fq[i] = feature_map(xq, p.fm);
     }
     double den = 1.0, don = 0.0;
     if (p.normalize) {
       den = p.eps;
-      for (int i = 0; i < dk; ++i) den += fq[i] * Z[i];
+      for (int i = 0; i < dk; ++i) den += Z[i] * fq[i];
     }
     for (int j = 0; j < dv; ++j) {
       double acc = 0.0;
