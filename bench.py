@@ -459,6 +459,7 @@ class BackwardOracleTimer(OracleTimer):
         dos = self.host_do if host is not None else self.do[:, :, :tp].to("cpu", torch.float64).numpy()
         t0 = time.perf_counter()
         self.orc.backward(qs, ks, vs, dos, feature_map=w.feature_map, gamma=w.gammas(),
+                          normalize=w.normalize,
                           nthreads=self.threads)
         return time.perf_counter() - t0
 
@@ -478,48 +479,66 @@ def backward_native(w, algorithm: str) -> bool:
 
 def backward_bytes(w, out_elem: int, algorithm: str, lseg: int = 0):
     """Algorithmic bytes per launch of every kernel of the backward, in launch order, for
-    the bench's call (no initial or final state): the input preparation (reversed copies,
-    psi), three prefills -- (do, v, psi(k)), reversed (k, q, do), reversed (v, do, psi(q));
-    two more for the lo halves of psi under ELU+1 with bf16 inputs -- and the output
-    finish (reversal back, psi')."""
+    the bench's call (no initial or final state).  The element-wise input preparation
+    (reversed copies where the reversed passes cannot run natively, psi(k) and psi(q) as
+    bf16 hi / lo pairs under ELU+1); the prefill (do, v, psi(k)); for the normalised form
+    the forward scan of Z (d_t, dd_t, dn_t as hi / lo, grad_q) and psi(q) / d_t; the
+    prefills reversed (k, q, do or dn) and reversed (v, do, psi(q) [/ d]); each prefill
+    once per bf16 half of its split operand; the reverse scan of the normaliser gradient;
+    the output finish."""
     BH = w.B * w.H
     e = 2 if w.dtype == "bf16" else 4
     elu = w.feature_map == "elu1"
     split = elu and w.dtype == "bf16"
+    norm = w.normalize
     native = backward_native(w, algorithm)
-    wk, wv = (not native) or elu, not native
+    halves = 2 if split else 1
+    wk, wv = (not native) or elu, (not native) or norm
     w_f32 = native or out_elem == 4 or elu
     ew = 4 if w_f32 else 2
-    nk, nv = BH * w.T * w.dk, BH * w.T * w.dv
+    nk, nv, nt = BH * w.T * w.dk, BH * w.T * w.dv, BH * w.T
     ops = []
-    n_in = (0 if native else 2 * nk + 2 * nv) + (2 * nk if elu else 0) + (2 * nk if split else 0)
-    if n_in:
-        ops.append(("bwd_reverse_inputs", 2 * n_in * e))
+    pre = (0 if native else 2 * nk + 2 * nv)
+    if elu:
+        pre += halves * nk * (1 if norm else 2)   # psi(k) (and psi(q) unnormalised)
+    if pre:
+        ops.append(("bwd_reverse_inputs", 2 * pre * e))
     wa = w.with_(dk=w.dv, dv=w.dk, feature_map="identity", normalize=False)
     wb = w.with_(normalize=False)
-    passes = [(wa, 4 if elu else out_elem)] * (2 if split else 1) + \
-        [(wb, ew if wv else out_elem)] + [(wa, ew if wk else out_elem)] * (2 if split else 1)
-    for pw, oe in passes:
+
+    def prefills(pw, oe, n):
         algo = effective_algorithm(pw, algorithm)
-        for name in kernel_names(pw, algo, "logdepth", lseg):
-            ops.append((name, kernel_bytes(pw, name, oe, algo, lseg)))
+        for _ in range(n):
+            for name in kernel_names(pw, algo, "logdepth", lseg):
+                ops.append((name, kernel_bytes(pw, name, oe, algo, lseg)))
+    prefills(wa, 4 if elu else out_elem, halves)
+    if norm:
+        # totals read k; the walk reads k, q, do, S do (hi and lo passes), writes dn (hi /
+        # lo), dd, 1 / d, grad_q
+        ops.append(("bwd_z_scan", nk * e + 2 * nk * e + nv * e + halves * nk * 4
+                    + halves * nv * e + 2 * nt * 4 + nk * out_elem))
+        ops.append(("bwd_scaled_psi_q", halves * (2 * nk * e + nt * 4)))
+    prefills(wb, ew if wv else out_elem, halves if norm else 1)
+    prefills(wa, ew if wk else out_elem, halves)
+    if norm:  # g scan: totals and walk read q and dd; the walk writes g
+        ops.append(("bwd_g_scan", 2 * (nk * e + nt * 4) + nk * 4))
     post = 0
     if wv:
-        post += nv * ew + nv * out_elem
+        post += nv * ew * (halves if norm else 1) + nv * out_elem
     if wk:
         post += nk * ew + nk * out_elem + (nk * 4 if split else 0) + (nk * e if elu else 0)
-    if elu:
-        post += nk * 4 + (nk * 4 if split else 0) + nk * e + nk * out_elem
+    if elu and not norm:
+        post += nk * 4 * halves + nk * e + nk * out_elem
+    if norm:
+        post += nk * 4  # the g term
     if post:
         ops.append(("bwd_reverse_outputs", post))
     return ops
 
 
 def backward_bench(args, w, info, dev):
-    """One backward of the unnormalised form (lin_attn_backward: grad_q, grad_k, grad_v for
-    a given grad_out) per step, timed like the prefill."""
-    if w.normalize:
-        w = w.with_(normalize=False, name=f"{w.name}_unnormalised")
+    """One backward (lin_attn_backward: grad_q, grad_k, grad_v for a given grad_out) per
+    step, timed like the prefill."""
     q, k, v = make_inputs(w, seed=info.rank, device=dev)
     g = torch.Generator(device=dev).manual_seed(1000 + info.rank)
     do = torch.randn((w.B, w.H, w.T, w.dv), generator=g, device=dev).to(q.dtype)
@@ -530,11 +549,15 @@ def backward_bench(args, w, info, dev):
     gv = torch.empty(v.shape, dtype=odt, device=dev)
     gam = w.gammas()
     ws = torch.empty(B.lin_attn_backward_workspace_bytes(q, v, chunk=w.C, feature_map=w.feature_map,
-                                                        out_dtype=args.out_dtype, gamma=gam),
+                                                        out_dtype=args.out_dtype, gamma=gam,
+                                                        normalize=w.normalize,
+                                                        algorithm=args.algorithm),
                      dtype=torch.uint8, device=dev)
     kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, out_dtype=args.out_dtype,
               kernel_path="tensor_core", algorithm=args.algorithm, workspace=ws,
               segment_chunks=args.segment_chunks)
+    if w.normalize:
+        kw.update(normalize=True)
 
     def step():
         B.lin_attn_backward(q, k, v, do, gq, gk, gv, **kw)

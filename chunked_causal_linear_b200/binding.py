@@ -71,7 +71,9 @@ class BackwardArgs(ctypes.Structure):
         ("out_dtype", ctypes.c_int), ("scan_mode", ctypes.c_int), ("kernel_path", ctypes.c_int),
         ("algorithm", ctypes.c_int), ("segment_chunks", ctypes.c_int),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-        ("stream", ctypes.c_void_p),
+        ("stream", ctypes.c_void_p), ("normalize", ctypes.c_int), ("eps", ctypes.c_float),
+        ("Z_init", ctypes.c_void_p), ("grad_Z_final", ctypes.c_void_p),
+        ("grad_Z_init", ctypes.c_void_p),
     ]
 
 
@@ -274,7 +276,9 @@ def lin_attn_prefill_host(q, k, v, out, S_final=None, Z_final=None, *, chunk=64,
 def make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init=None,
                        grad_S_final=None, grad_S_init=None, chunk=64, feature_map="identity",
                        gamma=None, out_dtype="as_input", scan="logdepth", kernel_path="auto",
-                       algorithm="auto", segment_chunks=0, workspace=None, stream=None):
+                       algorithm="auto", segment_chunks=0, workspace=None, stream=None,
+                       normalize=False, eps=0.0, Z_init=None, grad_Z_final=None,
+                       grad_Z_init=None):
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     garr, gptr = _gamma_array(gamma, H)
@@ -294,6 +298,9 @@ def make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init=None
     a.workspace = _ptr(workspace)
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = stream
+    a.normalize = int(bool(normalize))
+    a.eps = float(eps)
+    a.Z_init, a.grad_Z_final, a.grad_Z_init = _ptr(Z_init), _ptr(grad_Z_final), _ptr(grad_Z_init)
     return a, garr
 
 
@@ -301,11 +308,12 @@ def lin_attn_backward(q, k, v, grad_out, grad_q=None, grad_k=None, grad_v=None, 
                       S_init=None, grad_S_final=None, want_grad_S_init=False, grad_S_init=None,
                       chunk=64, feature_map="identity", gamma=None, out_dtype="as_input",
                       scan="logdepth", kernel_path="auto", algorithm="auto", segment_chunks=0,
-                      workspace=None, stream=None):
-    """Gradients of the unnormalised form for the loss <grad_out, out> + <grad_S_final,
-    S_final> (see the header).  q, k [B,H,T,dk], v, grad_out [B,H,T,dv] on the device.
-    Allocates the gradients not given.  Returns (grad_q, grad_k, grad_v, grad_S_init);
-    grad_S_init is None unless requested (want_grad_S_init or a tensor)."""
+                      workspace=None, stream=None, normalize=False, eps=0.0, Z_init=None,
+                      grad_Z_final=None, want_grad_Z_init=False, grad_Z_init=None):
+    """Gradients for the loss <grad_out, out> + <grad_S_final, S_final> (+ <grad_Z_final,
+    Z_final> normalised; see the header).  q, k [B,H,T,dk], v, grad_out [B,H,T,dv] on the
+    device.  Allocates the gradients not given.  Returns (grad_q, grad_k, grad_v, grad_S_init), plus grad_Z_init
+    when normalising; the state gradients are None unless requested."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     odt = torch.float32 if out_dtype == "f32" else q.dtype
@@ -315,14 +323,20 @@ def lin_attn_backward(q, k, v, grad_out, grad_q=None, grad_k=None, grad_v=None, 
     grad_v = mk(dv) if grad_v is None else grad_v
     if grad_S_init is None and want_grad_S_init:
         grad_S_init = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if grad_Z_init is None and want_grad_Z_init:
+        grad_Z_init = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
     a, keep = make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, S_init=S_init,
                                  grad_S_final=grad_S_final, grad_S_init=grad_S_init, chunk=chunk,
                                  feature_map=feature_map, gamma=gamma, out_dtype=out_dtype,
                                  scan=scan, kernel_path=kernel_path, algorithm=algorithm,
                                  segment_chunks=segment_chunks, workspace=workspace,
-                                 stream=_stream_handle(stream))
+                                 stream=_stream_handle(stream), normalize=normalize, eps=eps,
+                                 Z_init=Z_init, grad_Z_final=grad_Z_final,
+                                 grad_Z_init=grad_Z_init)
     _check("lin_attn_backward", load_library().lin_attn_backward(ctypes.byref(a)))
     del keep
+    if normalize:
+        return grad_q, grad_k, grad_v, grad_S_init, grad_Z_init
     return grad_q, grad_k, grad_v, grad_S_init
 
 
@@ -330,7 +344,8 @@ def lin_attn_backward_timed(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init
                             grad_S_final=None, grad_S_init=None, chunk=64, feature_map="identity",
                             gamma=None, out_dtype="as_input", scan="logdepth", kernel_path="auto",
                             algorithm="auto", segment_chunks=0, workspace=None,
-                            stream=None) -> list[tuple[str, float]]:
+                            stream=None, normalize=False,
+                            eps=0.0) -> list[tuple[str, float]]:
     """Runs the backward once with an event around every kernel; returns (name,
     milliseconds) per kernel in launch order (synchronous)."""
     a, keep = make_backward_args(q, k, v, grad_out, grad_q, grad_k, grad_v, S_init=S_init,
@@ -338,7 +353,7 @@ def lin_attn_backward_timed(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init
                                  feature_map=feature_map, gamma=gamma, out_dtype=out_dtype,
                                  scan=scan, kernel_path=kernel_path, algorithm=algorithm,
                                  segment_chunks=segment_chunks, workspace=workspace,
-                                 stream=_stream_handle(stream))
+                                 stream=_stream_handle(stream), normalize=normalize, eps=eps)
     cap = 48
     ms = (ctypes.c_float * cap)()
     names = (ctypes.c_char_p * cap)()
@@ -352,7 +367,7 @@ def lin_attn_backward_timed(q, k, v, grad_out, grad_q, grad_k, grad_v, *, S_init
 
 def lin_attn_backward_workspace_bytes(q, v, *, chunk=64, feature_map="identity",
                                       out_dtype="as_input", S_init=False, grad_S_final=False,
-                                      gamma=None) -> int:
+                                      gamma=None, normalize=False, algorithm="auto") -> int:
     """Workspace bytes of lin_attn_backward for these shapes and options (S_init /
     grad_S_final: whether they will be given)."""
     B, H, T, dk = q.shape
@@ -363,6 +378,8 @@ def lin_attn_backward_workspace_bytes(q, v, *, chunk=64, feature_map="identity",
     a.gamma = gptr
     a.dtype = DTYPES[q.dtype]
     a.out_dtype = OUT_DTYPES[out_dtype]
+    a.normalize = int(bool(normalize))
+    a.algorithm = ALGORITHMS[algorithm]
     # Only whether the states are given matters to the size; any non-null value says so.
     a.S_init = 16 if S_init else None
     a.grad_S_final = 16 if grad_S_final else None

@@ -70,14 +70,16 @@ __device__ __forceinline__ void store4(void* base, long long idx, float4 x, bool
   __stcs(reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + idx), u);
 }
 
-// dst[bh, t'] = f(src[bh, t] + src2[bh, t]) * g(x[bh, t']) for rows of d elements, where
-// t' = T-1-t when `flip`, else t; f = psi when `fm_src` is ELU+1, g = psi' of x when `x` is
-// given.  With `lo`, dst receives the part of the value that bf16 rounding drops
+// dst[bh, t'] = (f(src[bh, t] + src2[bh, t]) rs[bh, t] + src3[bh, t]) g(x[bh, t']) for rows
+// of d elements, where t' = T-1-t when `flip`, else t; f = psi when `fm_src` is ELU+1,
+// g = psi' of x when `x` is given (absent terms drop out).  With `lo`, dst receives the part of the value that bf16 rounding drops
 // (value - bf16(value), itself rounded to bf16): a bf16 hi + lo pair carries psi to about
 // 16 bits, like the split operands of the prefill's own kernels.
 struct RowJob {
   const void* src;
   const void* src2;  // added to src (same type), or nullptr
+  const void* src3;  // added after the row scale, or nullptr
+  const float* rs;   // per-row scale of (src + src2), indexed by the source row, or nullptr
   void* dst;
   const void* x;     // multiplier input (same layout as dst, type of the inputs) or nullptr
   int d;
@@ -107,6 +109,14 @@ __global__ void __launch_bounds__(256) row_jobs(RowJobs jobs, long long BH, long
     }
     if (J.fm_src == LA_FM_ELU1)
       a = make_float4(psi(a.x, 1), psi(a.y, 1), psi(a.z, 1), psi(a.w, 1));
+    if (J.rs) {
+      const float r = J.rs[row];
+      a = make_float4(a.x * r, a.y * r, a.z * r, a.w * r);
+    }
+    if (J.src3) {
+      const float4 b = load4(J.src3, row * J.d + col, J.src_f32);
+      a = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    }
     if (J.lo) {
       auto rest = [](float v) { return v - __bfloat162float(__float2bfloat16_rn(v)); };
       a = make_float4(rest(a.x), rest(a.y), rest(a.z), rest(a.w));
@@ -118,6 +128,194 @@ __global__ void __launch_bounds__(256) row_jobs(RowJobs jobs, long long BH, long
     }
     store4(J.dst, drow * J.d + col, a, J.dst_f32);
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// Decayed vector scans of the normalised form's gradient: y_t = gamma y_{t-1} + x_t over the
+// tokens of each (b, h) in scan order (t = 0 .. T-1, or T-1 .. 0 in reverse), x_t a
+// d-vector (d <= 128):
+//   mode 0 (forward)  x_t = psi(k_t), with gamma Z_init folded into the first element: y_t
+//                     is the normaliser Z_t.  Per token the walk forms the denominator
+//                     d_t = psi(q_t) . Z_t + eps, and from A_t = S_t do_t (the grad_q
+//                     pass's output, computed before the walk): do_t . n_t = psi(q_t) . A_t,
+//                     dd_t = -(do_t . n_t) / d_t^2, grad_q_t = psi'(q_t) (A_t / d_t +
+//                     dd_t Z_t), 1 / d_t and dn_t = do_t / d_t (the grad_v pass's value).
+//   mode 1 (reverse)  x_t = dd_t psi(q_t), with grad_Z_final folded into the first
+//                     element (token T-1, no decay): y_t is g_t, part of dpsi(k_t); the
+//                     walk writes it and grad_Z_init = gamma g_0.
+// Three launches: each segment's decayed total (one warp per segment of Ls tokens), the
+// exclusive scan over segments (one thread per (b, h, feature)), and the walk from each
+// segment's prefix.  Lane l holds features 4l .. 4l + 3.
+struct VecScan {
+  int BH, H;
+  long long T;
+  int d, dv;        // features of x (dk) and of do / o / dn (dv)
+  int Ls, NS;       // tokens per segment, segments per (b, h)
+  int mode;         // 0 or 1 (see above)
+  int fm;
+  bool in_f32;      // q, k, grad_out (and dn) are float32, else bf16
+  const void* x;    // k (mode 0) or q (mode 1)
+  const void* q;    // mode 0: psi(q) for the denominator
+  const void* dout;       // mode 0
+  const float* A;         // mode 0: S_t do_t [BH, T, d], and its lo pass (or nullptr)
+  const float* A_lo;
+  void* grad_q;           // mode 0: [BH, T, d], float32 or bf16
+  bool gq_f32;
+  float eps;
+  const float* init;      // Z_init (mode 0) or grad_Z_final (mode 1), [BH, d], or nullptr
+  float* tot;             // [BH, NS, d]: segment totals, then exclusive prefixes
+  float* dd;              // [BH, T]: written by mode 0, read by mode 1
+  float* inv_den;         // mode 0: [BH, T], 1 / d_t
+  void* dn;               // mode 0: [BH, T, dv] in the input type
+  void* dn_lo;            // mode 0: bf16 inputs: the residual dn - bf16(dn), else nullptr
+  bool dn_rev;            // mode 0: write dn's rows in reversed order
+  float* y_out;           // mode 1: g_t [BH, T, d]
+  bool y_rev;             // mode 1: write row T-1-t instead of t
+  float* init_grad;       // mode 1: grad_Z_init [BH, d] or nullptr
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// x_t for this lane's four features; `pos` is the scan position of token t.
+__device__ __forceinline__ float4 vs_x(const VecScan& p, long long bh, long long t, long long pos,
+                                       int col, float g) {
+  float4 a = load4(p.x, (bh * p.T + t) * p.d + col, p.in_f32);
+  a = make_float4(psi(a.x, p.fm), psi(a.y, p.fm), psi(a.z, p.fm), psi(a.w, p.fm));
+  if (p.mode == 1) {
+    const float w = p.dd[bh * p.T + t];
+    a = make_float4(a.x * w, a.y * w, a.z * w, a.w * w);
+  }
+  if (pos == 0 && p.init) {
+    const float4 z = *reinterpret_cast<const float4*>(p.init + bh * p.d + col);
+    const float w = p.mode == 0 ? g : 1.f;
+    a = make_float4(fmaf(w, z.x, a.x), fmaf(w, z.y, a.y), fmaf(w, z.z, a.z), fmaf(w, z.w, a.w));
+  }
+  return a;
+}
+
+__global__ void __launch_bounds__(128) vs_totals(VecScan p, GammaTable gt) {
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<long long>(p.BH) * p.NS) return;
+  const long long bh = wid / p.NS;
+  const int seg = static_cast<int>(wid - bh * p.NS);
+  const float g = gt.g[bh % p.H];
+  const int col = 4 * lane;
+  if (col >= p.d) return;
+  const long long p0 = static_cast<long long>(seg) * p.Ls, p1 = min(p.T, p0 + p.Ls);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long pos = p0; pos < p1; ++pos) {
+    const long long t = p.mode == 1 ? p.T - 1 - pos : pos;
+    const float4 x = vs_x(p, bh, t, pos, col, g);
+    acc = make_float4(fmaf(g, acc.x, x.x), fmaf(g, acc.y, x.y), fmaf(g, acc.z, x.z),
+                      fmaf(g, acc.w, x.w));
+  }
+  *reinterpret_cast<float4*>(p.tot + (bh * p.NS + seg) * p.d + col) = acc;
+}
+
+__global__ void vs_prefix(VecScan p, GammaTable gt) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(p.BH) * p.d) return;
+  const long long bh = idx / p.d;
+  const int f = static_cast<int>(idx - bh * p.d);
+  const float g = gt.g[bh % p.H];
+  const float gL = powf(g, static_cast<float>(p.Ls));
+  float P = 0.f;
+  for (int s = 0; s < p.NS; ++s) {
+    float* e = p.tot + (bh * p.NS + s) * p.d + f;
+    const float t = *e;
+    *e = P;
+    P = fmaf(gL, P, t);  // only the last segment can be short, and nothing follows it
+  }
+}
+
+__global__ void __launch_bounds__(128) vs_walk(VecScan p, GammaTable gt) {
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<long long>(p.BH) * p.NS) return;
+  const long long bh = wid / p.NS;
+  const int seg = static_cast<int>(wid - bh * p.NS);
+  const float g = gt.g[bh % p.H];
+  const int col = 4 * lane, vcol = 4 * lane;
+  const bool fx = col < p.d, fv = vcol < p.dv;
+  const long long p0 = static_cast<long long>(seg) * p.Ls, p1 = min(p.T, p0 + p.Ls);
+  float4 acc = fx ? *reinterpret_cast<const float4*>(p.tot + (bh * p.NS + seg) * p.d + col)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long pos = p0; pos < p1; ++pos) {
+    const long long t = p.mode == 1 ? p.T - 1 - pos : pos;
+    const long long row = bh * p.T + t;
+    if (fx) {
+      const float4 x = vs_x(p, bh, t, pos, col, g);
+      acc = make_float4(fmaf(g, acc.x, x.x), fmaf(g, acc.y, x.y), fmaf(g, acc.z, x.z),
+                        fmaf(g, acc.w, x.w));
+    }
+    if (p.mode == 0) {
+      float part = 0.f, part_n = 0.f;
+      float4 xq = make_float4(0.f, 0.f, 0.f, 0.f), A = xq;
+      if (fx) {
+        xq = load4(p.q, row * p.d + col, p.in_f32);
+        const float4 fq = make_float4(psi(xq.x, p.fm), psi(xq.y, p.fm), psi(xq.z, p.fm),
+                                      psi(xq.w, p.fm));
+        A = __ldcs(reinterpret_cast<const float4*>(p.A + row * p.d + col));
+        if (p.A_lo) {
+          const float4 b = __ldcs(reinterpret_cast<const float4*>(p.A_lo + row * p.d + col));
+          A = make_float4(A.x + b.x, A.y + b.y, A.z + b.z, A.w + b.w);
+        }
+        part = fq.x * acc.x + fq.y * acc.y + fq.z * acc.z + fq.w * acc.w;
+        part_n = fq.x * A.x + fq.y * A.y + fq.z * A.z + fq.w * A.w;
+      }
+      const float den = warp_sum(part) + p.eps;
+      const float r = 1.f / den;
+      const float ddt = -warp_sum(part_n) * r * r;
+      float4 dov = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (fv) dov = load4(p.dout, row * p.dv + vcol, p.in_f32);
+      if (fv) {
+        const float4 dn = make_float4(dov.x * r, dov.y * r, dov.z * r, dov.w * r);
+        const long long drow = p.dn_rev ? bh * p.T + (p.T - 1 - t) : row;
+        store4(p.dn, drow * p.dv + vcol, dn, p.in_f32);
+        if (p.dn_lo) {
+          auto rest = [](float x) { return x - __bfloat162float(__float2bfloat16_rn(x)); };
+          store4(p.dn_lo, drow * p.dv + vcol,
+                 make_float4(rest(dn.x), rest(dn.y), rest(dn.z), rest(dn.w)), false);
+        }
+      }
+      if (lane == 0) {
+        p.dd[row] = ddt;
+        p.inv_den[row] = r;
+      }
+      if (fx) {  // dpsi(q_t) = A_t / d_t + dd_t Z_t, times psi'(q_t)
+        const float4 gq = make_float4(fmaf(A.x, r, ddt * acc.x) * psi_prime(xq.x, p.fm),
+                                      fmaf(A.y, r, ddt * acc.y) * psi_prime(xq.y, p.fm),
+                                      fmaf(A.z, r, ddt * acc.z) * psi_prime(xq.z, p.fm),
+                                      fmaf(A.w, r, ddt * acc.w) * psi_prime(xq.w, p.fm));
+        store4(p.grad_q, row * p.d + col, gq, p.gq_f32);
+      }
+    } else if (fx) {
+      const long long wrow = p.y_rev ? bh * p.T + (p.T - 1 - t) : row;
+      __stcs(reinterpret_cast<float4*>(p.y_out + wrow * p.d + col), acc);
+    }
+  }
+  if (p.mode == 1 && p.init_grad && fx && p1 == p.T && p0 < p1)  // the segment ending at token 0
+    *reinterpret_cast<float4*>(p.init_grad + bh * p.d + col) =
+        make_float4(g * acc.x, g * acc.y, g * acc.z, g * acc.w);
+}
+
+cudaError_t launch_vec_scan(const VecScan& p, const GammaTable& gt, cudaStream_t s) {
+  const long long warps = static_cast<long long>(p.BH) * p.NS;
+  const unsigned wb = static_cast<unsigned>((warps + 3) / 4);
+  vs_totals<<<wb, 128, 0, s>>>(p, gt);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n = static_cast<long long>(p.BH) * p.d;
+  vs_prefix<<<static_cast<unsigned>((n + 127) / 128), 128, 0, s>>>(p, gt);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  vs_walk<<<wb, 128, 0, s>>>(p, gt);
+  return cudaGetLastError();
 }
 
 // dst[bh] = scale_h * (transpose ? src[bh]^T : src[bh]) for [rows x cols] float32
@@ -214,6 +412,21 @@ bool has_small_decay(const la_backward_args& a) {
   return false;
 }
 
+// Segments of the normaliser scans: about 32 warps per SM in all, at least 64 tokens each.
+void vec_segments(size_t BH, size_t T, int* Ls, int* NS) {
+  if (BH == 0 || T == 0) {
+    *Ls = 1;
+    *NS = 0;
+    return;
+  }
+  const size_t want = std::max<size_t>(1, (148 * 32 + BH - 1) / BH);
+  const size_t most = (T + 63) / 64;
+  const size_t ns = std::min(want, most);
+  const size_t ls = (T + ns - 1) / ns;
+  *Ls = static_cast<int>(ls);
+  *NS = static_cast<int>((T + ls - 1) / ls);
+}
+
 // Whether the two reversed passes run on the segmented kernels in reverse mode (reading
 // the inputs and writing the outputs in memory order) rather than on reversed copies.  A
 // pure function of the arguments: bf16 inputs, C = 64, dk = dv = 128, a tensor-core
@@ -232,13 +445,15 @@ bool native_reverse(const la_backward_args& a) {
 //   order [T, dk], each with its bf16 residual (lo) when the inputs are bf16.
 //   Outputs of the reversed passes Wk [T, dk], Wv [T, dv] where they cannot go straight to
 //   grad_k / grad_v: always without native reverse (float32 when multiplied by psi' or
-//   corrected, else the output type); with it, float32 and only where psi' or the
-//   small-decay terms still apply.  ELU+1: the grad_q pass's float32 output Wq [T, dk] and
+//   corrected, else the output type); with it, float32 and only where psi', the
+//   small-decay terms or the normalised form's lo pass still apply.  ELU+1: the grad_q pass's float32 output Wq [T, dk] and
 //   the lo passes' float32 outputs.
 //   Three [dk x dv] states per (b, h), then the prefill workspace.
 struct BwdLayout {
-  size_t kr, qr, dor, vr, pq, pk, pq_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC, pw, total;
-  bool native, elu, split, fix, wk, wv, w_f32;
+  size_t kr, qr, dor, vr, pq, pk, pq_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC;
+  size_t dn, dn_lo, Wv_lo, dd, inv_den, Wkg, vtot, pw, total;
+  int Ls, NS;  // the normaliser scans' segments
+  bool native, elu, split, fix, wk, wv, w_f32, norm;
 };
 
 BwdLayout bwd_layout(const la_backward_args& a) {
@@ -248,11 +463,12 @@ BwdLayout bwd_layout(const la_backward_args& a) {
   const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
   const bool out_f32 = a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32;
   l.native = native_reverse(a);
+  l.norm = a.normalize != 0;
   l.elu = a.feature_map == LA_FM_ELU1;
   l.split = l.elu && a.dtype == LA_DTYPE_BF16;
   l.fix = has_small_decay(a);
   l.wk = !l.native || l.elu || l.fix;
-  l.wv = !l.native || l.fix;
+  l.wv = !l.native || l.fix || a.normalize;
   l.w_f32 = l.native || out_f32 || l.elu || l.fix;
   const size_t ew = l.w_f32 ? 4 : 2;
   const size_t nk = BH * T * a.dk, nv = BH * T * a.dv, ns = BH * a.dk * a.dv * 4;
@@ -279,6 +495,17 @@ BwdLayout bwd_layout(const la_backward_args& a) {
   l.SA = take(a.S_init ? ns : 0);
   l.SB = take(a.grad_S_final ? ns : 0);
   l.SC = take(a.grad_S_final ? ns : 0);
+  // The normalised form: dn = do / d as hi / lo (reversed without native reverse), the lo
+  // pass's output of grad_v, dd, 1 / d, the g term of dpsi(k), and the scans' segment
+  // records.
+  vec_segments(BH, T, &l.Ls, &l.NS);
+  l.dn = take(l.norm ? nv * e : 0);
+  l.dn_lo = take(l.norm && l.split ? nv * e : 0);
+  l.Wv_lo = take(l.norm && l.split ? nv * 4 : 0);
+  l.dd = take(l.norm ? BH * T * 4 : 0);
+  l.inv_den = take(l.norm ? BH * T * 4 : 0);
+  l.Wkg = take(l.norm ? nk * 4 : 0);
+  l.vtot = take(l.norm ? BH * static_cast<size_t>(l.NS) * a.dk * 4 : 0);
   l.pw = off;
   off += lin_attn_prefill_workspace_bytes(a.B, a.H, a.T, a.dk, a.dv, a.C, 0);
   l.total = off;
@@ -323,8 +550,13 @@ int validate(const la_backward_args& a) {
   if (a.workspace && (reinterpret_cast<uintptr_t>(a.workspace) & 255u) != 0)
     return LA_ERR_INVALID_ARGUMENT;
   for (const void* p : {static_cast<const void*>(a.S_init), static_cast<const void*>(a.grad_S_final),
-                        static_cast<const void*>(a.grad_S_init)})
+                        static_cast<const void*>(a.grad_S_init), static_cast<const void*>(a.Z_init),
+                        static_cast<const void*>(a.grad_Z_final),
+                        static_cast<const void*>(a.grad_Z_init)})
     if (!aligned16(p)) return LA_ERR_INVALID_ARGUMENT;
+  if (a.normalize != 0 && a.normalize != 1) return LA_ERR_INVALID_ARGUMENT;
+  if (a.normalize && a.feature_map != LA_FM_ELU1) return LA_ERR_INVALID_ARGUMENT;
+  if (!(a.eps >= 0.f) || !std::isfinite(a.eps)) return LA_ERR_INVALID_ARGUMENT;
   // The three passes' shapes and options, checked as the prefill will check them (as
   // states-only calls, so that no output buffer is needed; q stands for every input).
   const long long BH = static_cast<long long>(a.B) * a.H;
@@ -385,12 +617,15 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
   if (BH == 0) return LA_OK;
   const size_t state_bytes = static_cast<size_t>(BH) * a.dk * a.dv * 4;
   if (a.T == 0) {
-    // No tokens: S_final = S_init, so dS_init = dS_final.
-    if (!a.grad_S_init) return LA_OK;
-    cudaError_t e = a.grad_S_final
-                        ? cudaMemcpyAsync(a.grad_S_init, a.grad_S_final, state_bytes,
-                                          cudaMemcpyDeviceToDevice, s)
-                        : cudaMemsetAsync(a.grad_S_init, 0, state_bytes, s);
+    // No tokens: S_final = S_init and Z_final = Z_init, so the gradients pass through.
+    auto pass = [&](float* dst, const float* src, size_t bytes) {
+      if (!dst) return cudaSuccess;
+      return src ? cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s)
+                 : cudaMemsetAsync(dst, 0, bytes, s);
+    };
+    cudaError_t e = pass(a.grad_S_init, a.grad_S_final, state_bytes);
+    if (e == cudaSuccess && a.normalize)
+      e = pass(a.grad_Z_init, a.grad_Z_final, static_cast<size_t>(BH) * a.dk * 4);
     return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
   }
 
@@ -420,8 +655,9 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
   // Inputs of the passes: reversed copies unless the reversed passes run natively; for
   // ELU+1, psi(q) (reversed likewise) and psi(k) in order, as hi / lo pairs for bf16.
   auto job = [](RowJobs& J, int& n, const void* src, const void* src2, void* dst, const void* x,
-                int d, int fm_src, int fm_x, bool flip, bool lo, bool sf, bool df, bool xf) {
-    J.j[n++] = RowJob{src, src2, dst, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
+                int d, int fm_src, int fm_x, bool flip, bool lo, bool sf, bool df, bool xf,
+                const void* src3 = nullptr, const float* rs = nullptr) {
+    J.j[n++] = RowJob{src, src2, src3, rs, dst, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
   };
   RowJobs pre{};
   int np = 0;
@@ -433,12 +669,15 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
         f, f, f);
     job(pre, np, a.v, nullptr, at(l.vr), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f, f, f);
   }
+  // (The normalised form's psi(q) is scaled by 1 / d_t, known only after its scan.)
   if (elu) {
-    job(pre, np, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f);
+    if (!l.norm)
+      job(pre, np, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f);
     job(pre, np, a.k, nullptr, at(l.pk), nullptr, a.dk, LA_FM_ELU1, 0, false, false, f, f, f);
   }
   if (l.split) {
-    job(pre, np, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f);
+    if (!l.norm)
+      job(pre, np, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f);
     job(pre, np, a.k, nullptr, at(l.pk_lo), nullptr, a.dk, LA_FM_ELU1, 0, false, true, f, f, f);
   }
   cudaError_t e = launch_rows(pre, np, BH, T, s, rec, "bwd_reverse_inputs");
@@ -490,6 +729,60 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
       run(p);
     }
   }
+  // The normalised form: Z_t by a forward scan whose walk forms d_t, dd_t, dn_t and grad_q.
+  // The two terms of dpsi(q_t) (A_t / d_t and Z_t dd_t) nearly cancel, and so do the two of
+  // dpsi(k_s) (G_s v_s and g_s): both are sums of psi terms weighted by (v_s - o_t) . do_t
+  // / d_t.  So nothing that meets such a cancellation passes through a bf16 rounding of
+  // dn_t or of the output: the grad_q pass runs on do (A_t = S_t do_t) and the walk takes
+  // do_t . n_t = psi(q_t) . A_t from it, both in float32; the dpsi(k) pass runs on do with
+  // the value psi(q_t) / d_t (split hi / lo).  The grad_v pass takes dn_t as its value,
+  // split into bf16 hi and lo: its largest entries come from the first tokens, where d_t
+  // is small, and would carry dn's rounding whole.
+  VecScan vs{};
+  if (l.norm) {
+    vs.BH = static_cast<int>(BH);
+    vs.H = a.H;
+    vs.T = T;
+    vs.d = a.dk;
+    vs.dv = a.dv;
+    vs.Ls = l.Ls;
+    vs.NS = l.NS;
+    vs.fm = a.feature_map;
+    vs.in_f32 = in_f32;
+    vs.q = a.q;
+    vs.dout = a.grad_out;
+    vs.A = static_cast<const float*>(at(l.Wq));
+    vs.A_lo = l.split ? static_cast<const float*>(at(l.Wq_lo)) : nullptr;
+    vs.grad_q = a.grad_q;
+    vs.gq_f32 = out_f32;
+    vs.eps = a.eps;
+    vs.tot = static_cast<float*>(at(l.vtot));
+    vs.dd = static_cast<float*>(at(l.dd));
+    vs.inv_den = static_cast<float*>(at(l.inv_den));
+    vs.dn = at(l.dn);
+    vs.dn_lo = l.split ? at(l.dn_lo) : nullptr;
+    vs.dn_rev = rv;
+    VecScan z = vs;
+    z.mode = 0;
+    z.x = a.k;
+    z.init = a.Z_init;
+    if (st == LA_OK && e == cudaSuccess) {
+      if (rec) rec->mark(s, "bwd_z_scan");
+      e = launch_vec_scan(z, gt, s);
+      // psi(q_t) / d_t (reversed without native reverse), hi / lo for bf16.
+      RowJobs pq{};
+      int n = 0;
+      const float* rs = static_cast<const float*>(at(l.inv_den));
+      job(pq, n, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f,
+          nullptr, rs);
+      if (l.split)
+        job(pq, n, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f,
+            nullptr, rs);
+      if (e == cudaSuccess) e = launch_rows(pq, n, BH, T, s, rec, "bwd_scaled_psi_q");
+      if (e != cudaSuccess) st = LA_ERR_CUDA;
+    }
+  }
+
   // grad_v: (k, q, do) in reverse time with the model's map; final state G_0.
   const int w_dtype = l.w_f32 ? LA_OUT_F32 : LA_OUT_AS_INPUT;
   {
@@ -497,11 +790,18 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
     p.reverse = l.native;
     p.q = rv ? at(l.kr) : a.k;
     p.k = rv ? at(l.qr) : a.q;
-    p.v = rv ? at(l.dor) : a.grad_out;
+    p.v = l.norm ? at(l.dn) : (rv ? at(l.dor) : a.grad_out);
     p.out = l.wv ? at(l.Wv) : a.grad_v;
     p.S_init = SB;
     p.S_final = a.grad_S_init;
     run(p);
+    if (l.norm && l.split) {  // the lo half of dn (linear in the value, from a zero state)
+      p.v = at(l.dn_lo);
+      p.out = at(l.Wv_lo);
+      p.S_init = nullptr;
+      p.S_final = nullptr;
+      run(p);
+    }
   }
   // dpsi(k): (v, do, psi(q)) in reverse time, identity map (lo half as for grad_q).
   {
@@ -521,7 +821,20 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
     }
   }
   e = cudaSuccess;
-  if (st == LA_OK && l.fix) {
+  // The normalised form: g_t = sum_{s >= t} gamma^(s-t) dd_s psi(q_s) (+ the final
+  // normaliser's gradient), part of dpsi(k_t), by a reverse scan; grad_Z_init = gamma g_0.
+  if (st == LA_OK && l.norm) {
+    VecScan gs = vs;
+    gs.mode = 1;
+    gs.x = a.q;
+    gs.init = a.grad_Z_final;
+    gs.y_out = static_cast<float*>(at(l.Wkg));
+    gs.y_rev = rv;
+    gs.init_grad = a.grad_Z_init;
+    if (rec) rec->mark(s, "bwd_g_scan");
+    e = launch_vec_scan(gs, gt, s);
+  }
+  if (st == LA_OK && e == cudaSuccess && l.fix) {
     if (rec) rec->mark(s, "bwd_fix_small_decay");
     fix_small_decay<<<static_cast<unsigned>(BH), 128, 0, s>>>(
         a.grad_S_final, a.k, a.v, static_cast<float*>(at(l.Wk)), static_cast<float*>(at(l.Wv)),
@@ -541,12 +854,13 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
     int n = 0;
     const bool wf = l.w_f32;
     if (l.wv)
-      job(post, n, at(l.Wv), nullptr, a.grad_v, nullptr, a.dv, LA_FM_IDENTITY, 0, rv, false, wf,
-          out_f32, f);
+      job(post, n, at(l.Wv), l.norm && l.split ? at(l.Wv_lo) : nullptr, a.grad_v, nullptr, a.dv,
+          LA_FM_IDENTITY, 0, rv, false, wf, out_f32, f);
     if (l.wk)
       job(post, n, at(l.Wk), l.split ? at(l.Wk_lo) : nullptr, a.grad_k, a.k, a.dk,
-          LA_FM_IDENTITY, a.feature_map, rv, false, wf, out_f32, f);
-    if (elu)  // grad_q = psi'(q) .* dpsi(q)
+          LA_FM_IDENTITY, a.feature_map, rv, false, wf, out_f32, f,
+          l.norm ? at(l.Wkg) : nullptr);
+    if (elu && !l.norm)  // grad_q = psi'(q) .* dpsi(q) (the normalised walk wrote it)
       job(post, n, at(l.Wq), l.split ? at(l.Wq_lo) : nullptr, a.grad_q, a.q, a.dk,
           LA_FM_IDENTITY, a.feature_map, false, false, true, out_f32, f);
     e = launch_rows(post, n, BH, T, s, rec, "bwd_reverse_outputs");

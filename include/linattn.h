@@ -299,7 +299,17 @@ int lin_attn_prefill_noalloc(const la_prefill_args* args);
  * their outputs reversed back.  Under ELU+1 with bf16 inputs, psi(k) and psi(q) enter
  * two passes as the value operand; they are split into bf16 hi and lo halves and those
  * passes run once per half, so that psi keeps about 16 bits as in the forward kernels.
- * The normalised form's gradient is not provided.
+ * The normalised form (o_t = n_t / d_t, n_t = psi(q_t) S_t, d_t = psi(q_t) . Z_t + eps)
+ * has, with dn_t = grad_out_t / d_t and dd_t = -(grad_out_t . n_t) / d_t^2,
+ *     grad_q_t = psi'(q_t) .* (S_t dn_t + Z_t dd_t),
+ *     grad_k_t = psi'(k_t) .* (G_t v_t + g_t),   grad_v_t = G_t^T psi(k_t),
+ *     G_t = psi(q_t) dn_t^T + gamma G_{t+1},  g_t = psi(q_t) dd_t + gamma g_{t+1}
+ *     (G_{T-1}, g_{T-1} include grad_S_final, grad_Z_final),
+ *     grad_S_init = gamma G_0,   grad_Z_init = gamma g_0.
+ * The same three prefills compute S_t grad_out_t, G_t v_t (with the value psi(q_t) / d_t)
+ * and grad_v (with the value dn_t, as bf16 hi and lo halves); decayed vector scans over
+ * the tokens add Z_t (forward: it also forms d_t, dd_t from psi(q_t) . S_t grad_out_t,
+ * and grad_q) and g_t (reverse).
  *
  *   q, k, v, grad_out  DEVICE, the forward's inputs and dL/dout, type `dtype`,
  *                      [B,H,T,dk] / [B,H,T,dk] / [B,H,T,dv] / [B,H,T,dv].
@@ -338,6 +348,16 @@ typedef struct la_backward_args {
   void* workspace;            /* DEVICE, 256-byte aligned, or NULL */
   size_t workspace_bytes;
   la_stream_t stream;
+  /* The normalised form (normalize = 1; requires LA_FM_ELU1): o_t = n_t / d_t with
+   * n_t = psi(q_t) S_t, d_t = psi(q_t) . Z_t + eps (the forward's eps).  The forward's
+   * output is not needed: n_t and d_t are recomputed.  Z_init: the forward's initial
+   * normaliser or NULL; grad_Z_final: dL/dZ_final or NULL; grad_Z_init: output dL/dZ_init
+   * or NULL (all float32 [B,H,dk]). */
+  int normalize;
+  float eps;
+  const float* Z_init;
+  const float* grad_Z_final;
+  float* grad_Z_init;
 } la_backward_args;
 
 int lin_attn_backward(const la_backward_args* args);

@@ -207,6 +207,13 @@ def _bwd_args(**kw):
     (dict(grad_k=0x8000000 + 16), 1),               # grad_k overlaps grad_q
     (dict(S_init=0x100004), 1), (dict(grad_S_final=0x100008), 1),
     (dict(grad_S_init=0x100002), 1), (dict(workspace=0x100010), 1),
+    # the normalised form: ELU+1 only, a valid eps, aligned normaliser states
+    (dict(normalize=1), 1), (dict(normalize=2, feature_map=1), 1),
+    (dict(normalize=1, feature_map=1, eps=-1.0), 1),
+    (dict(normalize=1, feature_map=1, eps=float("nan")), 1),
+    (dict(normalize=1, feature_map=1, Z_init=0x100004), 1),
+    (dict(normalize=1, feature_map=1, grad_Z_final=0x100008), 1),
+    (dict(normalize=1, feature_map=1, grad_Z_init=0x100004), 1),
 ])
 def test_backward_argument_errors_before_any_launch(lib, kw, status):
     a = _bwd_args(**kw)
@@ -256,3 +263,12 @@ def test_backward_workspace_bytes(lib):
     n2 = 2 * 3 * 100 * 128
     want = 4 * al(n2 * 2) + 4 * al(n2 * 4) + pw2  # ELU+1: psi(q), psi(k) hi / lo; Wk, Wq, lo
     assert B.lin_attn_backward_workspace_bytes(q2, q2, feature_map="elu1", out_dtype="f32") == want
+    # normalised: the scans' segment records hold segments of at least 64 tokens
+    ns_seg = min(-(-148 * 32 // 6), -(-100 // 64))
+    ls = -(-100 // ns_seg)
+    ns_seg = -(-100 // ls)
+    # dn as hi / lo, grad_v's float32 output and its lo pass's, dd, 1 / d, the g term
+    extra = (2 * al(n2 * 2) + 2 * al(n2 * 4) + 2 * al(6 * 100 * 4) + al(n2 * 4)
+             + al(6 * ns_seg * 128 * 4))
+    assert B.lin_attn_backward_workspace_bytes(q2, q2, feature_map="elu1", out_dtype="f32",
+                                               normalize=True) == want + extra

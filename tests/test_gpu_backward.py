@@ -185,3 +185,113 @@ def test_backward_full_size_retention_sampled_heads():
                                         feature_map=w.feature_map, gamma=[gam[h]])
         for name, x, r in zip(("grad_q", "grad_k", "grad_v"), got[:3], ref[:3]):
             assert_close(to_np(sl(x)), r, TOL_BF16, f"head {h} {name}")
+
+
+# ---------------------------------------------------------------------------------------
+# The normalised form (ELU+1).
+
+def _norm_problem(T, *, decay=False, dtype="bf16", dk=128, dv=128, H=3, seed=0, states=False):
+    w = Workload("bwdn", B=2, H=H, T=T, dk=dk, dv=dv, C=64, dtype=dtype, scale=0.5,
+                 feature_map="elu1", decay=decay, normalize=True)
+    q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
+    g = torch.Generator().manual_seed(2000 + seed)
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    do = torch.randn((2, H, T, dv), generator=g).to(tdt).cuda()
+    gamma = gammas_for(H, seed) if decay else None
+    st = {}
+    if states:
+        st = dict(S_init=(torch.randn((2, H, dk, dv), generator=g) * 0.3).cuda(),
+                  Z_init=(torch.rand((2, H, dk), generator=g) * 5.0 + 1.0).cuda(),
+                  grad_S_final=torch.randn((2, H, dk, dv), generator=g).cuda(),
+                  grad_Z_final=torch.randn((2, H, dk), generator=g).cuda())
+    return q, k, v, do, gamma, st
+
+
+def _norm_case(q, k, v, do, gamma, st, *, eps=0.0, chunk=64, **kw):
+    got = B.lin_attn_backward(q, k, v, do, chunk=chunk, feature_map="elu1", gamma=gamma,
+                              normalize=True, eps=eps, want_grad_S_init=True,
+                              want_grad_Z_init=True, **st, **kw)
+    torch.cuda.synchronize()
+    f64 = lambda t: None if t is None else to_np(t).astype(np.float64)
+    ref = default_oracle().backward(to_np(q), to_np(k), to_np(v), to_np(do).astype(np.float64),
+                                    feature_map="elu1", gamma=gamma, normalize=True, eps=eps,
+                                    S_init=f64(st.get("S_init")), Z_init=f64(st.get("Z_init")),
+                                    dS_final=f64(st.get("grad_S_final")),
+                                    dZ_final=f64(st.get("grad_Z_final")))
+    return got, ref
+
+
+def _check_norm(got, ref, tol, rounded=False):
+    for name, g, r in zip(("grad_q", "grad_k", "grad_v", "grad_S_init", "grad_Z_init"), got, ref):
+        if rounded and name in ("grad_q", "grad_k", "grad_v"):
+            assert_close_rounded_out(to_np(g), r, tol, name)
+        else:
+            assert_close(to_np(g), r, tol, name)
+
+
+@pytest.mark.parametrize("decay", [False, True])
+@pytest.mark.parametrize("path,algorithm,T", [
+    ("tensor_core", "auto", 1000), ("tensor_core", "auto", 3001), ("tensor_core", "chunked", 700),
+    ("fma", "chunked", 333)])
+def test_normalised_backward_matches_oracle(decay, path, algorithm, T):
+    q, k, v, do, gamma, st = _norm_problem(T, decay=decay)
+    got, ref = _norm_case(q, k, v, do, gamma, st, out_dtype="f32", kernel_path=path,
+                          algorithm=algorithm)
+    _check_norm(got, ref, TOL_BF16)
+
+
+@pytest.mark.parametrize("decay", [False, True])
+@pytest.mark.parametrize("T", [1, 65, 1500])
+def test_normalised_backward_with_states_and_eps(decay, T):
+    q, k, v, do, gamma, st = _norm_problem(T, decay=decay, states=True)
+    got, ref = _norm_case(q, k, v, do, gamma, st, eps=0.5, out_dtype="f32")
+    _check_norm(got, ref, TOL_BF16)
+
+
+def test_normalised_backward_fp32():
+    q, k, v, do, gamma, st = _norm_problem(300, dtype="f32", dk=32, dv=48, decay=True,
+                                           states=True)
+    got, ref = _norm_case(q, k, v, do, gamma, st, eps=0.25, chunk=32)
+    _check_norm(got, ref, TOL_F32)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_normalised_backward_other_dims(dk, dv):
+    # d = 64 is the 4096-token normalised workload's head size
+    q, k, v, do, gamma, st = _norm_problem(2000, dk=dk, dv=dv)
+    got, ref = _norm_case(q, k, v, do, gamma, st, out_dtype="f32")
+    _check_norm(got, ref, TOL_BF16)
+
+
+def test_normalised_backward_bf16_gradients():
+    q, k, v, do, gamma, st = _norm_problem(900)
+    got, ref = _norm_case(q, k, v, do, gamma, st)
+    assert all(g.dtype == torch.bfloat16 for g in got[:3])
+    _check_norm(got, ref, TOL_BF16, rounded=True)
+
+
+def test_normalised_backward_zero_tokens():
+    q, k, v, do, gamma, st = _norm_problem(0, states=True)
+    *_, gS, gZ = B.lin_attn_backward(q, k, v, do, feature_map="elu1", normalize=True,
+                                     want_grad_S_init=True, want_grad_Z_init=True, **st)
+    torch.cuda.synchronize()
+    assert torch.equal(gS, st["grad_S_final"]) and torch.equal(gZ, st["grad_Z_final"])
+
+
+def test_normalised_backward_full_size_sampled_heads():
+    """The 16,000-token normalised workload (B=2, H=32, d=128, ELU+1) in the benchmark's
+    configuration; the oracle recomputes (b, h) = (0, 0) and (1, 31) in full."""
+    w = WORKLOADS["ragged_b2h32"]
+    q, k, v = make_inputs(w, seed=0, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(5)
+    do = torch.randn(q.shape[:3] + (w.dv,), generator=g, device="cuda").to(torch.bfloat16)
+    got = B.lin_attn_backward(q, k, v, do, feature_map="elu1", normalize=True,
+                              out_dtype="f32", kernel_path="tensor_core")
+    torch.cuda.synchronize()
+    for b, h in ((0, 0), (1, 31)):
+        sl = lambda t: t[b:b + 1, h:h + 1]
+        ref = default_oracle().backward(to_np(sl(q)), to_np(sl(k)), to_np(sl(v)),
+                                        to_np(sl(do)).astype(np.float64), feature_map="elu1",
+                                        normalize=True)
+        for name, x, r in zip(("grad_q", "grad_k", "grad_v"), got[:3], ref[:3]):
+            assert_close(to_np(sl(x)), r, TOL_BF16, f"({b},{h}) {name}")
