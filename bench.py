@@ -498,11 +498,11 @@ def backward_bytes(w, out_elem: int, algorithm: str, lseg: int = 0):
     ew = 4 if w_f32 else 2
     nk, nv, nt = BH * w.T * w.dk, BH * w.T * w.dv, BH * w.T
     ops = []
-    pre = (0 if native else 2 * nk + 2 * nv)
-    if elu:
-        pre += halves * nk * (1 if norm else 2)   # psi(k) (and psi(q) unnormalised)
+    pre = 0 if native else 2 * (2 * nk + 2 * nv) * e  # reversed copies: read and write
+    if elu:  # psi(k) (and psi(q) unnormalised): one read, hi (and lo) written
+        pre += (1 if norm else 2) * (nk * e + halves * nk * e)
     if pre:
-        ops.append(("bwd_reverse_inputs", 2 * pre * e))
+        ops.append(("bwd_reverse_inputs", pre))
     wa = w.with_(dk=w.dv, dv=w.dk, feature_map="identity", normalize=False)
     wb = w.with_(normalize=False)
 
@@ -517,7 +517,7 @@ def backward_bytes(w, out_elem: int, algorithm: str, lseg: int = 0):
         # lo), dd, 1 / d, grad_q
         ops.append(("bwd_z_scan", nk * e + 2 * nk * e + nv * e + halves * nk * 4
                     + halves * nv * e + 2 * nt * 4 + nk * out_elem))
-        ops.append(("bwd_scaled_psi_q", halves * (2 * nk * e + nt * 4)))
+        ops.append(("bwd_scaled_psi_q", nk * e + nt * 4 + halves * nk * e))
     prefills(wb, ew if wv else out_elem, halves if norm else 1)
     prefills(wa, ew if wk else out_elem, halves)
     if norm:  # g scan: totals and walk read q and dd; the walk writes g

@@ -72,15 +72,17 @@ __device__ __forceinline__ void store4(void* base, long long idx, float4 x, bool
 
 // dst[bh, t'] = (f(src[bh, t] + src2[bh, t]) rs[bh, t] + src3[bh, t]) g(x[bh, t']) for rows
 // of d elements, where t' = T-1-t when `flip`, else t; f = psi when `fm_src` is ELU+1,
-// g = psi' of x when `x` is given (absent terms drop out).  With `lo`, dst receives the part of the value that bf16 rounding drops
-// (value - bf16(value), itself rounded to bf16): a bf16 hi + lo pair carries psi to about
-// 16 bits, like the split operands of the prefill's own kernels.
+// g = psi' of x when `x` is given (absent terms drop out).  With `lo`, dst2 also receives
+// the part of the value that bf16 rounding drops (value - bf16(value), itself rounded to
+// bf16): a bf16 hi + lo pair carries psi to about 16 bits, like the split operands of the
+// prefill's own kernels.
 struct RowJob {
   const void* src;
   const void* src2;  // added to src (same type), or nullptr
   const void* src3;  // added after the row scale, or nullptr
   const float* rs;   // per-row scale of (src + src2), indexed by the source row, or nullptr
   void* dst;
+  void* dst2;        // with `lo`: the value's bf16 residual goes here, the value to dst
   const void* x;     // multiplier input (same layout as dst, type of the inputs) or nullptr
   int d;
   int fm_src;        // la_feature_map applied to src
@@ -92,41 +94,97 @@ struct RowJobs {
   RowJob j[kMaxJobs];
 };
 
-// One 4-element group per thread and grid-stride loop; blockIdx.y selects the job.
-__global__ void __launch_bounds__(256) row_jobs(RowJobs jobs, long long BH, long long T) {
+// Eight consecutive elements (or four, for rows of 4 (mod 8) elements) of a bf16 or float32
+// row.
+template <int W>
+struct Vec {
+  float v[W];
+};
+template <int W>
+__device__ __forceinline__ Vec<W> loadw(const void* base, long long idx, bool f32) {
+  Vec<W> r;
+  if constexpr (W == 4) {
+    const float4 a = load4(base, idx, f32);
+    r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+  } else if (f32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+    const float4 a = __ldcs(p), b = __ldcs(p + 1);
+    r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+    r.v[4] = b.x; r.v[5] = b.y; r.v[6] = b.z; r.v[7] = b.w;
+  } else {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(
+        static_cast<const __nv_bfloat16*>(base) + idx));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h;
+      std::memcpy(&h, &w[e], 4);
+      const float2 f = __bfloat1622float2(h);
+      r.v[2 * e] = f.x;
+      r.v[2 * e + 1] = f.y;
+    }
+  }
+  return r;
+}
+template <int W>
+__device__ __forceinline__ void storew(void* base, long long idx, const Vec<W>& x, bool f32) {
+  if constexpr (W == 4) {
+    store4(base, idx, make_float4(x.v[0], x.v[1], x.v[2], x.v[3]), f32);
+  } else if (f32) {
+    float4* p = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
+    __stcs(p, make_float4(x.v[0], x.v[1], x.v[2], x.v[3]));
+    __stcs(p + 1, make_float4(x.v[4], x.v[5], x.v[6], x.v[7]));
+  } else {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h = __float22bfloat162_rn(make_float2(x.v[2 * e], x.v[2 * e + 1]));
+      std::memcpy(&w[e], &h, 4);
+    }
+    __stcs(reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + idx),
+           make_uint4(w[0], w[1], w[2], w[3]));
+  }
+}
+
+// One group of W elements per thread over a grid that covers the job (a memory-bound
+// element-wise pass wants every SM full of threads, each with its loads in flight, rather
+// than a few threads looping); blockIdx.y selects the job.  32-bit index arithmetic.
+template <int W>
+__device__ __forceinline__ void row_job_group(const RowJob& J, unsigned T, unsigned g) {
+  const unsigned gpr = static_cast<unsigned>(J.d / W);
+  const unsigned row = g / gpr, col = (g - row * gpr) * W;
+  const unsigned bh = row / T, t = row - bh * T;
+  const unsigned drow = J.flip ? bh * T + (T - 1 - t) : row;
+  const long long si = static_cast<long long>(row) * J.d + col;
+  const long long di = static_cast<long long>(drow) * J.d + col;
+  Vec<W> a = loadw<W>(J.src, si, J.src_f32), b{}, c{}, x{};
+  if (J.src2) b = loadw<W>(J.src2, si, J.src_f32);
+  if (J.src3) c = loadw<W>(J.src3, si, J.src_f32);
+  const bool dx = J.x && J.fm_x == LA_FM_ELU1;
+  if (dx) x = loadw<W>(J.x, di, J.x_f32);
+  const float r = J.rs ? J.rs[row] : 1.f;
+#pragma unroll
+  for (int e = 0; e < W; ++e) {
+    float v = a.v[e];
+    if (J.src2) v += b.v[e];
+    if (J.fm_src == LA_FM_ELU1) v = psi(v, 1);
+    v *= r;
+    if (J.src3) v += c.v[e];
+    if (dx) v *= psi_prime(x.v[e], 1);
+    a.v[e] = v;
+    if (J.lo) b.v[e] = v - __bfloat162float(__float2bfloat16_rn(v));
+  }
+  storew<W>(J.dst, di, a, J.dst_f32);
+  if (J.lo) storew<W>(J.dst2, di, b, J.dst_f32);
+}
+
+__global__ void __launch_bounds__(256) row_jobs(RowJobs jobs, unsigned T, unsigned rows) {
   const RowJob& J = jobs.j[blockIdx.y];
-  const long long gpr = J.d / 4;  // groups per row
-  const long long n = BH * T * gpr;
-  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < n;
-       g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = g / gpr, col = (g - row * gpr) * 4;
-    const long long bh = row / T, t = row - bh * T;
-    const long long drow = J.flip ? bh * T + (T - 1 - t) : row;
-    float4 a = load4(J.src, row * J.d + col, J.src_f32);
-    if (J.src2) {
-      const float4 b = load4(J.src2, row * J.d + col, J.src_f32);
-      a = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-    }
-    if (J.fm_src == LA_FM_ELU1)
-      a = make_float4(psi(a.x, 1), psi(a.y, 1), psi(a.z, 1), psi(a.w, 1));
-    if (J.rs) {
-      const float r = J.rs[row];
-      a = make_float4(a.x * r, a.y * r, a.z * r, a.w * r);
-    }
-    if (J.src3) {
-      const float4 b = load4(J.src3, row * J.d + col, J.src_f32);
-      a = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
-    }
-    if (J.lo) {
-      auto rest = [](float v) { return v - __bfloat162float(__float2bfloat16_rn(v)); };
-      a = make_float4(rest(a.x), rest(a.y), rest(a.z), rest(a.w));
-    }
-    if (J.x && J.fm_x == LA_FM_ELU1) {
-      const float4 x = load4(J.x, drow * J.d + col, J.x_f32);
-      a = make_float4(a.x * psi_prime(x.x, 1), a.y * psi_prime(x.y, 1),
-                      a.z * psi_prime(x.z, 1), a.w * psi_prime(x.w, 1));
-    }
-    store4(J.dst, drow * J.d + col, a, J.dst_f32);
+  const unsigned g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (J.d % 8 == 0) {
+    if (g < rows * static_cast<unsigned>(J.d / 8)) row_job_group<8>(J, T, g);
+  } else if (g < rows * static_cast<unsigned>(J.d / 4)) {
+    row_job_group<4>(J, T, g);
   }
 }
 
@@ -217,19 +275,48 @@ __global__ void __launch_bounds__(128) vs_totals(VecScan p, GammaTable gt) {
   *reinterpret_cast<float4*>(p.tot + (bh * p.NS + seg) * p.d + col) = acc;
 }
 
-__global__ void vs_prefix(VecScan p, GammaTable gt) {
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(p.BH) * p.d) return;
-  const long long bh = idx / p.d;
-  const int f = static_cast<int>(idx - bh * p.d);
+// Exclusive prefixes of the segment totals: one warp per (b, h) and four features, lane i
+// holding segment s0 + i of a block of 32; a decayed Hillis-Steele scan in registers
+// (every segment but the last spans Ls tokens, so each step's decay is gamma^(Ls * off)),
+// the block's total carried into the next block.
+__global__ void __launch_bounds__(128) vs_prefix(VecScan p, GammaTable gt) {
+  const long long wid = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int groups = (p.d + 3) / 4;
+  if (wid >= static_cast<long long>(p.BH) * groups) return;
+  const long long bh = wid / groups;
+  const int col = 4 * static_cast<int>(wid - bh * groups);
   const float g = gt.g[bh % p.H];
-  const float gL = powf(g, static_cast<float>(p.Ls));
-  float P = 0.f;
-  for (int s = 0; s < p.NS; ++s) {
-    float* e = p.tot + (bh * p.NS + s) * p.d + f;
-    const float t = *e;
-    *e = P;
-    P = fmaf(gL, P, t);  // only the last segment can be short, and nothing follows it
+  const float aL = powf(g, static_cast<float>(p.Ls));
+  float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < p.NS; s0 += 32) {
+    const int sg = s0 + lane;
+    float4* e = reinterpret_cast<float4*>(p.tot + (bh * p.NS + sg) * p.d + col);
+    float4 x = sg < p.NS ? *e : make_float4(0.f, 0.f, 0.f, 0.f);
+    float a = aL;  // gamma^(Ls * off)
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float4 y = make_float4(__shfl_up_sync(0xffffffffu, x.x, off),
+                                   __shfl_up_sync(0xffffffffu, x.y, off),
+                                   __shfl_up_sync(0xffffffffu, x.z, off),
+                                   __shfl_up_sync(0xffffffffu, x.w, off));
+      if (lane >= off)
+        x = make_float4(fmaf(a, y.x, x.x), fmaf(a, y.y, x.y), fmaf(a, y.z, x.z), fmaf(a, y.w, x.w));
+      a *= a;
+    }
+    // Inclusive over the block from the carry: x + aL^(lane + 1) carry; exclusive: the
+    // previous lane's, or the carry itself for lane 0.
+    const float w = powf(aL, static_cast<float>(lane + 1));
+    const float4 inc = make_float4(fmaf(w, carry.x, x.x), fmaf(w, carry.y, x.y),
+                                   fmaf(w, carry.z, x.z), fmaf(w, carry.w, x.w));
+    float4 exc = make_float4(__shfl_up_sync(0xffffffffu, inc.x, 1),
+                             __shfl_up_sync(0xffffffffu, inc.y, 1),
+                             __shfl_up_sync(0xffffffffu, inc.z, 1),
+                             __shfl_up_sync(0xffffffffu, inc.w, 1));
+    if (lane == 0) exc = carry;
+    if (sg < p.NS) *e = exc;
+    carry = make_float4(__shfl_sync(0xffffffffu, inc.x, 31), __shfl_sync(0xffffffffu, inc.y, 31),
+                        __shfl_sync(0xffffffffu, inc.z, 31), __shfl_sync(0xffffffffu, inc.w, 31));
   }
 }
 
@@ -310,8 +397,8 @@ cudaError_t launch_vec_scan(const VecScan& p, const GammaTable& gt, cudaStream_t
   vs_totals<<<wb, 128, 0, s>>>(p, gt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long n = static_cast<long long>(p.BH) * p.d;
-  vs_prefix<<<static_cast<unsigned>((n + 127) / 128), 128, 0, s>>>(p, gt);
+  const long long pw = static_cast<long long>(p.BH) * ((p.d + 3) / 4);  // warps
+  vs_prefix<<<static_cast<unsigned>((pw + 3) / 4), 128, 0, s>>>(p, gt);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   vs_walk<<<wb, 128, 0, s>>>(p, gt);
@@ -446,8 +533,8 @@ bool native_reverse(const la_backward_args& a) {
 //   Outputs of the reversed passes Wk [T, dk], Wv [T, dv] where they cannot go straight to
 //   grad_k / grad_v: always without native reverse (float32 when multiplied by psi' or
 //   corrected, else the output type); with it, float32 and only where psi', the
-//   small-decay terms or the normalised form's lo pass still apply.  ELU+1: the grad_q pass's float32 output Wq [T, dk] and
-//   the lo passes' float32 outputs.
+//   small-decay terms or the normalised form's lo pass still apply.  ELU+1: the grad_q
+//   pass's float32 output Wq [T, dk] and the lo passes' float32 outputs.
 //   Three [dk x dv] states per (b, h), then the prefill workspace.
 struct BwdLayout {
   size_t kr, qr, dor, vr, pq, pk, pq_lo, pk_lo, Wk, Wv, Wq, Wk_lo, Wq_lo, SA, SB, SC;
@@ -561,6 +648,9 @@ int validate(const la_backward_args& a) {
   // states-only calls, so that no output buffer is needed; q stands for every input).
   const long long BH = static_cast<long long>(a.B) * a.H;
   const bool empty = BH == 0 || a.T == 0;
+  // The element-wise kernels index rows and groups of four elements in 32 bits.
+  if (!empty && (BH * a.T >= (1LL << 31) || BH * a.T * (std::max(a.dk, a.dv) / 4) >= (1LL << 31)))
+    return LA_ERR_UNSUPPORTED;
   const int fms[3] = {LA_FM_IDENTITY, a.feature_map, LA_FM_IDENTITY};
   const int dks[3] = {a.dv, a.dk, a.dv}, dvs[3] = {a.dk, a.dv, a.dk};
   const bool native = native_reverse(a);
@@ -597,15 +687,15 @@ int validate(const la_backward_args& a) {
 cudaError_t launch_rows(const RowJobs& jobs, int n, long long BH, long long T, cudaStream_t s,
                         Recorder* rec, const char* name) {
   if (n == 0) return cudaSuccess;
-  // Enough 256-thread blocks to fill every SM several times over; each thread then walks
-  // its share with a grid stride.
   long long groups = 0;
-  for (int i = 0; i < n; ++i) groups = std::max(groups, BH * T * (jobs.j[i].d / 4));
-  long long blocks = (groups + 255) / 256;
-  blocks = std::min<long long>(blocks, 148LL * 8);
-  if (blocks < 1) blocks = 1;
+  for (int i = 0; i < n; ++i)
+    groups = std::max(groups, BH * T * (jobs.j[i].d / (jobs.j[i].d % 8 == 0 ? 8 : 4)));
+  // The kernel indexes groups and elements' rows in 32 bits.
+  if (groups >= (1LL << 31) || BH * T >= (1LL << 31)) return cudaErrorInvalidValue;
+  const long long blocks = std::max(1LL, (groups + 255) / 256);
   if (rec) rec->mark(s, name);
-  row_jobs<<<dim3(static_cast<unsigned>(blocks), n), 256, 0, s>>>(jobs, BH, T);
+  row_jobs<<<dim3(static_cast<unsigned>(blocks), n), 256, 0, s>>>(
+      jobs, static_cast<unsigned>(T), static_cast<unsigned>(BH * T));
   return cudaGetLastError();
 }
 
@@ -656,8 +746,8 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
   // ELU+1, psi(q) (reversed likewise) and psi(k) in order, as hi / lo pairs for bf16.
   auto job = [](RowJobs& J, int& n, const void* src, const void* src2, void* dst, const void* x,
                 int d, int fm_src, int fm_x, bool flip, bool lo, bool sf, bool df, bool xf,
-                const void* src3 = nullptr, const float* rs = nullptr) {
-    J.j[n++] = RowJob{src, src2, src3, rs, dst, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
+                const void* src3 = nullptr, const float* rs = nullptr, void* dst2 = nullptr) {
+    J.j[n++] = RowJob{src, src2, src3, rs, dst, dst2, x, d, fm_src, fm_x, flip, lo, sf, df, xf};
   };
   RowJobs pre{};
   int np = 0;
@@ -670,15 +760,13 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
     job(pre, np, a.v, nullptr, at(l.vr), nullptr, a.dv, LA_FM_IDENTITY, 0, true, false, f, f, f);
   }
   // (The normalised form's psi(q) is scaled by 1 / d_t, known only after its scan.)
-  if (elu) {
+  if (elu) {  // one job writes psi and, for bf16, its lo half
+    const bool sp = l.split;
     if (!l.norm)
-      job(pre, np, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f);
-    job(pre, np, a.k, nullptr, at(l.pk), nullptr, a.dk, LA_FM_ELU1, 0, false, false, f, f, f);
-  }
-  if (l.split) {
-    if (!l.norm)
-      job(pre, np, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f);
-    job(pre, np, a.k, nullptr, at(l.pk_lo), nullptr, a.dk, LA_FM_ELU1, 0, false, true, f, f, f);
+      job(pre, np, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, sp, f, f, f,
+          nullptr, nullptr, sp ? at(l.pq_lo) : nullptr);
+    job(pre, np, a.k, nullptr, at(l.pk), nullptr, a.dk, LA_FM_ELU1, 0, false, sp, f, f, f,
+        nullptr, nullptr, sp ? at(l.pk_lo) : nullptr);
   }
   cudaError_t e = launch_rows(pre, np, BH, T, s, rec, "bwd_reverse_inputs");
 
@@ -773,11 +861,8 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
       RowJobs pq{};
       int n = 0;
       const float* rs = static_cast<const float*>(at(l.inv_den));
-      job(pq, n, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, false, f, f, f,
-          nullptr, rs);
-      if (l.split)
-        job(pq, n, a.q, nullptr, at(l.pq_lo), nullptr, a.dk, LA_FM_ELU1, 0, rv, true, f, f, f,
-            nullptr, rs);
+      job(pq, n, a.q, nullptr, at(l.pq), nullptr, a.dk, LA_FM_ELU1, 0, rv, l.split, f, f, f,
+          nullptr, rs, l.split ? at(l.pq_lo) : nullptr);
       if (e == cudaSuccess) e = launch_rows(pq, n, BH, T, s, rec, "bwd_scaled_psi_q");
       if (e != cudaSuccess) st = LA_ERR_CUDA;
     }

@@ -320,7 +320,7 @@ int lin_attn_prefill_noalloc(const la_prefill_args* args);
  *   grad_S_init        DEVICE float32 [B,H,dk,dv] output, or NULL (not computed).
  *   The other fields as in la_prefill_args; every pass uses `algorithm`, `kernel_path`,
  *   `scan_mode` and `segment_chunks`.  Supported shapes: those of the prefill for both
- *   (dk, dv) and (dv, dk).  Workspace: lin_attn_backward_workspace_bytes(), or NULL to
+ *   (dk, dv) and (dv, dk), with B*H*T*max(dk, dv) / 4 < 2^31.  Workspace: lin_attn_backward_workspace_bytes(), or NULL to
  *   allocate on the stream.  Asynchronous; arguments are checked before any launch.
  */
 typedef struct la_backward_args {
