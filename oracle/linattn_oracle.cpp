@@ -40,7 +40,8 @@
 // S_init / Z_init may be NULL (zero initial state); the outputs may be NULL (skipped).
 //
 // la_oracle_backward differentiates both forms by hand, token by token (the chain rule
-// through the recurrence; see backward_pair), for the backward pass.
+// through the recurrence; see backward_pair), for the backward pass.  la_oracle_gla_forward
+// runs the gated (data-dependent decay) recurrence (see gla_pair).
 
 #include <cmath>
 #include <cstddef>
@@ -252,9 +253,81 @@ void backward_pair(const BackwardProblem& p, long long bh) {
     for (int i = 0; i < dk; ++i) p.dZ_init[bh * dk + i] = p.normalize ? gz[i] : 0.0;
 }
 
+// Gated linear attention ("Linear Attention and Retentive Networks ...", Gated Linear
+// Attention (GLA) and Hardware-Software Co-Design: the update S_t = G_t (.) S_{t-1} +
+// k_t^T v_t with the gate G_t = alpha_t 1^T), one (b, h) pair, token by token:
+//   S_t[i][j] = alpha_t[i] S_{t-1}[i][j] + k_t[i] v_t[j],   o_t[j] = sum_i q_t[i] S_t[i][j]
+// with S_{-1} = S_init (or zero).  No feature map and no normalisation, as on that page.
+struct GlaProblem {
+  const float* q;
+  const float* k;
+  const float* v;
+  const float* alpha;
+  long long T;
+  int dk, dv;
+  const double* S_init;
+  double* out;
+  double* S_final;
+};
+
+void gla_pair(const GlaProblem& p, long long bh) {
+  const int dk = p.dk, dv = p.dv;
+  const long long T = p.T;
+  const float* q = p.q + bh * T * dk;
+  const float* k = p.k + bh * T * dk;
+  const float* v = p.v + bh * T * dv;
+  const float* al = p.alpha + bh * T * dk;
+  std::vector<double> S(static_cast<size_t>(dk) * dv, 0.0);
+  if (p.S_init)
+    for (size_t e = 0; e < S.size(); ++e) S[e] = p.S_init[bh * dk * dv + e];
+  for (long long t = 0; t < T; ++t) {
+    for (int i = 0; i < dk; ++i) {
+      const double gate = static_cast<double>(al[t * dk + i]);
+      const double ki = static_cast<double>(k[t * dk + i]);
+      double* Si = &S[static_cast<size_t>(i) * dv];
+      for (int j = 0; j < dv; ++j) Si[j] = gate * Si[j] + ki * static_cast<double>(v[t * dv + j]);
+    }
+    if (p.out) {
+      for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i)
+          acc += static_cast<double>(q[t * dk + i]) * S[static_cast<size_t>(i) * dv + j];
+        p.out[(bh * T + t) * dv + j] = acc;
+      }
+    }
+  }
+  if (p.S_final)
+    for (size_t e = 0; e < S.size(); ++e) p.S_final[bh * dk * dv + e] = S[e];
+}
+
 }  // namespace
 
 extern "C" {
+
+// Gated linear attention forward (see gla_pair).  alpha [B, H, T, dk] float32 gates;
+// S_init [B, H, dk, dv] double or NULL; out [B, H, T, dv] and S_final double (each may be
+// NULL).  Returns 0, or 1 on an invalid argument.
+int la_oracle_gla_forward(const float* q, const float* k, const float* v, const float* alpha,
+                          int B, int H, long long T, int dk, int dv, const double* S_init,
+                          double* out, double* S_final, int nthreads) {
+  if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 1;
+  if (T > 0 && (!q || !k || !v || !alpha)) return 1;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return 0;
+  GlaProblem p{q, k, v, alpha, T, dk, dv, S_init, out, S_final};
+  long long workers = nthreads > 0 ? nthreads
+                                   : static_cast<long long>(std::thread::hardware_concurrency());
+  if (workers < 1) workers = 1;
+  if (workers > BH) workers = BH;
+  std::vector<std::thread> pool;
+  for (long long w = 0; w < workers; ++w)
+    pool.emplace_back([&p, w, workers, BH]() {
+      for (long long bh = w; bh < BH; bh += workers) gla_pair(p, bh);
+    });
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
 
 // Returns 0 on success, 1 on an invalid argument.  nthreads <= 0 means one thread per
 // hardware thread (capped at B*H).

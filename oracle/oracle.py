@@ -56,6 +56,11 @@ class Oracle:
         b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
             [ctypes.c_void_p, ctypes.c_int, ctypes.c_double] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
+        gl = self._lib.la_oracle_gla_forward
+        gl.restype = ctypes.c_int
+        gl.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                                              ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 3 + \
+            [ctypes.c_int]
         g = self._lib.la_oracle_feature_map
         g.restype = ctypes.c_int
         g.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int]
@@ -134,6 +139,27 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"la_oracle_backward returned {rc}")
         return dq, dk_, dv_, ds0, dz0
+
+
+    def gla_forward(self, q, k, v, alpha, *, S_init=None, want_out: bool = True,
+                    nthreads: int = 0):
+        """Gated linear attention's token loop: S_t = (alpha_t 1^T) (.) S_{t-1} + k_t^T v_t,
+        o_t = q_t S_t.  q, k, alpha [B, H, T, dk]; v [B, H, T, dv].  Returns (out float64 or
+        None, S_final [B, H, dk, dv])."""
+        q, k, v, al = (np.ascontiguousarray(a, dtype=np.float32) for a in (q, k, v, alpha))
+        B, H, T, dk = q.shape
+        dv = v.shape[-1]
+        if k.shape != q.shape or al.shape != q.shape or v.shape[:3] != (B, H, T):
+            raise ValueError("shape mismatch between q, k, v and alpha")
+        s0 = None if S_init is None else np.ascontiguousarray(S_init, dtype=np.float64)
+        out = np.empty((B, H, T, dv)) if want_out else None
+        S = np.empty((B, H, dk, dv))
+        ptr = lambda a: None if a is None else a.ctypes.data
+        rc = self._lib.la_oracle_gla_forward(ptr(q), ptr(k), ptr(v), ptr(al), B, H, T, dk, dv,
+                                             ptr(s0), ptr(out), ptr(S), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"la_oracle_gla_forward returned {rc}")
+        return out, S
 
 
 _default: Oracle | None = None
