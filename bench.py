@@ -680,6 +680,82 @@ def backward_bench(args, w, info, dev):
         print(json.dumps(line), flush=True)
 
 
+# Exponentials per second of one B200 from its unit counts: 148 SMs x 16 MUFU lanes
+# (ex2) per SM per clock x the 1965 MHz maximum SM clock.
+NOMINAL_EX2_PER_S = 148 * 16 * 1965e6
+METRIC_GLA = "gated linear-attn prefill tokens·heads/s at H=32,d=128; % of roofline"
+
+
+def gla_bench(args, info, dev):
+    """Gated linear attention (lin_attn_gla_prefill) on the 128k-token gated workload, one
+    prefill per step, timed like the main benchmark."""
+    from chunked_causal_linear_b200.workloads import GLA_WORKLOADS, make_gates
+    w = GLA_WORKLOADS["gla_128k"]
+    if args.heads:
+        w = w.with_(H=args.heads, name=f"{w.name}_h{args.heads}")
+    q, k, v = make_inputs(w, seed=info.rank, device=dev)
+    alpha = make_gates(w, seed=info.rank, device=dev)
+    out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
+    S = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(B.lin_attn_gla_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.C),
+                     dtype=torch.uint8, device=dev)
+    kw = dict(chunk=w.C, out_dtype="f32", workspace=ws)
+
+    def step():
+        B.lin_attn_gla_prefill(q, k, v, alpha, out, S, **kw)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = None if args.no_clocks else ClockSampler(info.local_rank)
+    if sampler:
+        sampler.start()
+    ranks.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ranks.barrier(info)
+    clocks = sampler.stop() if sampler else None
+    ms_max = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, info, dev)
+    per = [B.lin_attn_gla_prefill_timed(q, k, v, alpha, out, S, **kw)
+           for _ in range(max(1, args.kernel_timing_steps))]
+    names = ["gla_k1", "gla_k2", "gla_k3"]
+    kern_ms = {n: statistics.mean(x[i] for x in per) for i, n in enumerate(names)}
+    BH, NC, C = w.B * w.H, -(-w.T // w.C), w.C
+    R = w.dk * w.dv + w.dk
+    pairs = C * (C + 1) // 2
+    # K3: one exponential per (token pair in a chunk, key feature) plus one per (token,
+    # feature) for the prefix readout
+    ex2 = BH * NC * (pairs * w.dk + C * w.dk)
+    e_in = 2
+    bytes_ = {"gla_k1": BH * w.T * (w.dk * (e_in + 4) + w.dv * e_in) + BH * NC * R * 4,
+              "gla_k2": 2 * BH * NC * R * 4,
+              "gla_k3": BH * w.T * (w.dk * (2 * e_in + 4) + w.dv * e_in + w.dv * 4) + BH * NC * R * 4}
+    peak, peak_kind = measured_peaks()
+    hbm = {n: bytes_[n] / (kern_ms[n] / 1e3) / 1e9 / peak for n in names}
+    roofline = {"bound": "alu", "kernel": "gla_k3",
+                "achieved": ex2 / (kern_ms["gla_k3"] / 1e3) / 1e12, "peak": NOMINAL_EX2_PER_S / 1e12,
+                "unit": "Tex2/s", "frac": ex2 / (kern_ms["gla_k3"] / 1e3) / NOMINAL_EX2_PER_S,
+                "traffic": None,
+                "peak_source": "unit counts: 148 SMs x 16 ex2 per clock x 1965 MHz",
+                "hbm_frac_of_measured": hbm}
+    if info.is_root:
+        cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "C": w.C,
+               "inputs": "bf16", "gates": "float32 sigmoid(N(4, 1))", "out_dtype": "f32",
+               "kernel_path": "fma (CUDA cores)", "l2": "inputs larger than L2, no flush",
+               "parallelism": "replicas (one independent problem per GPU)"}
+        line = {"metric": METRIC_GLA, "value": info.world * w.tokens_heads / (ms_max / 1e3),
+                "unit": UNIT, "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+                "mode": "gla", "roofline": roofline, "kernels_ms": kern_ms, "clocks": clocks,
+                "gpu_launches": 3 * args.steps, "device_error": B.lin_attn_device_error()}
+        print(json.dumps(line), flush=True)
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
@@ -726,6 +802,9 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="instead of the prefill: the backward of the unnormalised form "
                          "(grad_q, grad_k, grad_v for a random grad_out)")
+    ap.add_argument("--gla", action="store_true",
+                    help="instead of the prefill: gated linear attention (data-dependent decay) "
+                         "on the 128k-token gated workload")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -755,6 +834,10 @@ def main():
         return
     if args.backward:
         backward_bench(args, w, info, dev)
+        ranks.finish(info)
+        return
+    if args.gla:
+        gla_bench(args, info, dev)
         ranks.finish(info)
         return
 

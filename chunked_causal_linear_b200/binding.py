@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = (
     "lin_attn_decode_step", "lin_attn_decode_step_f32", "lin_attn_device_error",
     "lin_attn_status_string", "lin_attn_version", "lin_attn_combine_states",
     "lin_attn_backward", "lin_attn_backward_workspace_bytes", "lin_attn_backward_timed",
+    "lin_attn_gla_prefill", "lin_attn_gla_workspace_bytes", "lin_attn_gla_prefill_timed",
 )
 
 
@@ -77,6 +78,17 @@ class BackwardArgs(ctypes.Structure):
     ]
 
 
+class GlaArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p), ("out", ctypes.c_void_p), ("S_final", ctypes.c_void_p),
+        ("S_init", ctypes.c_void_p), ("B", ctypes.c_int), ("H", ctypes.c_int),
+        ("T", ctypes.c_longlong), ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -111,6 +123,10 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_backward_workspace_bytes": (sz, [ctypes.POINTER(BackwardArgs)]),
         "lin_attn_backward_timed": (i, [ctypes.POINTER(BackwardArgs), ctypes.POINTER(f),
                                         ctypes.POINTER(ctypes.c_char_p), i, ctypes.POINTER(i)]),
+        "lin_attn_gla_prefill": (i, [ctypes.POINTER(GlaArgs)]),
+        "lin_attn_gla_workspace_bytes": (sz, [i, i, ll, i, i, i]),
+        "lin_attn_gla_prefill_timed": (i, [ctypes.POINTER(GlaArgs), ctypes.POINTER(f), i,
+                                           ctypes.POINTER(i)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -386,6 +402,51 @@ def lin_attn_backward_workspace_bytes(q, v, *, chunk=64, feature_map="identity",
     n = int(load_library().lin_attn_backward_workspace_bytes(ctypes.byref(a)))
     del garr
     return n
+
+
+def _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream):
+    B, H, T, dk = q.shape
+    a = GlaArgs()
+    a.q, a.k, a.v, a.alpha, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out)
+    a.S_final, a.S_init = _ptr(S_final), _ptr(S_init)
+    a.B, a.H, a.T, a.dk, a.dv, a.C = B, H, T, dk, v.shape[-1], int(chunk)
+    a.dtype = DTYPES[q.dtype]
+    a.out_dtype = OUT_DTYPES[out_dtype]
+    a.workspace = _ptr(workspace)
+    a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a.stream = _stream_handle(stream)
+    return a
+
+
+def lin_attn_gla_prefill(q, k, v, alpha, out=None, S_final=None, *, S_init=None, chunk=64,
+                         out_dtype="as_input", workspace=None, stream=None, want_state=True):
+    """Gated linear attention (see the header): q, k, alpha [B,H,T,dk] (alpha float32),
+    v [B,H,T,dv].  Returns (out, S_final)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if out is None:
+        odt = torch.float32 if out_dtype == "f32" else q.dtype
+        out = torch.empty((B, H, T, dv), dtype=odt, device=q.device)
+    if want_state and S_final is None:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    a = _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream)
+    _check("lin_attn_gla_prefill", load_library().lin_attn_gla_prefill(ctypes.byref(a)))
+    return out, S_final
+
+
+def lin_attn_gla_workspace_bytes(B, H, T, dk, dv, C) -> int:
+    return int(load_library().lin_attn_gla_workspace_bytes(B, H, T, dk, dv, C))
+
+
+def lin_attn_gla_prefill_timed(q, k, v, alpha, out, S_final=None, *, S_init=None, chunk=64,
+                               out_dtype="as_input", workspace=None, stream=None) -> list[float]:
+    """One GLA prefill with an event around each kernel; returns [K1, K2, K3] in ms."""
+    a = _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream)
+    ms = (ctypes.c_float * 4)()
+    n = ctypes.c_int(0)
+    _check("lin_attn_gla_prefill_timed",
+           load_library().lin_attn_gla_prefill_timed(ctypes.byref(a), ms, 4, ctypes.byref(n)))
+    return [float(ms[i]) for i in range(n.value)]
 
 
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024

@@ -1,0 +1,412 @@
+// Gated linear attention: the data-dependent decay of "Linear Attention and Retentive
+// Networks ..." (Gated Linear Attention (GLA) and Hardware-Software Co-Design):
+//     S_t = (alpha_t 1^T) (.) S_{t-1} + k_t^T v_t,      o_t = q_t S_t,
+// alpha_t a per-token, per-key-feature gate in [0, 1].  The scan page's three kernels with
+// the decayed monoid generalised from a scalar to a diagonal: a chunk scales what came before
+// it by a_c = prod_{j in c} alpha_j (a dk-vector), so (a1, S1) + (a2, S2) = (a1 a2,
+// diag(a2) S1 + S2) ("Log-Depth Chunked Linear-Attention Scan", Formulas, with the decay of
+// "C. Chunkwise Recurrent Representation" made per feature).  Within a chunk, with
+// L_j = sum_{r<=j} log alpha_r (per feature, from the chunk start):
+//   K1  S_loc = sum_j (k_j (.) e^(L_last - L_j)) v_j^T,   a_c = e^(L_last)
+//   K2  P_c = the exclusive prefix of (a_c, S_loc) over chunks (a carry per state element)
+//   K3  o_j = (q_j (.) e^(L_j)) P_c + sum_{i<=j} (sum_f q_j[f] k_i[f] e^(L_j[f] - L_i[f])) v_i
+// The kernels form these as powers of two of cumulative log2 gates.  Every exponent is
+// <= 0, so nothing overflows whatever the gates (a gate below 2^-126 counts as 2^-126).  The
+// intra-chunk scores take one exponential per (pair, feature) on the CUDA cores: exact, and
+// the reason this path is ALU-bound (the per-feature ratio does not factor into one matrix
+// product without rescaling that can overflow).
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/linattn.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace la {
+namespace {
+
+constexpr int kGlaThreads = 256;
+
+struct GlaParams {
+  int BH;
+  long long T;
+  int dk, dv, C;
+  int NC;        // chunks
+  int L_last;    // tokens in the last chunk
+  int R;         // floats per record: S [dk][dv] then a [dk]
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  void* out;
+  bool in_f32, out_f32;
+  float* rec;    // [BH][NC][R]
+  const float* S_init;
+  float* S_final;
+};
+
+__device__ __forceinline__ float ld(const void* p, long long i, bool f32) {
+  return f32 ? static_cast<const float*>(p)[i]
+             : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+__device__ __forceinline__ int chunk_len(const GlaParams& p, int c) {
+  return c == p.NC - 1 ? p.L_last : p.C;
+}
+
+// Loads rows [t0, t0 + L) of a [T, d] slice into sm[r * ld + f] as float32 (rows >= L zero).
+__device__ __forceinline__ void load_rows(float* sm, int lds, const void* g, bool f32,
+                                          long long base, int d, int C, int L) {
+  for (int e = threadIdx.x; e < C * d; e += blockDim.x) {
+    const int r = e / d, f = e - r * d;
+    sm[r * lds + f] = r < L ? ld(g, base + static_cast<long long>(r) * d + f, f32) : 0.f;
+  }
+}
+
+// Cumulative log2 of the gates down each feature column (sm holds the gates on entry).  A
+// gate below 2^-126 counts as 2^-126, so that sums stay finite (a zero gate would give
+// -inf - -inf); whatever passes through it is then below 2^-126 of its size.
+__device__ __forceinline__ void cum_log2(float* sm, int lds, int d, int L) {
+  for (int f = threadIdx.x; f < d; f += blockDim.x) {
+    float acc = 0.f;
+    for (int r = 0; r < L; ++r) {
+      acc += fmaxf(log2f(sm[r * lds + f]), -126.f);
+      sm[r * lds + f] = acc;
+    }
+  }
+}
+
+// K1: one CTA per (b*H + h, chunk): the chunk's summary and decay vector.
+__global__ void __launch_bounds__(kGlaThreads) gla_k1(GlaParams p) {
+  extern __shared__ float sm[];
+  const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
+  const int C = p.C, dk = p.dk, dv = p.dv, L = chunk_len(p, c);
+  float* sK = sm;            // [C][dk]
+  float* sA = sK + C * dk;   // [C][dk]: gates, then cumulative log2
+  float* sV = sA + C * dk;   // [C][dv]
+  const long long t0 = static_cast<long long>(c) * C;
+  load_rows(sK, dk, p.k, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dk, dk, C, L);
+  load_rows(sV, dv, p.v, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dv, dv, C, L);
+  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+    const int r = e / dk;
+    sA[e] = r < L ? p.alpha[(static_cast<long long>(bh) * p.T + t0) * dk + e] : 1.f;
+  }
+  __syncthreads();
+  cum_log2(sA, dk, dk, L);
+  __syncthreads();
+  float* rec = p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R;
+  // k_j (.) 2^(L_last - L_j), in place; the chunk's decay vector a_c = 2^(L_last).
+  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+    const int r = e / dk, f = e - r * dk;
+    sK[e] = r < L ? sK[e] * exp2f(sA[(L - 1) * dk + f] - sA[e]) : 0.f;
+  }
+  for (int f = threadIdx.x; f < dk; f += blockDim.x) rec[dk * dv + f] = exp2f(sA[(L - 1) * dk + f]);
+  __syncthreads();
+  // S[f][e] = sum_j K'[j][f] v[j][e]: an 8 x 8 tile of (f, e) per thread.
+  const int tiles_e = dv / 8, tiles = (dk / 8) * tiles_e;
+  for (int tile = threadIdx.x; tile < tiles; tile += blockDim.x) {
+    const int f0 = (tile / tiles_e) * 8, e0 = (tile % tiles_e) * 8;
+    float acc[8][8] = {};
+    for (int j = 0; j < L; ++j) {
+      float a[8], b[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        a[u] = sK[j * dk + f0 + u];
+        b[u] = sV[j * dv + e0 + u];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int w = 0; w < 8; w += 4)
+        *reinterpret_cast<float4*>(rec + (f0 + u) * dv + e0 + w) =
+            make_float4(acc[u][w], acc[u][w + 1], acc[u][w + 2], acc[u][w + 3]);
+  }
+}
+
+// K2: the exclusive prefix over chunks, one thread per float4 column of the state: record c
+// receives the state before chunk c, then P <- a_c (.) P + S_c (row f scaled by a_c[f]).
+__global__ void gla_k2(GlaParams p) {
+  const long long n4 = static_cast<long long>(p.dk) * p.dv / 4;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(p.BH) * n4) return;
+  const long long bh = idx / n4, col = idx - bh * n4;
+  const int f = static_cast<int>(col * 4 / p.dv);
+  float4 P = p.S_init ? reinterpret_cast<const float4*>(p.S_init + bh * p.dk * p.dv)[col]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  float* base = p.rec + bh * p.NC * p.R;
+  for (int c = 0; c < p.NC; ++c) {
+    float4* e = reinterpret_cast<float4*>(base + static_cast<long long>(c) * p.R) + col;
+    const float4 x = *e;
+    const float a = base[static_cast<long long>(c) * p.R + p.dk * p.dv + f];
+    *e = P;
+    P = make_float4(fmaf(a, P.x, x.x), fmaf(a, P.y, x.y), fmaf(a, P.z, x.z), fmaf(a, P.w, x.w));
+  }
+  if (p.S_final) reinterpret_cast<float4*>(p.S_final + bh * p.dk * p.dv)[col] = P;
+}
+
+// K3: one CTA per (b*H + h, chunk): the intra-chunk part with per-feature gate ratios and
+// the prefix read out through the gates' running products.
+__global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
+  extern __shared__ float sm[];
+  const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
+  const int C = p.C, dk = p.dk, dv = p.dv, L = chunk_len(p, c);
+  const int lk = dk + 1;       // padded rows: threads of a warp read different rows
+  float* sQ = sm;              // [C][lk]
+  float* sK = sQ + C * lk;     // [C][lk]
+  float* sL = sK + C * lk;     // [C][lk]: gates, then cumulative log2
+  float* sV = sL + C * lk;     // [C][dv]
+  float* sP = sV + C * dv;     // [dk][dv]
+  float* sS = sP + dk * dv;    // [C][C] scores
+  const long long t0 = static_cast<long long>(c) * C;
+  const long long rq = (static_cast<long long>(bh) * p.T + t0) * dk;
+  load_rows(sQ, lk, p.q, p.in_f32, rq, dk, C, L);
+  load_rows(sK, lk, p.k, p.in_f32, rq, dk, C, L);
+  load_rows(sV, dv, p.v, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dv, dv, C, L);
+  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+    const int r = e / dk, f = e - r * dk;
+    sL[r * lk + f] = r < L ? p.alpha[rq + e] : 1.f;
+  }
+  const float4* P4 = reinterpret_cast<const float4*>(p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R);
+  for (int e = threadIdx.x; e < dk * dv / 4; e += blockDim.x)
+    reinterpret_cast<float4*>(sP)[e] = P4[e];
+  __syncthreads();
+  cum_log2(sL, lk, dk, L);
+  __syncthreads();
+  // Scores A[j][i] = sum_f q_j[f] k_i[f] 2^(L_j[f] - L_i[f]) for i <= j (0 above).
+  for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
+    const int j = e / C, i = e - j * C;
+    float a = 0.f;
+    if (i <= j && j < L) {
+      const float* qj = sQ + j * lk;
+      const float* ki = sK + i * lk;
+      const float* Lj = sL + j * lk;
+      const float* Li = sL + i * lk;
+      for (int f = 0; f < dk; ++f) a = fmaf(qj[f] * ki[f], exp2f(Lj[f] - Li[f]), a);
+    }
+    sS[e] = a;
+  }
+  __syncthreads();
+  // q_j (.) 2^(L_j) for the prefix, in place.
+  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+    const int r = e / dk, f = e - r * dk;
+    sQ[r * lk + f] *= exp2f(sL[r * lk + f]);
+  }
+  __syncthreads();
+  // o[j][e] = sum_f q~[j][f] P[f][e] + sum_{i<=j} A[j][i] v[i][e]: a 4 x 8 tile per thread.
+  const int tiles_e = dv / 8, tiles = (C / 4) * tiles_e;
+  for (int tile = threadIdx.x; tile < tiles; tile += blockDim.x) {
+    const int j0 = (tile / tiles_e) * 4, e0 = (tile % tiles_e) * 8;
+    float acc[4][8] = {};
+    for (int f = 0; f < dk; ++f) {
+      float a[4], b[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = sQ[(j0 + u) * lk + f];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) b[w] = sP[f * dv + e0 + w];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+    }
+    for (int i = 0; i <= j0 + 3 && i < C; ++i) {
+      float a[4], b[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = sS[(j0 + u) * C + i];
+#pragma unroll
+      for (int w = 0; w < 8; ++w) b[w] = sV[i * dv + e0 + w];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (j0 + u >= L) continue;
+      const long long o = (static_cast<long long>(bh) * p.T + t0 + j0 + u) * dv + e0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        if (p.out_f32)
+          static_cast<float*>(p.out)[o + w] = acc[u][w];
+        else
+          static_cast<__nv_bfloat16*>(p.out)[o + w] = __float2bfloat16_rn(acc[u][w]);
+      }
+    }
+  }
+}
+
+size_t gla_smem_k1(int C, int dk, int dv) { return static_cast<size_t>(C) * (2 * dk + dv) * 4; }
+size_t gla_smem_k3(int C, int dk, int dv) {
+  return (static_cast<size_t>(C) * (3 * (dk + 1) + dv) + static_cast<size_t>(dk) * dv +
+          static_cast<size_t>(C) * C) * 4;
+}
+
+bool gla_dims_ok(int d) { return d >= 8 && d <= 128 && d % 8 == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  if (!a || !b || an == 0 || bn == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+size_t gla_ws(int B, int H, long long T, int dk, int dv, int C) {
+  if (B <= 0 || H <= 0 || T <= 0 || C <= 0) return 0;
+  const long long NC = (T + C - 1) / C;
+  return align256(static_cast<size_t>(B) * H * NC * (static_cast<size_t>(dk) * dv + dk) * 4);
+}
+
+int gla_validate(const la_gla_args& a) {
+  if (a.B < 0 || a.H < 0 || a.T < 0 || a.dk <= 0 || a.dv <= 0 || a.C <= 0)
+    return LA_ERR_INVALID_ARGUMENT;
+  if (a.dtype != LA_DTYPE_BF16 && a.dtype != LA_DTYPE_F32) return LA_ERR_INVALID_ARGUMENT;
+  if (a.out_dtype != LA_OUT_AS_INPUT && a.out_dtype != LA_OUT_F32) return LA_ERR_INVALID_ARGUMENT;
+  if (!gla_dims_ok(a.dk) || !gla_dims_ok(a.dv) || !(a.C == 16 || a.C == 32 || a.C == 64))
+    return LA_ERR_UNSUPPORTED;
+  const long long BH = static_cast<long long>(a.B) * a.H;
+  const long long NC = a.T > 0 ? (a.T + a.C - 1) / a.C : 0;
+  if (BH * NC > (1LL << 31) - 1) return LA_ERR_UNSUPPORTED;
+  if (a.workspace && (reinterpret_cast<uintptr_t>(a.workspace) & 255u)) return LA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a.S_init) || !aligned16(a.S_final)) return LA_ERR_INVALID_ARGUMENT;
+  if (BH > 0 && a.T > 0) {
+    if (!a.q || !a.k || !a.v || !a.alpha || !a.out) return LA_ERR_INVALID_ARGUMENT;
+    const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
+    const size_t eo = (a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32) ? 4 : 2;
+    const size_t nk = static_cast<size_t>(BH) * a.T * a.dk, nv = static_cast<size_t>(BH) * a.T * a.dv;
+    if (overlaps(a.out, nv * eo, a.q, nk * e) || overlaps(a.out, nv * eo, a.k, nk * e) ||
+        overlaps(a.out, nv * eo, a.v, nv * e) || overlaps(a.out, nv * eo, a.alpha, nk * 4))
+      return LA_ERR_INVALID_ARGUMENT;
+  }
+  return LA_OK;
+}
+
+int gla_prefill(const la_gla_args& a, Recorder* rec) {
+  int st = gla_validate(a);
+  if (st != LA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(a.stream);
+  const long long BH = static_cast<long long>(a.B) * a.H;
+  if (BH == 0) return LA_OK;
+  const size_t state_bytes = static_cast<size_t>(BH) * a.dk * a.dv * 4;
+  if (a.T == 0) {
+    if (!a.S_final) return LA_OK;
+    const cudaError_t e = a.S_init ? cudaMemcpyAsync(a.S_final, a.S_init, state_bytes,
+                                                     cudaMemcpyDeviceToDevice, s)
+                                   : cudaMemsetAsync(a.S_final, 0, state_bytes, s);
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+  const size_t need = gla_ws(a.B, a.H, a.T, a.dk, a.dv, a.C);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  bool owned = false;
+  if (ws) {
+    if (a.workspace_bytes < need) return LA_ERR_INVALID_ARGUMENT;
+  } else {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s) != cudaSuccess) {
+      cudaGetLastError();
+      return LA_ERR_OUT_OF_MEMORY;
+    }
+    owned = true;
+  }
+  GlaParams p;
+  p.BH = static_cast<int>(BH);
+  p.T = a.T;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.C = a.C;
+  p.NC = static_cast<int>((a.T + a.C - 1) / a.C);
+  p.L_last = static_cast<int>(a.T - static_cast<long long>(p.NC - 1) * a.C);
+  p.R = a.dk * a.dv + a.dk;
+  p.q = a.q;
+  p.k = a.k;
+  p.v = a.v;
+  p.alpha = a.alpha;
+  p.out = a.out;
+  p.in_f32 = a.dtype == LA_DTYPE_F32;
+  p.out_f32 = p.in_f32 || a.out_dtype == LA_OUT_F32;
+  p.rec = reinterpret_cast<float*>(ws);
+  p.S_init = a.S_init;
+  p.S_final = a.S_final;
+
+  const size_t s1 = gla_smem_k1(a.C, a.dk, a.dv), s3 = gla_smem_k3(a.C, a.dk, a.dv);
+  cudaError_t e = cudaFuncSetAttribute(gla_k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(s1));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gla_k3, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(s3));
+  const unsigned grid = static_cast<unsigned>(BH * p.NC);
+  if (e == cudaSuccess) {
+    if (rec) rec->mark(s, "gla_k1");
+    gla_k1<<<grid, kGlaThreads, s1, s>>>(p);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    const long long n = BH * a.dk * a.dv / 4;
+    if (rec) rec->mark(s, "gla_k2");
+    gla_k2<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) {
+    if (rec) rec->mark(s, "gla_k3");
+    gla_k3<<<grid, kGlaThreads, s3, s>>>(p);
+    e = cudaGetLastError();
+  }
+  if (rec) rec->mark(s);
+  if (owned) {
+    const cudaError_t e2 = cudaFreeAsync(ws, s);
+    if (e == cudaSuccess) e = e2;
+  }
+  return e == cudaSuccess ? LA_OK
+                          : (e == cudaErrorMemoryAllocation ? LA_ERR_OUT_OF_MEMORY : LA_ERR_CUDA);
+}
+
+}  // namespace
+}  // namespace la
+
+extern "C" int lin_attn_gla_prefill(const la_gla_args* args) {
+  if (!args) return LA_ERR_INVALID_ARGUMENT;
+  return la::gla_prefill(*args, nullptr);
+}
+
+extern "C" size_t lin_attn_gla_workspace_bytes(int B, int H, long long T, int dk, int dv, int C) {
+  return la::gla_ws(B, H, T, dk, dv, C);
+}
+
+extern "C" int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel_ms,
+                                          int max_kernels, int* n_kernels) {
+  if (!args || !kernel_ms || !n_kernels || max_kernels < 1) return LA_ERR_INVALID_ARGUMENT;
+  *n_kernels = 0;
+  cudaEvent_t ev[4];
+  const char* label[4] = {nullptr};
+  for (int i = 0; i < 4; ++i)
+    if (cudaEventCreate(&ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return LA_ERR_CUDA;
+    }
+  la::Recorder rec;
+  rec.ev = ev;
+  rec.label = label;
+  rec.cap = 4;
+  int st = la::gla_prefill(*args, &rec);
+  if (st == LA_OK && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(args->stream)) != cudaSuccess)
+    st = LA_ERR_CUDA;
+  if (st == LA_OK) {
+    int nk = 0;
+    for (int i = 0; i + 1 < rec.n && nk < max_kernels; ++i) {
+      float ms = 0.f;
+      cudaEventElapsedTime(&ms, ev[i], ev[i + 1]);
+      kernel_ms[nk++] = ms;
+    }
+    *n_kernels = nk;
+  }
+  for (int i = 0; i < 4; ++i) cudaEventDestroy(ev[i]);
+  return st;
+}

@@ -91,6 +91,31 @@ WORKLOADS: dict[str, Workload] = {
 }
 
 
+# Gated linear attention (data-dependent decay, "Linear Attention and Retentive Networks ...",
+# Gated Linear Attention (GLA) and Hardware-Software Co-Design) on the retention workload's
+# shape: gates alpha = sigmoid(x) per token and key feature, the page's parameterisation,
+# with x ~ N(4, 1) (gates mostly 0.95-0.99, some near 0.8).
+GLA_WORKLOADS: dict[str, Workload] = {
+    "gla_128k": Workload(
+        "gla_128k", B=1, H=32, T=131072, dk=128, dv=128, C=64, dtype="bf16",
+        scale=1.0 / math.sqrt(128.0), feature_map="identity", decay=False, normalize=False,
+        description="gated linear attention, B1 H32 T131072 d128 C64, bf16 N(0,1)/sqrt(128), "
+                    "gates sigmoid(N(4, 1)) in float32"),
+}
+
+
+def make_gates(w: Workload, seed: int = 0, device: str | torch.device = "cpu",
+               gen_device: str | torch.device | None = None, mean: float = 4.0,
+               std: float = 1.0) -> torch.Tensor:
+    """Draw the gates [B, H, T, dk] (float32) of a gated workload: sigmoid of N(mean, std)
+    from a generator seeded with ``seed`` + 1000003 (independent of q, k, v)."""
+    gen_device = torch.device(gen_device if gen_device is not None else device)
+    g = torch.Generator(device=gen_device)
+    g.manual_seed(int(seed) + 1000003)
+    x = torch.randn((w.B, w.H, w.T, w.dk), generator=g, device=gen_device, dtype=torch.float32)
+    return torch.sigmoid(x * std + mean).to(device)
+
+
 def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu",
                 gen_device: str | torch.device | None = None):
     """Draw (q, k, v) for workload ``w`` on ``device``.

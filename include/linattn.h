@@ -377,6 +377,53 @@ int lin_attn_backward_timed(const la_backward_args* args, float* kernel_ms,
 size_t lin_attn_backward_workspace_bytes(const la_backward_args* args);
 
 /*
+ * lin_attn_gla_prefill -- gated linear attention ("Linear Attention and Retentive Networks
+ * ...", Gated Linear Attention (GLA) and Hardware-Software Co-Design): the data-dependent
+ * decay
+ *     S_t = (alpha_t 1^T) (.) S_{t-1} + k_t^T v_t,     o_t = q_t S_t,
+ * S_{-1} = S_init (or zero), with a gate alpha_t[i] in [0, 1] per token and key feature
+ * (no feature map, no normalisation, as on that page).  The scan page's three kernels with
+ * the decayed monoid made per feature: K1 folds each chunk into (a_c, S_loc) with a_c the
+ * product of the chunk's gates, K2 carries the exclusive prefix over chunks (P <- a_c (.) P +
+ * S_loc, one thread per state element), K3 combines each chunk's intra part, whose score
+ * for tokens i <= j weighs feature f by prod_{i<r<=j} alpha_r[f], with the prefix read out
+ * through prod_{r<=j} alpha_r.  Gate products are formed as powers of two of cumulative
+ * log2 gates, every exponent <= 0; a gate below 2^-126 counts as 2^-126.  CUDA-core fp32
+ * kernels (the per-feature weights do not factor into one tensor-core product).
+ *   q, k      DEVICE [B,H,T,dk], v DEVICE [B,H,T,dv], bf16 or float32 per `dtype`
+ *   alpha     DEVICE float32 [B,H,T,dk]
+ *   out       DEVICE [B,H,T,dv], type per out_dtype; must not overlap the inputs
+ *   S_init    DEVICE float32 [B,H,dk,dv] or NULL;  S_final DEVICE float32 or NULL
+ * Shapes: dk, dv multiples of 8 in [8, 128]; C in {16, 32, 64}; T >= 0.  Workspace:
+ * lin_attn_gla_workspace_bytes() (one record of dk*dv + dk floats per chunk), or NULL to
+ * allocate on the stream.  Asynchronous; arguments are checked before any launch.
+ */
+typedef struct la_gla_args {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  void* out;
+  float* S_final;
+  const float* S_init;
+  int B, H;
+  long long T;
+  int dk, dv, C;
+  int dtype;              /* la_dtype of q, k, v */
+  int out_dtype;          /* la_out_dtype of out */
+  void* workspace;        /* DEVICE, 256-byte aligned, or NULL */
+  size_t workspace_bytes;
+  la_stream_t stream;
+} la_gla_args;
+
+int lin_attn_gla_prefill(const la_gla_args* args);
+size_t lin_attn_gla_workspace_bytes(int B, int H, long long T, int dk, int dv, int C);
+/* lin_attn_gla_prefill with a CUDA event around each of its three kernels; synchronises the
+ * stream and writes their durations (ms: K1, K2, K3) to kernel_ms.  For profiling. */
+int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel_ms, int max_kernels,
+                               int* n_kernels);
+
+/*
  * lin_attn_decode_step -- one recurrent step for every (b, h), the O(1) decode that the
  * prefill's final states feed ("The Recurrent Dual"; "B. Recurrent Representation").
  *   q, k      DEVICE bf16 [B,H,dk]   v DEVICE bf16 [B,H,dv]   out DEVICE bf16 [B,H,dv]

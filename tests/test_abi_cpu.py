@@ -272,3 +272,25 @@ def test_backward_workspace_bytes(lib):
              + al(6 * ns_seg * 128 * 4))
     assert B.lin_attn_backward_workspace_bytes(q2, q2, feature_map="elu1", out_dtype="f32",
                                                normalize=True) == want + extra
+
+
+def test_gla_argument_errors_before_any_launch(lib):
+    from chunked_causal_linear_b200.binding import GlaArgs
+    def args(**kw):
+        a = GlaArgs()
+        base = dict(q=0x1000, k=0x2000000, v=0x4000000, alpha=0x6000000, out=0x8000000, B=1,
+                    H=2, T=128, dk=64, dv=64, C=64, dtype=0, out_dtype=0)
+        base.update(kw)
+        for key, val in base.items():
+            setattr(a, key, val)
+        return a
+    cases = [(dict(B=-1), 1), (dict(dtype=5), 1), (dict(out_dtype=3), 1), (dict(dk=12), 2),
+             (dict(dv=136), 2), (dict(C=128), 2), (dict(alpha=0), 1), (dict(out=0), 1),
+             (dict(out=0x1000), 1), (dict(out=0x6000000 + 64), 1), (dict(S_init=0x100004), 1),
+             (dict(workspace=0x100010), 1), (dict(B=0), 0), (dict(H=0), 0)]
+    for kw, status in cases:
+        assert lib.lin_attn_gla_prefill(ctypes.byref(args(**kw))) == status, kw
+    assert lib.lin_attn_gla_prefill(None) == 1
+    # one record of dk*dv + dk floats per chunk, 256-byte aligned
+    n = lib.lin_attn_gla_workspace_bytes(2, 3, 100, 64, 32, 64)
+    assert n == (2 * 3 * 2 * (64 * 32 + 64) * 4 + 255) // 256 * 256

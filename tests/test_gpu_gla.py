@@ -1,0 +1,114 @@
+"""GPU parity of gated linear attention (lin_attn_gla_prefill) against the oracle's token
+loop, element by element on the same inputs (bf16 inputs: the oracle gets the same
+bf16-rounded values; the gates are float32 on both sides).  Tolerances: max |err| <=
+2e-2 * rms(oracle) for bf16 inputs, 1e-4 * rms for float32 (the kernels are float32
+throughout, so both sit far inside)."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from chunked_causal_linear_b200 import binding as B
+from chunked_causal_linear_b200.workloads import GLA_WORKLOADS, Workload, make_gates, make_inputs
+from gpu_common import TOL_BF16, TOL_F32, assert_close, to_np
+from oracle.oracle import default_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(T, *, dk=128, dv=128, dtype="bf16", H=3, seed=0, mean=4.0, std=1.0):
+    w = Workload("gla", B=2, H=H, T=T, dk=dk, dv=dv, C=64, dtype=dtype,
+                 scale=1.0 / math.sqrt(dk), feature_map="identity", decay=False, normalize=False)
+    q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
+    alpha = make_gates(w, seed=seed, device="cuda", gen_device="cpu", mean=mean, std=std)
+    return q, k, v, alpha
+
+
+def _oracle(q, k, v, alpha, S0=None):
+    return default_oracle().gla_forward(to_np(q), to_np(k), to_np(v), to_np(alpha),
+                                        S_init=None if S0 is None else to_np(S0).astype(np.float64))
+
+
+@pytest.mark.parametrize("C", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 1000, 3001])
+def test_gla_matches_oracle(C, T):
+    q, k, v, alpha = _problem(T)
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, chunk=C, out_dtype="f32")
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+@pytest.mark.parametrize("mean,std", [(0.0, 2.0), (8.0, 1.0), (-3.0, 1.0)])
+def test_gla_gate_ranges(mean, std):
+    # wide gates, gates near 1, and gates near 0 (state forgotten within a few tokens)
+    q, k, v, alpha = _problem(777, mean=mean, std=std)
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32")
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+def test_gla_exact_zero_and_unit_gates_and_initial_state():
+    q, k, v, alpha = _problem(500)
+    alpha[:, :, 100] = 0.0          # every feature forgets at token 100
+    alpha[:, :, 200:260, :64] = 1.0  # no decay on half the features for 60 tokens
+    S0 = (torch.randn((2, 3, 128, 128), generator=torch.Generator().manual_seed(9)) * 0.3).cuda()
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0, out_dtype="f32")
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle(q, k, v, alpha, S0)
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (32, 48), (128, 64), (8, 8)])
+def test_gla_fp32_and_other_dims(dk, dv):
+    q, k, v, alpha = _problem(300, dk=dk, dv=dv, dtype="f32")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, chunk=32)
+    torch.cuda.synchronize()
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    assert_close(to_np(out), o_ref, TOL_F32, "out")
+    assert_close(to_np(S), S_ref, TOL_F32, "S_final")
+
+
+def test_gla_bf16_output_and_workspace():
+    q, k, v, alpha = _problem(1000)
+    ws = torch.empty(B.lin_attn_gla_workspace_bytes(2, 3, 1000, 128, 128, 64), dtype=torch.uint8,
+                     device="cuda")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, workspace=ws)
+    out2, S2 = B.lin_attn_gla_prefill(q, k, v, alpha)
+    torch.cuda.synchronize()
+    assert out.dtype == torch.bfloat16
+    assert torch.equal(out, out2) and torch.equal(S, S2)
+    o_ref, _ = _oracle(q, k, v, alpha)
+    got, ref = to_np(out).astype(np.float64), o_ref
+    assert float(np.max(np.abs(got - ref) - (2e-2 * np.sqrt(np.mean(ref ** 2)) + 2 ** -8 * np.abs(ref)))) <= 0
+
+
+def test_gla_zero_tokens_return_the_initial_state():
+    q, k, v, alpha = _problem(0)
+    S0 = torch.randn((2, 3, 128, 128)).cuda()
+    _, S = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0)
+    torch.cuda.synchronize()
+    assert torch.equal(S, S0)
+
+
+def test_gla_full_size_sampled_heads():
+    """The 128k-token gated workload (B=1, H=32, T=131072, d=128) in the benchmark's
+    configuration; the oracle recomputes heads 0 and 31 in full."""
+    w = GLA_WORKLOADS["gla_128k"]
+    q, k, v = make_inputs(w, seed=0, device="cuda")
+    alpha = make_gates(w, seed=0, device="cuda")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32")
+    torch.cuda.synchronize()
+    for h in (0, 31):
+        sl = lambda t: t[:, h:h + 1]
+        o_ref, S_ref = _oracle(sl(q), sl(k), sl(v), sl(alpha))
+        assert_close(to_np(sl(out)), o_ref, TOL_BF16, f"head {h} out")
+        assert_close(to_np(sl(S)), S_ref, TOL_BF16, f"head {h} S_final")
