@@ -30,7 +30,7 @@
 namespace la {
 namespace {
 
-constexpr int kGlaThreads = 256;
+constexpr int kGlaThreads = 512;  // 16 warps: one or two CTAs per SM, latency hidden by warps
 
 struct GlaParams {
   int BH;
@@ -82,7 +82,9 @@ __device__ __forceinline__ void cum_log2(float* sm, int lds, int d, int L) {
 }
 
 // K1: one CTA per (b*H + h, chunk): the chunk's summary and decay vector.
-__global__ void __launch_bounds__(kGlaThreads) gla_k1(GlaParams p) {
+constexpr int kGlaThreads1 = 256;  // K1: two CTAs per SM (8 x 8 tiles, 94 registers)
+
+__global__ void __launch_bounds__(kGlaThreads1) gla_k1(GlaParams p) {
   extern __shared__ float sm[];
   const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
   const int C = p.C, dk = p.dk, dv = p.dv, L = chunk_len(p, c);
@@ -113,16 +115,16 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k1(GlaParams p) {
     const int f0 = (tile / tiles_e) * 8, e0 = (tile % tiles_e) * 8;
     float acc[8][8] = {};
     for (int j = 0; j < L; ++j) {
-      float a[8], b[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        a[u] = sK[j * dk + f0 + u];
-        b[u] = sV[j * dv + e0 + u];
-      }
+      const float4 a0 = *reinterpret_cast<const float4*>(sK + j * dk + f0);
+      const float4 a1 = *reinterpret_cast<const float4*>(sK + j * dk + f0 + 4);
+      const float4 b0 = *reinterpret_cast<const float4*>(sV + j * dv + e0);
+      const float4 b1 = *reinterpret_cast<const float4*>(sV + j * dv + e0 + 4);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u)
@@ -144,12 +146,24 @@ __global__ void gla_k2(GlaParams p) {
   float4 P = p.S_init ? reinterpret_cast<const float4*>(p.S_init + bh * p.dk * p.dv)[col]
                       : make_float4(0.f, 0.f, 0.f, 0.f);
   float* base = p.rec + bh * p.NC * p.R;
-  for (int c = 0; c < p.NC; ++c) {
-    float4* e = reinterpret_cast<float4*>(base + static_cast<long long>(c) * p.R) + col;
-    const float4 x = *e;
-    const float a = base[static_cast<long long>(c) * p.R + p.dk * p.dv + f];
-    *e = P;
-    P = make_float4(fmaf(a, P.x, x.x), fmaf(a, P.y, x.y), fmaf(a, P.z, x.z), fmaf(a, P.w, x.w));
+  constexpr int kB = 8;  // chunks whose records are loaded before the carry walks them
+  for (int c0 = 0; c0 < p.NC; c0 += kB) {
+    float4 x[kB];
+    float a[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (c0 + u >= p.NC) break;
+      const long long r = static_cast<long long>(c0 + u) * p.R;
+      x[u] = reinterpret_cast<const float4*>(base + r)[col];
+      a[u] = base[r + p.dk * p.dv + f];
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (c0 + u >= p.NC) break;
+      reinterpret_cast<float4*>(base + static_cast<long long>(c0 + u) * p.R)[col] = P;
+      P = make_float4(fmaf(a[u], P.x, x[u].x), fmaf(a[u], P.y, x[u].y), fmaf(a[u], P.z, x[u].z),
+                      fmaf(a[u], P.w, x[u].w));
+    }
   }
   if (p.S_final) reinterpret_cast<float4*>(p.S_final + bh * p.dk * p.dv)[col] = P;
 }
@@ -182,18 +196,27 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   __syncthreads();
   cum_log2(sL, lk, dk, L);
   __syncthreads();
-  // Scores A[j][i] = sum_f q_j[f] k_i[f] 2^(L_j[f] - L_i[f]) for i <= j (0 above).
+  // Scores A[j][i] = sum_f q_j[f] k_i[f] 2^(L_j[f] - L_i[f]) for i <= j: the upper triangle
+  // is zeroed, and the C (C + 1) / 2 pairs of the lower one are numbered row by row.
   for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
     const int j = e / C, i = e - j * C;
+    if (i > j) sS[e] = 0.f;
+  }
+  const int npairs = C * (C + 1) / 2;
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+    int j = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
+    while (j * (j + 1) / 2 > e) --j;           // guard the float root at row boundaries
+    while ((j + 1) * (j + 2) / 2 <= e) ++j;
+    const int i = e - j * (j + 1) / 2;
     float a = 0.f;
-    if (i <= j && j < L) {
+    if (j < L) {
       const float* qj = sQ + j * lk;
       const float* ki = sK + i * lk;
       const float* Lj = sL + j * lk;
       const float* Li = sL + i * lk;
       for (int f = 0; f < dk; ++f) a = fmaf(qj[f] * ki[f], exp2f(Lj[f] - Li[f]), a);
     }
-    sS[e] = a;
+    sS[j * C + i] = a;
   }
   __syncthreads();
   // q_j (.) 2^(L_j) for the prefix, in place.
@@ -202,42 +225,43 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
     sQ[r * lk + f] *= exp2f(sL[r * lk + f]);
   }
   __syncthreads();
-  // o[j][e] = sum_f q~[j][f] P[f][e] + sum_{i<=j} A[j][i] v[i][e]: a 4 x 8 tile per thread.
-  const int tiles_e = dv / 8, tiles = (C / 4) * tiles_e;
+  // o[j][e] = sum_f q~[j][f] P[f][e] + sum_{i<=j} A[j][i] v[i][e]: a 4 x 4 tile per thread.
+  const int tiles_e = dv / 4, tiles = (C / 4) * tiles_e;
   for (int tile = threadIdx.x; tile < tiles; tile += blockDim.x) {
-    const int j0 = (tile / tiles_e) * 4, e0 = (tile % tiles_e) * 8;
-    float acc[4][8] = {};
+    const int j0 = (tile / tiles_e) * 4, e0 = (tile % tiles_e) * 4;
+    float acc[4][4] = {};
     for (int f = 0; f < dk; ++f) {
-      float a[4], b[8];
+      float a[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) a[u] = sQ[(j0 + u) * lk + f];
-#pragma unroll
-      for (int w = 0; w < 8; ++w) b[w] = sP[f * dv + e0 + w];
+      const float4 b = *reinterpret_cast<const float4*>(sP + f * dv + e0);
+      const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], bv[w], acc[u][w]);
     }
     for (int i = 0; i <= j0 + 3 && i < C; ++i) {
-      float a[4], b[8];
+      float a[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) a[u] = sS[(j0 + u) * C + i];
-#pragma unroll
-      for (int w = 0; w < 8; ++w) b[w] = sV[i * dv + e0 + w];
+      const float4 b = *reinterpret_cast<const float4*>(sV + i * dv + e0);
+      const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], bv[w], acc[u][w]);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       if (j0 + u >= L) continue;
       const long long o = (static_cast<long long>(bh) * p.T + t0 + j0 + u) * dv + e0;
+      if (p.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) =
+            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+      } else {
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        if (p.out_f32)
-          static_cast<float*>(p.out)[o + w] = acc[u][w];
-        else
+        for (int w = 0; w < 4; ++w)
           static_cast<__nv_bfloat16*>(p.out)[o + w] = __float2bfloat16_rn(acc[u][w]);
       }
     }
@@ -345,7 +369,7 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
   const unsigned grid = static_cast<unsigned>(BH * p.NC);
   if (e == cudaSuccess) {
     if (rec) rec->mark(s, "gla_k1");
-    gla_k1<<<grid, kGlaThreads, s1, s>>>(p);
+    gla_k1<<<grid, kGlaThreads1, s1, s>>>(p);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) {
