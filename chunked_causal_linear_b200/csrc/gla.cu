@@ -30,6 +30,8 @@
 namespace la {
 namespace {
 
+// The intra-chunk weights factor into q 2^(L) and k 2^(-L) while L >= -kGlaFactorBound.
+constexpr float kGlaFactorBound = 100.f;
 constexpr int kGlaThreads = 512;  // 16 warps: one or two CTAs per SM, latency hidden by warps
 
 struct GlaParams {
@@ -196,33 +198,76 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   __syncthreads();
   cum_log2(sL, lk, dk, L);
   __syncthreads();
-  // Scores A[j][i] = sum_f q_j[f] k_i[f] 2^(L_j[f] - L_i[f]) for i <= j: the upper triangle
-  // is zeroed, and the C (C + 1) / 2 pairs of the lower one are numbered row by row.
+  // Scores A[j][i] = sum_f q_j[f] k_i[f] 2^(L_j[f] - L_i[f]) for i <= j (0 above the diagonal).
+  // When every L of the chunk is >= -kGlaFactorBound (the usual case), the weight factors
+  // exactly: q~_j = q_j 2^(L_j) and k~_i = k_i 2^(-L_i) stay within 2^kGlaFactorBound of q, k,
+  // and A = q~ k~^T is a plain product.  Otherwise (gates small enough for 2^(-L) to overflow)
+  // each (pair, feature) takes its own exponential, whose exponent is <= 0.
+  __shared__ int s_wide;
+  if (threadIdx.x == 0) s_wide = 0;
   for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
     const int j = e / C, i = e - j * C;
     if (i > j) sS[e] = 0.f;
   }
-  const int npairs = C * (C + 1) / 2;
-  for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
-    int j = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
-    while (j * (j + 1) / 2 > e) --j;           // guard the float root at row boundaries
-    while ((j + 1) * (j + 2) / 2 <= e) ++j;
-    const int i = e - j * (j + 1) / 2;
-    float a = 0.f;
-    if (j < L) {
-      const float* qj = sQ + j * lk;
-      const float* ki = sK + i * lk;
-      const float* Lj = sL + j * lk;
-      const float* Li = sL + i * lk;
-      for (int f = 0; f < dk; ++f) a = fmaf(qj[f] * ki[f], exp2f(Lj[f] - Li[f]), a);
-    }
-    sS[j * C + i] = a;
+  __syncthreads();
+  for (int e = threadIdx.x; e < L * dk; e += blockDim.x) {
+    const int r = e / dk, f = e - r * dk;
+    if (sL[r * lk + f] < -kGlaFactorBound) s_wide = 1;  // every writer stores 1
   }
   __syncthreads();
-  // q_j (.) 2^(L_j) for the prefix, in place.
-  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
-    const int r = e / dk, f = e - r * dk;
-    sQ[r * lk + f] *= exp2f(sL[r * lk + f]);
+  const int npairs = C * (C + 1) / 2;
+  if (!s_wide) {
+    for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+      const int r = e / dk, f = e - r * dk;
+      const float x = sL[r * lk + f];
+      sQ[r * lk + f] = r < L ? sQ[r * lk + f] * exp2f(x) : 0.f;
+      sK[r * lk + f] = r < L ? sK[r * lk + f] * exp2f(-x) : 0.f;
+    }
+    __syncthreads();
+    // 2 x 2 blocks of pairs over the lower triangle, numbered row by row.
+    const int h = C / 2, nblk = h * (h + 1) / 2;
+    for (int e = threadIdx.x; e < nblk; e += blockDim.x) {
+      int bj = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
+      while (bj * (bj + 1) / 2 > e) --bj;
+      while ((bj + 1) * (bj + 2) / 2 <= e) ++bj;
+      const int j = 2 * bj, i = 2 * (e - bj * (bj + 1) / 2);
+      const float* q0 = sQ + j * lk;
+      const float* k0 = sK + i * lk;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+      for (int f = 0; f < dk; ++f) {
+        const float x0 = q0[f], x1 = q0[lk + f], y0 = k0[f], y1 = k0[lk + f];
+        a00 = fmaf(x0, y0, a00);
+        a01 = fmaf(x0, y1, a01);
+        a10 = fmaf(x1, y0, a10);
+        a11 = fmaf(x1, y1, a11);
+      }
+      sS[j * C + i] = a00;
+      if (i + 1 <= j) sS[j * C + i + 1] = a01;  // above the diagonal stays zero
+      sS[(j + 1) * C + i] = a10;
+      sS[(j + 1) * C + i + 1] = a11;
+    }
+  } else {
+    for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+      int j = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
+      while (j * (j + 1) / 2 > e) --j;           // guard the float root at row boundaries
+      while ((j + 1) * (j + 2) / 2 <= e) ++j;
+      const int i = e - j * (j + 1) / 2;
+      float a = 0.f;
+      if (j < L) {
+        const float* qj = sQ + j * lk;
+        const float* ki = sK + i * lk;
+        const float* Lj = sL + j * lk;
+        const float* Li = sL + i * lk;
+        for (int f = 0; f < dk; ++f) a = fmaf(qj[f] * ki[f], exp2f(Lj[f] - Li[f]), a);
+      }
+      sS[j * C + i] = a;
+    }
+    __syncthreads();
+    // q_j (.) 2^(L_j) for the prefix, in place.
+    for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+      const int r = e / dk, f = e - r * dk;
+      sQ[r * lk + f] *= exp2f(sL[r * lk + f]);
+    }
   }
   __syncthreads();
   // o[j][e] = sum_f q~[j][f] P[f][e] + sum_{i<=j} A[j][i] v[i][e]: a 4 x 4 tile per thread.
