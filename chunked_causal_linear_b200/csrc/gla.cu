@@ -52,21 +52,55 @@ struct GlaParams {
   float* S_final;
 };
 
-__device__ __forceinline__ float ld(const void* p, long long i, bool f32) {
-  return f32 ? static_cast<const float*>(p)[i]
-             : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
-}
-
 __device__ __forceinline__ int chunk_len(const GlaParams& p, int c) {
   return c == p.NC - 1 ? p.L_last : p.C;
 }
 
-// Loads rows [t0, t0 + L) of a [T, d] slice into sm[r * ld + f] as float32 (rows >= L zero).
+// Loads rows [t0, t0 + L) of a [T, d] slice into sm[r * lds + f] as float32 (rows >= L zero),
+// eight elements per access (d is a multiple of 8): 16-byte loads of bf16, two of float32.
 __device__ __forceinline__ void load_rows(float* sm, int lds, const void* g, bool f32,
                                           long long base, int d, int C, int L) {
-  for (int e = threadIdx.x; e < C * d; e += blockDim.x) {
-    const int r = e / d, f = e - r * d;
-    sm[r * lds + f] = r < L ? ld(g, base + static_cast<long long>(r) * d + f, f32) : 0.f;
+  const int g8 = d / 8;
+  for (int e = threadIdx.x; e < C * g8; e += blockDim.x) {
+    const int r = e / g8, f = (e - r * g8) * 8;
+    float x[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (r < L) {
+      const long long i = base + static_cast<long long>(r) * d + f;
+      if (f32) {
+        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(g) + i);
+        const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(g) + i + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      } else {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(g) + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 h;
+          std::memcpy(&h, &w[k], 4);
+          const float2 v = __bfloat1622float2(h);
+          x[2 * k] = v.x;
+          x[2 * k + 1] = v.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sm[r * lds + f + k] = x[k];
+  }
+}
+
+// The gates of rows [t0, t0 + L) into sm[r * lds + f] (rows >= L: 1), float4 loads.
+__device__ __forceinline__ void load_gates(float* sm, int lds, const float* g, long long base,
+                                           int d, int C, int L) {
+  const int g4 = d / 4;
+  for (int e = threadIdx.x; e < C * g4; e += blockDim.x) {
+    const int r = e / g4, f = (e - r * g4) * 4;
+    const float4 a = r < L ? *reinterpret_cast<const float4*>(g + base + static_cast<long long>(r) * d + f)
+                           : make_float4(1.f, 1.f, 1.f, 1.f);
+    sm[r * lds + f] = a.x;
+    sm[r * lds + f + 1] = a.y;
+    sm[r * lds + f + 2] = a.z;
+    sm[r * lds + f + 3] = a.w;
   }
 }
 
@@ -96,10 +130,7 @@ __global__ void __launch_bounds__(kGlaThreads1) gla_k1(GlaParams p) {
   const long long t0 = static_cast<long long>(c) * C;
   load_rows(sK, dk, p.k, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dk, dk, C, L);
   load_rows(sV, dv, p.v, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dv, dv, C, L);
-  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
-    const int r = e / dk;
-    sA[e] = r < L ? p.alpha[(static_cast<long long>(bh) * p.T + t0) * dk + e] : 1.f;
-  }
+  load_gates(sA, dk, p.alpha, (static_cast<long long>(bh) * p.T + t0) * dk, dk, C, L);
   __syncthreads();
   cum_log2(sA, dk, dk, L);
   __syncthreads();
@@ -188,10 +219,7 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   load_rows(sQ, lk, p.q, p.in_f32, rq, dk, C, L);
   load_rows(sK, lk, p.k, p.in_f32, rq, dk, C, L);
   load_rows(sV, dv, p.v, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dv, dv, C, L);
-  for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
-    const int r = e / dk, f = e - r * dk;
-    sL[r * lk + f] = r < L ? p.alpha[rq + e] : 1.f;
-  }
+  load_gates(sL, lk, p.alpha, rq, dk, C, L);
   const float4* P4 = reinterpret_cast<const float4*>(p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R);
   for (int e = threadIdx.x; e < dk * dv / 4; e += blockDim.x)
     reinterpret_cast<float4*>(sP)[e] = P4[e];
@@ -349,6 +377,9 @@ int gla_validate(const la_gla_args& a) {
   if (!aligned16(a.S_init) || !aligned16(a.S_final)) return LA_ERR_INVALID_ARGUMENT;
   if (BH > 0 && a.T > 0) {
     if (!a.q || !a.k || !a.v || !a.alpha || !a.out) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.alpha) ||
+        !aligned16(a.out))
+      return LA_ERR_INVALID_ARGUMENT;
     const size_t e = a.dtype == LA_DTYPE_F32 ? 4 : 2;
     const size_t eo = (a.dtype == LA_DTYPE_F32 || a.out_dtype == LA_OUT_F32) ? 4 : 2;
     const size_t nk = static_cast<size_t>(BH) * a.T * a.dk, nv = static_cast<size_t>(BH) * a.T * a.dv;

@@ -287,7 +287,8 @@ def test_gla_argument_errors_before_any_launch(lib):
     cases = [(dict(B=-1), 1), (dict(dtype=5), 1), (dict(out_dtype=3), 1), (dict(dk=12), 2),
              (dict(dv=136), 2), (dict(C=128), 2), (dict(alpha=0), 1), (dict(out=0), 1),
              (dict(out=0x1000), 1), (dict(out=0x6000000 + 64), 1), (dict(S_init=0x100004), 1),
-             (dict(workspace=0x100010), 1), (dict(B=0), 0), (dict(H=0), 0)]
+             (dict(workspace=0x100010), 1), (dict(q=0x1008), 1), (dict(alpha=0x6000004), 1),
+             (dict(B=0), 0), (dict(H=0), 0)]
     for kw, status in cases:
         assert lib.lin_attn_gla_prefill(ctypes.byref(args(**kw))) == status, kw
     assert lib.lin_attn_gla_prefill(None) == 1
