@@ -295,3 +295,33 @@ def test_gla_argument_errors_before_any_launch(lib):
     # one record of dk*dv + dk floats per chunk, 256-byte aligned
     n = lib.lin_attn_gla_workspace_bytes(2, 3, 100, 64, 32, 64)
     assert n == (2 * 3 * 2 * (64 * 32 + 64) * 4 + 255) // 256 * 256
+
+
+def test_header_is_plain_c_and_the_binding_structs_match_it(tmp_path):
+    """The header compiles as strict C99, and every ctypes struct of the binding has the C
+    struct's size and field offsets (a field added or moved on one side only fails here)."""
+    import shutil
+    import subprocess
+    from chunked_causal_linear_b200 import binding as Bnd
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"la_prefill_args": Bnd.PrefillArgs, "la_backward_args": Bnd.BackwardArgs,
+               "la_gla_args": Bnd.GlaArgs}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "linattn.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", str(ROOT / "include"),
+                    str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
