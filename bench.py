@@ -699,7 +699,7 @@ def gla_bench(args, info, dev):
     S = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
     ws = torch.empty(B.lin_attn_gla_workspace_bytes(w.B, w.H, w.T, w.dk, w.dv, w.C),
                      dtype=torch.uint8, device=dev)
-    kw = dict(chunk=w.C, out_dtype="f32", workspace=ws)
+    kw = dict(chunk=w.C, out_dtype="f32", workspace=ws, kernel_path=args.gla_path)
 
     def step():
         B.lin_attn_gla_prefill(q, k, v, alpha, out, S, **kw)
@@ -722,7 +722,8 @@ def gla_bench(args, info, dev):
     ms_max = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, info, dev)
     per = [B.lin_attn_gla_prefill_timed(q, k, v, alpha, out, S, **kw)
            for _ in range(max(1, args.kernel_timing_steps))]
-    names = ["gla_k1", "gla_k2", "gla_k3"]
+    tc = args.gla_path == "tensor_core"
+    names = ["gla_tc_prep", "k1_tc", "gla_tc_k2", "k3_tc"] if tc else ["gla_k1", "gla_k2", "gla_k3"]
     kern_ms = {n: statistics.mean(x[i] for x in per) for i, n in enumerate(names)}
     BH, NC, C = w.B * w.H, -(-w.T // w.C), w.C
     R = w.dk * w.dv + w.dk
@@ -732,29 +733,46 @@ def gla_bench(args, info, dev):
     # logs stay above -100 (all of this workload's) the scores need no exponential per pair
     k3_flop = 2 * BH * NC * (C * w.dk * w.dv + pairs * w.dk + pairs * w.dv)
     e_in = 2
+    Rt = w.dk * w.dv
+    nk, nv = BH * w.T * w.dk, BH * w.T * w.dv
     bytes_ = {"gla_k1": BH * w.T * (w.dk * (e_in + 4) + w.dv * e_in) + BH * NC * R * 4,
               "gla_k2": 2 * BH * NC * R * 4,
-              "gla_k3": BH * w.T * (w.dk * (2 * e_in + 4) + w.dv * e_in + w.dv * 4) + BH * NC * R * 4}
+              "gla_k3": BH * w.T * (w.dk * (2 * e_in + 4) + w.dv * e_in + w.dv * 4) + BH * NC * R * 4,
+              # tensor cores: prep reads q, k, gates, writes three bf16 copies and a_c
+              "gla_tc_prep": nk * (2 * e_in + 4) + 3 * nk * e_in + BH * NC * w.dk * 4,
+              "k1_tc": nk * e_in + nv * e_in + BH * NC * Rt * 4,
+              "gla_tc_k2": 2 * BH * NC * Rt * 4 + BH * NC * w.dk * 4,
+              "k3_tc": 2 * nk * e_in + nv * e_in + BH * (NC - 1) * Rt * 4 + nv * 4}
     peak, peak_kind = measured_peaks()
     hbm = {n: bytes_[n] / (kern_ms[n] / 1e3) / 1e9 / peak for n in names}
-    roofline = {"bound": "alu", "kernel": "gla_k3",
-                "achieved": k3_flop / (kern_ms["gla_k3"] / 1e3) / 1e12,
-                "peak": NOMINAL_FP32_FLOPS / 1e12, "unit": "TFLOP/s (fp32, CUDA cores)",
-                "frac": k3_flop / (kern_ms["gla_k3"] / 1e3) / NOMINAL_FP32_FLOPS,
-                "traffic": None,
-                "peak_source": "unit counts: 148 SMs x 128 FMA lanes x 2 x 1965 MHz",
-                "hbm_frac_of_measured": hbm}
+    if tc:
+        dom = max(kern_ms, key=kern_ms.get)
+        roofline = {"bound": "hbm", "kernel": dom,
+                    "achieved": bytes_[dom] / (kern_ms[dom] / 1e3) / 1e9, "peak": peak,
+                    "unit": "GB/s", "frac": hbm[dom], "traffic": None,
+                    "algorithmic_bytes": bytes_[dom],
+                    "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                    "hbm_frac_of_measured": hbm}
+    else:
+        roofline = {"bound": "alu", "kernel": "gla_k3",
+                    "achieved": k3_flop / (kern_ms["gla_k3"] / 1e3) / 1e12,
+                    "peak": NOMINAL_FP32_FLOPS / 1e12, "unit": "TFLOP/s (fp32, CUDA cores)",
+                    "frac": k3_flop / (kern_ms["gla_k3"] / 1e3) / NOMINAL_FP32_FLOPS,
+                    "traffic": None,
+                    "peak_source": "unit counts: 148 SMs x 128 FMA lanes x 2 x 1965 MHz",
+                    "hbm_frac_of_measured": hbm}
     if info.is_root:
         cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "C": w.C,
                "inputs": "bf16", "gates": "float32 sigmoid(N(4, 1))", "out_dtype": "f32",
-               "kernel_path": "fma (CUDA cores)", "l2": "inputs larger than L2, no flush",
+               "kernel_path": "tensor_core (factored gates, bf16 operands)" if tc
+               else "fma (CUDA cores)", "l2": "inputs larger than L2, no flush",
                "parallelism": "replicas (one independent problem per GPU)"}
         line = {"metric": METRIC_GLA, "value": info.world * w.tokens_heads / (ms_max / 1e3),
                 "unit": UNIT, "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
                 "mode": "gla", "roofline": roofline, "kernels_ms": kern_ms, "clocks": clocks,
-                "gpu_launches": 3 * args.steps, "device_error": B.lin_attn_device_error()}
+                "gpu_launches": len(names) * args.steps, "device_error": B.lin_attn_device_error()}
         print(json.dumps(line), flush=True)
 
 
@@ -807,6 +825,9 @@ def main():
     ap.add_argument("--gla", action="store_true",
                     help="instead of the prefill: gated linear attention (data-dependent decay) "
                          "on the 128k-token gated workload")
+    ap.add_argument("--gla-path", default="fma", choices=["fma", "tensor_core"],
+                    help="GLA kernels: exact CUDA-core ones, or the tensor-core prefill on "
+                         "factored gates")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")

@@ -436,6 +436,14 @@ HostLayout host_layout(const la_prefill_args& a) {
 
 int prefill_with_args(const la_prefill_args& a, Recorder* rec) { return prefill(a, rec); }
 
+int* device_error_word() { return error_word_ptr(); }
+
+bool make_tile_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0,
+                   uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
+                   uint32_t box1) {
+  return make_map(m, dt, base, d0, d1, d2, stride1, stride2, box0, box1);
+}
+
 int check_prefill_args(const la_prefill_args& a) {
   Path path;
   const int st = validate(a, &path);

@@ -26,6 +26,7 @@
 #include "../../include/linattn.h"
 #include "common.cuh"
 #include "launch.h"
+#include "ptx.cuh"
 
 namespace la {
 namespace {
@@ -341,6 +342,112 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Tensor-core path (opt-in).  With every cumulative log of a chunk >= -kGlaFactorBound the
+// chunk's weights factor exactly: 2^(L_j - L_i) = 2^(L_j) 2^(-L_i) and 2^(L_last - L_j), so
+// gated attention is the plain (undecayed, identity-map) prefill of pre-scaled inputs:
+//   q~ = q (.) 2^L,  k~ = k (.) 2^-L  (the combine: o_j = q~_j P_c + sum_{i<=j} (q~_j . k~_i) v_i)
+//   k^ = k (.) 2^(L_last - L)         (the summary S_loc = sum_j k^_j v_j^T)
+// which the prefill's tcgen05 kernels k1_tc / k3_tc compute; between them the carry over
+// chunks scales the prefix by a_c per key feature.  q~, k~, k^ are rounded to bf16 (the
+// kernels' operand type).  A chunk whose gates are too small to factor sets the device error
+// word (kErrGateRange) and its results are not valid: this path is for gates of moderate size
+// (for example all >= 0.34 at C = 64), the CUDA-core path for any gates.
+
+// One CTA per (b*H + h, chunk): cumulative log2 gates, the three scaled copies, a_c.
+__global__ void __launch_bounds__(256) gla_tc_prep(GlaParams p, __nv_bfloat16* qt,
+                                                    __nv_bfloat16* kt, __nv_bfloat16* kh,
+                                                    float* ac, int* err) {
+  extern __shared__ float sm[];
+  const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
+  const int C = p.C, dk = p.dk, L = chunk_len(p, c);
+  float* sA = sm;  // [C][dk]
+  const long long base = (static_cast<long long>(bh) * p.T + static_cast<long long>(c) * C) * dk;
+  load_gates(sA, dk, p.alpha, base, dk, C, L);
+  __syncthreads();
+  cum_log2(sA, dk, dk, L);
+  __syncthreads();
+  const int g8 = dk / 8;
+  for (int e = threadIdx.x; e < L * g8; e += blockDim.x) {
+    const int r = e / g8, f0 = (e - r * g8) * 8;
+    const long long i = base + static_cast<long long>(r) * dk + f0;
+    const uint4 uq = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + i);
+    const uint4 uk = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + i);
+    const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+    uint32_t oq[4], ok[4], oh[4];
+    bool wide = false;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      __nv_bfloat162 hq, hk;
+      std::memcpy(&hq, &wq[m], 4);
+      std::memcpy(&hk, &wk[m], 4);
+      const float2 fq = __bfloat1622float2(hq), fk = __bfloat1622float2(hk);
+      const int f = f0 + 2 * m;
+      const float l0 = sA[r * dk + f], l1 = sA[r * dk + f + 1];
+      const float e0 = sA[(L - 1) * dk + f], e1 = sA[(L - 1) * dk + f + 1];
+      wide = wide || l0 < -kGlaFactorBound || l1 < -kGlaFactorBound;
+      const __nv_bfloat162 rq = __float22bfloat162_rn(make_float2(fq.x * exp2f(l0), fq.y * exp2f(l1)));
+      const __nv_bfloat162 rk = __float22bfloat162_rn(make_float2(fk.x * exp2f(-l0), fk.y * exp2f(-l1)));
+      const __nv_bfloat162 rh =
+          __float22bfloat162_rn(make_float2(fk.x * exp2f(e0 - l0), fk.y * exp2f(e1 - l1)));
+      std::memcpy(&oq[m], &rq, 4);
+      std::memcpy(&ok[m], &rk, 4);
+      std::memcpy(&oh[m], &rh, 4);
+    }
+    if (wide) report_error(err, kErrGateRange);
+    *reinterpret_cast<uint4*>(qt + i) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
+    *reinterpret_cast<uint4*>(kt + i) = make_uint4(ok[0], ok[1], ok[2], ok[3]);
+    *reinterpret_cast<uint4*>(kh + i) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+  }
+  for (int f = threadIdx.x; f < dk; f += blockDim.x)
+    ac[(static_cast<long long>(bh) * p.NC + c) * dk + f] = exp2f(sA[(L - 1) * dk + f]);
+}
+
+// The carry over chunks on the transposed records (S^T, [dv][dk] per chunk, as k1_tc writes
+// and k3_tc reads them): P^T[e][f] <- a_c[f] P^T[e][f] + S_c^T[e][f], exclusive, in place; one
+// thread per float4 of the state, eight chunks loaded ahead.  The state before chunk 0 is
+// S_init^T (or zero); the state after the last chunk goes to S_final ([dk][dv]).
+__global__ void gla_tc_k2(GlaParams p, const float* ac) {
+  const long long n4 = static_cast<long long>(p.dk) * p.dv / 4;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(p.BH) * n4) return;
+  const long long bh = idx / n4, col = idx - bh * n4;
+  const int e = static_cast<int>(col * 4 / p.dk), f4 = static_cast<int>(col * 4 % p.dk);
+  const long long sd = static_cast<long long>(p.dk) * p.dv;
+  float4 P = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.S_init) {
+    const float* S0 = p.S_init + bh * sd;
+    P = make_float4(S0[(f4 + 0) * p.dv + e], S0[(f4 + 1) * p.dv + e], S0[(f4 + 2) * p.dv + e],
+                    S0[(f4 + 3) * p.dv + e]);
+  }
+  float* base = p.rec + bh * p.NC * sd;
+  const float* abase = ac + bh * p.NC * p.dk + f4;
+  constexpr int kB = 8;
+  for (int c0 = 0; c0 < p.NC; c0 += kB) {
+    float4 x[kB], a[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (c0 + u >= p.NC) break;
+      x[u] = reinterpret_cast<const float4*>(base + static_cast<long long>(c0 + u) * sd)[col];
+      a[u] = *reinterpret_cast<const float4*>(abase + static_cast<long long>(c0 + u) * p.dk);
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (c0 + u >= p.NC) break;
+      reinterpret_cast<float4*>(base + static_cast<long long>(c0 + u) * sd)[col] = P;
+      P = make_float4(fmaf(a[u].x, P.x, x[u].x), fmaf(a[u].y, P.y, x[u].y),
+                      fmaf(a[u].z, P.z, x[u].z), fmaf(a[u].w, P.w, x[u].w));
+    }
+  }
+  if (p.S_final) {
+    float* Sf = p.S_final + bh * sd;
+    Sf[(f4 + 0) * p.dv + e] = P.x;
+    Sf[(f4 + 1) * p.dv + e] = P.y;
+    Sf[(f4 + 2) * p.dv + e] = P.z;
+    Sf[(f4 + 3) * p.dv + e] = P.w;
+  }
+}
+
 size_t gla_smem_k1(int C, int dk, int dv) { return static_cast<size_t>(C) * (2 * dk + dv) * 4; }
 size_t gla_smem_k3(int C, int dk, int dv) {
   return (static_cast<size_t>(C) * (3 * (dk + 1) + dv) + static_cast<size_t>(dk) * dv +
@@ -357,10 +464,33 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return a0 < b0 + bn && b0 < a0 + an;
 }
 
+// Workspace of either path.  CUDA cores: one record of dk*dv + dk floats per chunk.  Tensor
+// cores: q~, k~, k^ (bf16, the inputs' shape), a record of dk*dv floats per chunk and a_c.
+struct GlaLayout {
+  size_t rec, qt, kt, kh, ac, total;
+};
+GlaLayout gla_layout(int B, int H, long long T, int dk, int dv, int C) {
+  GlaLayout l{};
+  if (B <= 0 || H <= 0 || T <= 0 || C <= 0) return l;
+  const size_t BH = static_cast<size_t>(B) * H, NC = static_cast<size_t>((T + C - 1) / C);
+  const size_t fma = align256(BH * NC * (static_cast<size_t>(dk) * dv + dk) * 4);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  l.rec = take(BH * NC * static_cast<size_t>(dk) * dv * 4);
+  l.qt = take(BH * static_cast<size_t>(T) * dk * 2);
+  l.kt = take(BH * static_cast<size_t>(T) * dk * 2);
+  l.kh = take(BH * static_cast<size_t>(T) * dk * 2);
+  l.ac = take(BH * NC * dk * 4);
+  l.total = off > fma ? off : fma;
+  return l;
+}
+
 size_t gla_ws(int B, int H, long long T, int dk, int dv, int C) {
-  if (B <= 0 || H <= 0 || T <= 0 || C <= 0) return 0;
-  const long long NC = (T + C - 1) / C;
-  return align256(static_cast<size_t>(B) * H * NC * (static_cast<size_t>(dk) * dv + dk) * 4);
+  return gla_layout(B, H, T, dk, dv, C).total;
 }
 
 int gla_validate(const la_gla_args& a) {
@@ -369,6 +499,11 @@ int gla_validate(const la_gla_args& a) {
   if (a.dtype != LA_DTYPE_BF16 && a.dtype != LA_DTYPE_F32) return LA_ERR_INVALID_ARGUMENT;
   if (a.out_dtype != LA_OUT_AS_INPUT && a.out_dtype != LA_OUT_F32) return LA_ERR_INVALID_ARGUMENT;
   if (!gla_dims_ok(a.dk) || !gla_dims_ok(a.dv) || !(a.C == 16 || a.C == 32 || a.C == 64))
+    return LA_ERR_UNSUPPORTED;
+  if (a.kernel_path < LA_PATH_AUTO || a.kernel_path > LA_PATH_FMA) return LA_ERR_INVALID_ARGUMENT;
+  if (a.kernel_path == LA_PATH_TENSOR_CORE &&
+      !(a.dtype == LA_DTYPE_BF16 && a.C == 64 && (a.dk == 64 || a.dk == 128) &&
+        (a.dv == 64 || a.dv == 128) && a.T < (1LL << 31)))
     return LA_ERR_UNSUPPORTED;
   const long long BH = static_cast<long long>(a.B) * a.H;
   const long long NC = a.T > 0 ? (a.T + a.C - 1) / a.C : 0;
@@ -436,6 +571,82 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
   p.S_init = a.S_init;
   p.S_final = a.S_final;
 
+  if (a.kernel_path == LA_PATH_TENSOR_CORE) {
+    const GlaLayout l = gla_layout(a.B, a.H, a.T, a.dk, a.dv, a.C);
+    auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
+    float* ac = reinterpret_cast<float*>(ws + l.ac);
+    p.rec = reinterpret_cast<float*>(ws + l.rec);
+    PrefillParams pp{};
+    pp.BH = p.BH;
+    pp.H = a.H;
+    pp.T = a.T;
+    pp.dk = a.dk;
+    pp.dv = a.dv;
+    pp.C = a.C;
+    pp.NC = p.NC;
+    pp.L_last = p.L_last;
+    pp.R = a.dk * a.dv;
+    pp.rec = p.rec;
+    pp.has_init = a.S_init != nullptr;
+    pp.Ls = 1;
+    pp.G = 1;
+    pp.err = device_error_word();
+    GammaTable gt;
+    for (int h = 0; h < kMaxHeads; ++h) gt.g[h] = 1.f;
+    const Flags fl{0, false, false, p.out_f32};
+    const uint64_t T = static_cast<uint64_t>(a.T), BHu = static_cast<uint64_t>(BH);
+    const uint64_t dk = a.dk, dv = a.dv;
+    TcMaps m1, m3;
+    bool ok = make_tile_map(&m1.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.kh), dk, T, BHu, dk * 2,
+                            T * dk * 2, 64, 64) &&
+              make_tile_map(&m1.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, dv, T, BHu, dv * 2,
+                            T * dv * 2, 64, 64) &&
+              make_tile_map(&m1.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.rec, dk, dv,
+                            BHu * static_cast<uint64_t>(p.NC), dk * 4, dk * dv * 4, 32,
+                            static_cast<uint32_t>(dv));
+    m3 = m1;
+    ok = ok &&
+         make_tile_map(&m3.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.qt), dk, T, BHu, dk * 2,
+                       T * dk * 2, 64, 64) &&
+         make_tile_map(&m3.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.kt), dk, T, BHu, dk * 2,
+                       T * dk * 2, 64, 64) &&
+         (p.out_f32 ? make_tile_map(&m3.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, dv, T, BHu,
+                                    dv * 4, T * dv * 4, 32, 64)
+                    : make_tile_map(&m3.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, dv, T, BHu,
+                                    dv * 2, T * dv * 2, 64, 64));
+    cudaError_t e = ok ? cudaSuccess : cudaErrorInvalidValue;
+    const size_t sp = static_cast<size_t>(a.C) * a.dk * 4;
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gla_tc_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(sp));
+    if (e == cudaSuccess) {
+      if (rec) rec->mark(s, "gla_tc_prep");
+      gla_tc_prep<<<static_cast<unsigned>(BH * p.NC), 256, sp, s>>>(p, bf(l.qt), bf(l.kt),
+                                                                   bf(l.kh), ac, pp.err);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+      if (rec) rec->mark(s, "k1_tc");
+      e = launch_k1_tc(pp, gt, m1, fl, s);
+    }
+    if (e == cudaSuccess) {
+      const long long n = BH * a.dk * a.dv / 4;
+      if (rec) rec->mark(s, "gla_tc_k2");
+      gla_tc_k2<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p, ac);
+      e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+      if (rec) rec->mark(s, "k3_tc");
+      e = launch_k3_tc(pp, gt, m3, fl, s);
+    }
+    if (rec) rec->mark(s);
+    if (owned) {
+      const cudaError_t e2 = cudaFreeAsync(ws, s);
+      if (e == cudaSuccess) e = e2;
+    }
+    return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+  }
+
   const size_t s1 = gla_smem_k1(a.C, a.dk, a.dv), s3 = gla_smem_k3(a.C, a.dk, a.dv);
   cudaError_t e = cudaFuncSetAttribute(gla_k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(s1));
@@ -484,9 +695,10 @@ extern "C" int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel
                                           int max_kernels, int* n_kernels) {
   if (!args || !kernel_ms || !n_kernels || max_kernels < 1) return LA_ERR_INVALID_ARGUMENT;
   *n_kernels = 0;
-  cudaEvent_t ev[4];
-  const char* label[4] = {nullptr};
-  for (int i = 0; i < 4; ++i)
+  constexpr int kEv = 8;
+  cudaEvent_t ev[kEv];
+  const char* label[kEv] = {nullptr};
+  for (int i = 0; i < kEv; ++i)
     if (cudaEventCreate(&ev[i]) != cudaSuccess) {
       for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
       return LA_ERR_CUDA;
@@ -494,7 +706,7 @@ extern "C" int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel
   la::Recorder rec;
   rec.ev = ev;
   rec.label = label;
-  rec.cap = 4;
+  rec.cap = kEv;
   int st = la::gla_prefill(*args, &rec);
   if (st == LA_OK && cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(args->stream)) != cudaSuccess)
     st = LA_ERR_CUDA;
@@ -507,6 +719,6 @@ extern "C" int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel
     }
     *n_kernels = nk;
   }
-  for (int i = 0; i < 4; ++i) cudaEventDestroy(ev[i]);
+  for (int i = 0; i < kEv; ++i) cudaEventDestroy(ev[i]);
   return st;
 }

@@ -12,6 +12,14 @@ namespace la {
 // The argument checks of the prefill alone: LA_OK when prefill_with_args(a) would launch.
 int check_prefill_args(const la_prefill_args& a);
 
+// The device error word of the current device (every kernel receives it).
+int* device_error_word();
+
+// A 3D tiled TMA map (d0 innermost) with the 128-byte swizzle, as the prefill's kernels use.
+bool make_tile_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0,
+                   uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
+                   uint32_t box1);
+
 enum Dtype : int { kBF16 = 0, kF32 = 1 };
 
 struct Flags {

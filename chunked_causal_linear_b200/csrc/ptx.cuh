@@ -15,6 +15,7 @@ enum : int {
   kErrTmaTimeout = 1,
   kErrMmaTimeout = 2,
   kErrBadShape = 3,
+  kErrGateRange = 4,  // gated attention on the tensor cores: a chunk's gates too small to factor
 };
 
 __device__ __forceinline__ void report_error(int* err, int code) {

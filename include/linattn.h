@@ -414,6 +414,14 @@ typedef struct la_gla_args {
   void* workspace;        /* DEVICE, 256-byte aligned, or NULL */
   size_t workspace_bytes;
   la_stream_t stream;
+  /* la_kernel_path.  LA_PATH_AUTO / LA_PATH_FMA: the CUDA-core kernels above, exact for any
+   * gates.  LA_PATH_TENSOR_CORE (bf16, C = 64, dk, dv in {64, 128}): while every chunk's
+   * cumulative log2 gates stay >= -100 (for example all gates >= 0.34), the weights factor
+   * as 2^(L_j) 2^(-L_i), and the call runs the prefill's tcgen05 kernels on q (.) 2^L,
+   * k (.) 2^-L and k (.) 2^(L_last - L) (rounded to bf16), with the carry over chunks scaling
+   * the prefix per key feature.  A chunk outside that range sets the device error word to 4
+   * (lin_attn_device_error) and the call's results are not valid. */
+  int kernel_path;
 } la_gla_args;
 
 int lin_attn_gla_prefill(const la_gla_args* args);

@@ -112,3 +112,59 @@ def test_gla_full_size_sampled_heads():
         o_ref, S_ref = _oracle(sl(q), sl(k), sl(v), sl(alpha))
         assert_close(to_np(sl(out)), o_ref, TOL_BF16, f"head {h} out")
         assert_close(to_np(sl(S)), S_ref, TOL_BF16, f"head {h} S_final")
+
+
+# ---------------------------------------------------------------------------------------
+# The tensor-core path (opt-in): gates whose chunk logs stay >= -100 factor exactly, but the
+# factored operands q (.) 2^L, k (.) 2^-L and k (.) 2^(L_last - L) are rounded to bf16 (the
+# prefill's identity-map kernels split no operand), so every product carries two bf16
+# roundings (2 * 2^-9 relative) where the retention path's exact bf16 inputs carry none.
+# Bound: 2^-4 * rms = 2 * 2^-9 per product times 16 for the maximum over ~10^6 outputs and
+# the few terms that average it when small gates shorten the memory.  Measured: up to
+# 1.4e-2 (gates sigmoid(N(4, 1))) and 3.3e-2 (sigmoid(N(3, 1)), d = 64).
+TOL_GLA_TC = 2.0 ** -4
+
+@pytest.mark.parametrize("T", [65, 1000, 3001])
+def test_gla_tensor_core_path_matches_oracle(T):
+    q, k, v, alpha = _problem(T)
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+    torch.cuda.synchronize()
+    assert B.lin_attn_device_error() == 0
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    assert_close(to_np(out), o_ref, TOL_GLA_TC, "out")
+    assert_close(to_np(S), S_ref, TOL_GLA_TC, "S_final")
+
+
+def test_gla_tensor_core_path_with_initial_state_and_d64():
+    q, k, v, alpha = _problem(1500, dk=64, dv=128, mean=3.0)
+    S0 = (torch.randn((2, 3, 64, 128), generator=torch.Generator().manual_seed(4)) * 0.3).cuda()
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0, out_dtype="f32",
+                                    kernel_path="tensor_core")
+    torch.cuda.synchronize()
+    assert B.lin_attn_device_error() == 0
+    o_ref, S_ref = _oracle(q, k, v, alpha, S0)
+    assert_close(to_np(out), o_ref, TOL_GLA_TC, "out")
+    assert_close(to_np(S), S_ref, TOL_GLA_TC, "S_final")
+
+
+def test_gla_tensor_core_path_flags_gates_it_cannot_factor():
+    # gates around 0.05: a chunk's cumulative log2 passes -100 within ~25 tokens
+    q, k, v, alpha = _problem(300, mean=-3.0)
+    B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+    torch.cuda.synchronize()
+    assert B.lin_attn_device_error() == 4  # reading it clears it
+    assert B.lin_attn_device_error() == 0
+
+
+def test_gla_tensor_core_path_full_size_sampled_heads():
+    w = GLA_WORKLOADS["gla_128k"]
+    q, k, v = make_inputs(w, seed=0, device="cuda")
+    alpha = make_gates(w, seed=0, device="cuda")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+    torch.cuda.synchronize()
+    assert B.lin_attn_device_error() == 0
+    for h in (0, 31):
+        sl = lambda t: t[:, h:h + 1]
+        o_ref, S_ref = _oracle(sl(q), sl(k), sl(v), sl(alpha))
+        assert_close(to_np(sl(out)), o_ref, TOL_GLA_TC, f"head {h} out")
+        assert_close(to_np(sl(S)), S_ref, TOL_GLA_TC, f"head {h} S_final")
