@@ -39,11 +39,15 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
-def test_library_links_no_torch():
+def test_library_links_no_torch(lib):
+    # The libraries the build declared it needs (the dynamic section's NEEDED entries of the
+    # library built here), independent of the search path.
     import subprocess
     from chunked_causal_linear_b200.binding import LIB_PATH
-    out = subprocess.run(["ldd", str(LIB_PATH)], capture_output=True, text=True).stdout
-    assert "torch" not in out and "c10" not in out
+    out = subprocess.run(["readelf", "-d", str(LIB_PATH)], capture_output=True, text=True,
+                         check=True).stdout
+    needed = [l for l in out.splitlines() if "NEEDED" in l]
+    assert needed and not any("torch" in l or "c10" in l for l in needed), needed
 
 
 def test_status_strings_and_version(lib):
