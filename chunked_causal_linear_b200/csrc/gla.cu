@@ -422,7 +422,7 @@ __global__ void gla_tc_k2(GlaParams p, const float* ac) {
   }
   float* base = p.rec + bh * p.NC * sd;
   const float* abase = ac + bh * p.NC * p.dk + f4;
-  constexpr int kB = 8;
+  constexpr int kB = 16;
   for (int c0 = 0; c0 < p.NC; c0 += kB) {
     float4 x[kB], a[kB];
 #pragma unroll

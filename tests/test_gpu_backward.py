@@ -295,3 +295,12 @@ def test_normalised_backward_full_size_sampled_heads():
                                         normalize=True)
         for name, x, r in zip(("grad_q", "grad_k", "grad_v"), got[:3], ref[:3]):
             assert_close(to_np(sl(x)), r, TOL_BF16, f"({b},{h}) {name}")
+
+
+def test_normalised_backward_small_and_extreme_decays():
+    # gamma = 0, 1e-7 (below 2^-20: the final-state gradient's terms are added directly),
+    # 2^-19, 0.5 and 1, with every state gradient given and requested
+    q, k, v, do, _, st = _norm_problem(700, decay=True, H=5, states=True)
+    gamma = [0.0, 1e-7, 2.0 ** -19, 0.5, 1.0]
+    got, ref = _norm_case(q, k, v, do, gamma, st, eps=0.1, out_dtype="f32")
+    _check_norm(got, ref, TOL_BF16)
