@@ -10,11 +10,13 @@
 //   K1  S_loc = sum_j (k_j (.) e^(L_last - L_j)) v_j^T,   a_c = e^(L_last)
 //   K2  P_c = the exclusive prefix of (a_c, S_loc) over chunks (a carry per state element)
 //   K3  o_j = (q_j (.) e^(L_j)) P_c + sum_{i<=j} (sum_f q_j[f] k_i[f] e^(L_j[f] - L_i[f])) v_i
-// The kernels form these as powers of two of cumulative log2 gates.  Every exponent is
-// <= 0, so nothing overflows whatever the gates (a gate below 2^-126 counts as 2^-126).  The
-// intra-chunk scores take one exponential per (pair, feature) on the CUDA cores: exact, and
-// the reason this path is ALU-bound (the per-feature ratio does not factor into one matrix
-// product without rescaling that can overflow).
+// The kernels form these as powers of two of cumulative log2 gates, every exponent <= 0,
+// so nothing overflows whatever the gates (a gate below 2^-126 counts as 2^-126).  Two paths:
+//   CUDA cores (default; gla_k1, gla_k2, gla_k3): exact in float32 for any gates.  K3's
+//     scores factor as (q (.) 2^L) . (k (.) 2^-L) when the chunk's logs stay >= -100 (plain
+//     dot products), else take one exponential per (pair, feature).
+//   Tensor cores (opt-in; gla_tc_prep, the prefill's k1_tc / k3_tc, gla_tc_k2): the factored
+//     operands in bf16 through the prefill's tcgen05 kernels, for gates that factor.
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
