@@ -41,8 +41,10 @@
 //
 // la_oracle_backward differentiates both forms by hand, token by token (the chain rule
 // through the recurrence; see backward_pair), for the backward pass.  la_oracle_gla_forward
-// runs the gated (data-dependent decay) recurrence (see gla_pair).
+// runs the gated (data-dependent decay) recurrence (see gla_pair), la_oracle_gla_backward its
+// gradients (see gla_backward_pair).
 
+#include <algorithm>
 #include <cmath>
 #include <cstddef>
 #include <cstdint>
@@ -300,9 +302,138 @@ void gla_pair(const GlaProblem& p, long long bh) {
     for (size_t e = 0; e < S.size(); ++e) p.S_final[bh * dk * dv + e] = S[e];
 }
 
+// Gradients of the gated loop (see gla_pair) for L = <dout, out> + <dS_final, S_final>, by
+// the chain rule one token at a time: with G_t = dL/dS_t,
+//   dq_t[i] = sum_j S_t[i][j] do_t[j]                        (forward sweep)
+//   G_t = q_t do_t^T + diag(alpha_{t+1}) G_{t+1},  G_{T-1} = q_{T-1} do_{T-1}^T + dS_final
+//   dk_t[i] = sum_j G_t[i][j] v_t[j],  dv_t[j] = sum_i G_t[i][j] k_t[i]
+//   dalpha_t[i] = sum_j G_t[i][j] S_{t-1}[i][j],  dS_init = diag(alpha_0) G_0
+// The reverse sweep needs S_{t-1}: the forward sweep keeps S every kGlaCheck tokens and each
+// block is recomputed from its checkpoint.
+constexpr long long kGlaCheck = 64;
+
+struct GlaBackwardProblem {
+  const float* q;
+  const float* k;
+  const float* v;
+  const float* alpha;
+  const double* dout;
+  long long T;
+  int dk, dv;
+  const double* S_init;
+  const double* dS_final;
+  double* dq;
+  double* dk_out;
+  double* dv_out;
+  double* dalpha;
+  double* dS_init;
+};
+
+void gla_backward_pair(const GlaBackwardProblem& p, long long bh) {
+  const int dk = p.dk, dv = p.dv;
+  const long long T = p.T;
+  const size_t sd = static_cast<size_t>(dk) * dv;
+  const float* q = p.q + bh * T * dk;
+  const float* k = p.k + bh * T * dk;
+  const float* v = p.v + bh * T * dv;
+  const float* al = p.alpha + bh * T * dk;
+  const double* dout = p.dout + bh * T * dv;
+  auto step = [&](std::vector<double>& S, long long t) {  // S_{t-1} -> S_t
+    for (int i = 0; i < dk; ++i) {
+      const double gate = static_cast<double>(al[t * dk + i]), ki = static_cast<double>(k[t * dk + i]);
+      for (int j = 0; j < dv; ++j)
+        S[static_cast<size_t>(i) * dv + j] = gate * S[static_cast<size_t>(i) * dv + j] +
+                                             ki * static_cast<double>(v[t * dv + j]);
+    }
+  };
+  // Forward sweep: dq, and S before every block of kGlaCheck tokens.
+  const long long nblk = (T + kGlaCheck - 1) / kGlaCheck;
+  std::vector<double> S(sd, 0.0), checks(static_cast<size_t>(nblk) * sd);
+  if (p.S_init)
+    for (size_t e = 0; e < sd; ++e) S[e] = p.S_init[bh * sd + e];
+  for (long long t = 0; t < T; ++t) {
+    if (t % kGlaCheck == 0) std::copy(S.begin(), S.end(), checks.begin() + (t / kGlaCheck) * sd);
+    step(S, t);
+    for (int i = 0; i < dk; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < dv; ++j) acc += S[static_cast<size_t>(i) * dv + j] * dout[t * dv + j];
+      p.dq[(bh * T + t) * dk + i] = acc;
+    }
+  }
+  // Reverse sweep, block by block from the last.
+  std::vector<double> G(sd, 0.0), prev(static_cast<size_t>(kGlaCheck) * sd);
+  if (p.dS_final)
+    for (size_t e = 0; e < sd; ++e) G[e] = p.dS_final[bh * sd + e];
+  for (long long b = nblk - 1; b >= 0; --b) {
+    const long long t0 = b * kGlaCheck, t1 = std::min(T, t0 + kGlaCheck);
+    std::vector<double> Sb(checks.begin() + b * sd, checks.begin() + (b + 1) * sd);
+    for (long long t = t0; t < t1; ++t) {  // prev[t - t0] = S_{t-1}
+      std::copy(Sb.begin(), Sb.end(), prev.begin() + (t - t0) * sd);
+      step(Sb, t);
+    }
+    for (long long t = t1 - 1; t >= t0; --t) {
+      const double* Sp = &prev[(t - t0) * sd];
+      for (int i = 0; i < dk; ++i) {
+        const double qi = static_cast<double>(q[t * dk + i]);
+        for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] += qi * dout[t * dv + j];
+      }
+      for (int i = 0; i < dk; ++i) {
+        double gk = 0.0, ga = 0.0;
+        for (int j = 0; j < dv; ++j) {
+          gk += G[static_cast<size_t>(i) * dv + j] * static_cast<double>(v[t * dv + j]);
+          ga += G[static_cast<size_t>(i) * dv + j] * Sp[static_cast<size_t>(i) * dv + j];
+        }
+        p.dk_out[(bh * T + t) * dk + i] = gk;
+        p.dalpha[(bh * T + t) * dk + i] = ga;
+      }
+      for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i)
+          acc += G[static_cast<size_t>(i) * dv + j] * static_cast<double>(k[t * dk + i]);
+        p.dv_out[(bh * T + t) * dv + j] = acc;
+      }
+      for (int i = 0; i < dk; ++i) {  // G_{t-1} receives diag(alpha_t) G_t
+        const double gate = static_cast<double>(al[t * dk + i]);
+        for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= gate;
+      }
+    }
+  }
+  if (p.dS_init)
+    for (size_t e = 0; e < sd; ++e) p.dS_init[bh * sd + e] = G[e];
+}
+
 }  // namespace
 
 extern "C" {
+
+// Gradients of the gated loop (see gla_backward_pair).  dout [B, H, T, dv] double,
+// dS_final [B, H, dk, dv] double or NULL; writes dq, dk, dalpha [B, H, T, dk], dv
+// [B, H, T, dv] and dS_init [B, H, dk, dv] (may be NULL), all double.
+int la_oracle_gla_backward(const float* q, const float* k, const float* v, const float* alpha,
+                           const double* dout, int B, int H, long long T, int dk, int dv,
+                           const double* S_init, const double* dS_final, double* dq,
+                           double* dk_out, double* dv_out, double* dalpha, double* dS_init,
+                           int nthreads) {
+  if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return 1;
+  if (T > 0 && (!q || !k || !v || !alpha || !dout || !dq || !dk_out || !dv_out || !dalpha))
+    return 1;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH == 0) return 0;
+  GlaBackwardProblem p{q, k, v, alpha, dout, T, dk, dv, S_init, dS_final, dq, dk_out, dv_out,
+                       dalpha, dS_init};
+  long long workers = nthreads > 0 ? nthreads
+                                   : static_cast<long long>(std::thread::hardware_concurrency());
+  if (workers < 1) workers = 1;
+  if (workers > BH) workers = BH;
+  std::vector<std::thread> pool;
+  for (long long w = 0; w < workers; ++w)
+    pool.emplace_back([&p, w, workers, BH]() {
+      for (long long bh = w; bh < BH; bh += workers) gla_backward_pair(p, bh);
+    });
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
 
 // Gated linear attention forward (see gla_pair).  alpha [B, H, T, dk] float32 gates;
 // S_init [B, H, dk, dv] double or NULL; out [B, H, T, dv] and S_final double (each may be

@@ -56,6 +56,11 @@ class Oracle:
         b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int] + \
             [ctypes.c_void_p, ctypes.c_int, ctypes.c_double] + [ctypes.c_void_p] * 9 + [ctypes.c_int]
+        gb = self._lib.la_oracle_gla_backward
+        gb.restype = ctypes.c_int
+        gb.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
+                                              ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 7 + \
+            [ctypes.c_int]
         gl = self._lib.la_oracle_gla_forward
         gl.restype = ctypes.c_int
         gl.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int, ctypes.c_int, ctypes.c_longlong,
@@ -160,6 +165,29 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"la_oracle_gla_forward returned {rc}")
         return out, S
+
+
+    def gla_backward(self, q, k, v, alpha, dout, *, S_init=None, dS_final=None,
+                     nthreads: int = 0):
+        """Gradients of <dout, out> + <dS_final, S_final> through the gated loop.  Returns
+        (dq, dk, dv, dalpha, dS_init), float64."""
+        q, k, v, al = (np.ascontiguousarray(a, dtype=np.float32) for a in (q, k, v, alpha))
+        do = np.ascontiguousarray(dout, dtype=np.float64)
+        B, H, T, dk = q.shape
+        dv = v.shape[-1]
+        if k.shape != q.shape or al.shape != q.shape or v.shape[:3] != (B, H, T) or do.shape != v.shape:
+            raise ValueError("shape mismatch between q, k, v, alpha and dout")
+        f64 = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+        s0, dsf = f64(S_init), f64(dS_final)
+        dq = np.empty((B, H, T, dk)); dk_ = np.empty((B, H, T, dk)); dv_ = np.empty((B, H, T, dv))
+        da = np.empty((B, H, T, dk)); ds0 = np.empty((B, H, dk, dv))
+        ptr = lambda a: None if a is None else a.ctypes.data
+        rc = self._lib.la_oracle_gla_backward(ptr(q), ptr(k), ptr(v), ptr(al), ptr(do), B, H, T,
+                                              dk, dv, ptr(s0), ptr(dsf), ptr(dq), ptr(dk_), ptr(dv_),
+                                              ptr(da), ptr(ds0), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"la_oracle_gla_backward returned {rc}")
+        return dq, dk_, dv_, da, ds0
 
 
 _default: Oracle | None = None
