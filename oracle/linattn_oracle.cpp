@@ -393,8 +393,8 @@ void gla_backward_pair(const GlaBackwardProblem& p, long long bh) {
         p.dv_out[(bh * T + t) * dv + j] = acc;
       }
       for (int i = 0; i < dk; ++i) {  // G_{t-1} receives diag(alpha_t) G_t
-        const double gate = static_cast<double>(al[t * dk + i]);
-        for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= gate;
+        const double at = al[t * dk + i];
+        for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= at;
       }
     }
   }

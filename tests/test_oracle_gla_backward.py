@@ -125,7 +125,7 @@ MUTANTS = {
         "ga += G[static_cast<size_t>(i) * dv + j] * Sp[static_cast<size_t>(i) * dv + j];",
         "ga += G[static_cast<size_t>(i) * dv + j] * Sb[static_cast<size_t>(i) * dv + j];"),
     "reverse_sweep_without_the_gate": (
-        "for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= gate;",
+        "for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= at;",
         "for (int j = 0; j < dv; ++j) G[static_cast<size_t>(i) * dv + j] *= 1.0;"),
     "checkpoint_after_the_step": (
         "if (t % kGlaCheck == 0) std::copy(S.begin(), S.end(), checks.begin() + (t / kGlaCheck) * sd);\n    step(S, t);",
