@@ -266,19 +266,22 @@ def clocks_bad(c) -> bool:
 
 
 class OracleTimer:
-    """Times the oracle on the first T' tokens of every (b, h) of the workload, T' sized
-    for about `target_s` seconds of host work."""
+    """Times the oracle on the first T' tokens of every (b, h) of the workload `w`, T' sized
+    for about `target_s` seconds of host work.  q, k, v may hold fewer tokens than the
+    workload (a sample drawn with its recipe); T' never exceeds what they hold."""
 
     def __init__(self, w, q, k, v, target_s: float):
         from oracle.oracle import default_oracle
         self.orc = default_oracle()
         self.w = w
+        self.avail = int(q.shape[2])
         self.threads = max(1, min(len(os.sched_getaffinity(0)), w.B * w.H))
-        probe_t = min(w.T, 512)
+        probe_t = min(self.avail, 512)
         self.inputs = (q, k, v)
         dt = self._run(probe_t)
-        self.tp = min(w.T, max(probe_t, int(probe_t * target_s / max(dt, 1e-6))))
+        self.tp = min(self.avail, max(probe_t, int(probe_t * target_s / max(dt, 1e-6))))
         self.host = [t[:, :, :self.tp].to("cpu", torch.float32).numpy() for t in (q, k, v)]
+        self.last_s = dt
 
     def _run(self, tp, host=None):
         w = self.w
@@ -294,32 +297,50 @@ class OracleTimer:
         self.last_s = dt
         return self.w.B * self.w.H * self.tp / dt
 
+    @property
+    def sample_tokens_heads(self) -> int:
+        return self.w.B * self.w.H * self.tp
+
     def sample(self):
         return (f"first {self.tp} of {self.w.T} tokens of all {self.w.B * self.w.H} (b,h) "
-                f"pairs, full fp64 token loop, {self.last_s:.1f} s per run on "
+                f"pairs, full fp64 token loop, {self.last_s:.2f} s per run on "
                 f"{self.threads} threads")
 
 
 def reference_arm(args, w, info):
+    """The oracle as the reference arm: every step is one oracle run over a bounded sample
+    of the workload (its first T' tokens of every (b, h)), sized so that warm-up plus timed
+    steps take about --reference-total-s seconds.  `value` is the sample's tokens*heads
+    over its measured time (the token loop's cost is the same for every token), and
+    `ms_per_step` is the measured time of one sample step; the time a whole-workload step
+    would take at that rate is reported beside it, labelled as extrapolated."""
     if not info.is_root:
         return
+    n_runs = args.warmup + args.steps
+    per_step_s = max(0.05, min(args.reference_step_s, args.reference_total_s / n_runs))
     # The oracle's cost per token does not depend on the values; draw the sample's inputs
-    # on the CPU with the workload's recipe.
+    # on the CPU with the workload's recipe, never more tokens than a step can use.
     probe = w.with_(T=min(w.T, 1 << 15))
     q, k, v = make_inputs(probe, seed=0, device="cpu")
-    timer = OracleTimer(w.with_(T=probe.T), q, k, v, target_s=args.reference_step_s)
-    per_step = []
-    for i in range(args.warmup + args.steps):
+    timer = OracleTimer(w, q, k, v, target_s=per_step_s)
+    per_step, secs = [], []
+    for i in range(n_runs):
         r = timer.rate()
         if i >= args.warmup:
             per_step.append(r)
+            secs.append(timer.last_s)
     value = statistics.median(per_step)
+    step_s = statistics.median(secs)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * w.B * w.H * w.T / value,
+        "ms_per_step": 1000.0 * step_s,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args),
+        "sample": {"tokens_heads_per_step": timer.sample_tokens_heads, "tokens": timer.tp,
+                   "of_tokens": w.T, "seconds_per_step": step_s,
+                   "extrapolated": timer.tp < w.T,
+                   "extrapolated_full_workload_ms": 1000.0 * w.tokens_heads / value},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": timer.threads, "kind": "oracle",
                          "sample": timer.sample()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -805,7 +826,10 @@ def main():
     ap.add_argument("--kernel-timing-steps", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-baseline-s", type=float, default=15.0)
-    ap.add_argument("--reference-step-s", type=float, default=10.0)
+    ap.add_argument("--reference-step-s", type=float, default=10.0,
+                    help="reference arm: upper bound on the seconds of one sample step")
+    ap.add_argument("--reference-total-s", type=float, default=120.0,
+                    help="reference arm: warm-up plus timed steps take about this long")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
