@@ -48,10 +48,11 @@ FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
-K2_NAMES = {"logdepth": ["k2_reduce", "k2_scan_totals", "k2_downsweep"],
+K2_NAMES = {"logdepth": ["k2_reduce", "k2_block_scan", "k2_downsweep"],
             "sequential": ["k2_sequential"]}
+SCAN_BLOCK_ELEMS = 2048  # the log-depth scan's one-level limit (lin_attn_scan_plan)
 KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce": "scan.cu",
-                  "k2_scan_totals": "scan.cu", "k2_downsweep": "scan.cu",
+                  "k2_block_scan": "scan.cu", "k2_downsweep": "scan.cu",
                   "k2_sequential": "scan.cu", "k1_seg": "seg_kernels.cu",
                   "k3_seg": "seg_kernels.cu"}
 
@@ -68,7 +69,7 @@ def effective_algorithm(w, requested: str) -> str:
 def kernel_names(w, algo: str, scan: str, lseg: int = 0) -> list[str]:
     k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
     n, _, _ = layout(w, algo, lseg)
-    k2 = ["k2_scan_totals"] if scan == "logdepth" and n <= 32 else K2_NAMES[scan]
+    k2 = ["k2_block_scan"] if scan == "logdepth" and n <= SCAN_BLOCK_ELEMS else K2_NAMES[scan]
     return [k1, *k2, k3]
 
 
@@ -92,7 +93,7 @@ def layout(w, algo: str = "chunked", lseg: int = 0):
     n = NC
     if algo == "segmented":
         n = -(-NC // segment_length(w, lseg))
-    Ls = max(1, -(-n // 32))
+    Ls = max(16, -(-n // SCAN_BLOCK_ELEMS)) if n > SCAN_BLOCK_ELEMS else n
     G = -(-n // Ls)
     R = w.dk * w.dv + (w.dk if w.normalize else 0)
     return n, G, R
@@ -107,9 +108,12 @@ def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked", lseg: int =
     if name.startswith("k1"):
         return BH * w.T * (w.dk + w.dv) * e_in + rec
     if name == "k2_reduce":
-        return rec
-    if name == "k2_scan_totals":
-        return 2 * BH * G * R * 4 + BH * R * 4
+        return rec + BH * G * R * 4
+    if name == "k2_block_scan":
+        # One level: the records read once (the second read of a CTA's slab comes from L2)
+        # and written once; two levels: the same over the segment folds.  Plus the final
+        # states.
+        return 2 * (rec if n <= SCAN_BLOCK_ELEMS else BH * G * R * 4) + BH * R * 4
     if name == "k2_downsweep":
         return 2 * rec + BH * G * R * 4
     if name == "k2_sequential":
@@ -361,8 +365,11 @@ def sweep_scan(args, dev):
                                                             w.normalize),
                          dtype=torch.uint8, device=dev)
         out = torch.empty((w.B, w.H, w.T, w.dv), dtype=torch.float32, device=dev)
-        row = {"sweep": "k2_scan", "workload": w.name, "chunks": -(-w.T // w.C),
-               "columns": w.B * w.H * (w.dk * w.dv + (w.dk if w.normalize else 0))}
+        nc = -(-w.T // w.C)
+        row = {"sweep": "k2_scan", "workload": w.name, "chunks": nc,
+               "columns": w.B * w.H * (w.dk * w.dv + (w.dk if w.normalize else 0)),
+               "depth_logdepth": B.lin_attn_scan_plan(nc)["depth"],
+               "depth_sequential": nc, "ceil_log2_chunks": math.ceil(math.log2(nc))}
         for scan in ("logdepth", "sequential"):
             kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=w.gammas(),
                       normalize=w.normalize, scan=scan, kernel_path="tensor_core",
@@ -797,6 +804,17 @@ def gla_bench(args, info, dev):
         print(json.dumps(line), flush=True)
 
 
+def scan_depth(w, args) -> dict:
+    """The implemented K2 depth (dependent combine steps per column) of this run."""
+    algo = effective_algorithm(w, args.algorithm)
+    n, _, _ = layout(w, algo, getattr(args, "segment_chunks", 0))
+    try:
+        d = B.lin_attn_scan_plan(n, args.scan)["depth"]
+    except Exception:  # library not built (CPU-only tooling)
+        d = None
+    return {"elements": n, "depth": d, "ceil_log2_elements": math.ceil(math.log2(max(n, 2)))}
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
@@ -806,6 +824,7 @@ def config_of(w, args):
             **({"segment_chunks": segment_length(w, getattr(args, "segment_chunks", 0))}
                if effective_algorithm(w, args.algorithm) == "segmented" else {}),
             "kernel_path": "tensor_core", "l2": "inputs larger than L2, no flush",
+            "scan_depth": scan_depth(w, args),
             "parallelism": "replicas (one independent problem per GPU)"}
 
 

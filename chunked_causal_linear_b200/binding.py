@@ -33,6 +33,7 @@ EXPORTED_SYMBOLS = (
     "lin_attn_status_string", "lin_attn_version", "lin_attn_combine_states",
     "lin_attn_backward", "lin_attn_backward_workspace_bytes", "lin_attn_backward_timed",
     "lin_attn_gla_prefill", "lin_attn_gla_workspace_bytes", "lin_attn_gla_prefill_timed",
+    "lin_attn_scan_plan",
 )
 
 
@@ -118,6 +119,8 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_device_error": (i, [ctypes.POINTER(ctypes.c_int)]),
         "lin_attn_status_string": (ctypes.c_char_p, [i]),
         "lin_attn_version": (i, []),
+        "lin_attn_scan_plan": (i, [ll, i, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i),
+                                   ctypes.POINTER(i), ctypes.POINTER(ll)]),
         "lin_attn_combine_states": (i, [vp, vp, i, i, ctypes.POINTER(ll), i, i, i, i, vp, vp,
                                         vp, vp]),
         "lin_attn_backward": (i, [ctypes.POINTER(BackwardArgs)]),
@@ -512,6 +515,19 @@ def lin_attn_device_error() -> int:
 
 def lin_attn_status_string(status: int) -> str:
     return load_library().lin_attn_status_string(int(status)).decode()
+
+
+def lin_attn_scan_plan(n: int, scan: str = "logdepth") -> dict:
+    """K2's shape for a scan over n elements: segment length and count, blocked-scan groups
+    and elements per group, and the dependent-step depth."""
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    depth = ctypes.c_longlong(0)
+    _check("lin_attn_scan_plan",
+           load_library().lin_attn_scan_plan(int(n), SCAN_MODES[scan],
+                                             *(ctypes.byref(x) for x in vals),
+                                             ctypes.byref(depth)))
+    return {"segment_len": vals[0].value, "segments": vals[1].value, "groups": vals[2].value,
+            "per_group": vals[3].value, "depth": depth.value}
 
 
 def lin_attn_version() -> int:

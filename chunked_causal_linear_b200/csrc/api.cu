@@ -23,8 +23,7 @@ __device__ int g_error_word = 0;
 
 namespace {
 
-constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
-constexpr int kMaxSegments = 32;
+constexpr int kVersion = 1 * 10000 + 1 * 100 + 0;
 
 struct Layout {
   long long BH = 0;
@@ -42,13 +41,19 @@ Layout make_layout(int B, int H, long long T, int dk, int dv, int C, int normali
   l.NC = static_cast<int>(nc);
   l.L_last = static_cast<int>(T - (nc - 1) * C);
   l.R = dk * dv + (normalize ? dk : 0);
-  l.Ls = static_cast<int>((nc + kMaxSegments - 1) / kMaxSegments);
-  if (l.Ls < 1) l.Ls = 1;
-  l.G = static_cast<int>((nc + l.Ls - 1) / l.Ls);
+  const ScanPlan sp = scan_plan(nc);
+  l.Ls = sp.Ls;
+  l.G = sp.G;
   l.rec_off = 0;
   l.rec_bytes = align256(static_cast<size_t>(l.BH) * nc * l.R * sizeof(float));
   l.tot_off = l.rec_off + l.rec_bytes;
-  l.tot_bytes = align256(static_cast<size_t>(l.BH) * l.G * l.R * sizeof(float));
+  // Segment folds of the two-level scan.  Sized for min(2048, ceil(NC / 16)) segments, a
+  // bound on the segment count of any scan of at most NC elements, so that the segmented
+  // algorithm's scan over its (fewer) segment records fits in the same space.
+  const long long gmax = nc > kScanBlockElems
+                             ? std::min<long long>(kScanBlockElems, (nc + kScanMinSegment - 1) / kScanMinSegment)
+                             : 0;
+  l.tot_bytes = align256(static_cast<size_t>(l.BH) * gmax * l.R * sizeof(float));
   l.total = l.tot_off + l.tot_bytes;
   return l;
 }
@@ -314,8 +319,9 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     ps.L_last = static_cast<int>(a.T - static_cast<long long>(NS - 1) * Lseg * a.C);
     ps.rec = sp.srec;
     ps.tot = reinterpret_cast<float*>(ws + srec_bytes);
-    ps.Ls = (NS + kMaxSegments - 1) / kMaxSegments;
-    ps.G = (NS + ps.Ls - 1) / ps.Ls;
+    const ScanPlan spl = scan_plan(NS);
+    ps.Ls = spl.Ls;
+    ps.G = spl.G;
     TcMaps m;
     const uint64_t T = static_cast<uint64_t>(a.T);
     bool ok = make_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, a.dk, T, BH, a.dk * 2ull,
@@ -728,6 +734,26 @@ const char* lin_attn_status_string(int status) {
     case LA_ERR_INTERNAL: return "LA_ERR_INTERNAL";
     default: return "LA_ERR_UNKNOWN";
   }
+}
+
+int lin_attn_scan_plan(long long n, int scan_mode, int* segment_len, int* segments,
+                       int* groups, int* per_group, long long* depth) {
+  if (n < 1 || (scan_mode != LA_SCAN_LOGDEPTH && scan_mode != LA_SCAN_SEQUENTIAL))
+    return LA_ERR_INVALID_ARGUMENT;
+  la::ScanPlan pl = la::scan_plan(n);
+  if (scan_mode == LA_SCAN_SEQUENTIAL) {
+    pl.Ls = static_cast<int>(n > (1LL << 31) - 1 ? (1LL << 31) - 1 : n);
+    pl.G = 1;
+    pl.NG = 1;
+    pl.E = pl.Ls;
+    pl.depth = n;
+  }
+  if (segment_len) *segment_len = pl.Ls;
+  if (segments) *segments = pl.G;
+  if (groups) *groups = pl.NG;
+  if (per_group) *per_group = pl.E;
+  if (depth) *depth = pl.depth;
+  return LA_OK;
 }
 
 int lin_attn_version(void) { return la::kVersion; }

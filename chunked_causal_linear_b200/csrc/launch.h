@@ -57,7 +57,22 @@ cudaError_t launch_k3_fma(const PrefillParams& p, const GammaTable& gt, const vo
                           const void* k, const void* v, void* out, int dtype, Flags f,
                           cudaStream_t s);
 
-// K2: scan of the chunk records (mode 0 log-depth over segments, 1 sequential carry).
+// The log-depth K2's shape for n scan elements: up to kScanBlockElems elements one blocked
+// scan (NG groups of E elements, Hillis-Steele over the groups); beyond that G segments of
+// Ls >= kScanMinSegment elements, their folds scanned by the blocked scan.  `depth` is the
+// longest chain of dependent combine steps: 2E + log2 NG (+ 2 Ls with segments).
+constexpr long long kScanBlockElems = 2048;
+constexpr long long kScanMinSegment = 16;
+struct ScanPlan {
+  int Ls = 1;  // elements per segment (n itself with one level)
+  int G = 1;   // segments (1 with one level)
+  int NG = 1;  // groups of the blocked scan (a power of two, <= 128)
+  int E = 0;   // elements per group
+  long long depth = 0;
+};
+ScanPlan scan_plan(long long n);
+
+// K2: scan of the chunk records (mode 0 log-depth, 1 sequential carry).
 cudaError_t launch_k2(const PrefillParams& p, const GammaTable& gt, int mode, Flags f,
                       cudaStream_t s, Recorder* rec = nullptr);
 

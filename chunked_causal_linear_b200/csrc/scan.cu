@@ -10,18 +10,26 @@
 // after K2, record c holds P_c, the state before chunk c, and P_0 = 0.  The inclusive
 // total (the state after the last token) goes to S_final / Z_final.
 //
-// Log-depth mode ("Implementation notes": a Blelloch or Hillis-Steele scan) splits the
-// chunk axis into G <= 32 segments of Ls chunks (when Ls = 1, i.e. at most 32 elements,
-// k2_scan_totals alone scans the records in place):
-//   k2_reduce       one pass over the records: each segment's aggregate (parallel over
-//                   segments and columns);
-//   k2_scan_totals  Hillis-Steele scan of the G segment aggregates, ceil(log2 G) rounds
-//                   in shared memory, giving each segment's exclusive prefix;
-//   k2_downsweep    second pass: each segment re-scans its chunks from its prefix and
-//                   writes P_c in place.
-// Sequential mode (comparison only) carries the state through every chunk in order.
-// Both modes read and write float4 columns; a warp touches 512 contiguous bytes of a
-// record per step.
+// Log-depth mode ("Implementation notes": a Blelloch or Hillis-Steele scan; "Verification":
+// ceil(log2 N_C) rounds) is a work-efficient blocked scan (Brent's arrangement of
+// Hillis-Steele).  One CTA takes a slab of 8 float4 columns (128 contiguous bytes of every
+// record) and up to 2048 elements of the chunk axis, split over NG <= 128 groups of E <= 16
+// consecutive elements, one thread per (group, column):
+//   k2_block_scan   pass 1: each thread folds its E elements (E dependent steps);
+//                   Hillis-Steele over the NG group folds in shared memory (log2 NG
+//                   rounds); pass 2: each thread re-reads its elements (from L2: a CTA's
+//                   slab is at most 256 KB) and writes their exclusive prefixes in place
+//                   (E steps).  Depth 2E + log2 NG, e.g. 16 + 7 + 16 at N_C = 2048; the
+//                   records cross HBM once each way, as in the sequential carry.
+// Beyond 2048 elements one level more: segments of Ls >= 16 chunks, G = ceil(N_C / Ls)
+// <= 2048 of them:
+//   k2_reduce       each segment's fold (Ls steps, parallel over segments and columns);
+//   k2_block_scan   the scan above over the G segment folds, giving each segment's
+//                   exclusive prefix;
+//   k2_downsweep    each segment re-scans its chunks from its prefix, in place (Ls steps).
+// Depth 2 Ls + 2E + log2 NG (55 at N_C = 16384).
+// Sequential mode (comparison only) carries the state through every chunk in order
+// (depth N_C).  Every mode reads and writes float4 columns.
 // A caller-given state before token 0 (S_init, Z_init) is the scan's first element: the
 // exclusive prefix of chunk 0 is that state, and every later prefix carries it decayed by
 // gamma^(tokens before the chunk) -- the same monoid with one more element in front.
@@ -35,6 +43,8 @@ namespace {
 
 constexpr int kScanThreads = 128;
 constexpr int kUnroll = 8;
+constexpr int kSlab = 8;         // float4 columns per block-scan CTA (128 contiguous bytes)
+constexpr int kMaxGroups = 128;  // groups per block-scan CTA (1024 threads)
 
 __device__ __forceinline__ float4 axpy4(float a, float4 x, float4 y) {
   return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
@@ -80,20 +90,20 @@ __device__ __forceinline__ float4 read_init(const PrefillParams& p, int bh, int 
 // receives the carry before chunk c, then carry <- a_c carry + x_c.  The next batch of
 // loads is issued before the current batch is stored, so a thread always has loads in
 // flight (in-place read-then-write streams reach copy bandwidth only this way).
-template <bool DECAY>
+template <bool DECAY, int U = kUnroll>
 __device__ __forceinline__ float4 carry_in_place(float4* base, long long stride, int cbeg,
                                                  int cend, int last, float gC, float aL,
                                                  float4 carry) {
-  float4 x[kUnroll], y[kUnroll];
+  float4 x[U], y[U];
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u)
+  for (int u = 0; u < U; ++u)
     if (cbeg + u < cend) x[u] = base[static_cast<long long>(cbeg + u) * stride];
-  for (int c0 = cbeg; c0 < cend; c0 += kUnroll) {
+  for (int c0 = cbeg; c0 < cend; c0 += U) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-      if (c0 + kUnroll + u < cend) y[u] = base[static_cast<long long>(c0 + kUnroll + u) * stride];
+    for (int u = 0; u < U; ++u)
+      if (c0 + U + u < cend) y[u] = base[static_cast<long long>(c0 + U + u) * stride];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       if (c0 + u < cend) {
         base[static_cast<long long>(c0 + u) * stride] = carry;
         const float a = DECAY ? (c0 + u == last ? aL : gC) : 1.f;
@@ -101,7 +111,7 @@ __device__ __forceinline__ float4 carry_in_place(float4* base, long long stride,
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) x[u] = y[u];
+    for (int u = 0; u < U; ++u) x[u] = y[u];
   }
   return carry;
 }
@@ -153,55 +163,73 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
   reinterpret_cast<float4*>(p.tot + (static_cast<long long>(bh) * p.G + s) * p.R)[col4] = agg;
 }
 
-// Hillis-Steele scan of the segment aggregates.  Block (32 float4 columns) x (32
-// segments); ceil(log2 G) rounds in shared memory.
+// Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of kSlab float4
+// columns); NG groups of E consecutive elements (NG a power of two, NG * E >= N).
 template <bool DECAY>
-__global__ void __launch_bounds__(1024) k2_scan_totals(PrefillParams p, GammaTable gt) {
-  __shared__ float4 sX[32][33];
-  __shared__ float sA[32];
+__global__ void __launch_bounds__(kSlab * kMaxGroups, 1)
+k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
+  __shared__ float4 sX[kMaxGroups * kSlab];
+  __shared__ float sA[kMaxGroups];
   const int R4 = p.R / 4;
-  const int ncb = (R4 + 31) / 32;
-  const int bh = blockIdx.x / ncb;
-  const int col4 = (blockIdx.x % ncb) * 32 + threadIdx.x;
-  const int s = threadIdx.y;
-  const bool live = s < p.G && col4 < R4;
+  const int nslab = (R4 + kSlab - 1) / kSlab;
+  const int bh = blockIdx.x / nslab;
+  const int c8 = threadIdx.x % kSlab;
+  const int col4 = (blockIdx.x % nslab) * kSlab + c8;
+  const int gi = threadIdx.x / kSlab;
+  const bool live = col4 < R4;
   const float g = DECAY ? gt.g[bh % p.H] : 1.f;
+  const float gC = DECAY ? powf(g, static_cast<float>(p.C)) : 1.f;
+  const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
+  const int e0 = min(p.NC, gi * E);
+  const int e1 = min(p.NC, e0 + E);
+  float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) + col4;
 
-  // Segment decay: product of its chunks' decays.
-  float a = 1.f;
-  if (DECAY && s < p.G) {
-    const int cbeg = s * p.Ls;
-    const int cend = min(p.NC, cbeg + p.Ls);
-    const float tokens = static_cast<float>(cend == p.NC
-                                                ? static_cast<long long>(cend - cbeg - 1) * p.C + p.L_last
-                                                : static_cast<long long>(cend - cbeg) * p.C);
-    a = powf(g, tokens);
+  // Pass 1: this group's fold, agg = sum_e (decay after e within the group) x_e.
+  float4 agg = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (live) {
+    for (int c0 = e0; c0 < e1; c0 += kUnroll) {
+      float4 x[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (c0 + u < e1) x[u] = base[static_cast<long long>(c0 + u) * R4];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (c0 + u < e1) agg = axpy4(DECAY ? (c0 + u == p.NC - 1 ? aL : gC) : 1.f, agg, x[u]);
+    }
   }
-  float4* tot = reinterpret_cast<float4*>(p.tot + static_cast<long long>(bh) * p.G * p.R);
-  float4 x = live ? tot[static_cast<long long>(s) * R4 + col4] : make_float4(0.f, 0.f, 0.f, 0.f);
-
-  for (int d = 1; d < p.G; d <<= 1) {
-    sX[s][threadIdx.x] = x;
-    if (threadIdx.x == 0) sA[s] = a;
+  // The group's decay: gamma^(tokens of its elements).
+  float A = 1.f;
+  if (DECAY && e1 > e0) {
+    const long long tokens = e1 == p.NC
+                                 ? static_cast<long long>(e1 - e0 - 1) * p.C + p.L_last
+                                 : static_cast<long long>(e1 - e0) * p.C;
+    A = powf(g, static_cast<float>(tokens));
+  }
+  // Hillis-Steele over the groups: after round r, group gi holds the fold of groups
+  // gi - 2^(r+1) + 1 .. gi, and A their decay.
+  for (int d = 1; d < NG; d <<= 1) {
+    sX[gi * kSlab + c8] = agg;
+    if (c8 == 0) sA[gi] = A;
     __syncthreads();
-    if (s >= d) {
-      x = axpy4(a, sX[s - d][threadIdx.x], x);
-      a = sA[s - d] * a;
+    if (gi >= d) {
+      agg = axpy4(A, sX[(gi - d) * kSlab + c8], agg);
+      A *= sA[gi - d];
     }
     __syncthreads();
   }
-  // `a` is now the product of the decays of segments 0 .. s: the initial state reaches
-  // the end of segment s scaled by it.
-  const float4 init = (p.S_init || p.Z_init) && live ? read_init(p, bh, col4 * 4)
-                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-  x = axpy4(a, init, x);
-  // Inclusive -> exclusive.
-  sX[s][threadIdx.x] = x;
+  // Inclusive -> exclusive over groups; the initial state enters with the decay of every
+  // group before this one.
+  sX[gi * kSlab + c8] = agg;
+  if (c8 == 0) sA[gi] = A;
   __syncthreads();
-  if (live) {
-    tot[static_cast<long long>(s) * R4 + col4] = s > 0 ? sX[s - 1][threadIdx.x] : init;
-    if (s == p.G - 1) write_final(p, bh, col4 * 4, x);
-  }
+  if (!live || e0 >= e1) return;
+  const float4 init = p.has_init ? read_init(p, bh, col4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 carry = init;
+  if (gi > 0) carry = axpy4(sA[gi - 1], init, sX[(gi - 1) * kSlab + c8]);
+  // Pass 2: exclusive prefixes of this group's elements, in place (re-read from L2, so
+  // four loads in flight suffice and keep the thread within 64 registers).
+  carry = carry_in_place<DECAY, 4>(base, R4, e0, e1, p.NC - 1, gC, aL, carry);
+  if (e1 == p.NC) write_final(p, bh, col4 * 4, carry);
 }
 
 // Second pass: each segment writes its chunks' exclusive prefixes in place.
@@ -226,6 +254,16 @@ __global__ void __launch_bounds__(kScanThreads) k2_downsweep(PrefillParams p, Ga
 }
 
 template <bool DECAY>
+cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_t s) {
+  const ScanPlan bp = scan_plan(p.NC);  // p.NC <= kScanBlockElems: a single block level
+  const int R4 = p.R / 4;
+  const long long nslab = (R4 + kSlab - 1) / kSlab;
+  k2_block_scan<DECAY><<<static_cast<unsigned>(nslab * p.BH), kSlab * bp.NG, 0, s>>>(
+      p, gt, bp.NG, bp.E);
+  return cudaGetLastError();
+}
+
+template <bool DECAY>
 cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStream_t s,
                Recorder* rec) {
   const int R4 = p.R / 4;
@@ -235,23 +273,28 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
     k2_sequential<DECAY><<<static_cast<unsigned>(nblk * p.BH), kScanThreads, 0, s>>>(p, gt);
     return cudaGetLastError();
   }
-  const long long grid = nblk * p.G * p.BH;
-  const long long ncb = (R4 + 31) / 32;
-  if (p.Ls == 1) {
-    // Every segment is one element: the Hillis-Steele scan alone, in place on the records.
-    PrefillParams q = p;
-    q.tot = p.rec;
-    if (rec) rec->mark(s, "k2_scan_totals");
-    k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(q, gt);
-    return cudaGetLastError();
+  if (p.NC <= kScanBlockElems) {
+    // One block level: the blocked scan alone, in place on the records.
+    if (rec) rec->mark(s, "k2_block_scan");
+    return block_scan<DECAY>(p, gt, s);
   }
+  // Two levels: segment folds, the blocked scan over them, the per-segment sweep.
+  const ScanPlan plan = scan_plan(p.NC);
+  if (plan.Ls != p.Ls || plan.G != p.G) return cudaErrorInvalidValue;
+  const long long grid = nblk * p.G * p.BH;
   if (rec) rec->mark(s, "k2_reduce");
   k2_reduce<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (rec) rec->mark(s, "k2_scan_totals");
-  k2_scan_totals<DECAY><<<static_cast<unsigned>(ncb * p.BH), dim3(32, 32), 0, s>>>(p, gt);
-  e = cudaGetLastError();
+  // The scan over segments: one element per segment, each of Ls chunks (the last one
+  // holding what is left).
+  PrefillParams q = p;
+  q.rec = p.tot;
+  q.NC = p.G;
+  q.C = p.C * p.Ls;
+  q.L_last = static_cast<int>(p.T - static_cast<long long>(p.G - 1) * p.Ls * p.C);
+  if (rec) rec->mark(s, "k2_block_scan");
+  e = block_scan<DECAY>(q, gt, s);
   if (e != cudaSuccess) return e;
   if (rec) rec->mark(s, "k2_downsweep");
   k2_downsweep<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);
@@ -259,6 +302,31 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
 }
 
 }  // namespace
+
+ScanPlan scan_plan(long long n) {
+  ScanPlan pl;
+  if (n <= 0) return pl;
+  long long m = n;  // elements of the block level
+  if (n > kScanBlockElems) {
+    long long ls = (n + kScanBlockElems - 1) / kScanBlockElems;
+    if (ls < kScanMinSegment) ls = kScanMinSegment;
+    pl.Ls = static_cast<int>(ls);
+    pl.G = static_cast<int>((n + ls - 1) / ls);
+    m = pl.G;
+  } else {
+    pl.Ls = static_cast<int>(n);
+    pl.G = 1;
+  }
+  int ng = 1, lg = 0;
+  while (ng < m && ng < kMaxGroups) {
+    ng <<= 1;
+    ++lg;
+  }
+  pl.NG = ng;
+  pl.E = static_cast<int>((m + ng - 1) / ng);
+  pl.depth = 2LL * pl.E + lg + (n > kScanBlockElems ? 2LL * pl.Ls : 0);
+  return pl;
+}
 
 cudaError_t launch_k2(const PrefillParams& p, const GammaTable& gt, int mode, Flags f,
                       cudaStream_t s, Recorder* rec) {

@@ -25,7 +25,8 @@
  *       ("Formulas"; decay placement from "C. Chunkwise Recurrent Representation").
  *   K2  exclusive associative scan of the summaries across chunks
  *       ((a1,S1,Z1) + (a2,S2,Z2) = (a1 a2, a2 S1 + S2, a2 Z1 + Z2), a = gamma^L), either
- *       log-depth over segments of chunks or a sequential carry (comparison mode).
+ *       log-depth (a blocked Hillis-Steele scan, see lin_attn_scan_plan) or a sequential
+ *       carry (comparison mode).
  *   K3  per chunk: the intra-chunk causal part (psi(Q) psi(K)^T masked with gamma^(i-j))
  *       plus Theta_i psi(q_i) P_c with the chunk's exclusive prefix P_c, Theta_i =
  *       gamma^(i+1), then the normalisation.
@@ -77,7 +78,7 @@ typedef enum {
 typedef enum { LA_FM_IDENTITY = 0, LA_FM_ELU1 = 1 } la_feature_map;
 
 typedef enum {
-  LA_SCAN_LOGDEPTH = 0,   /* K2 over segments of chunks: reduce, log-depth scan, sweep */
+  LA_SCAN_LOGDEPTH = 0,   /* K2 as a blocked log-depth scan (lin_attn_scan_plan) */
   LA_SCAN_SEQUENTIAL = 1  /* K2 as one sequential carry over chunks (comparison only) */
 } la_scan_mode;
 
@@ -203,8 +204,8 @@ int lin_attn_prefill_ex(const la_prefill_args* args);
  * before every kernel launch and after the last one; synchronises the stream and writes
  * each kernel's device duration (milliseconds, launch order) to kernel_ms[0 ..].
  * *n_kernels receives the number of kernels the prefill launched: K1, the scan's kernels
- * (3 for the log-depth scan over more than 32 elements, 1 for at most 32 elements or for
- * the sequential carry), K3.  For profiling;
+ * (3 for the log-depth scan over more than 2048 elements, 1 for at most 2048 elements or
+ * for the sequential carry), K3.  For profiling;
  * the results are identical to lin_attn_prefill_ex.
  */
 int lin_attn_prefill_timed(const la_prefill_args* args, float* kernel_ms, int max_kernels,
@@ -457,6 +458,23 @@ int lin_attn_device_error(int* code);
 
 /* A static, human-readable name for a la_status value. */
 const char* lin_attn_status_string(int status);
+
+/*
+ * lin_attn_scan_plan -- the shape of K2 for a scan over n elements (chunks, or segments of
+ * the segmented algorithm), without touching a device.  "Log-Depth Chunked Linear-Attention
+ * Scan" (Implementation notes, Verification) asks for a Blelloch or Hillis-Steele scan in
+ * ceil(log2 n) rounds.  The log-depth mode (scan_mode LA_SCAN_LOGDEPTH) arranges it the
+ * work-efficient way: n <= 2048 elements are cut into *groups (a power of two, at most 128)
+ * of *per_group consecutive elements; each thread folds its group, a Hillis-Steele scan
+ * combines the group folds in log2(*groups) rounds, and each thread re-scans its group
+ * from the result.  Beyond 2048 elements, *segments segments of *segment_len (>= 16)
+ * elements are folded first and that scan runs over the segment folds.  *depth receives
+ * the longest chain of dependent combine steps: 2 per_group + log2 groups (+ 2 segment_len
+ * with segments); for scan_mode LA_SCAN_SEQUENTIAL it is n.  Any output pointer may be
+ * NULL.  Returns LA_ERR_INVALID_ARGUMENT for n < 1 or an unknown mode.
+ */
+int lin_attn_scan_plan(long long n, int scan_mode, int* segment_len, int* segments,
+                       int* groups, int* per_group, long long* depth);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int lin_attn_version(void);

@@ -8,6 +8,7 @@ import math
 import re
 from pathlib import Path
 
+import numpy as np
 import pytest
 
 ROOT = Path(__file__).resolve().parent.parent
@@ -55,7 +56,7 @@ def test_status_strings_and_version(lib):
     for code, name in b.STATUS_NAMES.items():
         assert b.lin_attn_status_string(code) == name
     assert b.lin_attn_status_string(99) == "LA_ERR_UNKNOWN"
-    assert b.lin_attn_version() == 10000
+    assert b.lin_attn_version() == 10100
 
 
 def expected_workspace(B, H, T, dk, dv, C, normalize):
@@ -63,10 +64,9 @@ def expected_workspace(B, H, T, dk, dv, C, normalize):
         return 0
     nc = -(-T // C)
     R = dk * dv + (dk if normalize else 0)
-    ls = max(1, -(-nc // 32))
-    G = -(-nc // ls)
+    gmax = min(2048, -(-nc // 16)) if nc > 2048 else 0
     a256 = lambda x: (x + 255) // 256 * 256
-    return a256(B * H * nc * R * 4) + a256(B * H * G * R * 4)
+    return a256(B * H * nc * R * 4) + a256(B * H * gmax * R * 4)
 
 
 @pytest.mark.parametrize("shape", [(1, 2, 256, 32, 32, 32, 1), (4, 16, 4096, 64, 64, 64, 1),
@@ -79,10 +79,107 @@ def test_workspace_bytes(lib, shape):
     assert lin_attn_prefill_workspace_bytes(*shape) == expected_workspace(*shape)
 
 
-def test_scan_segments_are_at_most_32():
-    for nc in (1, 2, 31, 32, 33, 64, 250, 2048, 16384, 100000):
-        ls = max(1, math.ceil(nc / 32))
-        assert math.ceil(nc / ls) <= 32
+SCAN_SIZES = (1, 2, 3, 7, 31, 32, 33, 64, 127, 128, 129, 250, 1000, 2047, 2048, 2049, 4096,
+              16384, 32768, 32769, 100000, 1 << 20)
+
+
+@pytest.mark.parametrize("n", SCAN_SIZES)
+def test_scan_plan_shape_and_depth(lib, n):
+    from chunked_causal_linear_b200 import binding as B
+    p = B.lin_attn_scan_plan(n)
+    ng, e, ls, g = p["groups"], p["per_group"], p["segment_len"], p["segments"]
+    assert ng & (ng - 1) == 0 and 1 <= ng <= 128
+    if n <= 2048:
+        assert (ls, g) == (n, 1)
+        m = n
+    else:
+        assert ls >= 16 and g == -(-n // ls) and g <= 2048 and (g - 1) * ls < n
+        m = g
+    assert ng * e >= m and (ng // 2) * e < m or ng == 1
+    assert e <= 16 or n > 32768
+    want = 2 * e + int(math.log2(ng)) + (2 * ls if n > 2048 else 0)
+    assert p["depth"] == want
+    if n <= 32768:
+        assert p["depth"] <= 2 * 16 + 2 * 16 + 7
+    assert B.lin_attn_scan_plan(n, "sequential")["depth"] == n
+
+
+def _blocked_scan_model(x, a, init, plan):
+    """Host restatement of the log-depth arrangement the plan describes (fold each group,
+    Hillis-Steele over group folds, re-scan each group), to check that the plan's groups
+    and segments cover every element exactly once; returns exclusive prefixes and total."""
+    def blocked(xs, as_, init_):
+        m = len(xs)
+        ng, e = plan_block(m)
+        folds, decays = [], []
+        for gi in range(ng):
+            agg, A = np.zeros_like(xs[0]), 1.0
+            for j in range(gi * e, min(m, gi * e + e)):
+                agg = as_[j] * agg + xs[j]
+                A *= as_[j]
+            folds.append(agg)
+            decays.append(A)
+        d = 1
+        while d < ng:
+            nf, nd = list(folds), list(decays)
+            for gi in range(d, ng):
+                nf[gi] = decays[gi] * folds[gi - d] + folds[gi]
+                nd[gi] = decays[gi] * decays[gi - d]
+            folds, decays = nf, nd
+            d *= 2
+        out = [None] * m
+        total = None
+        for gi in range(ng):
+            carry = init_ if gi == 0 else decays[gi - 1] * init_ + folds[gi - 1]
+            for j in range(gi * e, min(m, gi * e + e)):
+                out[j] = carry
+                carry = as_[j] * carry + xs[j]
+            if min(m, gi * e + e) == m and gi * e < m:
+                total = carry
+        return out, total
+
+    def plan_block(m):
+        ng = 1
+        while ng < m and ng < 128:
+            ng *= 2
+        return ng, -(-m // ng)
+
+    n = len(x)
+    if n <= 2048:
+        return blocked(x, a, init)
+    ls, g = plan["segment_len"], plan["segments"]
+    segs = [range(s * ls, min(n, s * ls + ls)) for s in range(g)]
+    sx, sa = [], []
+    for r in segs:
+        agg, A = np.zeros_like(x[0]), 1.0
+        for j in r:
+            agg = a[j] * agg + x[j]
+            A *= a[j]
+        sx.append(agg)
+        sa.append(A)
+    pref, total = blocked(sx, sa, init)
+    out = [None] * n
+    for s, r in enumerate(segs):
+        carry = pref[s]
+        for j in r:
+            out[j] = carry
+            carry = a[j] * carry + x[j]
+    return out, total
+
+
+@pytest.mark.parametrize("n", [1, 5, 64, 129, 2048, 2049, 5000])
+def test_scan_plan_covers_every_element(lib, n):
+    from chunked_causal_linear_b200 import binding as B
+    rng = np.random.default_rng(n)
+    x = [rng.standard_normal(2) for _ in range(n)]
+    a = list(rng.uniform(0.5, 1.0, n))
+    init = rng.standard_normal(2)
+    got, total = _blocked_scan_model(x, a, init, B.lin_attn_scan_plan(n))
+    carry = init.copy()
+    for j in range(n):
+        np.testing.assert_allclose(got[j], carry, rtol=1e-12, atol=1e-12)
+        carry = a[j] * carry + x[j]
+    np.testing.assert_allclose(total, carry, rtol=1e-12, atol=1e-12)
 
 
 def _args(**kw):

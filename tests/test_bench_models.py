@@ -36,8 +36,8 @@ def test_backward_bytes_are_three_prefills_on_the_retention_workload():
     w = WORKLOADS["retention_128k"]
     ops = bench.backward_bytes(w, 4, "auto")
     names = [n for n, _ in ops]
-    # reverse-mode passes: no element-wise kernel, three (k1_seg, k2_scan_totals, k3_seg)
-    assert names == ["k1_seg", "k2_scan_totals", "k3_seg"] * 3
+    # reverse-mode passes: no element-wise kernel, three (k1_seg, k2_block_scan, k3_seg)
+    assert names == ["k1_seg", "k2_block_scan", "k3_seg"] * 3
     k3 = [b for n, b in ops if n == "k3_seg"]
     assert len(set(k3)) == 1 and k3[0] == bench.kernel_bytes(w, "k3_seg", 4, "segmented")
 
