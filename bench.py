@@ -35,6 +35,7 @@ from pathlib import Path
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from chunked_causal_linear_b200 import binding as B  # noqa: E402
@@ -815,6 +816,94 @@ def scan_depth(w, args) -> dict:
     return {"elements": n, "depth": d, "ceil_log2_elements": math.ceil(math.log2(max(n, 2)))}
 
 
+METRIC_DEC = "causal linear-attn decode steps: state bytes/s; % of roofline"
+DECODE_CASES = ((8, 32), (64, 32), (1, 32))  # (B, H) at dk = dv = 128
+
+
+def decode_bytes(Bn, H, dk, dv, e_in, e_out, with_z):
+    """Bytes one decode step must move: the state read and written once, q, k, v read, the
+    output written (and Z read and written when it is kept)."""
+    per = 2 * dk * dv * 4 + (2 * dk + dv) * e_in + dv * e_out + (2 * dk * 4 if with_z else 0)
+    return Bn * H * per
+
+
+def decode_bench(args, dev):
+    """One decode step for every (b, h) at dk = dv = 128, bf16 q, k, v and output, float32
+    state: the retention form (identity map, per-head decay) and the normalised ELU+1 form.
+    The steps are captured in a CUDA graph (64 steps) and the graph replayed, so the time is
+    the kernels' own; each case is first checked against the oracle (one step from the
+    same state)."""
+    from oracle.oracle import default_oracle
+    peak, peak_kind = measured_peaks()
+    dk = dv = 128
+    nsteps = 64
+    for Bn, H in DECODE_CASES:
+        for form in ("retention", "normalised"):
+            norm = form == "normalised"
+            fm = "elu1" if norm else "identity"
+            gam = None if norm else [float(1 - 2.0 ** (-5 - 3 * h / 31)) for h in range(H)]
+            g = torch.Generator(device=dev).manual_seed(0)
+            scale = 0.5 if norm else 128 ** -0.5
+            q, k, v = (torch.randn((Bn, H, d), generator=g, device=dev).mul_(scale)
+                       .to(torch.bfloat16) for d in (dk, dk, dv))
+            S = torch.randn((Bn, H, dk, dv), generator=g, device=dev).mul_(0.1)
+            Z = torch.rand((Bn, H, dk), generator=g, device=dev).add_(1.0) if norm else None
+            out = torch.empty((Bn, H, dv), dtype=torch.bfloat16, device=dev)
+            kw = dict(feature_map=fm, gamma=gam, normalize=norm)
+            # Parity: one step against the oracle from the same state (a sample of heads).
+            S0 = S.cpu().numpy()
+            Z0 = Z.cpu().numpy() if Z is not None else None
+            B.lin_attn_decode_step(q, k, v, S, Z, out=out, **kw)
+            torch.cuda.synchronize()
+            f = lambda t: t.float().cpu().numpy()[:, :, None]
+            o_ref, S_ref, _ = default_oracle().forward(
+                f(q), f(k), f(v), feature_map=fm, normalize=norm,
+                gamma=None if gam is None else np.asarray(gam, dtype=np.float64),
+                S_init=S0, Z_init=Z0)
+            got = out.float().cpu().numpy()
+            err_o = float(np.max(np.abs(got - o_ref[:, :, 0])) / np.sqrt(np.mean(o_ref ** 2)))
+            err_S = float(np.max(np.abs(S.cpu().numpy() - S_ref)) / np.sqrt(np.mean(S_ref ** 2)))
+            # Time: a graph of nsteps steps, replayed.
+            stream = torch.cuda.Stream(device=dev)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                B.lin_attn_decode_step(q, k, v, S, Z, out=out, stream=stream, **kw)
+                stream.synchronize()
+                with torch.cuda.graph(graph, stream=stream):
+                    for _ in range(nsteps):
+                        B.lin_attn_decode_step(q, k, v, S, Z, out=out, stream=stream, **kw)
+            for _ in range(max(3, args.warmup)):
+                graph.replay()
+            torch.cuda.synchronize()
+            reps = max(5, args.steps // 4)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1000.0 / (reps * nsteps)
+            nb = decode_bytes(Bn, H, dk, dv, 2, 2, norm)
+            gbs = nb / (us * 1e-6) / 1e9
+            line = {
+                "metric": METRIC_DEC, "workload": f"decode_b{Bn}h{H}_d128_{form}",
+                "B": Bn, "H": H, "dk": dk, "dv": dv, "heads": Bn * H,
+                "us_per_step": us, "steps_per_s": 1e6 / us,
+                "tokens_heads_per_s": Bn * H * 1e6 / us, "bytes_per_step": nb,
+                "roofline": {"bound": "hbm", "kernel": "decode_tiles", "achieved": gbs,
+                             "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                             "peak_source": peak_kind},
+                "parity_vs_oracle": {"out_max_err_over_rms": err_o, "S_max_err_over_rms": err_S,
+                                     "bound": 2e-2},
+                "timing": f"CUDA graph of {nsteps} steps replayed {reps} times, CUDA events",
+                "state_bytes": Bn * H * dk * dv * 4,
+                "l2": "state larger than L2" if Bn * H * dk * dv * 4 > 126e6 else
+                      "state fits in L2 (a step re-reads it from L2)",
+            }
+            print(json.dumps(line), flush=True)
+            del graph
+
+
 def config_of(w, args):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
             "C": w.C, "inputs": w.dtype, "feature_map": w.feature_map,
@@ -871,6 +960,9 @@ def main():
     ap.add_argument("--gla-path", default="fma", choices=["fma", "tensor_core"],
                     help="GLA kernels: exact CUDA-core ones, or the tensor-core prefill on "
                          "factored gates")
+    ap.add_argument("--decode", action="store_true",
+                    help="instead of the prefill: the decode step (state in place) at B.H = "
+                         "256, 2048 and 32, dk = dv = 128, one JSON line per case")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with this many heads instead (smaller cases for "
                          "profiler captures; every other size unchanged)")
@@ -904,6 +996,10 @@ def main():
         return
     if args.gla:
         gla_bench(args, info, dev)
+        ranks.finish(info)
+        return
+    if args.decode:
+        decode_bench(args, dev)
         ranks.finish(info)
         return
 

@@ -2,11 +2,20 @@
 //   S <- gamma S + psi(k) v^T,  Z <- gamma Z + psi(k),
 //   o  = psi(q) S / (psi(q) . Z + eps)   or   psi(q) S
 // ("Linear Attention and Retentive Networks ...", "The Recurrent Dual" and
-// "B. Recurrent Representation").  One CTA per (b, h); thread j owns value column j and
-// streams the state column S[:, j] (coalesced across threads), so each state element is
-// read and written exactly once.  The step is memory-bound: 8 dk dv bytes of state
-// traffic per (b, h).
+// "B. Recurrent Representation").  The step is memory-bound: each state element is read
+// and written once, 8 dk dv bytes of state traffic per (b, h).
+//
+// decode_tiles (dk a multiple of 16 up to 128, dv a multiple of 4 up to 256, 16-byte
+// aligned tensors): the state of one (b, h) is cut into dk / 16 tiles of 16 rows (key
+// features), one CTA each, and those CTAs form one thread-block cluster.  A thread streams
+// float4 columns of its rows (every row is contiguous), so a step is one wave of
+// independent 16-byte loads over the whole GPU.  Each CTA reduces psi(q) . S over its rows
+// in shared memory; the cluster then adds the tiles' partial outputs (and denominators)
+// through distributed shared memory in a fixed order, each CTA finishing a share of the
+// value features.  No atomics and no scratch memory: the result does not depend on timing.
+// decode_step (any dk, dv up to 256): one CTA per (b, h), thread j streams state column j.
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -88,9 +97,175 @@ decode_step(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   }
 }
 
+constexpr int kTileRows = 16;
+constexpr int kTileThreads = 256;
+
+// Four consecutive values as float (bf16: one 8-byte load; float: one 16-byte load).
+__device__ __forceinline__ float4 ld4(const float* p, long long i) {
+  return *reinterpret_cast<const float4*>(p + i);
+}
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* p, long long i) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p + i);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void st4(float* p, long long i, float4 x) {
+  *reinterpret_cast<float4*>(p + i) = x;
+}
+__device__ __forceinline__ void st4(__nv_bfloat16* p, long long i, float4 x) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p + i) = u;
+}
+
+template <typename T, int FM, bool DECAY, bool NORM>
+__global__ void __launch_bounds__(kTileThreads)
+decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+             T* __restrict__ out, float* __restrict__ S, float* __restrict__ Z, int H, int dk,
+             int dv, float eps, GammaTable gt) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  __shared__ float sq[kTileRows], sk[kTileRows];
+  __shared__ float4 sAcc[kTileThreads];
+  __shared__ float4 sPart[64];  // this tile's partial psi(q) . S, dv / 4 float4
+  __shared__ float sDen;
+  const int nt = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int bh = blockIdx.x / nt;
+  const int i0 = rank * kTileRows;
+  const int tid = threadIdx.x;
+  const float g = DECAY ? gt.g[bh % H] : 1.f;
+
+  if (tid < 32) {
+    // Rows i0 .. i0 + 15: psi(q), psi(k), the Z update and this tile's share of psi(q) . Z.
+    float part = 0.f;
+    if (tid < kTileRows) {
+      const long long i = static_cast<long long>(bh) * dk + i0 + tid;
+      const float fq = feature<FM>(static_cast<float>(q[i]));
+      const float fk = feature<FM>(static_cast<float>(k[i]));
+      sq[tid] = fq;
+      sk[tid] = fk;
+      if (Z) {
+        const float z = fmaf(g, Z[i], fk);
+        Z[i] = z;
+        part = fq * z;
+      }
+    }
+    if (NORM) {
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (tid == 0) sDen = part;
+    }
+  }
+  __syncthreads();
+
+  const int dv4 = dv / 4;
+  const int lanes = kTileThreads / dv4;  // row lanes (>= 4)
+  const int c4 = tid % dv4, rl = tid / dv4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (rl < lanes && rl < kTileRows) {
+    const float4 vj = ld4(v, static_cast<long long>(bh) * dv + 4 * c4);
+    float* Sb = S + (static_cast<long long>(bh) * dk + i0) * dv + 4 * c4;
+    constexpr int kMax = kTileRows / 4;  // rows per thread when lanes >= 4
+    float4 s[kMax];
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+      const int r = rl + m * lanes;
+      if (r < kTileRows) s[m] = *reinterpret_cast<const float4*>(Sb + static_cast<long long>(r) * dv);
+    }
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+      const int r = rl + m * lanes;
+      if (r < kTileRows) {
+        const float a = sk[r], b = sq[r];
+        float4 x = s[m];
+        x.x = fmaf(a, vj.x, g * x.x);
+        x.y = fmaf(a, vj.y, g * x.y);
+        x.z = fmaf(a, vj.z, g * x.z);
+        x.w = fmaf(a, vj.w, g * x.w);
+        *reinterpret_cast<float4*>(Sb + static_cast<long long>(r) * dv) = x;
+        acc.x = fmaf(b, x.x, acc.x);
+        acc.y = fmaf(b, x.y, acc.y);
+        acc.z = fmaf(b, x.z, acc.z);
+        acc.w = fmaf(b, x.w, acc.w);
+      }
+    }
+  }
+  sAcc[tid] = acc;
+  __syncthreads();
+  if (tid < dv4) {
+    float4 t = sAcc[tid];
+    for (int r = 1; r < lanes && r < kTileRows; ++r) {
+      const float4 u = sAcc[r * dv4 + tid];
+      t.x += u.x;
+      t.y += u.y;
+      t.z += u.z;
+      t.w += u.w;
+    }
+    sPart[tid] = t;
+  }
+  cl.sync();
+  // Value features c4 = rank, rank + nt, ...: the tiles' partials added in rank order.
+  for (int c = rank + nt * tid; c < dv4; c += nt * kTileThreads) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    for (int j = 0; j < nt; ++j) {
+      const float4 u = *cl.map_shared_rank(&sPart[c], j);
+      o.x += u.x;
+      o.y += u.y;
+      o.z += u.z;
+      o.w += u.w;
+      if (NORM) den += *cl.map_shared_rank(&sDen, j);
+    }
+    if (NORM) {
+      const float d = den + eps;
+      o.x /= d;
+      o.y /= d;
+      o.z /= d;
+      o.w /= d;
+    }
+    st4(out, static_cast<long long>(bh) * dv + 4 * c, o);
+  }
+  cl.sync();  // no CTA leaves while another still reads its shared memory
+}
+
+bool tiles_ok(const void* q, const void* k, const void* v, const void* out, const float* S,
+              const float* Z, int dk, int dv) {
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return dk % kTileRows == 0 && dk <= 8 * kTileRows && dv % 4 == 0 && dv <= 256 && a16(q) &&
+         a16(k) && a16(v) && a16(out) && a16(S) && a16(Z);
+}
+
+template <typename T, int FM, bool DECAY, bool NORM>
+cudaError_t go_tiles(const void* q, const void* k, const void* v, void* out, float* S, float* Z,
+                     int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
+                     cudaStream_t s) {
+  const int nt = dk / kTileRows;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(BH) * nt);
+  cfg.blockDim = dim3(kTileThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nt;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tiles<T, FM, DECAY, NORM>, static_cast<const T*>(q),
+                            static_cast<const T*>(k), static_cast<const T*>(v),
+                            static_cast<T*>(out), S, Z, H, dk, dv, eps, gt);
+}
+
 template <typename T, int FM, bool DECAY, bool NORM>
 cudaError_t go(const void* q, const void* k, const void* v, void* out, float* S, float* Z,
                int BH, int H, int dk, int dv, float eps, const GammaTable& gt, cudaStream_t s) {
+  if (tiles_ok(q, k, v, out, S, Z, dk, dv))
+    return go_tiles<T, FM, DECAY, NORM>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
   decode_step<T, FM, DECAY, NORM><<<BH, kDecThreads, 0, s>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
       static_cast<T*>(out), S, Z, H, dk, dv, eps, gt);

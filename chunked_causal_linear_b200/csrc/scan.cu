@@ -12,9 +12,9 @@
 //
 // Log-depth mode ("Implementation notes": a Blelloch or Hillis-Steele scan; "Verification":
 // ceil(log2 N_C) rounds) is a work-efficient blocked scan (Brent's arrangement of
-// Hillis-Steele).  One CTA takes a slab of 8 float4 columns (128 contiguous bytes of every
-// record) and up to 2048 elements of the chunk axis, split over NG <= 128 groups of E <= 16
-// consecutive elements, one thread per (group, column):
+// Hillis-Steele).  One CTA of 1024 threads takes up to 2048 elements of the chunk axis, split
+// over NG <= 128 groups of E <= 16 consecutive elements, and a slab of 1024 / NG float4
+// columns (128 contiguous bytes of every record or more), one thread per (group, column):
 //   k2_block_scan   pass 1: each thread folds its E elements (E dependent steps);
 //                   Hillis-Steele over the NG group folds in shared memory (log2 NG
 //                   rounds); pass 2: each thread re-reads its elements (from L2: a CTA's
@@ -43,8 +43,8 @@ namespace {
 
 constexpr int kScanThreads = 128;
 constexpr int kUnroll = 8;
-constexpr int kSlab = 8;         // float4 columns per block-scan CTA (128 contiguous bytes)
-constexpr int kMaxGroups = 128;  // groups per block-scan CTA (1024 threads)
+constexpr int kBlockThreads = 1024;  // block-scan CTA: groups x slab columns
+constexpr int kMaxGroups = 128;      // groups per block-scan CTA (slab of at least 8 float4)
 
 __device__ __forceinline__ float4 axpy4(float a, float4 x, float4 y) {
   return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
@@ -163,13 +163,15 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
   reinterpret_cast<float4*>(p.tot + (static_cast<long long>(bh) * p.G + s) * p.R)[col4] = agg;
 }
 
-// Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of kSlab float4
-// columns); NG groups of E consecutive elements (NG a power of two, NG * E >= N).
+// Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of W = 1024 / NG
+// float4 columns: at least 128 contiguous bytes of every record); NG groups of E consecutive
+// elements (NG a power of two, NG * E >= N).
 template <bool DECAY>
-__global__ void __launch_bounds__(kSlab * kMaxGroups, 1)
+__global__ void __launch_bounds__(kBlockThreads, 1)
 k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
-  __shared__ float4 sX[kMaxGroups * kSlab];
-  __shared__ float sA[kMaxGroups];
+  __shared__ float4 sX[kBlockThreads];
+  __shared__ float sA[kBlockThreads];
+  const int kSlab = kBlockThreads / NG;  // W
   const int R4 = p.R / 4;
   const int nslab = (R4 + kSlab - 1) / kSlab;
   const int bh = blockIdx.x / nslab;
@@ -257,8 +259,9 @@ template <bool DECAY>
 cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_t s) {
   const ScanPlan bp = scan_plan(p.NC);  // p.NC <= kScanBlockElems: a single block level
   const int R4 = p.R / 4;
-  const long long nslab = (R4 + kSlab - 1) / kSlab;
-  k2_block_scan<DECAY><<<static_cast<unsigned>(nslab * p.BH), kSlab * bp.NG, 0, s>>>(
+  const int W = kBlockThreads / bp.NG;
+  const long long nslab = (R4 + W - 1) / W;
+  k2_block_scan<DECAY><<<static_cast<unsigned>(nslab * p.BH), kBlockThreads, 0, s>>>(
       p, gt, bp.NG, bp.E);
   return cudaGetLastError();
 }
