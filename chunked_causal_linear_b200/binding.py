@@ -33,7 +33,7 @@ EXPORTED_SYMBOLS = (
     "lin_attn_status_string", "lin_attn_version", "lin_attn_combine_states",
     "lin_attn_backward", "lin_attn_backward_workspace_bytes", "lin_attn_backward_timed",
     "lin_attn_gla_prefill", "lin_attn_gla_workspace_bytes", "lin_attn_gla_prefill_timed",
-    "lin_attn_scan_plan",
+    "lin_attn_scan_plan", "lin_attn_check_wait_timeout",
 )
 
 
@@ -119,6 +119,7 @@ def load_library(path: Path | str | None = None) -> ctypes.CDLL:
         "lin_attn_device_error": (i, [ctypes.POINTER(ctypes.c_int)]),
         "lin_attn_status_string": (ctypes.c_char_p, [i]),
         "lin_attn_version": (i, []),
+        "lin_attn_check_wait_timeout": (i, [ctypes.c_uint, vp]),
         "lin_attn_scan_plan": (i, [ll, i, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i),
                                    ctypes.POINTER(i), ctypes.POINTER(ll)]),
         "lin_attn_combine_states": (i, [vp, vp, i, i, ctypes.POINTER(ll), i, i, i, i, vp, vp,
@@ -515,6 +516,13 @@ def lin_attn_device_error() -> int:
 
 def lin_attn_status_string(status: int) -> str:
     return load_library().lin_attn_status_string(int(status)).decode()
+
+
+def lin_attn_check_wait_timeout(timeout_us: int = 1000, stream=None) -> None:
+    """Launches the library's bounded-wait check (one wait that must give up); read the
+    result with lin_attn_device_error() (code 5)."""
+    _check("lin_attn_check_wait_timeout",
+           load_library().lin_attn_check_wait_timeout(int(timeout_us), _stream_handle(stream)))
 
 
 def lin_attn_scan_plan(n: int, scan: str = "logdepth") -> dict:

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -256,7 +257,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
   if (ws) {
     if (a.workspace_bytes < l.total) return LA_ERR_INVALID_ARGUMENT;
   } else {
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), l.total, s);
+    cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), l.total, s);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return LA_ERR_OUT_OF_MEMORY;
@@ -444,6 +445,12 @@ int prefill_with_args(const la_prefill_args& a, Recorder* rec) { return prefill(
 
 int* device_error_word() { return error_word_ptr(); }
 
+cudaError_t workspace_alloc(void** p, size_t bytes, cudaStream_t s) {
+  const char* inj = std::getenv("LA_FAULT_INJECT");
+  if (inj && std::strcmp(inj, "alloc") == 0) return cudaErrorMemoryAllocation;
+  return cudaMallocAsync(p, bytes, s);
+}
+
 bool make_tile_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0,
                    uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
                    uint32_t box1) {
@@ -542,7 +549,7 @@ int lin_attn_prefill_host(const la_prefill_args* host_args, void* device_buffer,
     if (device_buffer_bytes < hl.total || (reinterpret_cast<uintptr_t>(buf) & 255u))
       return LA_ERR_INVALID_ARGUMENT;
   } else {
-    if (cudaMallocAsync(reinterpret_cast<void**>(&buf), hl.total, s) != cudaSuccess) {
+    if (la::workspace_alloc(reinterpret_cast<void**>(&buf), hl.total, s) != cudaSuccess) {
       cudaGetLastError();
       return LA_ERR_OUT_OF_MEMORY;
     }

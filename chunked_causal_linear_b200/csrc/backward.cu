@@ -730,7 +730,7 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
   if (ws) {
     if (a.workspace_bytes < l.total) return LA_ERR_INVALID_ARGUMENT;
   } else {
-    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), l.total, s) != cudaSuccess) {
+    if (workspace_alloc(reinterpret_cast<void**>(&ws), l.total, s) != cudaSuccess) {
       cudaGetLastError();
       return LA_ERR_OUT_OF_MEMORY;
     }

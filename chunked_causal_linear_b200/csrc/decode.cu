@@ -6,7 +6,7 @@
 // and written once, 8 dk dv bytes of state traffic per (b, h).
 //
 // decode_tiles (dk a multiple of 16 up to 128, dv a multiple of 4 up to 256, 16-byte
-// aligned tensors): the state of one (b, h) is cut into dk / 16 tiles of 16 rows (key
+// aligned tensors): the state of one (b, h) is cut into tiles of 16 or 64 rows (key
 // features), one CTA each, and those CTAs form one thread-block cluster.  A thread streams
 // float4 columns of its rows (every row is contiguous), so a step is one wave of
 // independent 16-byte loads over the whole GPU.  Each CTA reduces psi(q) . S over its rows
@@ -121,28 +121,47 @@ __device__ __forceinline__ void st4(__nv_bfloat16* p, long long i, float4 x) {
   *reinterpret_cast<uint2*>(p + i) = u;
 }
 
-template <typename T, int FM, bool DECAY, bool NORM>
+template <typename T, int FM, bool DECAY, bool NORM, int TR>
 __global__ void __launch_bounds__(kTileThreads)
 decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
              T* __restrict__ out, float* __restrict__ S, float* __restrict__ Z, int H, int dk,
              int dv, float eps, GammaTable gt) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
-  __shared__ float sq[kTileRows], sk[kTileRows];
+  __shared__ float sq[TR], sk[TR];
   __shared__ float4 sAcc[kTileThreads];
   __shared__ float4 sPart[64];  // this tile's partial psi(q) . S, dv / 4 float4
   __shared__ float sDen;
   const int nt = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
   const int bh = blockIdx.x / nt;
-  const int i0 = rank * kTileRows;
+  const int i0 = rank * TR;
   const int tid = threadIdx.x;
   const float g = DECAY ? gt.g[bh % H] : 1.f;
 
-  if (tid < 32) {
-    // Rows i0 .. i0 + 15: psi(q), psi(k), the Z update and this tile's share of psi(q) . Z.
+  // The tile's state rows first (they depend on nothing else): thread (row lane rl,
+  // float4 column c4) loads rows rl, rl + lanes, ... of the tile.
+  const int dv4 = dv / 4;
+  const int lanes = kTileThreads / dv4;  // row lanes (>= 4)
+  const int c4 = tid % dv4, rl = tid / dv4;
+  const bool active = rl < lanes && rl < TR;
+  constexpr int kMax = TR / 4;  // rows per thread (lanes >= 4)
+  float* Sb = S + (static_cast<long long>(bh) * dk + i0) * dv + 4 * c4;
+  float4 s[kMax];
+  if (active) {
+#pragma unroll
+    for (int m = 0; m < kMax; ++m) {
+      const int r = rl + m * lanes;
+      if (r < TR) s[m] = *reinterpret_cast<const float4*>(Sb + static_cast<long long>(r) * dv);
+    }
+  }
+  float4 vj = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) vj = ld4(v, static_cast<long long>(bh) * dv + 4 * c4);
+
+  if (tid < 32 * ((TR + 31) / 32)) {
+    // Rows i0 .. i0 + TR - 1: psi(q), psi(k), the Z update and this tile's psi(q) . Z.
     float part = 0.f;
-    if (tid < kTileRows) {
+    if (tid < TR) {
       const long long i = static_cast<long long>(bh) * dk + i0 + tid;
       const float fq = feature<FM>(static_cast<float>(q[i]));
       const float fk = feature<FM>(static_cast<float>(k[i]));
@@ -156,30 +175,24 @@ decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
     }
     if (NORM) {
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (tid == 0) sDen = part;
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if ((tid & 31) == 0) sAcc[tid >> 5].x = part;  // per-warp sums, read below
     }
   }
   __syncthreads();
+  if (NORM && tid == 0) {
+    float d = 0.f;
+    for (int w = 0; w < (TR + 31) / 32; ++w) d += sAcc[w].x;
+    sDen = d;
+  }
+  __syncthreads();
 
-  const int dv4 = dv / 4;
-  const int lanes = kTileThreads / dv4;  // row lanes (>= 4)
-  const int c4 = tid % dv4, rl = tid / dv4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (rl < lanes && rl < kTileRows) {
-    const float4 vj = ld4(v, static_cast<long long>(bh) * dv + 4 * c4);
-    float* Sb = S + (static_cast<long long>(bh) * dk + i0) * dv + 4 * c4;
-    constexpr int kMax = kTileRows / 4;  // rows per thread when lanes >= 4
-    float4 s[kMax];
+  if (active) {
 #pragma unroll
     for (int m = 0; m < kMax; ++m) {
       const int r = rl + m * lanes;
-      if (r < kTileRows) s[m] = *reinterpret_cast<const float4*>(Sb + static_cast<long long>(r) * dv);
-    }
-#pragma unroll
-    for (int m = 0; m < kMax; ++m) {
-      const int r = rl + m * lanes;
-      if (r < kTileRows) {
+      if (r < TR) {
         const float a = sk[r], b = sq[r];
         float4 x = s[m];
         x.x = fmaf(a, vj.x, g * x.x);
@@ -198,7 +211,7 @@ decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
   __syncthreads();
   if (tid < dv4) {
     float4 t = sAcc[tid];
-    for (int r = 1; r < lanes && r < kTileRows; ++r) {
+    for (int r = 1; r < lanes && r < TR; ++r) {
       const float4 u = sAcc[r * dv4 + tid];
       t.x += u.x;
       t.y += u.y;
@@ -232,6 +245,13 @@ decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
   cl.sync();  // no CTA leaves while another still reads its shared memory
 }
 
+// Rows per CTA: 64 (four tiles in flight per thread pair of rows: 8 loads of 16 bytes per
+// thread at dv = 128) when that still gives every SM two CTAs, else 16.
+int tile_rows(long long BH, int dk) {
+  if (dk % 64 == 0 && BH * (dk / 64) >= 2 * 148) return 64;
+  return 16;
+}
+
 bool tiles_ok(const void* q, const void* k, const void* v, const void* out, const float* S,
               const float* Z, int dk, int dv) {
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
@@ -239,11 +259,11 @@ bool tiles_ok(const void* q, const void* k, const void* v, const void* out, cons
          a16(k) && a16(v) && a16(out) && a16(S) && a16(Z);
 }
 
-template <typename T, int FM, bool DECAY, bool NORM>
-cudaError_t go_tiles(const void* q, const void* k, const void* v, void* out, float* S, float* Z,
-                     int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
-                     cudaStream_t s) {
-  const int nt = dk / kTileRows;
+template <typename T, int FM, bool DECAY, bool NORM, int TR>
+cudaError_t go_tiles_r(const void* q, const void* k, const void* v, void* out, float* S,
+                       float* Z, int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
+                       cudaStream_t s) {
+  const int nt = dk / TR;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(BH) * nt);
   cfg.blockDim = dim3(kTileThreads);
@@ -256,9 +276,18 @@ cudaError_t go_tiles(const void* q, const void* k, const void* v, void* out, flo
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tiles<T, FM, DECAY, NORM>, static_cast<const T*>(q),
+  return cudaLaunchKernelEx(&cfg, decode_tiles<T, FM, DECAY, NORM, TR>, static_cast<const T*>(q),
                             static_cast<const T*>(k), static_cast<const T*>(v),
                             static_cast<T*>(out), S, Z, H, dk, dv, eps, gt);
+}
+
+template <typename T, int FM, bool DECAY, bool NORM>
+cudaError_t go_tiles(const void* q, const void* k, const void* v, void* out, float* S, float* Z,
+                     int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
+                     cudaStream_t s) {
+  if (tile_rows(BH, dk) == 64)
+    return go_tiles_r<T, FM, DECAY, NORM, 64>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
+  return go_tiles_r<T, FM, DECAY, NORM, 16>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
 }
 
 template <typename T, int FM, bool DECAY, bool NORM>

@@ -547,7 +547,7 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
   if (ws) {
     if (a.workspace_bytes < need) return LA_ERR_INVALID_ARGUMENT;
   } else {
-    if (cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s) != cudaSuccess) {
+    if (workspace_alloc(reinterpret_cast<void**>(&ws), need, s) != cudaSuccess) {
       cudaGetLastError();
       return LA_ERR_OUT_OF_MEMORY;
     }

@@ -15,6 +15,11 @@ int check_prefill_args(const la_prefill_args& a);
 // The device error word of the current device (every kernel receives it).
 int* device_error_word();
 
+// Workspace allocation of every entry point that allocates (cudaMallocAsync on the
+// stream).  With the environment variable LA_FAULT_INJECT=alloc it fails without
+// allocating, so that callers' handling of LA_ERR_OUT_OF_MEMORY can be tested.
+cudaError_t workspace_alloc(void** p, size_t bytes, cudaStream_t s);
+
 // A 3D tiled TMA map (d0 innermost) with the 128-byte swizzle, as the prefill's kernels use.
 bool make_tile_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0,
                    uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,

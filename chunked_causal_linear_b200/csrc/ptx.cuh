@@ -16,6 +16,7 @@ enum : int {
   kErrMmaTimeout = 2,
   kErrBadShape = 3,
   kErrGateRange = 4,  // gated attention on the tensor cores: a chunk's gates too small to factor
+  kErrWaitCheck = 5,  // lin_attn_check_wait_timeout: the deliberate wait gave up, as it should
 };
 
 __device__ __forceinline__ void report_error(int* err, int code) {

@@ -129,7 +129,9 @@ typedef enum {
  *   feature_map  la_feature_map.  normalize != 0 requires LA_FM_ELU1 (the identity map
  *             gives a denominator of indefinite sign).
  * Uses the log-depth scan, LA_ALGO_AUTO and eps = 0.  The workspace is allocated with
- * cudaMallocAsync / cudaFreeAsync on `stream` (LA_ERR_OUT_OF_MEMORY on failure).
+ * cudaMallocAsync / cudaFreeAsync on `stream` (LA_ERR_OUT_OF_MEMORY on failure; with
+ * the environment variable LA_FAULT_INJECT=alloc every library-side allocation fails
+ * this way without allocating, for testing callers' handling of it).
  * T == 0 zero-fills S_final / Z_final.  Returns a la_status.
  */
 int lin_attn_prefill(const void* q, const void* k, const void* v, void* out,
@@ -453,8 +455,23 @@ int lin_attn_decode_step_f32(const float* q, const float* k, const float* v, flo
                              la_stream_t stream);
 
 /* Reads and clears the device-side error word that kernels set when an internal check
- * or a bounded wait fails (0 = none).  Synchronises the current device. */
+ * or a bounded wait fails (0 = none).  Synchronises the current device.  Codes: 1 a TMA
+ * load never landed, 2 an MMA or a hand-off between warps never completed (each after
+ * about two seconds), 3 an internal shape check failed, 4 gated attention: gates the
+ * tensor-core kernels cannot factor, 5 the deliberate wait of lin_attn_check_wait_timeout
+ * gave up.  While the word is set, the tensor-core kernels launched afterwards skip their
+ * work (so one failure costs one bounded wait, not one per CTA). */
 int lin_attn_device_error(int* code);
+
+/*
+ * lin_attn_check_wait_timeout -- exercises the failure detection above without faulting
+ * anything (no passage of the pages corresponds to it; it is a diagnostic).  Launches one
+ * small kernel on `stream` in which one thread waits, with a limit of timeout_us
+ * microseconds, on an mbarrier that nothing arrives on; the wait gives up, and the kernel
+ * records code 5 in the device error word and returns.  Read and clear it with
+ * lin_attn_device_error.  timeout_us in [1, 10^6]; LA_ERR_INVALID_ARGUMENT otherwise.
+ */
+int lin_attn_check_wait_timeout(unsigned int timeout_us, la_stream_t stream);
 
 /* A static, human-readable name for a la_status value. */
 const char* lin_attn_status_string(int status);
