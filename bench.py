@@ -60,7 +60,7 @@ KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce
 
 def effective_algorithm(w, requested: str) -> str:
     """The algorithm the library runs for this workload on the tensor-core path."""
-    seg_ok = (w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv == 128
+    seg_ok = (w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv in (64, 128)
               and not (w.feature_map == "elu1" and w.decay))
     if requested == "segmented" or (requested == "auto" and seg_ok):
         return "segmented"
@@ -751,8 +751,9 @@ def gla_bench(args, info, dev):
     ms_max = ranks.max_over_ranks(e0.elapsed_time(e1) / args.steps, info, dev)
     per = [B.lin_attn_gla_prefill_timed(q, k, v, alpha, out, S, **kw)
            for _ in range(max(1, args.kernel_timing_steps))]
-    tc = args.gla_path == "tensor_core"
-    names = ["gla_tc_prep", "k1_tc", "gla_tc_k2", "k3_tc"] if tc else ["gla_k1", "gla_k2", "gla_k3"]
+    tc = args.gla_path in ("tensor_core", "auto")  # auto: the tensor cores at this shape
+    names = (["gla_k1_seg", "gla_scan", "gla_k3_seg", "gla_fixup"] if tc
+             else ["gla_k1", "gla_k2", "gla_k3"])
     kern_ms = {n: statistics.mean(x[i] for x in per) for i, n in enumerate(names)}
     BH, NC, C = w.B * w.H, -(-w.T // w.C), w.C
     R = w.dk * w.dv + w.dk
@@ -762,16 +763,18 @@ def gla_bench(args, info, dev):
     # logs stay above -100 (all of this workload's) the scores need no exponential per pair
     k3_flop = 2 * BH * NC * (C * w.dk * w.dv + pairs * w.dk + pairs * w.dv)
     e_in = 2
-    Rt = w.dk * w.dv
-    nk, nv = BH * w.T * w.dk, BH * w.T * w.dv
+    NS = -(-NC // segment_length(w))  # the tensor-core path's segments (automatic length)
     bytes_ = {"gla_k1": BH * w.T * (w.dk * (e_in + 4) + w.dv * e_in) + BH * NC * R * 4,
               "gla_k2": 2 * BH * NC * R * 4,
               "gla_k3": BH * w.T * (w.dk * (2 * e_in + 4) + w.dv * e_in + w.dv * 4) + BH * NC * R * 4,
-              # tensor cores: prep reads q, k, gates, writes three bf16 copies and a_c
-              "gla_tc_prep": nk * (2 * e_in + 4) + 3 * nk * e_in + BH * NC * w.dk * 4,
-              "k1_tc": nk * e_in + nv * e_in + BH * NC * Rt * 4,
-              "gla_tc_k2": 2 * BH * NC * Rt * 4 + BH * NC * w.dk * 4,
-              "k3_tc": 2 * nk * e_in + nv * e_in + BH * (NC - 1) * Rt * 4 + nv * 4}
+              # tensor cores, per token*head: K1 reads k, v, gates; K3 reads q, k, v, gates and
+              # writes the float32 output; per segment a record of R floats (K1 writes it,
+              # the scan reads and writes it, K3 reads its state part); one flag per chunk
+              "gla_k1_seg": BH * w.T * (w.dk * (e_in + 4) + w.dv * e_in) + BH * NS * R * 4,
+              "gla_scan": 2 * BH * NS * R * 4 + BH * w.dk * w.dv * 4,
+              "gla_k3_seg": BH * w.T * (w.dk * (2 * e_in + 4) + w.dv * e_in + w.dv * 4)
+              + BH * NS * w.dk * w.dv * 4 + BH * NC,
+              "gla_fixup": BH * NC}
     peak, peak_kind = measured_peaks()
     hbm = {n: bytes_[n] / (kern_ms[n] / 1e3) / 1e9 / peak for n in names}
     if tc:
@@ -793,8 +796,9 @@ def gla_bench(args, info, dev):
     if info.is_root:
         cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv, "C": w.C,
                "inputs": "bf16", "gates": "float32 sigmoid(N(4, 1))", "out_dtype": "f32",
-               "kernel_path": "tensor_core (factored gates, bf16 operands)" if tc
-               else "fma (CUDA cores)", "l2": "inputs larger than L2, no flush",
+               "kernel_path": "tensor_core (segmented, factored hi/lo operands)" if tc
+               else "fma (CUDA cores)", "segments": NS if tc else None,
+               "l2": "inputs larger than L2, no flush",
                "parallelism": "replicas (one independent problem per GPU)"}
         line = {"metric": METRIC_GLA, "value": info.world * w.tokens_heads / (ms_max / 1e3),
                 "unit": UNIT, "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
@@ -957,9 +961,9 @@ def main():
     ap.add_argument("--gla", action="store_true",
                     help="instead of the prefill: gated linear attention (data-dependent decay) "
                          "on the 128k-token gated workload")
-    ap.add_argument("--gla-path", default="fma", choices=["fma", "tensor_core"],
-                    help="GLA kernels: exact CUDA-core ones, or the tensor-core prefill on "
-                         "factored gates")
+    ap.add_argument("--gla-path", default="auto", choices=["auto", "fma", "tensor_core"],
+                    help="GLA kernels: the library's choice (tensor cores at this shape), the "
+                         "CUDA-core ones, or the tensor-core ones")
     ap.add_argument("--decode", action="store_true",
                     help="instead of the prefill: the decode step (state in place) at B.H = "
                          "256, 2048 and 32, dk = dv = 128, one JSON line per case")

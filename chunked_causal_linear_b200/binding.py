@@ -87,7 +87,7 @@ class GlaArgs(ctypes.Structure):
         ("T", ctypes.c_longlong), ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
         ("dtype", ctypes.c_int), ("out_dtype", ctypes.c_int), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("stream", ctypes.c_void_p),
-        ("kernel_path", ctypes.c_int),
+        ("kernel_path", ctypes.c_int), ("segment_chunks", ctypes.c_int),
     ]
 
 
@@ -410,7 +410,7 @@ def lin_attn_backward_workspace_bytes(q, v, *, chunk=64, feature_map="identity",
 
 
 def _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream,
-              kernel_path="auto"):
+              kernel_path="auto", segment_chunks=0):
     B, H, T, dk = q.shape
     a = GlaArgs()
     a.q, a.k, a.v, a.alpha, a.out = _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out)
@@ -422,12 +422,13 @@ def _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace,
     a.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     a.stream = _stream_handle(stream)
     a.kernel_path = KERNEL_PATHS[kernel_path]
+    a.segment_chunks = int(segment_chunks)
     return a
 
 
 def lin_attn_gla_prefill(q, k, v, alpha, out=None, S_final=None, *, S_init=None, chunk=64,
                          out_dtype="as_input", workspace=None, stream=None, want_state=True,
-                         kernel_path="auto"):
+                         kernel_path="auto", segment_chunks=0):
     """Gated linear attention (see the header): q, k, alpha [B,H,T,dk] (alpha float32),
     v [B,H,T,dv].  Returns (out, S_final)."""
     B, H, T, dk = q.shape
@@ -438,7 +439,7 @@ def lin_attn_gla_prefill(q, k, v, alpha, out=None, S_final=None, *, S_init=None,
     if want_state and S_final is None:
         S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     a = _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream,
-                  kernel_path)
+                  kernel_path, segment_chunks)
     _check("lin_attn_gla_prefill", load_library().lin_attn_gla_prefill(ctypes.byref(a)))
     return out, S_final
 
@@ -449,11 +450,12 @@ def lin_attn_gla_workspace_bytes(B, H, T, dk, dv, C) -> int:
 
 def lin_attn_gla_prefill_timed(q, k, v, alpha, out, S_final=None, *, S_init=None, chunk=64,
                                out_dtype="as_input", workspace=None, stream=None,
-                               kernel_path="auto") -> list[float]:
+                               kernel_path="auto", segment_chunks=0) -> list[float]:
     """One GLA prefill with an event around each kernel; returns their durations in ms, in
-    launch order (CUDA cores: K1, K2, K3; tensor cores: prep, k1_tc, carry, k3_tc)."""
+    launch order (CUDA cores: K1, K2, K3; tensor cores: gla_k1_seg, gla_scan, gla_k3_seg,
+    gla_fixup)."""
     a = _gla_args(q, k, v, alpha, out, S_final, S_init, chunk, out_dtype, workspace, stream,
-                  kernel_path)
+                  kernel_path, segment_chunks)
     ms = (ctypes.c_float * 8)()
     n = ctypes.c_int(0)
     _check("lin_attn_gla_prefill_timed",

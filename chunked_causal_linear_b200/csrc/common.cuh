@@ -67,4 +67,26 @@ __device__ __forceinline__ int chunk_len(const SegParams& p, int c) {
   return c == p.NC - 1 ? p.L_last : p.C;
 }
 
+// Gated linear attention on the tensor cores (segmented, dv = 128): one record per segment,
+// R = dk * dv + dk floats: the segment's fold S^T (dv rows of dk), then its decay vector.
+struct GlaSegParams {
+  int BH;
+  long long T;
+  int dk;
+  int NC;          // chunks of 64 tokens
+  int L_last;      // valid tokens in the last chunk
+  int Lseg;        // chunks per segment
+  int NS;          // segments per (b, h)
+  int R;           // floats per record
+  float* srec;     // [BH, NS, R]: segment folds, turned into exclusive prefixes by the scan
+  void* out;       // [BH, T, 128], bf16 or fp32
+  unsigned char* steep;  // [BH, NC]: 1 where the chunk's intra part is left to the fix-up
+  bool has_init;   // segment 0 starts from a given state
+  int* err;
+};
+
+__device__ __forceinline__ int chunk_len(const GlaSegParams& p, int c) {
+  return c == p.NC - 1 ? p.L_last : 64;
+}
+
 }  // namespace la

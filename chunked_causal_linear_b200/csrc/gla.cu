@@ -12,15 +12,19 @@
 //   K3  o_j = (q_j (.) e^(L_j)) P_c + sum_{i<=j} (sum_f q_j[f] k_i[f] e^(L_j[f] - L_i[f])) v_i
 // The kernels form these as powers of two of cumulative log2 gates, every exponent <= 0,
 // so nothing overflows whatever the gates (a gate below 2^-126 counts as 2^-126).  Two paths:
-//   CUDA cores (default; gla_k1, gla_k2, gla_k3): exact in float32 for any gates.  K3's
-//     scores factor as (q (.) 2^L) . (k (.) 2^-L) when the chunk's logs stay >= -100 (plain
-//     dot products), else take one exponential per (pair, feature).
-//   Tensor cores (opt-in; gla_tc_prep, the prefill's k1_tc / k3_tc, gla_tc_k2): the factored
-//     operands in bf16 through the prefill's tcgen05 kernels, for gates that factor.
+//   Tensor cores (default for bf16, C = 64, dk in {64, 128}, dv = 128; gla_seg.cu): the
+//     segmented arrangement on tcgen05 with hi / lo split factored operands.  Chunks whose
+//     gates are too small for the factored scores are flagged there, and gla_k3 in fix-up
+//     mode adds their exact intra-chunk part.
+//   CUDA cores (every other shape, or kernel_path LA_PATH_FMA; gla_k1, gla_k2, gla_k3):
+//     exact in float32 for any gates.  K3's scores factor as (q (.) 2^L) . (k (.) 2^-L) when
+//     the chunk's logs stay >= -100 (plain dot products), else take one exponential per
+//     (pair, feature).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -53,6 +57,9 @@ struct GlaParams {
   float* rec;    // [BH][NC][R]
   const float* S_init;
   float* S_final;
+  // Fix-up mode of gla_k3: [BH][NC] flags; only flagged chunks run, they compute the
+  // intra-chunk part alone and add it to `out` (which holds the prefix part).
+  const unsigned char* steep;
 };
 
 __device__ __forceinline__ int chunk_len(const GlaParams& p, int c) {
@@ -208,6 +215,8 @@ __global__ void gla_k2(GlaParams p) {
 // the prefix read out through the gates' running products.
 __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   extern __shared__ float sm[];
+  if (p.steep && !p.steep[blockIdx.x]) return;  // fix-up mode: flagged chunks only
+  const bool fix = p.steep != nullptr;
   const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
   const int C = p.C, dk = p.dk, dv = p.dv, L = chunk_len(p, c);
   const int lk = dk + 1;       // padded rows: threads of a warp read different rows
@@ -223,9 +232,12 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   load_rows(sK, lk, p.k, p.in_f32, rq, dk, C, L);
   load_rows(sV, dv, p.v, p.in_f32, (static_cast<long long>(bh) * p.T + t0) * dv, dv, C, L);
   load_gates(sL, lk, p.alpha, rq, dk, C, L);
-  const float4* P4 = reinterpret_cast<const float4*>(p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R);
-  for (int e = threadIdx.x; e < dk * dv / 4; e += blockDim.x)
-    reinterpret_cast<float4*>(sP)[e] = P4[e];
+  if (!fix) {
+    const float4* P4 =
+        reinterpret_cast<const float4*>(p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R);
+    for (int e = threadIdx.x; e < dk * dv / 4; e += blockDim.x)
+      reinterpret_cast<float4*>(sP)[e] = P4[e];
+  }
   __syncthreads();
   cum_log2(sL, lk, dk, L);
   __syncthreads();
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
   for (int tile = threadIdx.x; tile < tiles; tile += blockDim.x) {
     const int j0 = (tile / tiles_e) * 4, e0 = (tile % tiles_e) * 4;
     float acc[4][4] = {};
-    for (int f = 0; f < dk; ++f) {
+    for (int f = 0; f < (fix ? 0 : dk); ++f) {
       float a[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) a[u] = sQ[(j0 + u) * lk + f];
@@ -333,120 +345,22 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
       if (j0 + u >= L) continue;
       const long long o = (static_cast<long long>(bh) * p.T + t0 + j0 + u) * dv + e0;
       if (p.out_f32) {
-        *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) =
-            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + o);
+        if (fix) {
+          const float4 x = *dst;
+          acc[u][0] += x.x;
+          acc[u][1] += x.y;
+          acc[u][2] += x.z;
+          acc[u][3] += x.w;
+        }
+        *dst = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
       } else {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + o;
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-          static_cast<__nv_bfloat16*>(p.out)[o + w] = __float2bfloat16_rn(acc[u][w]);
+          dst[w] = __float2bfloat16_rn(fix ? acc[u][w] + __bfloat162float(dst[w]) : acc[u][w]);
       }
     }
-  }
-}
-
-// ---------------------------------------------------------------------------------------
-// Tensor-core path (opt-in).  With every cumulative log of a chunk >= -kGlaFactorBound the
-// chunk's weights factor exactly: 2^(L_j - L_i) = 2^(L_j) 2^(-L_i) and 2^(L_last - L_j), so
-// gated attention is the plain (undecayed, identity-map) prefill of pre-scaled inputs:
-//   q~ = q (.) 2^L,  k~ = k (.) 2^-L  (the combine: o_j = q~_j P_c + sum_{i<=j} (q~_j . k~_i) v_i)
-//   k^ = k (.) 2^(L_last - L)         (the summary S_loc = sum_j k^_j v_j^T)
-// which the prefill's tcgen05 kernels k1_tc / k3_tc compute; between them the carry over
-// chunks scales the prefix by a_c per key feature.  q~, k~, k^ are rounded to bf16 (the
-// kernels' operand type).  A chunk whose gates are too small to factor sets the device error
-// word (kErrGateRange) and its results are not valid: this path is for gates of moderate size
-// (for example all >= 0.34 at C = 64), the CUDA-core path for any gates.
-
-// One CTA per (b*H + h, chunk): cumulative log2 gates, the three scaled copies, a_c.
-__global__ void __launch_bounds__(256) gla_tc_prep(GlaParams p, __nv_bfloat16* qt,
-                                                    __nv_bfloat16* kt, __nv_bfloat16* kh,
-                                                    float* ac, int* err) {
-  extern __shared__ float sm[];
-  const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
-  const int C = p.C, dk = p.dk, L = chunk_len(p, c);
-  float* sA = sm;  // [C][dk]
-  const long long base = (static_cast<long long>(bh) * p.T + static_cast<long long>(c) * C) * dk;
-  load_gates(sA, dk, p.alpha, base, dk, C, L);
-  __syncthreads();
-  cum_log2(sA, dk, dk, L);
-  __syncthreads();
-  const int g8 = dk / 8;
-  for (int e = threadIdx.x; e < L * g8; e += blockDim.x) {
-    const int r = e / g8, f0 = (e - r * g8) * 8;
-    const long long i = base + static_cast<long long>(r) * dk + f0;
-    const uint4 uq = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + i);
-    const uint4 uk = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k) + i);
-    const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
-    uint32_t oq[4], ok[4], oh[4];
-    bool wide = false;
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      __nv_bfloat162 hq, hk;
-      std::memcpy(&hq, &wq[m], 4);
-      std::memcpy(&hk, &wk[m], 4);
-      const float2 fq = __bfloat1622float2(hq), fk = __bfloat1622float2(hk);
-      const int f = f0 + 2 * m;
-      const float l0 = sA[r * dk + f], l1 = sA[r * dk + f + 1];
-      const float e0 = sA[(L - 1) * dk + f], e1 = sA[(L - 1) * dk + f + 1];
-      wide = wide || l0 < -kGlaFactorBound || l1 < -kGlaFactorBound;
-      const __nv_bfloat162 rq = __float22bfloat162_rn(make_float2(fq.x * exp2f(l0), fq.y * exp2f(l1)));
-      const __nv_bfloat162 rk = __float22bfloat162_rn(make_float2(fk.x * exp2f(-l0), fk.y * exp2f(-l1)));
-      const __nv_bfloat162 rh =
-          __float22bfloat162_rn(make_float2(fk.x * exp2f(e0 - l0), fk.y * exp2f(e1 - l1)));
-      std::memcpy(&oq[m], &rq, 4);
-      std::memcpy(&ok[m], &rk, 4);
-      std::memcpy(&oh[m], &rh, 4);
-    }
-    if (wide) report_error(err, kErrGateRange);
-    *reinterpret_cast<uint4*>(qt + i) = make_uint4(oq[0], oq[1], oq[2], oq[3]);
-    *reinterpret_cast<uint4*>(kt + i) = make_uint4(ok[0], ok[1], ok[2], ok[3]);
-    *reinterpret_cast<uint4*>(kh + i) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-  }
-  for (int f = threadIdx.x; f < dk; f += blockDim.x)
-    ac[(static_cast<long long>(bh) * p.NC + c) * dk + f] = exp2f(sA[(L - 1) * dk + f]);
-}
-
-// The carry over chunks on the transposed records (S^T, [dv][dk] per chunk, as k1_tc writes
-// and k3_tc reads them): P^T[e][f] <- a_c[f] P^T[e][f] + S_c^T[e][f], exclusive, in place; one
-// thread per float4 of the state, eight chunks loaded ahead.  The state before chunk 0 is
-// S_init^T (or zero); the state after the last chunk goes to S_final ([dk][dv]).
-__global__ void gla_tc_k2(GlaParams p, const float* ac) {
-  const long long n4 = static_cast<long long>(p.dk) * p.dv / 4;
-  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long long>(p.BH) * n4) return;
-  const long long bh = idx / n4, col = idx - bh * n4;
-  const int e = static_cast<int>(col * 4 / p.dk), f4 = static_cast<int>(col * 4 % p.dk);
-  const long long sd = static_cast<long long>(p.dk) * p.dv;
-  float4 P = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (p.S_init) {
-    const float* S0 = p.S_init + bh * sd;
-    P = make_float4(S0[(f4 + 0) * p.dv + e], S0[(f4 + 1) * p.dv + e], S0[(f4 + 2) * p.dv + e],
-                    S0[(f4 + 3) * p.dv + e]);
-  }
-  float* base = p.rec + bh * p.NC * sd;
-  const float* abase = ac + bh * p.NC * p.dk + f4;
-  constexpr int kB = 16;
-  for (int c0 = 0; c0 < p.NC; c0 += kB) {
-    float4 x[kB], a[kB];
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      if (c0 + u >= p.NC) break;
-      x[u] = reinterpret_cast<const float4*>(base + static_cast<long long>(c0 + u) * sd)[col];
-      a[u] = *reinterpret_cast<const float4*>(abase + static_cast<long long>(c0 + u) * p.dk);
-    }
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      if (c0 + u >= p.NC) break;
-      reinterpret_cast<float4*>(base + static_cast<long long>(c0 + u) * sd)[col] = P;
-      P = make_float4(fmaf(a[u].x, P.x, x[u].x), fmaf(a[u].y, P.y, x[u].y),
-                      fmaf(a[u].z, P.z, x[u].z), fmaf(a[u].w, P.w, x[u].w));
-    }
-  }
-  if (p.S_final) {
-    float* Sf = p.S_final + bh * sd;
-    Sf[(f4 + 0) * p.dv + e] = P.x;
-    Sf[(f4 + 1) * p.dv + e] = P.y;
-    Sf[(f4 + 2) * p.dv + e] = P.z;
-    Sf[(f4 + 3) * p.dv + e] = P.w;
   }
 }
 
@@ -466,33 +380,37 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return a0 < b0 + bn && b0 < a0 + an;
 }
 
-// Workspace of either path.  CUDA cores: one record of dk*dv + dk floats per chunk.  Tensor
-// cores: q~, k~, k^ (bf16, the inputs' shape), a record of dk*dv floats per chunk and a_c.
+// Workspace of either path: one record of dk*dv + dk floats per chunk (the CUDA-core path's
+// chunk records; the tensor-core path's segment records, at most one per chunk), then one
+// byte per chunk (the tensor-core path's fix-up flags).
 struct GlaLayout {
-  size_t rec, qt, kt, kh, ac, total;
+  size_t rec, flags, total;
 };
 GlaLayout gla_layout(int B, int H, long long T, int dk, int dv, int C) {
   GlaLayout l{};
   if (B <= 0 || H <= 0 || T <= 0 || C <= 0) return l;
   const size_t BH = static_cast<size_t>(B) * H, NC = static_cast<size_t>((T + C - 1) / C);
-  const size_t fma = align256(BH * NC * (static_cast<size_t>(dk) * dv + dk) * 4);
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t o = off;
-    off = align256(off + bytes);
-    return o;
-  };
-  l.rec = take(BH * NC * static_cast<size_t>(dk) * dv * 4);
-  l.qt = take(BH * static_cast<size_t>(T) * dk * 2);
-  l.kt = take(BH * static_cast<size_t>(T) * dk * 2);
-  l.kh = take(BH * static_cast<size_t>(T) * dk * 2);
-  l.ac = take(BH * NC * dk * 4);
-  l.total = off > fma ? off : fma;
+  l.rec = 0;
+  l.flags = align256(BH * NC * (static_cast<size_t>(dk) * dv + dk) * 4);
+  l.total = l.flags + align256(BH * NC);
   return l;
 }
 
 size_t gla_ws(int B, int H, long long T, int dk, int dv, int C) {
   return gla_layout(B, H, T, dk, dv, C).total;
+}
+
+bool gla_tc_shape(const la_gla_args& a) {
+  return a.dtype == LA_DTYPE_BF16 && a.C == 64 && (a.dk == 64 || a.dk == 128) && a.dv == 128 &&
+         a.T < (1LL << 31);
+}
+
+bool gla_device_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  return major == 10;
 }
 
 int gla_validate(const la_gla_args& a) {
@@ -503,10 +421,8 @@ int gla_validate(const la_gla_args& a) {
   if (!gla_dims_ok(a.dk) || !gla_dims_ok(a.dv) || !(a.C == 16 || a.C == 32 || a.C == 64))
     return LA_ERR_UNSUPPORTED;
   if (a.kernel_path < LA_PATH_AUTO || a.kernel_path > LA_PATH_FMA) return LA_ERR_INVALID_ARGUMENT;
-  if (a.kernel_path == LA_PATH_TENSOR_CORE &&
-      !(a.dtype == LA_DTYPE_BF16 && a.C == 64 && (a.dk == 64 || a.dk == 128) &&
-        (a.dv == 64 || a.dv == 128) && a.T < (1LL << 31)))
-    return LA_ERR_UNSUPPORTED;
+  if (a.kernel_path == LA_PATH_TENSOR_CORE && !gla_tc_shape(a)) return LA_ERR_UNSUPPORTED;
+  if (a.segment_chunks < 0 || a.segment_chunks > 1024) return LA_ERR_INVALID_ARGUMENT;
   const long long BH = static_cast<long long>(a.B) * a.H;
   const long long NC = a.T > 0 ? (a.T + a.C - 1) / a.C : 0;
   if (BH * NC > (1LL << 31) - 1) return LA_ERR_UNSUPPORTED;
@@ -572,74 +488,59 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
   p.rec = reinterpret_cast<float*>(ws);
   p.S_init = a.S_init;
   p.S_final = a.S_final;
+  p.steep = nullptr;
 
-  if (a.kernel_path == LA_PATH_TENSOR_CORE) {
+  const bool tc = a.kernel_path != LA_PATH_FMA && gla_tc_shape(a) && gla_device_sm100();
+  if (a.kernel_path == LA_PATH_TENSOR_CORE && !tc) {
+    if (owned) cudaFreeAsync(ws, s);
+    return LA_ERR_UNSUPPORTED;
+  }
+  if (tc) {
     const GlaLayout l = gla_layout(a.B, a.H, a.T, a.dk, a.dv, a.C);
-    auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(ws + off); };
-    float* ac = reinterpret_cast<float*>(ws + l.ac);
-    p.rec = reinterpret_cast<float*>(ws + l.rec);
-    PrefillParams pp{};
-    pp.BH = p.BH;
-    pp.H = a.H;
-    pp.T = a.T;
-    pp.dk = a.dk;
-    pp.dv = a.dv;
-    pp.C = a.C;
-    pp.NC = p.NC;
-    pp.L_last = p.L_last;
-    pp.R = a.dk * a.dv;
-    pp.rec = p.rec;
-    pp.has_init = a.S_init != nullptr;
-    pp.Ls = 1;
-    pp.G = 1;
-    pp.err = device_error_word();
-    GammaTable gt;
-    for (int h = 0; h < kMaxHeads; ++h) gt.g[h] = 1.f;
-    const Flags fl{0, false, false, p.out_f32};
+    GlaSegParams sp{};
+    sp.BH = p.BH;
+    sp.T = a.T;
+    sp.dk = a.dk;
+    sp.NC = p.NC;
+    sp.L_last = p.L_last;
+    sp.Lseg = a.segment_chunks > 0 ? std::min(a.segment_chunks, p.NC)
+                                   : default_segment_chunks(BH, p.NC);
+    sp.NS = (p.NC + sp.Lseg - 1) / sp.Lseg;
+    sp.R = p.R;
+    sp.srec = reinterpret_cast<float*>(ws + l.rec);
+    sp.out = a.out;
+    sp.steep = ws + l.flags;
+    sp.has_init = a.S_init != nullptr;
+    sp.err = device_error_word();
     const uint64_t T = static_cast<uint64_t>(a.T), BHu = static_cast<uint64_t>(BH);
     const uint64_t dk = a.dk, dv = a.dv;
-    TcMaps m1, m3;
-    bool ok = make_tile_map(&m1.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.kh), dk, T, BHu, dk * 2,
-                            T * dk * 2, 64, 64) &&
-              make_tile_map(&m1.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, dv, T, BHu, dv * 2,
-                            T * dv * 2, 64, 64) &&
-              make_tile_map(&m1.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.rec, dk, dv,
-                            BHu * static_cast<uint64_t>(p.NC), dk * 4, dk * dv * 4, 32,
-                            static_cast<uint32_t>(dv));
-    m3 = m1;
-    ok = ok &&
-         make_tile_map(&m3.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.qt), dk, T, BHu, dk * 2,
-                       T * dk * 2, 64, 64) &&
-         make_tile_map(&m3.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, bf(l.kt), dk, T, BHu, dk * 2,
-                       T * dk * 2, 64, 64) &&
-         (p.out_f32 ? make_tile_map(&m3.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.out, dv, T, BHu,
-                                    dv * 4, T * dv * 4, 32, 64)
-                    : make_tile_map(&m3.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, dv, T, BHu,
-                                    dv * 2, T * dv * 2, 64, 64));
+    GlaSegMaps m;
+    const bool ok =
+        make_tile_map(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.q, dk, T, BHu, dk * 2, T * dk * 2,
+                      64, 64) &&
+        make_tile_map(&m.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.k, dk, T, BHu, dk * 2, T * dk * 2,
+                      64, 64) &&
+        make_tile_map(&m.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.v, dv, T, BHu, dv * 2, T * dv * 2,
+                      64, 64) &&
+        make_plain_map(&m.a, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.alpha, dk, T, BHu, dk * 4,
+                       T * dk * 4, static_cast<uint32_t>(dk), 64) &&
+        make_tile_map(&m.rec, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sp.srec, dk, dv,
+                      BHu * static_cast<uint64_t>(sp.NS), dk * 4, static_cast<uint64_t>(p.R) * 4,
+                      32, static_cast<uint32_t>(dv));
     cudaError_t e = ok ? cudaSuccess : cudaErrorInvalidValue;
-    const size_t sp = static_cast<size_t>(a.C) * a.dk * 4;
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gla_tc_prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(sp));
+    if (e == cudaSuccess) e = launch_gla_seg(sp, m, a.S_init, a.S_final, p.out_f32, s, rec);
+    // The exact intra-chunk part of the chunks the tensor-core combine flagged.
     if (e == cudaSuccess) {
-      if (rec) rec->mark(s, "gla_tc_prep");
-      gla_tc_prep<<<static_cast<unsigned>(BH * p.NC), 256, sp, s>>>(p, bf(l.qt), bf(l.kt),
-                                                                   bf(l.kh), ac, pp.err);
-      e = cudaGetLastError();
-    }
-    if (e == cudaSuccess) {
-      if (rec) rec->mark(s, "k1_tc");
-      e = launch_k1_tc(pp, gt, m1, fl, s);
-    }
-    if (e == cudaSuccess) {
-      const long long n = BH * a.dk * a.dv / 4;
-      if (rec) rec->mark(s, "gla_tc_k2");
-      gla_tc_k2<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p, ac);
-      e = cudaGetLastError();
-    }
-    if (e == cudaSuccess) {
-      if (rec) rec->mark(s, "k3_tc");
-      e = launch_k3_tc(pp, gt, m3, fl, s);
+      const size_t s3 = gla_smem_k3(a.C, a.dk, a.dv);
+      e = cudaFuncSetAttribute(gla_k3, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(s3));
+      GlaParams pf = p;
+      pf.steep = sp.steep;
+      if (e == cudaSuccess) {
+        if (rec) rec->mark(s, "gla_fixup");
+        gla_k3<<<static_cast<unsigned>(BH * p.NC), kGlaThreads, s3, s>>>(pf);
+        e = cudaGetLastError();
+      }
     }
     if (rec) rec->mark(s);
     if (owned) {

@@ -99,6 +99,25 @@ cudaError_t launch_k1_seg(const SegParams& sp, const GammaTable& gt, const TcMap
 cudaError_t launch_k3_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                           cudaStream_t s);
 
+// Gated linear attention on the tensor cores, segmented (gla_seg.cu): bf16 q, k, v,
+// float32 gates, C = 64, dk in {64, 128}, dv = 128.  K1 (segment folds), the scan over
+// segments (writes S_final), K3 (the combine; flags the chunks whose intra part the
+// CUDA-core fix-up must add).
+struct GlaSegMaps {
+  CUtensorMap q, k, v, a, rec;
+};
+cudaError_t launch_gla_seg(const GlaSegParams& sp, const GlaSegMaps& m, const float* S_init,
+                           float* S_final, bool out_f32, cudaStream_t s, Recorder* rec);
+
+// A 3D tiled TMA map without swizzle (d0 innermost), for float32 gate tiles.
+bool make_plain_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0,
+                    uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
+                    uint32_t box1);
+
+// Chunks per segment chosen automatically for BH heads of NC chunks (about four segments
+// per SM, at most 64 chunks each).
+int default_segment_chunks(long long BH, int NC);
+
 // One recurrent decode step for every (b, h).
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* out, float* S,
                           float* Z, int BH, int H, int dk, int dv, int dtype, Flags f,

@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
+#include "tile_util.cuh"
 
 namespace la {
 namespace {
@@ -38,49 +39,6 @@ namespace {
 constexpr int kC = 64;
 constexpr int kThreads = 256;  // 8 warps: two warps per TMEM lane quarter share its columns
 constexpr int kWarps = kThreads / 32;
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  const uint32_t a = smem_u32(p);
-  return p + ((1024u - (a & 1023u)) & 1023u);
-}
-
-__device__ __forceinline__ void unpack8(uint4 raw, float (&x)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(h[e]);
-    x[2 * e] = f.x;
-    x[2 * e + 1] = f.y;
-  }
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
-  uint4 raw;
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
-  return raw;
-}
-
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-  hi = pack8(x);
-  float h[8], r[8];
-  unpack8(hi, h);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) r[e] = x[e] - h[e];
-  lo = pack8(r);
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-// A shared-memory descriptor advanced by a byte offset: the start address field holds
-// address >> 4 in its low 14 bits and every operand of these kernels lies below 256 KB, so
-// the addition never carries out of the field.
-__device__ __forceinline__ uint64_t desc_at(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
-
 
 // ---------------------------------------------------------------------------------------
 // K1s, warp-specialised: one CTA per (b*H + h, segment).
@@ -382,11 +340,15 @@ struct K3sSmem {
 };
 
 
-template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV>
+template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV, int DVR>
 __global__ void __launch_bounds__(kThreads3, 1)
 k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
        const __grid_constant__ CUtensorMap tm_v, SegParams sp, GammaTable gt) {
+  // The MMAs run at dv = 128 (value features on the 128 TMEM lanes); a problem with
+  // DVR = 64 value features leaves the upper half of the V tile zero, so its lanes of the
+  // prefix, X and N stay zero and are never stored.
   constexpr int DV = 128;
+  static_assert(DVR == 64 || DVR == 128, "value features");
   using L_ = K3sSmem<DK, FM, DECAY, OUTF32>;
   constexpr bool kSplitQK = FM == 1;
   constexpr uint32_t kTmemCols = 512;
@@ -467,7 +429,16 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   }
   const float g64 = DECAY ? powf(g, static_cast<float>(kC)) : 1.f;
   if constexpr (NORM) {
-    if (tid < DK) sZP[tid] = srec[DK * DV + tid];
+    if (tid < DK) sZP[tid] = srec[DK * DVR + tid];
+  }
+  if constexpr (DVR < DV) {
+    // The V tiles' upper 64 value features: zero once, never loaded.
+    for (int e = tid; e < 2 * (kC * 128 / 16); e += kThreads3) {
+      const int st = e / (kC * 128 / 16), o = e % (kC * 128 / 16);
+      reinterpret_cast<uint4*>(base + st * L_::kStage + L_::kQ + L_::kK + kC * 128)[o] =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -516,7 +487,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         uint32_t u[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float4 f = src[q4 * 8 + e];
+          const float4 f = row < DVR ? src[q4 * 8 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
           u[4 * e] = __float_as_uint(f.x);
           u[4 * e + 1] = __float_as_uint(f.y);
           u[4 * e + 2] = __float_as_uint(f.z);
@@ -787,8 +758,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       const int t_hi = rev ? 32 : min(32, L - 32 * half);
 #pragma unroll
       for (int tt = 0; tt < 32; ++tt) {
-        if (tt >= t_lo && tt < t_hi) {
-          const long long idx = (row0 + tt) * DV + j;
+        if (tt >= t_lo && tt < t_hi && j < DVR) {
+          const long long idx = (row0 + tt) * DVR + j;
           if constexpr (OUTF32)
             __stcs(static_cast<float*>(sp.out) + idx, no[tt]);
           else
@@ -807,14 +778,14 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         uint8_t* sK = sQ + L_::kQ;
         uint8_t* sV = sK + L_::kK;
         const int t0 = rev ? static_cast<int>(sp.T) - (cb + i + 1) * kC : (cb + i) * kC;
-        mbar_arrive_expect_tx(&full[i & 1], L_::kStage);
+        mbar_arrive_expect_tx(&full[i & 1], L_::kQ + L_::kK + DVR * kC * 2);
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) {
           tma_load_3d(sQ + b * kC * 128, &tm_q, &full[i & 1], b * 64, t0, bh);
           tma_load_3d(sK + b * kC * 128, &tm_k, &full[i & 1], b * 64, t0, bh);
         }
 #pragma unroll
-        for (int b = 0; b < DV / 64; ++b)
+        for (int b = 0; b < DVR / 64; ++b)
           tma_load_3d(sV + b * kC * 128, &tm_v, &full[i & 1], b * 64, t0, bh);
         ++loads;
       }
@@ -948,7 +919,8 @@ cudaError_t k1s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
 
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV>
 cudaError_t k3s_go_r(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
-  auto kern = k3_seg<DK, FM, DECAY, NORM, OUTF32, REV>;
+  auto kern = sp.dv == 64 ? k3_seg<DK, FM, DECAY, NORM, OUTF32, REV, 64>
+                          : k3_seg<DK, FM, DECAY, NORM, OUTF32, REV, 128>;
   const uint32_t sm = K3sSmem<DK, FM, DECAY, OUTF32>::kTotal;
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
@@ -966,7 +938,6 @@ cudaError_t k3s_go_o(const SegParams& sp, const GammaTable& gt, const TcMaps& m,
 template <int DK, int DV, int FM, bool DECAY, bool NORM>
 cudaError_t k3s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                    cudaStream_t s) {
-  static_assert(DV == 128, "the segmented combine needs dv = 128");
   if constexpr (FM == 1 && DECAY) {
     return cudaErrorInvalidValue;  // excluded by seg_supported (shared memory budget)
   } else {
@@ -994,20 +965,23 @@ cudaError_t k3s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
 bool seg_supported(int dk, int dv, int C, int fm, bool decay) {
   // ELU+1 with decay needs both the psi lo tiles and the decayed key tiles double
   // buffered, which does not fit in shared memory next to the two stages.
-  return C == kC && (dk == 64 || dk == 128) && dv == 128 && !(fm == 1 && decay);
+  return C == kC && (dk == 64 || dk == 128) && (dv == 64 || dv == 128) && !(fm == 1 && decay);
 }
 
 cudaError_t launch_k1_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                           cudaStream_t s) {
   if (sp.dk == 64 && sp.dv == 128) LA_SEG_FLAGS(64, 128, k1s_go);
   if (sp.dk == 128 && sp.dv == 128) LA_SEG_FLAGS(128, 128, k1s_go);
+  if (sp.dk == 64 && sp.dv == 64) LA_SEG_FLAGS(64, 64, k1s_go);
+  if (sp.dk == 128 && sp.dv == 64) LA_SEG_FLAGS(128, 64, k1s_go);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_k3_seg(const SegParams& sp, const GammaTable& gt, const TcMaps& m, Flags f,
                           cudaStream_t s) {
-  if (sp.dk == 64 && sp.dv == 128) LA_SEG_FLAGS(64, 128, k3s_go);
-  if (sp.dk == 128 && sp.dv == 128) LA_SEG_FLAGS(128, 128, k3s_go);
+  // k3s_go_r picks the kernel for sp.dv (64 or 128); the MMA geometry is the same.
+  if (sp.dk == 64 && (sp.dv == 128 || sp.dv == 64)) LA_SEG_FLAGS(64, 128, k3s_go);
+  if (sp.dk == 128 && (sp.dv == 128 || sp.dv == 64)) LA_SEG_FLAGS(128, 128, k3s_go);
   return cudaErrorInvalidValue;
 }
 

@@ -386,20 +386,30 @@ size_t lin_attn_backward_workspace_bytes(const la_backward_args* args);
  *     S_t = (alpha_t 1^T) (.) S_{t-1} + k_t^T v_t,     o_t = q_t S_t,
  * S_{-1} = S_init (or zero), with a gate alpha_t[i] in [0, 1] per token and key feature
  * (no feature map, no normalisation, as on that page).  The scan page's three kernels with
- * the decayed monoid made per feature: K1 folds each chunk into (a_c, S_loc) with a_c the
- * product of the chunk's gates, K2 carries the exclusive prefix over chunks (P <- a_c (.) P +
- * S_loc, one thread per state element), K3 combines each chunk's intra part, whose score
- * for tokens i <= j weighs feature f by prod_{i<r<=j} alpha_r[f], with the prefix read out
- * through prod_{r<=j} alpha_r.  Gate products are formed as powers of two of cumulative
- * log2 gates, every exponent <= 0; a gate below 2^-126 counts as 2^-126.  CUDA-core fp32
- * kernels (the per-feature weights do not factor into one tensor-core product).
+ * the decayed monoid made per feature: (a1, S1) + (a2, S2) = (a1 a2, diag(a2) S1 + S2), a
+ * the product of the gates.  Within a chunk the score for tokens i <= j weighs feature f by
+ * prod_{i<r<=j} alpha_r[f], the prefix is read out through prod_{r<=j} alpha_r; gate
+ * products are powers of two of cumulative log2 gates (a gate below 2^-126 counts as
+ * 2^-126).  Two paths:
+ *   Tensor cores (default for bf16 inputs, C = 64, dk in {64, 128}, dv = 128 on sm_100):
+ *     the segmented arrangement.  Per segment of chunks a fold into (a_s, S_s), an exclusive
+ *     scan over segments, then a combine that walks each segment's chunks carrying the state
+ *     in TMEM.  The scores, the prefix product and the state update are tcgen05 MMAs on the
+ *     factored operands q (.) 2^(W+L) and k (.) 2^-(W+L) (a per-feature window offset W keeps
+ *     every factor within 2^60), each split into bf16 hi + lo, so products keep ~16 bits.
+ *     Chunks whose gates fall so fast that their own factors would leave that range (an
+ *     average gate below ~0.5 over the chunk in some feature) take an exact CUDA-core pass
+ *     for their intra-chunk scores.  Exact to float32 accumulation for any gates.
+ *   CUDA cores (every other shape, or kernel_path LA_PATH_FMA): per-chunk float32 kernels,
+ *     exact for any gates.
  *   q, k      DEVICE [B,H,T,dk], v DEVICE [B,H,T,dv], bf16 or float32 per `dtype`
  *   alpha     DEVICE float32 [B,H,T,dk]
  *   out       DEVICE [B,H,T,dv], type per out_dtype; must not overlap the inputs
  *   S_init    DEVICE float32 [B,H,dk,dv] or NULL;  S_final DEVICE float32 or NULL
  * Shapes: dk, dv multiples of 8 in [8, 128]; C in {16, 32, 64}; T >= 0.  Workspace:
- * lin_attn_gla_workspace_bytes() (one record of dk*dv + dk floats per chunk), or NULL to
- * allocate on the stream.  Asynchronous; arguments are checked before any launch.
+ * lin_attn_gla_workspace_bytes() (one record of dk*dv + dk floats and one byte per chunk),
+ * or NULL to allocate on the stream.  Asynchronous; arguments are checked before any
+ * launch.
  */
 typedef struct la_gla_args {
   const void* q;
@@ -417,20 +427,20 @@ typedef struct la_gla_args {
   void* workspace;        /* DEVICE, 256-byte aligned, or NULL */
   size_t workspace_bytes;
   la_stream_t stream;
-  /* la_kernel_path.  LA_PATH_AUTO / LA_PATH_FMA: the CUDA-core kernels above, exact for any
-   * gates.  LA_PATH_TENSOR_CORE (bf16, C = 64, dk, dv in {64, 128}): while every chunk's
-   * cumulative log2 gates stay >= -100 (for example all gates >= 0.34), the weights factor
-   * as 2^(L_j) 2^(-L_i), and the call runs the prefill's tcgen05 kernels on q (.) 2^L,
-   * k (.) 2^-L and k (.) 2^(L_last - L) (rounded to bf16), with the carry over chunks scaling
-   * the prefix per key feature.  A chunk outside that range sets the device error word to 4
-   * (lin_attn_device_error) and the call's results are not valid. */
+  /* la_kernel_path.  LA_PATH_AUTO: the tensor cores where their shape rule holds, else the
+   * CUDA cores.  LA_PATH_TENSOR_CORE: the tensor cores or LA_ERR_UNSUPPORTED.  LA_PATH_FMA:
+   * the CUDA cores. */
   int kernel_path;
+  /* Tensor-core path: chunks per segment, 0 to choose automatically (about four segments
+   * per SM, at most 64 chunks); at most 1024. */
+  int segment_chunks;
 } la_gla_args;
 
 int lin_attn_gla_prefill(const la_gla_args* args);
 size_t lin_attn_gla_workspace_bytes(int B, int H, long long T, int dk, int dv, int C);
-/* lin_attn_gla_prefill with a CUDA event around each of its three kernels; synchronises the
- * stream and writes their durations (ms: K1, K2, K3) to kernel_ms.  For profiling. */
+/* lin_attn_gla_prefill with a CUDA event around each of its kernels; synchronises the
+ * stream and writes their durations (ms, launch order: K1, K2, K3 on the CUDA cores;
+ * gla_k1_seg, gla_scan, gla_k3_seg, the fix-up on the tensor cores) to kernel_ms. */
 int lin_attn_gla_prefill_timed(const la_gla_args* args, float* kernel_ms, int max_kernels,
                                int* n_kernels);
 

@@ -391,17 +391,17 @@ def test_gla_argument_errors_before_any_launch(lib):
              (dict(workspace=0x100010), 1), (dict(q=0x1008), 1), (dict(alpha=0x6000004), 1),
              (dict(kernel_path=5), 1), (dict(kernel_path=1, dtype=1), 2),
              (dict(kernel_path=1, C=32), 2), (dict(kernel_path=1, dk=32), 2),
-             (dict(B=0), 0), (dict(H=0), 0)]
+             (dict(kernel_path=1, dv=64), 2), (dict(segment_chunks=-1), 1),
+             (dict(segment_chunks=1025), 1), (dict(B=0), 0), (dict(H=0), 0)]
     for kw, status in cases:
         assert lib.lin_attn_gla_prefill(ctypes.byref(args(**kw))) == status, kw
     assert lib.lin_attn_gla_prefill(None) == 1
-    # enough for either path: CUDA cores, one record of dk*dv + dk floats per chunk; tensor
-    # cores, a record of dk*dv floats per chunk, three bf16 copies of q / k, a_c
+    # enough for either path: one record of dk*dv + dk floats per chunk (the CUDA cores' chunk
+    # records, or the tensor cores' segment records, at most one per chunk), then one flag
+    # byte per chunk
     al = lambda x: (x + 255) // 256 * 256
     n = lib.lin_attn_gla_workspace_bytes(2, 3, 100, 64, 32, 64)
-    fma = al(2 * 3 * 2 * (64 * 32 + 64) * 4)
-    tc = al(2 * 3 * 2 * 64 * 32 * 4) + 3 * al(2 * 3 * 100 * 64 * 2) + al(2 * 3 * 2 * 64 * 4)
-    assert n == max(fma, tc)
+    assert n == al(2 * 3 * 2 * (64 * 32 + 64) * 4) + al(2 * 3 * 2)
 
 
 def test_header_is_plain_c_and_the_binding_structs_match_it(tmp_path):

@@ -1,8 +1,8 @@
 """GPU parity of gated linear attention (lin_attn_gla_prefill) against the oracle's token
 loop, element by element on the same inputs (bf16 inputs: the oracle gets the same
 bf16-rounded values; the gates are float32 on both sides).  Tolerances: max |err| <=
-2e-2 * rms(oracle) for bf16 inputs, 1e-4 * rms for float32 (the kernels are float32
-throughout, so both sit far inside)."""
+2e-2 * rms(oracle) for bf16 inputs (both paths), 1e-4 * rms for float32 inputs (CUDA
+cores)."""
 
 from __future__ import annotations
 
@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _problem(T, *, dk=128, dv=128, dtype="bf16", H=3, seed=0, mean=4.0, std=1.0):
+    """B2 H3 inputs N(0,1)/sqrt(dk) and gates sigmoid(N(mean, std)), CPU-drawn."""
     w = Workload("gla", B=2, H=H, T=T, dk=dk, dv=dv, C=64, dtype=dtype,
                  scale=1.0 / math.sqrt(dk), feature_map="identity", decay=False, normalize=False)
     q, k, v = make_inputs(w, seed=seed, device="cuda", gen_device="cpu")
@@ -99,13 +100,13 @@ def test_gla_zero_tokens_return_the_initial_state():
     assert torch.equal(S, S0)
 
 
-def test_gla_full_size_sampled_heads():
-    """The 128k-token gated workload (B=1, H=32, T=131072, d=128) in the benchmark's
-    configuration; the oracle recomputes heads 0 and 31 in full."""
+def test_gla_full_size_sampled_heads_cuda_cores():
+    """The 128k-token gated workload (B=1, H=32, T=131072, d=128) on the CUDA-core path;
+    the oracle recomputes heads 0 and 31 in full."""
     w = GLA_WORKLOADS["gla_128k"]
     q, k, v = make_inputs(w, seed=0, device="cuda")
     alpha = make_gates(w, seed=0, device="cuda")
-    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="fma")
     torch.cuda.synchronize()
     for h in (0, 31):
         sl = lambda t: t[:, h:h + 1]
@@ -115,56 +116,87 @@ def test_gla_full_size_sampled_heads():
 
 
 # ---------------------------------------------------------------------------------------
-# The tensor-core path (opt-in): gates whose chunk logs stay >= -100 factor exactly, but the
-# factored operands q (.) 2^L, k (.) 2^-L and k (.) 2^(L_last - L) are rounded to bf16 (the
-# prefill's identity-map kernels split no operand), so every product carries two bf16
-# roundings (2 * 2^-9 relative) where the retention path's exact bf16 inputs carry none.
-# Bound: 2^-4 * rms = 2 * 2^-9 per product times 16 for the maximum over ~10^6 outputs and
-# the few terms that average it when small gates shorten the memory.  Measured: up to
-# 1.4e-2 (gates sigmoid(N(4, 1))) and 3.3e-2 (sigmoid(N(3, 1)), d = 64).
-TOL_GLA_TC = 2.0 ** -4
+# The tensor-core path (the default for bf16, C = 64, dk in {64, 128}, dv = 128): segmented,
+# factored operands split into bf16 hi + lo, a renormalised window per feature, and the
+# exact CUDA-core fix-up for chunks whose gates fall too fast to factor.  Held to the same
+# 2e-2 rms bound as every bf16 path, against the oracle; the CUDA-core path beside it.
 
-@pytest.mark.parametrize("T", [65, 1000, 3001])
-def test_gla_tensor_core_path_matches_oracle(T):
-    q, k, v, alpha = _problem(T)
-    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+def _both_paths(q, k, v, alpha, S0=None, **kw):
+    out_t, S_t = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0, out_dtype="f32",
+                                        kernel_path="tensor_core", **kw)
+    out_f, S_f = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0, out_dtype="f32",
+                                        kernel_path="fma")
     torch.cuda.synchronize()
     assert B.lin_attn_device_error() == 0
+    return (out_t, S_t), (out_f, S_f)
+
+
+@pytest.mark.parametrize("dk", [64, 128])
+@pytest.mark.parametrize("mean,std", [(4.0, 1.0), (8.0, 1.0), (0.0, 2.0), (-3.0, 1.0), (2.0, 3.0)])
+@pytest.mark.parametrize("seg", [0, 1, 4, 7])
+def test_gla_tensor_core_path_gate_ranges(dk, mean, std, seg):
+    """Gates near 1 (long windows), moderate, wide, and small (every chunk takes the exact
+    fix-up); segments of 1, 4, 7 chunks and the automatic length; ragged T."""
+    q, k, v, alpha = _problem(1000, dk=dk, mean=mean, std=std, seed=seg)
+    (out, S), (out_f, S_f) = _both_paths(q, k, v, alpha, segment_chunks=seg)
     o_ref, S_ref = _oracle(q, k, v, alpha)
-    assert_close(to_np(out), o_ref, TOL_GLA_TC, "out")
-    assert_close(to_np(S), S_ref, TOL_GLA_TC, "S_final")
+    assert_close(to_np(out), o_ref, TOL_BF16, "out (tensor cores)")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final (tensor cores)")
+    assert_close(to_np(out_f), o_ref, TOL_BF16, "out (CUDA cores)")
+    assert_close(to_np(S_f), S_ref, TOL_BF16, "S_final (CUDA cores)")
 
 
-def test_gla_tensor_core_path_with_initial_state_and_d64():
-    q, k, v, alpha = _problem(1500, dk=64, dv=128, mean=3.0)
-    S0 = (torch.randn((2, 3, 64, 128), generator=torch.Generator().manual_seed(4)) * 0.3).cuda()
-    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, S_init=S0, out_dtype="f32",
-                                    kernel_path="tensor_core")
-    torch.cuda.synchronize()
-    assert B.lin_attn_device_error() == 0
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 129, 3001])
+def test_gla_tensor_core_path_lengths_and_initial_state(T):
+    q, k, v, alpha = _problem(T, mean=3.0)
+    S0 = (torch.randn((2, 3, 128, 128), generator=torch.Generator().manual_seed(T)) * 0.3).cuda()
+    (out, S), _ = _both_paths(q, k, v, alpha, S0, segment_chunks=3)
     o_ref, S_ref = _oracle(q, k, v, alpha, S0)
-    assert_close(to_np(out), o_ref, TOL_GLA_TC, "out")
-    assert_close(to_np(S), S_ref, TOL_GLA_TC, "S_final")
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
 
 
-def test_gla_tensor_core_path_flags_gates_it_cannot_factor():
-    # gates around 0.05: a chunk's cumulative log2 passes -100 within ~25 tokens
-    q, k, v, alpha = _problem(300, mean=-3.0)
-    B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+def test_gla_tensor_core_path_mixed_windows_and_zero_gates():
+    """One head's features decay at very different rates (a few near 0, most near 1), a
+    zero gate on every feature mid-sequence, and unit gates on half the features: windows,
+    rebases and steep chunks all occur within the same segments."""
+    q, k, v, alpha = _problem(2000, mean=5.0, seed=5)
+    alpha[:, :, :, :8] = torch.sigmoid(torch.randn_like(alpha[:, :, :, :8]) - 4.0)
+    alpha[:, :, 700] = 0.0
+    alpha[:, :, 1000:1500, 64:] = 1.0
+    (out, S), _ = _both_paths(q, k, v, alpha, segment_chunks=8)
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+def test_gla_tensor_core_path_bf16_output():
+    q, k, v, alpha = _problem(1000, mean=-1.0)
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, kernel_path="tensor_core", segment_chunks=4)
     torch.cuda.synchronize()
-    assert B.lin_attn_device_error() == 4  # reading it clears it
-    assert B.lin_attn_device_error() == 0
+    assert out.dtype == torch.bfloat16
+    o_ref, S_ref = _oracle(q, k, v, alpha)
+    got, ref = to_np(out).astype(np.float64), o_ref
+    assert float(np.max(np.abs(got - ref) - (2e-2 * np.sqrt(np.mean(ref ** 2)) + 2 ** -8 * np.abs(ref)))) <= 0
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+
+
+def test_gla_tensor_core_path_refuses_other_shapes():
+    q, k, v, alpha = _problem(100, dk=128, dv=64)
+    with pytest.raises(B.LinAttnError):
+        B.lin_attn_gla_prefill(q, k, v, alpha, kernel_path="tensor_core")
 
 
 def test_gla_tensor_core_path_full_size_sampled_heads():
+    """The 128k-token gated workload in the benchmark's configuration (the default path)."""
     w = GLA_WORKLOADS["gla_128k"]
     q, k, v = make_inputs(w, seed=0, device="cuda")
     alpha = make_gates(w, seed=0, device="cuda")
-    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32", kernel_path="tensor_core")
+    out, S = B.lin_attn_gla_prefill(q, k, v, alpha, out_dtype="f32")
     torch.cuda.synchronize()
     assert B.lin_attn_device_error() == 0
-    for h in (0, 31):
+    for h in (0, 17, 31):
         sl = lambda t: t[:, h:h + 1]
         o_ref, S_ref = _oracle(sl(q), sl(k), sl(v), sl(alpha))
-        assert_close(to_np(sl(out)), o_ref, TOL_GLA_TC, f"head {h} out")
-        assert_close(to_np(sl(S)), S_ref, TOL_GLA_TC, f"head {h} S_final")
+        assert_close(to_np(sl(out)), o_ref, TOL_BF16, f"head {h} out")
+        assert_close(to_np(sl(S)), S_ref, TOL_BF16, f"head {h} S_final")

@@ -62,11 +62,12 @@ def test_tensor_core_path(dk, dv, T, mode):
 @pytest.mark.parametrize("mode", sorted(MODES))
 @pytest.mark.parametrize("T,seg", [(1, 0), (64, 1), (100, 1), (257, 2), (1000, 3), (1000, 7),
                                    (1000, 16), (4485, 0), (4485, 5)])
-@pytest.mark.parametrize("dk", [64, 128])
-def test_segmented_path(dk, T, seg, mode):
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 128), (64, 64), (128, 64)])
+def test_segmented_path(dk, dv, T, seg, mode):
     """Segments of `seg` chunks (0 = automatic): the prefix carried through several chunks
-    inside a segment, segment prefixes from the scan, a ragged last chunk."""
-    w, q, k, v, gamma = _case(T, dk, 128, 64, mode)
+    inside a segment, segment prefixes from the scan, a ragged last chunk.  dv = 64 runs the
+    combine at 128 value lanes with the upper half of V zero."""
+    w, q, k, v, gamma = _case(T, dk, dv, 64, mode)
     if mode == "decay_norm":
         # ELU+1 with decay is not offered by the segmented kernels (shared memory); an
         # explicit request is refused and `auto` runs the chunked algorithm.
@@ -101,12 +102,13 @@ def test_fma_path_f32(T, dk, dv, C, mode):
 @pytest.mark.parametrize("path", ["tensor_core", "fma"])
 @pytest.mark.parametrize("T", [100, 1000])
 @pytest.mark.parametrize("algorithm", ["chunked", "segmented"])
-def test_bf16_output(T, path, mode, algorithm):
+@pytest.mark.parametrize("dv", [64, 128])
+def test_bf16_output(T, path, mode, algorithm, dv):
     if path == "fma" and algorithm == "segmented":
         pytest.skip("the segmented algorithm runs on the tensor-core kernels only")
     if mode == "decay_norm" and algorithm == "segmented":
         pytest.skip("ELU+1 with decay runs on the chunked algorithm only")
-    w, q, k, v, gamma = _case(T, 128, 128, 64, mode)
+    w, q, k, v, gamma = _case(T, 128, dv, 64, mode)
     out, S, Z = gpu_prefill(q, k, v, C=64, feature_map=w.feature_map, gamma=gamma,
                             normalize=w.normalize, kernel_path=path, out_dtype="as_input",
                             algorithm=algorithm, segment_chunks=3)
@@ -119,7 +121,7 @@ def test_bf16_output(T, path, mode, algorithm):
 
 @pytest.mark.parametrize("mode", ["norm", "retention"])
 @pytest.mark.parametrize("T", [100, 1000, 64 * 70 + 5])
-@pytest.mark.parametrize("dv,algorithm", [(64, "chunked"), (128, "segmented")])
+@pytest.mark.parametrize("dv,algorithm", [(64, "chunked"), (128, "segmented"), (64, "segmented")])
 def test_scan_modes_agree_with_oracle(T, mode, dv, algorithm):
     w, q, k, v, gamma = _case(T, 64, dv, 64, mode)
     for scan in ("logdepth", "sequential"):
