@@ -273,6 +273,18 @@ __device__ __forceinline__ void tmem_ld16x2_x16(uint32_t taddr, float (&r)[16]) 
       : "r"(taddr));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem] with 32-bit (tf32) operands; A holds one float per column
+// (row m in lane m, k in column k).
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

@@ -333,10 +333,11 @@ struct K3sSmem {
   static constexpr uint32_t kLo = FM == 1 ? kQ + kK : 0;  // lo tiles of psi(Q), psi(K)
   static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
+  static constexpr uint32_t kQf = FM == 0 ? kC * DK * 4 : 0;  // float32 copy of Q (tf32 X)
   static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC;
   static constexpr uint32_t kBars = 15;
   static constexpr uint32_t kTotal =
-      2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
+      2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kQf + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
 };
 
 
@@ -351,6 +352,14 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   static_assert(DVR == 64 || DVR == 128, "value features");
   using L_ = K3sSmem<DK, FM, DECAY, OUTF32>;
   constexpr bool kSplitQK = FM == 1;
+  // The unnormalised identity-map forward reads the prefix for X straight from its TMEM
+  // accumulator as a tf32 operand (Q copied to float32, exact for bf16 inputs), instead of
+  // splitting it into bf16 hi / lo every chunk: no per-chunk pass over the state.  tf32
+  // keeps 10 mantissa bits of P (error ~2^-11 relative per term, about 3e-3 of rms(o) at
+  // the largest of 10^8 outputs); the normalised form (whose bound is far tighter relative
+  // to its outputs, see the precision notes) and the backward's reversed passes keep the
+  // split.  Heads decaying faster than gamma ~ 0.52 (no renormalised window) keep it too.
+  constexpr bool kTf32X = FM == 0 && !NORM && !REV;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColS = 0, kColN = 128, kColP = 192;
   constexpr uint32_t kColPH = kColP + DK, kColPL = kColPH + DK / 2;
@@ -364,7 +373,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   uint8_t* sKpp = sLo + 2 * L_::kLo;         // [2] x (hi, lo)
   uint8_t* sAh = sKpp + 2 * L_::kKpp;
   uint8_t* sAl = sAh + L_::kA;
-  float* sZP = reinterpret_cast<float*>(sAl + L_::kA);
+  uint8_t* sQf = sAl + L_::kA;  // float32 copy of the chunk's Q (tf32 prefix product)
+  float* sZP = reinterpret_cast<float*>(sQf + L_::kQf);
   float* sZpart = sZP + DK;        // [8][DK]
   float* sDenX = sZpart + 8 * DK;  // [2][kC]
   float* sDen = sDenX + 2 * kC;
@@ -473,6 +483,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     if (W < 2) W = 1;
   }
   const bool renorm = W >= 2;
+  // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
+  const bool tf32x = kTf32X && (!DECAY || renorm);
 
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
@@ -612,6 +624,45 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         }
       }
 
+      if (tf32x) {
+        // tf32 prefix product: X reads P~ in place.  A window's first chunk turns P~ back
+        // into P first; then the chunk's Q goes to float32 (K-major, 128-byte swizzle, 32
+        // features per row) once the previous chunk's X has read the copy.
+        if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
+        tc_fence_after();
+        if (DECAY && i > 0 && i % W == 0) {
+          const float c_w = powf(g, static_cast<float>(kC * W));
+#pragma unroll
+          for (int q4 = 0; q4 < kHalf / 32; ++q4) {
+            const uint32_t col = pcol + q4 * 32;
+            float rr[32];
+            tmem_ld32(tmem + lane_base + kColP + col, rr);
+            tmem_ld_wait();
+            uint32_t u[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * c_w);
+            tmem_st32(tmem + lane_base + kColP + col, u);
+          }
+          tmem_st_wait();
+        }
+        for (int e = tw; e < kC * DK / 8; e += kXfThreads) {
+          const int r = e / (DK / 8), c8 = e % (DK / 8);
+          const uint4 raw =
+              *reinterpret_cast<const uint4*>(sQ + (c8 / 8) * (kC * 128) + sw128_offset(r, c8 % 8));
+          float x[8];
+          unpack8(raw, x);
+          const int f0 = c8 * 8;
+          uint8_t* dst = sQf + (f0 / 32) * (kC * 128);
+          *reinterpret_cast<float4*>(dst + sw128_offset(r, (f0 % 32) / 4)) =
+              make_float4(x[0], x[1], x[2], x[3]);
+          *reinterpret_cast<float4*>(dst + sw128_offset(r, (f0 % 32) / 4 + 1)) =
+              make_float4(x[4], x[5], x[6], x[7]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(pready);
+        continue;
+      }
       // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of
       // the key features.
       if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
@@ -810,6 +861,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     const uint64_t dKpm = smem_desc_sw128(kp0 + L_::kK, kC * 128, 1024);
     const uint64_t dAh = smem_desc_sw128(smem_u32(sAh), 16, 1024);
     const uint64_t dAl = smem_desc_sw128(smem_u32(sAl), 16, 1024);
+    const uint64_t dQf = smem_desc_sw128(smem_u32(sQf), 16, 1024);  // float32 Q, K-major
     constexpr uint32_t kStageD = L_::kStage >> 4, kLoD = L_::kLo >> 4, kKppD = L_::kKpp >> 4;
 
     auto issue_scores = [&](int i) -> bool {
@@ -844,7 +896,17 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       if (!wait(pready, i & 1, kErrMmaTimeout)) break;
       if (i > 1 && !wait(&xfree[s], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
       tc_fence_after();
-      if (has_prefix) {
+      if (tf32x) {
+        if (has_prefix) {
+          constexpr uint32_t idt = instr_desc(kFmtTF32, kFmtTF32, kKMajor, kKMajor, 128, 64);
+#pragma unroll
+          for (int kk = 0; kk < DK / 8; ++kk) {
+            const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
+            mma_tf32_ts(tmem + kColX[s], tmem + kColP + kk * 8, desc_at(dQf, off), idt,
+                        kk > 0 ? 1u : 0u);
+          }
+        }
+      } else if (has_prefix) {
         constexpr uint32_t idx = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 128, 64);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
