@@ -226,7 +226,7 @@ int to_status(cudaError_t e) {
   return LA_ERR_CUDA;
 }
 
-int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
+int prefill(const la_prefill_args& a, Recorder* rec = nullptr, bool exact_prefix = false) {
   Path path;
   int st = validate(a, &path);
   if (st != LA_OK) return st;
@@ -312,6 +312,7 @@ int prefill(const la_prefill_args& a, Recorder* rec = nullptr) {
     sp.out = a.out;
     sp.has_init = p.has_init;
     sp.reverse = a.reverse != 0;
+    sp.tf32_prefix = !exact_prefix;
     sp.err = p.err;
     const size_t srec_bytes = align256(static_cast<size_t>(BH) * NS * l.R * sizeof(float));
     PrefillParams ps = p;  // the scan over segments: one scan element per segment
@@ -441,7 +442,9 @@ HostLayout host_layout(const la_prefill_args& a) {
 
 }  // namespace
 
-int prefill_with_args(const la_prefill_args& a, Recorder* rec) { return prefill(a, rec); }
+int prefill_with_args(const la_prefill_args& a, Recorder* rec, bool exact_prefix) {
+  return prefill(a, rec, exact_prefix);
+}
 
 int* device_error_word() { return error_word_ptr(); }
 

@@ -797,7 +797,7 @@ int backward(const la_backward_args& a, Recorder* rec = nullptr) {
     if (st != LA_OK) return;
     p.workspace = at(l.pw);
     p.workspace_bytes = l.total - l.pw;
-    const int r = prefill_with_args(p, rec);
+    const int r = prefill_with_args(p, rec, /*exact_prefix=*/true);
     if (r != LA_OK) st = r == LA_ERR_INVALID_ARGUMENT || r == LA_ERR_UNSUPPORTED ? LA_ERR_INTERNAL : r;
   };
   // grad_q (or, for ELU+1, dpsi(q) in float32): (do, v, psi(k)) in order, identity map;

@@ -60,6 +60,7 @@ struct SegParams {
   bool has_init;   // segment 0 starts from a given state (its prefix is not zero)
   bool reverse;    // the sequence runs from token T - 1 down to token 0: chunk c covers
                    // tokens [T - 64 (c + 1), T - 64 c), its position p is token T-64c-1-p
+  bool tf32_prefix;  // the identity-map, unnormalised combine may read the prefix as tf32
   int* err;
 };
 

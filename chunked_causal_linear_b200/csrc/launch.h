@@ -53,7 +53,10 @@ struct Recorder {
 
 // The full prefill of lin_attn_prefill_ex (validation, workspace, launches), optionally
 // recording an event before every kernel.
-int prefill_with_args(const la_prefill_args& a, Recorder* rec = nullptr);
+// exact_prefix: keep the bf16 hi / lo split of the carried prefix in the combine even where
+// the forward reads it as tf32 (the backward's passes, whose sums cancel).
+int prefill_with_args(const la_prefill_args& a, Recorder* rec = nullptr,
+                      bool exact_prefix = false);
 
 // CUDA-core fp32 FMA kernels (any supported shape, float32 or bf16 inputs).
 cudaError_t launch_k1_fma(const PrefillParams& p, const GammaTable& gt, const void* k,

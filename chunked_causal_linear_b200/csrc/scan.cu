@@ -166,8 +166,10 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
 // Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of W = 1024 / NG
 // float4 columns: at least 128 contiguous bytes of every record); NG groups of E consecutive
 // elements (NG a power of two, NG * E >= N).
-template <bool DECAY>
-__global__ void __launch_bounds__(kBlockThreads, 1)
+// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 8 for long groups; 1 for groups
+// of one element, which keeps a thread within 32 registers (two CTAs per SM).
+template <bool DECAY, int U>
+__global__ void __launch_bounds__(kBlockThreads, U == 1 ? 2 : 1)
 k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   __shared__ float4 sX[kBlockThreads];
   __shared__ float sA[kBlockThreads];
@@ -189,13 +191,13 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   // Pass 1: this group's fold, agg = sum_e (decay after e within the group) x_e.
   float4 agg = make_float4(0.f, 0.f, 0.f, 0.f);
   if (live) {
-    for (int c0 = e0; c0 < e1; c0 += kUnroll) {
-      float4 x[kUnroll];
+    for (int c0 = e0; c0 < e1; c0 += U) {
+      float4 x[U];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
+      for (int u = 0; u < U; ++u)
         if (c0 + u < e1) x[u] = base[static_cast<long long>(c0 + u) * R4];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
+      for (int u = 0; u < U; ++u)
         if (c0 + u < e1) agg = axpy4(DECAY ? (c0 + u == p.NC - 1 ? aL : gC) : 1.f, agg, x[u]);
     }
   }
@@ -230,7 +232,7 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   if (gi > 0) carry = axpy4(sA[gi - 1], init, sX[(gi - 1) * kSlab + c8]);
   // Pass 2: exclusive prefixes of this group's elements, in place (re-read from L2, so
   // four loads in flight suffice and keep the thread within 64 registers).
-  carry = carry_in_place<DECAY, 4>(base, R4, e0, e1, p.NC - 1, gC, aL, carry);
+  carry = carry_in_place<DECAY, (U > 1 ? U / 2 : 1)>(base, R4, e0, e1, p.NC - 1, gC, aL, carry);
   if (e1 == p.NC) write_final(p, bh, col4 * 4, carry);
 }
 
@@ -261,8 +263,11 @@ cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_
   const int R4 = p.R / 4;
   const int W = kBlockThreads / bp.NG;
   const long long nslab = (R4 + W - 1) / W;
-  k2_block_scan<DECAY><<<static_cast<unsigned>(nslab * p.BH), kBlockThreads, 0, s>>>(
-      p, gt, bp.NG, bp.E);
+  const unsigned grid = static_cast<unsigned>(nslab * p.BH);
+  if (bp.E == 1)
+    k2_block_scan<DECAY, 1><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
+  else
+    k2_block_scan<DECAY, kUnroll><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   return cudaGetLastError();
 }
 

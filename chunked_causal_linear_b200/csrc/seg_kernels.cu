@@ -358,7 +358,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   // keeps 10 mantissa bits of P (error ~2^-11 relative per term, about 3e-3 of rms(o) at
   // the largest of 10^8 outputs); the normalised form (whose bound is far tighter relative
   // to its outputs, see the precision notes) and the backward's reversed passes keep the
-  // split.  Heads decaying faster than gamma ~ 0.52 (no renormalised window) keep it too.
+  // split, and so do the backward's passes (sp.tf32_prefix false: their sums cancel) and
+  // heads decaying faster than gamma ~ 0.52 (no renormalised window).
   constexpr bool kTf32X = FM == 0 && !NORM && !REV;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColS = 0, kColN = 128, kColP = 192;
@@ -484,7 +485,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   }
   const bool renorm = W >= 2;
   // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
-  const bool tf32x = kTf32X && (!DECAY || renorm);
+  const bool tf32x = kTf32X && sp.tf32_prefix && (!DECAY || renorm);
 
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
