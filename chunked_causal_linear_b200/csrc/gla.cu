@@ -213,11 +213,10 @@ __global__ void gla_k2(GlaParams p) {
 
 // K3: one CTA per (b*H + h, chunk): the intra-chunk part with per-feature gate ratios and
 // the prefix read out through the gates' running products.
-__global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
+__device__ __forceinline__ void gla_k3_chunk(const GlaParams& p, int id) {
   extern __shared__ float sm[];
-  if (p.steep && !p.steep[blockIdx.x]) return;  // fix-up mode: flagged chunks only
   const bool fix = p.steep != nullptr;
-  const int bh = static_cast<int>(blockIdx.x / p.NC), c = static_cast<int>(blockIdx.x % p.NC);
+  const int bh = id / p.NC, c = id % p.NC;
   const int C = p.C, dk = p.dk, dv = p.dv, L = chunk_len(p, c);
   const int lk = dk + 1;       // padded rows: threads of a warp read different rows
   float* sQ = sm;              // [C][lk]
@@ -361,6 +360,21 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
           dst[w] = __float2bfloat16_rn(fix ? acc[u][w] + __bfloat162float(dst[w]) : acc[u][w]);
       }
     }
+  }
+}
+
+// One CTA per chunk; in fix-up mode a grid of a few CTAs per SM walks every chunk and
+// takes the flagged ones (usually none), so that the common case costs one short launch.
+__global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
+  if (!p.steep) {
+    gla_k3_chunk(p, static_cast<int>(blockIdx.x));
+    return;
+  }
+  const int n = p.BH * p.NC;
+  for (int id = static_cast<int>(blockIdx.x); id < n; id += static_cast<int>(gridDim.x)) {
+    if (!p.steep[id]) continue;  // the same id for every thread of the CTA
+    gla_k3_chunk(p, id);
+    __syncthreads();  // the next flagged chunk reuses shared memory
   }
 }
 
@@ -538,7 +552,8 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
       pf.steep = sp.steep;
       if (e == cudaSuccess) {
         if (rec) rec->mark(s, "gla_fixup");
-        gla_k3<<<static_cast<unsigned>(BH * p.NC), kGlaThreads, s3, s>>>(pf);
+        const long long nf = std::min<long long>(BH * p.NC, 2 * 148);
+        gla_k3<<<static_cast<unsigned>(nf), kGlaThreads, s3, s>>>(pf);
         e = cudaGetLastError();
       }
     }

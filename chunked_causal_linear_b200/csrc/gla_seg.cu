@@ -144,15 +144,24 @@ __device__ __forceinline__ int chunk_mode(float* sW, const float* sLc, float* sB
   return mode;
 }
 
-// The factored operand of one 128B-swizzled bf16 tile (q or k) in place as hi, with lo
-// beside it: x (.) 2^(base + sign * L) for rows < L (zero past them).  Thread (cc, rg):
-// 8 consecutive features of rows rg, rg + RG, ...
+// The factored operand of one 128B-swizzled bf16 tile (q or k): x (.) 2^(base + sign * L) for
+// rows < L (zero past them), split into bf16 hi, written in place, and lo, returned in `lo`
+// (kRows x uint4) for factor_tile_store_lo once every thread has read the gate tile.
+// Thread (cc, rg): 8 consecutive features of rows rg, rg + RG, ...
+template <int DK>
+struct FactorShape {
+  static constexpr int NCC = DK / 8;
+  static constexpr int RG = kXf / NCC;
+  static constexpr int kRows = kC / RG;
+};
+
 template <int DK, int SIGN>
-__device__ __forceinline__ void factor_tile(uint8_t* tile, uint8_t* lo, const float* sA,
-                                            const float* sBase, int tw, int L) {
-  constexpr int NCC = DK / 8;
-  constexpr int RG = kXf / NCC;
-  constexpr int kRows = kC / RG;
+__device__ __forceinline__ void factor_tile(uint8_t* tile, const float* sA, const float* sBase,
+                                            int tw, int L,
+                                            uint4 (&lo)[FactorShape<DK>::kRows]) {
+  constexpr int NCC = FactorShape<DK>::NCC;
+  constexpr int RG = FactorShape<DK>::RG;
+  constexpr int kRows = FactorShape<DK>::kRows;
   const int cc = tw % NCC, rg = tw / NCC;
   const uint32_t boff = (cc / 8) * (kC * 128);
   float base[8];
@@ -173,32 +182,45 @@ __device__ __forceinline__ void factor_tile(uint8_t* tile, uint8_t* lo, const fl
 #pragma unroll
     for (int e = 0; e < 8; ++e)
       x[e] = r < L ? x[e] * exp2f(base[e] + static_cast<float>(SIGN) * lv[e]) : 0.f;
-    uint4 hi, l;
-    split8(x, hi, l);
-    const uint32_t off = boff + sw128_offset(r, cc % 8);
-    *reinterpret_cast<uint4*>(tile + off) = hi;
-    *reinterpret_cast<uint4*>(lo + off) = l;
+    uint4 hi;
+    split8(x, hi, lo[k]);
+    *reinterpret_cast<uint4*>(tile + boff + sw128_offset(r, cc % 8)) = hi;
   }
+}
+
+// The lo halves of factor_tile, into a tile of the same layout.
+template <int DK>
+__device__ __forceinline__ void factor_tile_store_lo(uint8_t* lo_tile, int tw,
+                                                     const uint4 (&lo)[FactorShape<DK>::kRows]) {
+  constexpr int NCC = FactorShape<DK>::NCC;
+  constexpr int RG = FactorShape<DK>::RG;
+  constexpr int kRows = FactorShape<DK>::kRows;
+  const int cc = tw % NCC, rg = tw / NCC;
+  const uint32_t boff = (cc / 8) * (kC * 128);
+#pragma unroll
+  for (int k = 0; k < kRows; ++k)
+    *reinterpret_cast<uint4*>(lo_tile + boff + sw128_offset(rg + k * RG, cc % 8)) = lo[k];
 }
 
 // ---------------------------------------------------------------------------------------
 // gla_k1_seg: one CTA per (b*H + h, segment), 320 threads.
 //   warps 0-7  transform: cumulative log gates, the chunk's mode, the key operand
-//              (hi in place, lo beside the stage); a rebase scales the accumulator in TMEM
-//              (after the previous chunk's MMAs); at the end the epilogue applies 2^W and
-//              stores the record.
-//   warp 8     producer: TMA loads of K, V, alpha into a two-stage ring.
+//              (hi in place, lo over the gate tile once every thread has read it); a rebase
+//              scales the accumulator in TMEM (after the previous chunk's MMAs); at the end
+//              the epilogue applies 2^W and stores the record.
+//   warp 8     producer: TMA loads of K, V, alpha into a three-stage ring.
 //   warp 9     MMA issuer: V^T K' into one TMEM accumulator (M = dv = 128, N = DK).
 
 constexpr int kThreadsK1 = 320;
-constexpr int kStagesK1 = 2;
+constexpr int kStagesK1 = 3;
 
 template <int DK>
 struct GK1Smem {
   static constexpr uint32_t kK = DK * kC * 2;
   static constexpr uint32_t kV = 128 * kC * 2;
   static constexpr uint32_t kG = kC * DK * 4;
-  static constexpr uint32_t kStage = kK + kV + kK + kG;  // K (hi in place), V, K lo, gates
+  // K (hi in place), V, the gate tile (cumulative logs, then the lo half of K)
+  static constexpr uint32_t kStage = kK + kV + kG;
   static constexpr uint32_t kIn = kStagesK1 * kStage;
   static constexpr uint32_t kS = DK * 128 * 4;  // staging of S^T, aliases the inputs
   static constexpr uint32_t kRegion = kIn > kS ? kIn : kS;
@@ -283,8 +305,8 @@ gla_k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
       const int st = i % kStagesK1;
       const int L = chunk_len(sp, cb + i);
       uint8_t* sK = base + st * L_::kStage;
-      uint8_t* sKl = sK + L_::kK + L_::kV;
-      float* sA = reinterpret_cast<float*>(sKl + L_::kK);
+      uint8_t* sKl = sK + L_::kK + L_::kV;  // the gate tile, reused for the lo half of K
+      float* sA = reinterpret_cast<float*>(sKl);
       wait(&full[st], (i / kStagesK1) & 1, kErrTmaTimeout);
       chunk_cumlog<DK>(sA, sTot, sLc, tw, L, false);
       const int mode = chunk_mode<DK>(sW, sLc, sBq, sBk, sScale, sScale2, sRed, tw, warp, lane);
@@ -311,7 +333,10 @@ gla_k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         tmem_st_wait();
         tc_fence_before();
       }
-      factor_tile<DK, -1>(sK, sKl, sA, sBk, tw, L);
+      uint4 klo[FactorShape<DK>::kRows];
+      factor_tile<DK, -1>(sK, sA, sBk, tw, L, klo);
+      named_barrier(1, kXf);  // every thread has read the gate tile
+      factor_tile_store_lo<DK>(sKl, tw, klo);
       fence_async_smem();
       mbar_arrive(&ops[st]);
     }
@@ -357,7 +382,7 @@ gla_k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
         if (i >= kStagesK1 && !wait(&empty[st], ((i / kStagesK1) - 1) & 1, kErrMmaTimeout)) break;
         uint8_t* sK = base + st * L_::kStage;
         uint8_t* sV = sK + L_::kK;
-        uint8_t* sA = sK + 2 * L_::kK + L_::kV;
+        uint8_t* sA = sV + L_::kV;
         const int t0 = (cb + i) * kC;
         mbar_arrive_expect_tx(&full[st], L_::kK + L_::kV + L_::kG);
 #pragma unroll
@@ -405,7 +430,8 @@ gla_k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 // gla_k3_seg: one CTA per (b*H + h, segment), 576 threads, the roles of the prefill's
 // segmented combine:
 //   warps 0-7   transform: cumulative log gates, the chunk's mode, the factored q~ and k~
-//               (hi in place over the staged tiles, lo beside them); then the prefix operand:
+//               (hi in place over the staged tiles, lo over the stage's gate tile once every
+//               thread has read it); then the prefix operand:
 //               P~ from TMEM -> (rebase: times 2^W) -> bf16 hi / lo into TMEM, and on a
 //               rebase the state written back for the chunk's update.
 //   warps 8-15  epilogue: causal mask of the scores into A (hi / lo), then o = X + N,
@@ -413,8 +439,7 @@ gla_k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUt
 //   warp 16     producer: TMA loads of Q, K, V and the gates into a two-stage ring.
 //   warp 17     MMA issuer: scores q~ k~^T, X = P~^T q~^T, P~ += V^T k~, N = V^T A^T.
 // TMEM columns: scores [0, 64), X [64, 128) and [448, 512), N [128, 192), P~ [192, 192 + DK),
-// its bf16 hi / lo after it.  At DK = 128 the lo tiles are single-buffered (shared memory),
-// so a chunk's operands are written once the previous chunk's MMAs are done.
+// its bf16 hi / lo after it.
 
 constexpr int kThreadsK3 = 576;
 constexpr int kEp = 256;  // epilogue threads, warps 8-15
@@ -426,14 +451,14 @@ struct GK3Smem {
   static constexpr uint32_t kK = DK * kC * 2;
   static constexpr uint32_t kV = DV * kC * 2;
   static constexpr uint32_t kG = kC * DK * 4;
+  // Q, K (hi in place), V, the gate tile (cumulative logs, then the lo halves of q~ and k~:
+  // kG = kQ + kK)
   static constexpr uint32_t kStage = kQ + kK + kV + kG;
-  static constexpr int kLoBufs = DK == 128 ? 1 : 2;
-  static constexpr uint32_t kLo = kQ + kK;  // lo tiles of q~, k~
+  static_assert(kG == kQ + kK, "the lo tiles fill the gate tile");
   static constexpr uint32_t kA = kC * kC * 2;
   static constexpr uint32_t kSmallFloats = 6 * DK + kXf + 16 + 4;
   static constexpr uint32_t kBars = 15;
-  static constexpr uint32_t kTotal =
-      2 * kStage + kLoBufs * kLo + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
+  static constexpr uint32_t kTotal = 2 * kStage + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
 };
 
 template <int DK, bool OUTF32>
@@ -443,7 +468,6 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
            GlaSegParams sp) {
   constexpr int DV = 128;
   using L_ = GK3Smem<DK>;
-  constexpr int kLoBufs = L_::kLoBufs;
   constexpr uint32_t kTmemCols = 512;
   constexpr uint32_t kColS = 0, kColN = 128, kColP = 192;
   constexpr uint32_t kColPH = kColP + DK, kColPL = kColPH + DK / 2;
@@ -453,8 +477,7 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
-  uint8_t* sLo = base + 2 * L_::kStage;  // [kLoBufs] x (q~ lo, k~ lo)
-  uint8_t* sAh = sLo + kLoBufs * L_::kLo;
+  uint8_t* sAh = base + 2 * L_::kStage;
   uint8_t* sAl = sAh + L_::kA;
   float* sW = reinterpret_cast<float*>(sAl + L_::kA);
   float* sLc = sW + DK;
@@ -556,20 +579,25 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       const bool last = i == n - 1;
       uint8_t* sQ = base + s * L_::kStage;
       uint8_t* sK = sQ + L_::kQ;
-      float* sA = reinterpret_cast<float*>(sK + L_::kK + L_::kV);
-      uint8_t* sQl = sLo + (kLoBufs == 1 ? 0 : s) * L_::kLo;
+      uint8_t* sQl = sK + L_::kK + L_::kV;  // the gate tile, reused for the lo halves
       uint8_t* sKl = sQl + L_::kQ;
+      float* sA = reinterpret_cast<float*>(sQl);
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
       chunk_cumlog<DK>(sA, sTot, sLc, tw, L, false);
       const int mode = chunk_mode<DK>(sW, sLc, sBq, sBk, sScale, sScale2, sRed, tw, warp, lane);
       if (tw == 0) sMode[s] = mode;
-      // Every MMA of the previous chunk is done (the lo tiles are free, and the state is
-      // final before the prefix pass below).
-      if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
-      factor_tile<DK, 1>(sQ, sQl, sA, sBq, tw, L);
-      factor_tile<DK, -1>(sK, sKl, sA, sBk, tw, L);
+      {
+        uint4 qlo[FactorShape<DK>::kRows], klo[FactorShape<DK>::kRows];
+        factor_tile<DK, 1>(sQ, sA, sBq, tw, L, qlo);
+        factor_tile<DK, -1>(sK, sA, sBk, tw, L, klo);
+        named_barrier(1, kXf);  // every thread has read the gate tile
+        factor_tile_store_lo<DK>(sQl, tw, qlo);
+        factor_tile_store_lo<DK>(sKl, tw, klo);
+      }
       fence_async_smem();
       mbar_arrive(&ops[s]);
+      // The state is final before the prefix pass (the previous chunk's MMAs are done).
+      if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
 
       // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of the
       // key features: P = P~ 2^W on a rebase (and, for the chunk's update, times 2^(L_last)
@@ -708,13 +736,13 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     const uint64_t dKk = smem_desc_sw128(a0 + L_::kQ, 16, 1024);                 // k~, K-major
     const uint64_t dKm = smem_desc_sw128(a0 + L_::kQ, kC * 128, 1024);           // k~, MN-major
     const uint64_t dVm = smem_desc_sw128(a0 + L_::kQ + L_::kK, kC * 128, 1024);  // V, MN-major
-    const uint32_t lo0 = smem_u32(sLo);
+    const uint32_t lo0 = a0 + L_::kQ + L_::kK + L_::kV;  // stage 0's gate tile: q~ lo, k~ lo
     const uint64_t dQlk = smem_desc_sw128(lo0, 16, 1024);
     const uint64_t dKlk = smem_desc_sw128(lo0 + L_::kQ, 16, 1024);
     const uint64_t dKlm = smem_desc_sw128(lo0 + L_::kQ, kC * 128, 1024);
     const uint64_t dAh = smem_desc_sw128(smem_u32(sAh), 16, 1024);
     const uint64_t dAl = smem_desc_sw128(smem_u32(sAl), 16, 1024);
-    constexpr uint32_t kStageD = L_::kStage >> 4, kLoD = kLoBufs == 1 ? 0 : (L_::kLo >> 4);
+    constexpr uint32_t kStageD = L_::kStage >> 4, kLoD = kStageD;
 
     auto issue_scores = [&](int i) -> bool {
       const int s = i & 1;
