@@ -267,7 +267,9 @@ int lin_attn_combine_states(const float* S_parts, const float* Z_parts, int part
  *   - A problem whose workspace (lin_attn_prefill_workspace_bytes) exceeds
  *     LA_NOALLOC_SCRATCH_BYTES returns LA_ERR_UNSUPPORTED and launches nothing.
  *   - The first call on each device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *     device current) and keeps it; make that first call before any stream capture, and
+ *     do not use this entry point across a reset of the device (cudaDeviceReset), which
+ *     would leave the kept address stale.
  *   - Every call shares the array and it keeps the last call's contents; the kernels
  *     write all workspace bytes before reading them, so no clearing is needed.  Calls
  *     whose work overlaps on the GPU race on the array: serialise them.

@@ -309,8 +309,10 @@ void gla_pair(const GlaProblem& p, long long bh) {
 //   dk_t[i] = sum_j G_t[i][j] v_t[j],  dv_t[j] = sum_i G_t[i][j] k_t[i]
 //   dalpha_t[i] = sum_j G_t[i][j] S_{t-1}[i][j],  dS_init = diag(alpha_0) G_0
 // The reverse sweep needs S_{t-1}: the forward sweep keeps S every kGlaCheck tokens and each
-// block is recomputed from its checkpoint.
-constexpr long long kGlaCheck = 64;
+// block is recomputed from its checkpoint.  kGlaCheck is about sqrt(T) (at least 64), so the
+// checkpoints and one block's states take O(sqrt(T) dk dv) memory per thread; the values are
+// the same for any interval (the recomputation repeats the forward sweep's operations).
+constexpr long long kGlaCheckMin = 64;
 
 struct GlaBackwardProblem {
   const float* q;
@@ -338,6 +340,8 @@ void gla_backward_pair(const GlaBackwardProblem& p, long long bh) {
   const float* v = p.v + bh * T * dv;
   const float* al = p.alpha + bh * T * dk;
   const double* dout = p.dout + bh * T * dv;
+  const long long kGlaCheck = std::max<long long>(
+      kGlaCheckMin, static_cast<long long>(std::ceil(std::sqrt(static_cast<double>(T)))));
   auto step = [&](std::vector<double>& S, long long t) {  // S_{t-1} -> S_t
     for (int i = 0; i < dk; ++i) {
       const double gate = static_cast<double>(al[t * dk + i]), ki = static_cast<double>(k[t * dk + i]);

@@ -3,8 +3,8 @@
 Checked against: central finite differences of the oracle's own gated forward (every input,
 the gates included); float64 autograd through a brute-force parallel form built from products
 of the gates; and, for gates constant per head, the retention backward (the oracle's pinned
-la_oracle_backward).  The reverse sweep recomputes S from checkpoints every 64 tokens, so the
-sequences here cross block boundaries.  Planted mistakes must each fail a pin.
+la_oracle_backward).  The reverse sweep recomputes S from checkpoints every max(64,
+ceil(sqrt(T))) tokens, so the sequences here cross block boundaries.  Planted mistakes must each fail a pin.
 """
 
 from __future__ import annotations
@@ -113,6 +113,20 @@ def _pins(o: Oracle) -> dict[str, bool]:
     res["constant_gates_are_retention"] = all(_rel(x, y) < 1e-11 for x, y in
                                               zip((g_gla[0], g_gla[1], g_gla[2], g_gla[4]), g_ret[:4]))
     return res
+
+
+def test_gla_backward_long_sequence_crosses_many_checkpoints():
+    """T = 4500: the checkpoint interval is ceil(sqrt(T)) = 68 tokens, so the reverse sweep
+    recomputes 67 blocks; with gates constant per head the gradients must equal the retention
+    backward's (the oracle's separately pinned la_oracle_backward)."""
+    o = default_oracle()
+    q, k, v, a, do, S0, dSf = _problem(7, T=4500)
+    gam = [float(np.float32(0.999)), float(np.float32(0.97))]
+    ac = np.broadcast_to(np.asarray(gam, dtype=np.float32)[None, :, None, None], a.shape).copy()
+    g_gla = o.gla_backward(q, k, v, ac, do, S_init=S0, dS_final=dSf)
+    g_ret = o.backward(q, k, v, do, feature_map="identity", gamma=gam, S_init=S0, dS_final=dSf)
+    for x, y in zip((g_gla[0], g_gla[1], g_gla[2], g_gla[4]), g_ret[:4]):
+        assert _rel(x, y) < 1e-10
 
 
 def test_gla_backward_pins_hold():
