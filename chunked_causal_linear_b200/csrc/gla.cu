@@ -370,11 +370,21 @@ __global__ void __launch_bounds__(kGlaThreads) gla_k3(GlaParams p) {
     gla_k3_chunk(p, static_cast<int>(blockIdx.x));
     return;
   }
+  // The flags of kGlaThreads chunks at a time, read by all threads at once.
+  __shared__ unsigned char s_flag[kGlaThreads];
   const int n = p.BH * p.NC;
-  for (int id = static_cast<int>(blockIdx.x); id < n; id += static_cast<int>(gridDim.x)) {
-    if (!p.steep[id]) continue;  // the same id for every thread of the CTA
-    gla_k3_chunk(p, id);
-    __syncthreads();  // the next flagged chunk reuses shared memory
+  for (int b0 = static_cast<int>(blockIdx.x) * kGlaThreads; b0 < n;
+       b0 += static_cast<int>(gridDim.x) * kGlaThreads) {
+    const int my = b0 + static_cast<int>(threadIdx.x);
+    const unsigned char f = my < n ? p.steep[my] : 0;
+    s_flag[threadIdx.x] = f;
+    if (!__syncthreads_or(f)) continue;
+    for (int j = 0; j < kGlaThreads && b0 + j < n; ++j) {
+      if (!s_flag[j]) continue;  // the same j for every thread of the CTA
+      gla_k3_chunk(p, b0 + j);
+      __syncthreads();  // the next flagged chunk reuses shared memory
+    }
+    __syncthreads();  // s_flag is rewritten next round
   }
 }
 
@@ -552,7 +562,7 @@ int gla_prefill(const la_gla_args& a, Recorder* rec) {
       pf.steep = sp.steep;
       if (e == cudaSuccess) {
         if (rec) rec->mark(s, "gla_fixup");
-        const long long nf = std::min<long long>(BH * p.NC, 2 * 148);
+        const long long nf = std::min<long long>((BH * p.NC + kGlaThreads - 1) / kGlaThreads, 2 * 148);
         gla_k3<<<static_cast<unsigned>(nf), kGlaThreads, s3, s>>>(pf);
         e = cudaGetLastError();
       }

@@ -166,10 +166,12 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
 // Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of W = 1024 / NG
 // float4 columns: at least 128 contiguous bytes of every record); NG groups of E consecutive
 // elements (NG a power of two, NG * E >= N).
-// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 8 for long groups; 1 for groups
-// of one element, which keeps a thread within 32 registers (two CTAs per SM).
+// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 4 for longer groups, 1 for groups
+// of one element.  Either keeps a thread within 32 registers: two CTAs per SM, so that one
+// CTA's loads overlap the other's Hillis-Steele rounds and stores (one CTA of 1024 threads
+// per SM left DRAM half idle: measured 50 % of its peak, warps 48 % active).
 template <bool DECAY, int U>
-__global__ void __launch_bounds__(kBlockThreads, U == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kBlockThreads, 2)
 k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   __shared__ float4 sX[kBlockThreads];
   __shared__ float sA[kBlockThreads];
@@ -267,7 +269,7 @@ cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_
   if (bp.E == 1)
     k2_block_scan<DECAY, 1><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   else
-    k2_block_scan<DECAY, kUnroll><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
+    k2_block_scan<DECAY, 4><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   return cudaGetLastError();
 }
 

@@ -765,7 +765,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         named_barrier(2, kEpThreads);
         if (tw < kC) {
           const float den_loc = sDenPart[tw] + sDenPart[kC + tw];
-          sDen[tw] = (has_prefix ? fmaf(sTh[tw], sDenX[s * kC + tw], den_loc) : den_loc) + sp.eps;
+          // The reciprocal, so that the 32 outputs of a thread take multiplications.
+          sDen[tw] = 1.f / ((has_prefix ? fmaf(sTh[tw], sDenX[s * kC + tw], den_loc) : den_loc) + sp.eps);
         }
       }
       mbar_arrive(aready);
@@ -798,10 +799,10 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 dn = *reinterpret_cast<const float4*>(sDen + 32 * half + 4 * q);
-          no[4 * q] /= dn.x;
-          no[4 * q + 1] /= dn.y;
-          no[4 * q + 2] /= dn.z;
-          no[4 * q + 3] /= dn.w;
+          no[4 * q] *= dn.x;
+          no[4 * q + 1] *= dn.y;
+          no[4 * q + 2] *= dn.z;
+          no[4 * q + 3] *= dn.w;
         }
       }
       const long long row0 = static_cast<long long>(bh) * sp.T + t0 + 32 * half;
