@@ -52,14 +52,23 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 K2_NAMES = {"logdepth": ["k2_reduce", "k2_block_scan", "k2_downsweep"],
             "sequential": ["k2_sequential"]}
 SCAN_BLOCK_ELEMS = 2048  # the log-depth scan's one-level limit (lin_attn_scan_plan)
-KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k2_reduce": "scan.cu",
+KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k1_fma": "fma_kernels.cu",
+                  "k3_fma": "fma_kernels.cu", "k2_reduce": "scan.cu",
                   "k2_block_scan": "scan.cu", "k2_downsweep": "scan.cu",
                   "k2_sequential": "scan.cu", "k1_seg": "seg_kernels.cu",
                   "k3_seg": "seg_kernels.cu"}
 
 
+def kernel_path_for(w) -> str:
+    """The kernels a workload runs on: the tensor cores for bf16 inputs, the CUDA-core FMA
+    kernels for float32 inputs (the small float32 workload)."""
+    return "fma" if w.dtype == "f32" else "tensor_core"
+
+
 def effective_algorithm(w, requested: str) -> str:
-    """The algorithm the library runs for this workload on the tensor-core path."""
+    """The algorithm the library runs for this workload (the FMA kernels are chunked)."""
+    if kernel_path_for(w) == "fma":
+        return "chunked"
     seg_ok = (w.dtype == "bf16" and w.C == 64 and w.dk in (64, 128) and w.dv in (64, 128)
               and not (w.feature_map == "elu1" and w.decay))
     if requested == "segmented" or (requested == "auto" and seg_ok):
@@ -69,6 +78,8 @@ def effective_algorithm(w, requested: str) -> str:
 
 def kernel_names(w, algo: str, scan: str, lseg: int = 0) -> list[str]:
     k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
+    if kernel_path_for(w) == "fma":
+        k1, k3 = "k1_fma", "k3_fma"
     n, _, _ = layout(w, algo, lseg)
     k2 = ["k2_block_scan"] if scan == "logdepth" and n <= SCAN_BLOCK_ELEMS else K2_NAMES[scan]
     return [k1, *k2, k3]
@@ -119,7 +130,7 @@ def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked", lseg: int =
         return 2 * rec + BH * G * R * 4
     if name == "k2_sequential":
         return 2 * rec + BH * R * 4
-    if name == "k3_tc":
+    if name in ("k3_tc", "k3_fma"):
         return BH * w.T * (2 * w.dk + w.dv) * e_in + BH * (n - 1) * R * 4 + BH * w.T * w.dv * out_elem
     if name == "k3_seg":
         return BH * w.T * (2 * w.dk + w.dv) * e_in + rec + BH * w.T * w.dv * out_elem
@@ -916,7 +927,9 @@ def config_of(w, args):
             "algorithm": effective_algorithm(w, args.algorithm),
             **({"segment_chunks": segment_length(w, getattr(args, "segment_chunks", 0))}
                if effective_algorithm(w, args.algorithm) == "segmented" else {}),
-            "kernel_path": "tensor_core", "l2": "inputs larger than L2, no flush",
+            "kernel_path": kernel_path_for(w),
+            "l2": "inputs larger than L2, no flush" if w.B * w.H * w.T * (2 * w.dk + w.dv)
+            * (2 if w.dtype == "bf16" else 4) > 126e6 else "inputs fit in L2 (latency case)",
             "scan_depth": scan_depth(w, args),
             "parallelism": "replicas (one independent problem per GPU)"}
 
@@ -1019,7 +1032,7 @@ def main():
     gam = w.gammas()
     algo = effective_algorithm(w, args.algorithm)
     kw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
-              scan=args.scan, kernel_path="tensor_core", workspace=ws, out_dtype=args.out_dtype,
+              scan=args.scan, kernel_path=kernel_path_for(w), workspace=ws, out_dtype=args.out_dtype,
               algorithm=algo, segment_chunks=args.segment_chunks)
 
     def step():
@@ -1089,7 +1102,7 @@ def main():
         Sh = torch.empty(S.shape, dtype=torch.float32).pin_memory()
         Zh = torch.empty(Z.shape, dtype=torch.float32).pin_memory() if Z is not None else None
         hkw = dict(chunk=w.C, feature_map=w.feature_map, gamma=gam, normalize=w.normalize,
-                   scan=args.scan, kernel_path="tensor_core", out_dtype=args.out_dtype,
+                   scan=args.scan, kernel_path=kernel_path_for(w), out_dtype=args.out_dtype,
                    algorithm=algo)
         dbuf = torch.empty(B.lin_attn_prefill_host_buffer_bytes(qh, vh, chunk=w.C,
                                                                 normalize=w.normalize,
@@ -1123,7 +1136,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32",
             "data": "synthetic", "config": config_of(w, args), "roofline": roofline,
             "step_roofline": step_roof, "kernels_ms": kern_ms, "cpu_baseline": cpu,
             "e2e": e2e, "clocks": clocks, "remeasured": remeasured,

@@ -166,15 +166,15 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
 // Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of W = 1024 / NG
 // float4 columns: at least 128 contiguous bytes of every record); NG groups of E consecutive
 // elements (NG a power of two, NG * E >= N).
-// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 4 for longer groups, 1 for groups
-// of one element.  Either keeps a thread within 32 registers: two CTAs per SM, so that one
-// CTA's loads overlap the other's Hillis-Steele rounds and stores (one CTA of 1024 threads
-// per SM left DRAM half idle: measured 50 % of its peak, warps 48 % active).
+// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 8 for longer groups (64
+// registers, one CTA per SM; two CTAs of 32 registers measured slower), 1 for groups of one
+// element (32 registers, two CTAs per SM).
 template <bool DECAY, int U>
-__global__ void __launch_bounds__(kBlockThreads, 2)
+__global__ void __launch_bounds__(kBlockThreads, U == 1 ? 2 : 1)
 k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   __shared__ float4 sX[kBlockThreads];
   __shared__ float sA[kBlockThreads];
+  __shared__ float sG[2];
   const int kSlab = kBlockThreads / NG;  // W
   const int R4 = p.R / 4;
   const int nslab = (R4 + kSlab - 1) / kSlab;
@@ -183,15 +183,23 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   const int col4 = (blockIdx.x % nslab) * kSlab + c8;
   const int gi = threadIdx.x / kSlab;
   const bool live = col4 < R4;
-  const float g = DECAY ? gt.g[bh % p.H] : 1.f;
-  const float gC = DECAY ? powf(g, static_cast<float>(p.C)) : 1.f;
-  const float aL = DECAY ? powf(g, static_cast<float>(p.L_last)) : 1.f;
+  // The element decays gamma^C and gamma^(L_last), once per CTA.
+  if (DECAY && threadIdx.x == 0) {
+    const float g = gt.g[bh % p.H];
+    sG[0] = powf(g, static_cast<float>(p.C));
+    sG[1] = powf(g, static_cast<float>(p.L_last));
+  }
+  if (DECAY) __syncthreads();
+  const float gC = DECAY ? sG[0] : 1.f;
+  const float aL = DECAY ? sG[1] : 1.f;
   const int e0 = min(p.NC, gi * E);
   const int e1 = min(p.NC, e0 + E);
   float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) + col4;
 
-  // Pass 1: this group's fold, agg = sum_e (decay after e within the group) x_e.
+  // Pass 1: this group's fold, agg = sum_e (decay after e within the group) x_e, and the
+  // group's decay A, the product of its elements' decays.
   float4 agg = make_float4(0.f, 0.f, 0.f, 0.f);
+  float A = 1.f;
   if (live) {
     for (int c0 = e0; c0 < e1; c0 += U) {
       float4 x[U];
@@ -200,16 +208,12 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
         if (c0 + u < e1) x[u] = base[static_cast<long long>(c0 + u) * R4];
 #pragma unroll
       for (int u = 0; u < U; ++u)
-        if (c0 + u < e1) agg = axpy4(DECAY ? (c0 + u == p.NC - 1 ? aL : gC) : 1.f, agg, x[u]);
+        if (c0 + u < e1) {
+          const float a = DECAY ? (c0 + u == p.NC - 1 ? aL : gC) : 1.f;
+          agg = axpy4(a, agg, x[u]);
+          A *= a;
+        }
     }
-  }
-  // The group's decay: gamma^(tokens of its elements).
-  float A = 1.f;
-  if (DECAY && e1 > e0) {
-    const long long tokens = e1 == p.NC
-                                 ? static_cast<long long>(e1 - e0 - 1) * p.C + p.L_last
-                                 : static_cast<long long>(e1 - e0) * p.C;
-    A = powf(g, static_cast<float>(tokens));
   }
   // Hillis-Steele over the groups: after round r, group gi holds the fold of groups
   // gi - 2^(r+1) + 1 .. gi, and A their decay.
@@ -269,7 +273,7 @@ cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_
   if (bp.E == 1)
     k2_block_scan<DECAY, 1><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   else
-    k2_block_scan<DECAY, 4><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
+    k2_block_scan<DECAY, kUnroll><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   return cudaGetLastError();
 }
 
