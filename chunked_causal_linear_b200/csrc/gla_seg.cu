@@ -181,7 +181,7 @@ __device__ __forceinline__ void factor_tile(uint8_t* tile, const float* sA, cons
     unpack8(raw[k], x);
 #pragma unroll
     for (int e = 0; e < 8; ++e)
-      x[e] = r < L ? x[e] * exp2f(base[e] + static_cast<float>(SIGN) * lv[e]) : 0.f;
+      x[e] = r < L ? x[e] * exp2_approx(base[e] + static_cast<float>(SIGN) * lv[e]) : 0.f;
     uint4 hi;
     split8(x, hi, lo[k]);
     *reinterpret_cast<uint4*>(tile + boff + sw128_offset(r, cc % 8)) = hi;

@@ -333,6 +333,14 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 // ---------------------------------------------------------------------------------------
 // Small numeric helpers
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32: about 2^-22
+// relative; results below 2^-126 flush to zero, far below anything they multiply).
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // psi: ELU+1 (x + 1 for x > 0, e^x otherwise; the fast exponential, about 2^-21 relative,
 // far below the 2^-16 of the split bf16 operands) or the identity.
 template <int FM>
