@@ -334,7 +334,7 @@ struct K3sSmem {
   static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
   static constexpr uint32_t kQf = FM == 0 ? kC * DK * 4 : 0;  // float32 copy of Q (tf32 X)
-  static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC;
+  static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC + 40;
   static constexpr uint32_t kBars = 15;
   static constexpr uint32_t kTotal =
       2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kQf + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
@@ -383,7 +383,9 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   float* sPow = sTh + kC;
   float* sXi = sPow + kC;          // [2][kC]
   float* sDenPart = sXi + 2 * kC;  // [2][kC]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDenPart + 2 * kC);
+  float* sCw = sDenPart + 2 * kC;  // [17] gamma^(64 m)
+  float* sCwInv = sCw + 20;        // [17] gamma^(-64 m)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sCwInv + 20);
   uint64_t* full = bars;           // [2]
   uint64_t* ops = bars + 2;        // [2]
   uint64_t* pready = bars + 4;
@@ -433,10 +435,31 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   // Tile row r holds chunk position p = r, or p = 63 - r in reverse (the tile is loaded in
   // memory order); sTh is indexed by tile row, sPow by position difference.  The direction
   // is a template parameter: the causal kernel carries no trace of the reverse one.
+  // Decayed prefix kept as P = c P~ (TMEM holds P~): within a window of W chunks the
+  // state update adds V^T (Xi .* psi(K)) / c, the epilogue scales X by c, and only the
+  // window's first chunk rescales P~ in TMEM, instead of every chunk writing gamma^L P
+  // back.  c = gamma^(64 m) m chunks into the window; W keeps 1 / c <= 2^60.  Heads with
+  // gamma < ~0.52 (and gamma = 0) keep W = 1: P itself, decayed every chunk.
+  int W = 1;
+  if constexpr (DECAY) {
+    if (g > 0.f) {
+      const float lg = -log2f(g);
+      W = lg > 0.f ? static_cast<int>(fminf(16.f, 60.f / (64.f * lg))) : 16;
+    }
+    if (W < 2) W = 1;
+  }
+  const bool renorm = W >= 2;
   constexpr bool rev = REV;
   if (tid < kC) {
     sTh[tid] = DECAY ? powf(g, static_cast<float>((rev ? kC - 1 - tid : tid) + 1)) : 1.f;
     sPow[tid] = DECAY ? powf(g, static_cast<float>(tid)) : 1.f;
+  }
+  // Window factors gamma^(64 m) and their inverses (m <= W <= 16), so that no role needs a
+  // power per chunk.
+  if (DECAY && renorm && tid >= kC && tid < kC + 17) {
+    const int m = tid - kC;
+    sCw[m] = powf(g, static_cast<float>(kC * m));
+    sCwInv[m] = powf(g, -static_cast<float>(kC * m));
   }
   const float g64 = DECAY ? powf(g, static_cast<float>(kC)) : 1.f;
   if constexpr (NORM) {
@@ -470,20 +493,6 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     return false;
   };
 
-  // Decayed prefix kept as P = c P~ (TMEM holds P~): within a window of W chunks the
-  // state update adds V^T (Xi .* psi(K)) / c, the epilogue scales X by c, and only the
-  // window's first chunk rescales P~ in TMEM, instead of every chunk writing gamma^L P
-  // back.  c = gamma^(64 m) m chunks into the window; W keeps 1 / c <= 2^60.  Heads with
-  // gamma < ~0.52 (and gamma = 0) keep W = 1: P itself, decayed every chunk.
-  int W = 1;
-  if constexpr (DECAY) {
-    if (g > 0.f) {
-      const float lg = -log2f(g);
-      W = lg > 0.f ? static_cast<int>(fminf(16.f, 60.f / (64.f * lg))) : 16;
-    }
-    if (W < 2) W = 1;
-  }
-  const bool renorm = W >= 2;
   // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
   const bool tf32x = kTf32X && sp.tf32_prefix && (!DECAY || renorm);
 
@@ -527,8 +536,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       float* xi = sXi + s * kC;
       if (tw < kC) {
         const int p = rev ? kC - 1 - tw : tw;
-        xi[tw] = p < L ? (DECAY ? powf(g, static_cast<float>(L - 1 - p - (renorm ? kC * (i % W + 1) : 0)))
-                                : 1.f)
+        xi[tw] = p < L ? (DECAY ? sPow[L - 1 - p] * (renorm ? sCwInv[i % W + 1] : 1.f) : 1.f)
                        : 0.f;
       }
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
@@ -632,7 +640,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
         tc_fence_after();
         if (DECAY && i > 0 && i % W == 0) {
-          const float c_w = powf(g, static_cast<float>(kC * W));
+          const float c_w = sCw[W];
 #pragma unroll
           for (int q4 = 0; q4 < kHalf / 32; ++q4) {
             const uint32_t col = pcol + q4 * 32;
@@ -670,7 +678,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       tc_fence_after();
       // A window's first chunk turns P~ back into P (c = gamma^(64 W) since the last one).
       const bool rescale = renorm && i > 0 && i % W == 0;
-      const float c_w = rescale ? powf(g, static_cast<float>(kC * W)) : 1.f;
+      const float c_w = rescale ? sCw[W] : 1.f;
 #pragma unroll
       for (int q4 = 0; q4 < kHalf / 32; ++q4) {
         const uint32_t col = pcol + q4 * 32;
@@ -785,7 +793,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       // first global store.
       if (has_prefix) {
         // X was computed from P~: the chunk's Theta carries the window factor c.
-        const float c = renorm ? powf(g, static_cast<float>(kC * (i % W))) : 1.f;
+        const float c = renorm ? sCw[i % W] : 1.f;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 th = *reinterpret_cast<const float4*>(sTh + 32 * half + 4 * q);
