@@ -200,7 +200,13 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   // group's decay A, the product of its elements' decays.
   float4 agg = make_float4(0.f, 0.f, 0.f, 0.f);
   float A = 1.f;
-  if (live) {
+  if (U == 1) {
+    // One element per group: it stays in registers for pass 2.
+    if (live && e0 < e1) {
+      agg = base[static_cast<long long>(e0) * R4];
+      A = DECAY ? (e0 == p.NC - 1 ? aL : gC) : 1.f;
+    }
+  } else if (live) {
     for (int c0 = e0; c0 < e1; c0 += U) {
       float4 x[U];
 #pragma unroll
@@ -215,6 +221,8 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
         }
     }
   }
+  const float4 x_own = agg;  // the group's own fold and decay (U == 1: the element itself)
+  const float a_own = A;
   // Hillis-Steele over the groups: after round r, group gi holds the fold of groups
   // gi - 2^(r+1) + 1 .. gi, and A their decay.
   for (int d = 1; d < NG; d <<= 1) {
@@ -236,6 +244,12 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   const float4 init = p.has_init ? read_init(p, bh, col4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
   float4 carry = init;
   if (gi > 0) carry = axpy4(sA[gi - 1], init, sX[(gi - 1) * kSlab + c8]);
+  if (U == 1) {
+    // The element's exclusive prefix; the state after it is a carry + x.
+    base[static_cast<long long>(e0) * R4] = carry;
+    if (e1 == p.NC) write_final(p, bh, col4 * 4, axpy4(a_own, carry, x_own));
+    return;
+  }
   // Pass 2: exclusive prefixes of this group's elements, in place (re-read from L2, so
   // four loads in flight suffice and keep the thread within 64 registers).
   carry = carry_in_place<DECAY, (U > 1 ? U / 2 : 1)>(base, R4, e0, e1, p.NC - 1, gC, aL, carry);
