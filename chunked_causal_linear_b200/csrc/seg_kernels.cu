@@ -28,8 +28,6 @@
 
 #include <cuda_bf16.h>
 
-#include <algorithm>
-
 #include "common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
@@ -325,59 +323,6 @@ constexpr int kThreads3 = 576;
 constexpr int kXfThreads = 256;  // transform warps 0-7
 constexpr int kEpThreads = 256;  // epilogue warps 8-15
 
-// The segments of a persistent CTA, j = blockIdx.x, blockIdx.x + gridDim.x, ... of the BH * NS
-// segments (j = bh * NS + seg), walked chunk by chunk.  Every role keeps its own cursor and
-// takes the same steps, so the roles agree on every chunk's (head, segment, position).
-struct SegCursor {
-  int j, bh, seg, cb, n, l;
-  __device__ __forceinline__ void at(const SegParams& sp, int jj) {
-    j = jj;
-    bh = jj / sp.NS;
-    seg = jj % sp.NS;
-    cb = seg * sp.Lseg;
-    n = min(sp.NC, cb + sp.Lseg) - cb;
-    l = 0;
-  }
-  __device__ __forceinline__ void next(const SegParams& sp) {
-    if (++l >= n) at(sp, j + static_cast<int>(gridDim.x));
-  }
-};
-
-// Chunks this CTA walks in all its segments.
-__device__ __forceinline__ int cta_chunks(const SegParams& sp) {
-  int total = 0;
-  for (int j = static_cast<int>(blockIdx.x); j < sp.BH * sp.NS; j += static_cast<int>(gridDim.x)) {
-    const int cb = (j % sp.NS) * sp.Lseg;
-    total += min(sp.NC, cb + sp.Lseg) - cb;
-  }
-  return total;
-}
-
-// The decay of one head as the combine uses it.  Decayed prefix kept as P = c P~ (TMEM
-// holds P~): within a window of W chunks the state update adds V^T (Xi .* psi(K)) / c, the
-// epilogue scales X by c, and only the window's first chunk rescales P~ in TMEM, instead of
-// every chunk writing gamma^L P back.  c = gamma^(64 m) m chunks into the window; W keeps
-// 1 / c <= 2^60.  Heads with gamma < ~0.52 (and gamma = 0) keep W = 1: P itself, decayed
-// every chunk.
-struct HeadDecay {
-  float g = 1.f, g64 = 1.f, ginv64 = 1.f, gW = 1.f;  // gamma, gamma^64, gamma^-64, gamma^(64 W)
-  int W = 1;
-  bool renorm = false;
-  __device__ __forceinline__ void set(float gamma) {
-    g = gamma;
-    g64 = powf(g, 64.f);
-    W = 1;
-    if (g > 0.f) {
-      const float lg = -log2f(g);
-      W = lg > 0.f ? static_cast<int>(fminf(16.f, 60.f / (64.f * lg))) : 16;
-    }
-    if (W < 2) W = 1;
-    renorm = W >= 2;
-    ginv64 = renorm ? powf(g, -64.f) : 1.f;
-    gW = renorm ? powf(g, 64.f * W) : 1.f;
-  }
-};
-
 template <int DK, int FM, bool DECAY, bool OUTF32>
 struct K3sSmem {
   static constexpr int DV = 128;
@@ -389,7 +334,7 @@ struct K3sSmem {
   static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
   static constexpr uint32_t kQf = FM == 0 ? kC * DK * 4 : 0;  // float32 copy of Q (tf32 X)
-  static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC;
+  static constexpr uint32_t kSmallFloats = 9 * DK + 9 * kC + 40;
   static constexpr uint32_t kBars = 15;
   static constexpr uint32_t kTotal =
       2 * kStage + 2 * kLo + 2 * kKpp + 2 * kA + kQf + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
@@ -434,11 +379,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   float* sZpart = sZP + DK;        // [8][DK]
   float* sDenX = sZpart + 8 * DK;  // [2][kC]
   float* sDen = sDenX + 2 * kC;
-  float* sTh = sDen + kC;          // the epilogue's per-head tables (set at segment starts)
+  float* sTh = sDen + kC;
   float* sPow = sTh + kC;
   float* sXi = sPow + kC;          // [2][kC]
   float* sDenPart = sXi + 2 * kC;  // [2][kC]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDenPart + 2 * kC);
+  float* sCw = sDenPart + 2 * kC;  // [17] gamma^(64 m)
+  float* sCwInv = sCw + 20;        // [17] gamma^(-64 m)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sCwInv + 20);
   uint64_t* full = bars;           // [2]
   uint64_t* ops = bars + 2;        // [2]
   uint64_t* pready = bars + 4;
@@ -454,7 +401,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 
   if (error_pending(sp.err)) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_all = cta_chunks(sp);  // chunks over all of this CTA's segments
+  const int seg = static_cast<int>(blockIdx.x % sp.NS);
+  const int bh = static_cast<int>(blockIdx.x / sp.NS);
+  const int cb = seg * sp.Lseg;
+  const int ce = min(sp.NC, cb + sp.Lseg);
+  const int n = ce - cb;
+  const float g = DECAY ? gt.g[bh % sp.H] : 1.f;
+  const float* srec = sp.srec + (static_cast<long long>(bh) * sp.NS + seg) * sp.R;
 
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -480,10 +433,38 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     tmem_relinquish();
   }
   // Tile row r holds chunk position p = r, or p = 63 - r in reverse (the tile is loaded in
-  // memory order).  The direction is a template parameter: the causal kernel carries no
-  // trace of the reverse one.  Per-head decay values live in each role's registers, set at
-  // each segment's first chunk (a CTA's segments may belong to different heads).
+  // memory order); sTh is indexed by tile row, sPow by position difference.  The direction
+  // is a template parameter: the causal kernel carries no trace of the reverse one.
+  // Decayed prefix kept as P = c P~ (TMEM holds P~): within a window of W chunks the
+  // state update adds V^T (Xi .* psi(K)) / c, the epilogue scales X by c, and only the
+  // window's first chunk rescales P~ in TMEM, instead of every chunk writing gamma^L P
+  // back.  c = gamma^(64 m) m chunks into the window; W keeps 1 / c <= 2^60.  Heads with
+  // gamma < ~0.52 (and gamma = 0) keep W = 1: P itself, decayed every chunk.
+  int W = 1;
+  if constexpr (DECAY) {
+    if (g > 0.f) {
+      const float lg = -log2f(g);
+      W = lg > 0.f ? static_cast<int>(fminf(16.f, 60.f / (64.f * lg))) : 16;
+    }
+    if (W < 2) W = 1;
+  }
+  const bool renorm = W >= 2;
   constexpr bool rev = REV;
+  if (tid < kC) {
+    sTh[tid] = DECAY ? powf(g, static_cast<float>((rev ? kC - 1 - tid : tid) + 1)) : 1.f;
+    sPow[tid] = DECAY ? powf(g, static_cast<float>(tid)) : 1.f;
+  }
+  // Window factors gamma^(64 m) and their inverses (m <= W <= 16), so that no role needs a
+  // power per chunk.
+  if (DECAY && renorm && tid >= kC && tid < kC + 17) {
+    const int m = tid - kC;
+    sCw[m] = powf(g, static_cast<float>(kC * m));
+    sCwInv[m] = powf(g, -static_cast<float>(kC * m));
+  }
+  const float g64 = DECAY ? powf(g, static_cast<float>(kC)) : 1.f;
+  if constexpr (NORM) {
+    if (tid < DK) sZP[tid] = srec[DK * DVR + tid];
+  }
   if constexpr (DVR < DV) {
     // The V tiles' upper 64 value features: zero once, never loaded.
     for (int e = tid; e < 2 * (kC * 128 / 16); e += kThreads3) {
@@ -513,19 +494,14 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   };
 
   // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
-  auto use_tf32x = [&](const HeadDecay& hd) { return kTf32X && sp.tf32_prefix && (!DECAY || hd.renorm); };
-  auto head_gamma = [&](int bh) { return DECAY ? gt.g[bh % sp.H] : 1.f; };
-  auto seg_rec = [&](const SegCursor& c) {
-    return sp.srec + (static_cast<long long>(c.bh) * sp.NS + c.seg) * sp.R;
-  };
+  const bool tf32x = kTf32X && sp.tf32_prefix && (!DECAY || renorm);
 
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
     const int tw = tid;
     constexpr int kHalf = DK / 2;  // key features of P handled by this thread
     const uint32_t pcol = static_cast<uint32_t>(warp >> 2) * kHalf;
-    // A segment's exclusive prefix into the TMEM state: row (lane) of P^T, this thread's half.
-    auto load_prefix = [&](const float* srec) {
+    {  // the segment's exclusive prefix: row (lane) of P^T, this thread's half
       const int row = (warp & 3) * 32 + lane;
       const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
 #pragma unroll
@@ -542,28 +518,15 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
       }
       tmem_st_wait();
-    };
+    }
     constexpr int NCC = DK / 8;
     constexpr int RG = kXfThreads / NCC;
     constexpr int kRows = kC / RG;
     const int cc = tw % NCC, rg = tw / NCC;
-    SegCursor cur;
-    cur.at(sp, static_cast<int>(blockIdx.x));
-    HeadDecay hd;
-    bool tf32x = false;
-    float pw_full = 1.f;  // tw < kC: gamma^(63 - p), the weight of position p in a full chunk
-    float inv_w = 1.f;    // tw < kC: gamma^(-64 (m + 1)), m chunks into the window
-    for (int i = 0; i < n_all; ++i, cur.next(sp)) {
+    for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      const bool first = cur.l == 0;
-      if (first) {
-        hd.set(head_gamma(cur.bh));
-        tf32x = use_tf32x(hd);
-        if (DECAY && tw < kC) pw_full = powf(hd.g, static_cast<float>(kC - 1 - (rev ? kC - 1 - tw : tw)));
-      }
-      const int L = chunk_len(sp, cur.cb + cur.l);
-      const bool last = cur.l == cur.n - 1;
-      const int wpos = cur.l % hd.W;  // chunks into the renormalised window
+      const int L = chunk_len(sp, cb + i);
+      const bool last = i == n - 1;
       uint8_t* sQ = base + s * L_::kStage;
       uint8_t* sK = sQ + L_::kQ;
       uint8_t* sQl = sLo + s * L_::kLo;
@@ -573,15 +536,10 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       float* xi = sXi + s * kC;
       if (tw < kC) {
         const int p = rev ? kC - 1 - tw : tw;
-        if (DECAY && hd.renorm) inv_w = wpos == 0 ? hd.ginv64 : inv_w * hd.ginv64;
-        const float pw = L == kC ? pw_full : powf(hd.g, static_cast<float>(L - 1 - p));
-        xi[tw] = p < L ? (DECAY ? pw * (hd.renorm ? inv_w : 1.f) : 1.f) : 0.f;
+        xi[tw] = p < L ? (DECAY ? sPow[L - 1 - p] * (renorm ? sCwInv[i % W + 1] : 1.f) : 1.f)
+                       : 0.f;
       }
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
-      if constexpr (NORM) {
-        // A new segment's incoming Z (after this thread's own last update of the old one).
-        if (first && tw < DK) sZP[tw] = seg_rec(cur)[DK * DVR + tw];
-      }
       named_barrier(1, kXfThreads);
 
       float zacc[8];
@@ -657,7 +615,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       mbar_arrive(&ops[s]);
 
       // gamma^L: Theta of the chunk's last token for a full chunk.
-      const float a_c = DECAY ? (L == kC ? hd.g64 : powf(hd.g, static_cast<float>(L))) : 1.f;
+      const float a_c = DECAY ? (L == kC ? g64 : powf(g, static_cast<float>(L))) : 1.f;
       if constexpr (NORM) {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -681,9 +639,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         // features per row) once the previous chunk's X has read the copy.
         if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
         tc_fence_after();
-        if (first) load_prefix(seg_rec(cur));
-        if (DECAY && !first && wpos == 0) {
-          const float c_w = hd.gW;
+        if (DECAY && i > 0 && i % W == 0) {
+          const float c_w = sCw[W];
 #pragma unroll
           for (int q4 = 0; q4 < kHalf / 32; ++q4) {
             const uint32_t col = pcol + q4 * 32;
@@ -715,14 +672,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         mbar_arrive(pready);
         continue;
       }
-      // Prefix operand for chunk i (the state after chunk i - 1, or a new segment's exclusive
-      // prefix), this thread's half of the key features.
+      // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of
+      // the key features.
       if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
       tc_fence_after();
-      if (first) load_prefix(seg_rec(cur));
       // A window's first chunk turns P~ back into P (c = gamma^(64 W) since the last one).
-      const bool rescale = DECAY && hd.renorm && !first && wpos == 0;
-      const float c_w = rescale ? hd.gW : 1.f;
+      const bool rescale = renorm && i > 0 && i % W == 0;
+      const float c_w = rescale ? sCw[W] : 1.f;
 #pragma unroll
       for (int q4 = 0; q4 < kHalf / 32; ++q4) {
         const uint32_t col = pcol + q4 * 32;
@@ -749,7 +705,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         tmem_st16(tmem + lane_base + kColPH + col / 2, hi);
         tmem_st16(tmem + lane_base + kColPL + col / 2, lo);
         if constexpr (DECAY) {
-          if (!hd.renorm && !last) {
+          if (!renorm && !last) {
             uint32_t u[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * a_c);
@@ -766,31 +722,12 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     const int tw = tid - kXfThreads;
     const int quarter = warp & 3, half = (warp - 8) >> 2;
     const int j = quarter * 32 + lane;  // value feature of this thread's output column
-    SegCursor cur;
-    cur.at(sp, static_cast<int>(blockIdx.x));
-    HeadDecay hd;
-    float cwin = 1.f;  // gamma^(64 m), m chunks into the renormalised window
-    for (int i = 0; i < n_all; ++i, cur.next(sp)) {
+    for (int i = 0; i < n; ++i) {
       const int s = i & 1;
-      const bool first = cur.l == 0;
-      if (first) {
-        // The head's tables: Theta by tile row, gamma^d by position difference.  Written by
-        // this role alone, between two barriers of the role (everyone is done with the
-        // previous segment's, then everyone sees the new ones).
-        hd.set(head_gamma(cur.bh));
-        named_barrier(2, kEpThreads);
-        if (tw < kC) {
-          sTh[tw] = DECAY ? powf(hd.g, static_cast<float>((rev ? kC - 1 - tw : tw) + 1)) : 1.f;
-          sPow[tw] = DECAY ? powf(hd.g, static_cast<float>(tw)) : 1.f;
-        }
-        named_barrier(2, kEpThreads);
-      }
-      if (DECAY && hd.renorm) cwin = cur.l % hd.W == 0 ? 1.f : cwin * hd.g64;
-      const long long t0 = rev ? sp.T - static_cast<long long>(cur.cb + cur.l + 1) * kC
-                               : static_cast<long long>(cur.cb + cur.l) * kC;
-      const int L = chunk_len(sp, cur.cb + cur.l);
-      const bool has_prefix = !(cur.seg == 0 && cur.l == 0) || sp.has_init;
-      const int bh = cur.bh;
+      const long long t0 = rev ? sp.T - static_cast<long long>(cb + i + 1) * kC
+                               : static_cast<long long>(cb + i) * kC;
+      const int L = chunk_len(sp, cb + i);
+      const bool has_prefix = !(seg == 0 && i == 0) || sp.has_init;
       wait(sdone, i & 1, kErrMmaTimeout);
       wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout);
       tc_fence_after();
@@ -856,7 +793,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       // first global store.
       if (has_prefix) {
         // X was computed from P~: the chunk's Theta carries the window factor c.
-        const float c = hd.renorm ? cwin : 1.f;
+        const float c = renorm ? sCw[i % W] : 1.f;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 th = *reinterpret_cast<const float4*>(sTh + 32 * half + 4 * q);
@@ -895,16 +832,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       int loads = 0;
-      SegCursor cur;
-      cur.at(sp, static_cast<int>(blockIdx.x));
-      for (int i = 0; i < n_all; ++i, cur.next(sp)) {
+      for (int i = 0; i < n; ++i) {
         // Stage i & 1 is free once N(i - 2), the last MMA reading it, is done.
         if (i >= 2 && !wait(&empty[i & 1], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
         uint8_t* sQ = base + (i & 1) * L_::kStage;
         uint8_t* sK = sQ + L_::kQ;
         uint8_t* sV = sK + L_::kK;
-        const int c = cur.cb + cur.l, bh = cur.bh;
-        const int t0 = rev ? static_cast<int>(sp.T) - (c + 1) * kC : c * kC;
+        const int t0 = rev ? static_cast<int>(sp.T) - (cb + i + 1) * kC : (cb + i) * kC;
         mbar_arrive_expect_tx(&full[i & 1], L_::kQ + L_::kK + DVR * kC * 2);
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) {
@@ -960,19 +894,11 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       mma_commit(sdone);
       return true;
     };
-    SegCursor cur;
-    cur.at(sp, static_cast<int>(blockIdx.x));
-    HeadDecay hd;
-    bool tf32x = false;
     issue_scores(0);
-    for (int i = 0; i < n_all && !failed; ++i, cur.next(sp)) {
+    for (int i = 0; i < n && !failed; ++i) {
       const int s = i & 1;
-      if (cur.l == 0) {
-        hd.set(head_gamma(cur.bh));
-        tf32x = use_tf32x(hd);
-      }
-      const bool last = cur.l == cur.n - 1;
-      const bool has_prefix = !(cur.seg == 0 && cur.l == 0) || sp.has_init;
+      const bool last = i == n - 1;
+      const bool has_prefix = !(seg == 0 && i == 0) || sp.has_init;
       const uint64_t q = dQk + s * kStageD, ql = dQlk + s * kLoD;
       const uint64_t v = dVm + s * kStageD;
 
@@ -1028,8 +954,8 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       mma_commit(ndone);
       mma_commit(&empty[s]);
 
-      // The next chunk's scores go in right behind N(i) (across a segment boundary too).
-      if (i + 1 < n_all && !issue_scores(i + 1)) break;
+      // The next chunk's scores go in right behind N(i).
+      if (i + 1 < n && !issue_scores(i + 1)) break;
     }
     if (failed) {
       // Let the issued MMAs finish before TMEM is given up (bounded).
@@ -1063,19 +989,6 @@ cudaError_t k1s_go(const SegParams& sp, const GammaTable& gt, const TcMaps& m, F
   return cudaGetLastError();
 }
 
-// Streaming multiprocessors of the current device (cached per device).
-int sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cache[dev]) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
-  }
-  return cache[dev];
-}
-
 template <int DK, int FM, bool DECAY, bool NORM, bool OUTF32, bool REV>
 cudaError_t k3s_go_r(const SegParams& sp, const GammaTable& gt, const TcMaps& m, cudaStream_t s) {
   auto kern = sp.dv == 64 ? k3_seg<DK, FM, DECAY, NORM, OUTF32, REV, 64>
@@ -1083,8 +996,7 @@ cudaError_t k3s_go_r(const SegParams& sp, const GammaTable& gt, const TcMaps& m,
   const uint32_t sm = K3sSmem<DK, FM, DECAY, OUTF32>::kTotal;
   cudaError_t e = set_smem(kern, sm);
   if (e != cudaSuccess) return e;
-  // Persistent: one CTA per SM (one fits), each walking every gridDim-th segment.
-  const long long grid = std::min<long long>(static_cast<long long>(sp.BH) * sp.NS, sm_count());
+  const long long grid = static_cast<long long>(sp.BH) * sp.NS;
   kern<<<static_cast<unsigned>(grid), kThreads3, sm, s>>>(m.q, m.k, m.v, sp, gt);
   return cudaGetLastError();
 }
