@@ -61,16 +61,20 @@ def gpu_prefill(q, k, v, *, C, feature_map, gamma, normalize, **kw):
     return out, S, Z
 
 
-def oracle_prefill(q, k, v, *, feature_map, gamma, normalize, heads=None, want_out=True):
-    """Oracle on host copies of q, k, v.
+def oracle_prefill(q, k, v, *, feature_map, gamma, normalize, heads=None, want_out=True,
+                   S_init=None, Z_init=None):
+    """Oracle on host copies of q, k, v (and of the initial state, when given).
 
     `heads` selects (b, h) pairs (default: all); the selected pairs run as one oracle call
     (one thread each) and come back stacked as [n, T, d] / [n, dk, dv] / [n, dk].
     """
     g = None if gamma is None else np.asarray(gamma, dtype=np.float64)
     if heads is None:
+        s0 = None if S_init is None else to_np(S_init).astype(np.float64)
+        z0 = None if Z_init is None else to_np(Z_init).astype(np.float64)
         return default_oracle().forward(to_np(q), to_np(k), to_np(v), feature_map=feature_map,
-                                        gamma=g, normalize=normalize, want_out=want_out)
+                                        gamma=g, normalize=normalize, want_out=want_out,
+                                        S_init=s0, Z_init=z0)
     sel = lambda t: torch.stack([t[b, h] for b, h in heads])[None]
     gs = None if g is None else np.array([g[h] for _, h in heads])
     o, S, Z = default_oracle().forward(to_np(sel(q)), to_np(sel(k)), to_np(sel(v)),
