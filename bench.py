@@ -180,7 +180,7 @@ def measured_peaks() -> tuple[float, str]:
 def source_hash(fname: str) -> str:
     csrc = ROOT / "chunked_causal_linear_b200" / "csrc"
     h = hashlib.sha256()
-    for f in sorted({fname, "ptx.cuh", "common.cuh"}):
+    for f in sorted({fname, "ptx.cuh", "common.cuh", "tile_util.cuh"}):
         h.update((csrc / f).read_bytes())
     return h.hexdigest()[:16]
 
