@@ -259,6 +259,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+        "=r"(u[14]), "=r"(u[15])
+      : "r"(taddr));
+}
+
 // The 16-lane shape for 64-row accumulators (rows in lanes 0-15 of each quarter): lanes
 // 0-15 of the warp receive TMEM lanes 0-15 of the warp's quarter at columns
 // [taddr, taddr + 16), lanes 16-31 the same TMEM lanes at columns [taddr + 16, taddr + 32).
@@ -314,6 +325,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&u)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+      ::"r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]),
+        "r"(u[6]), "r"(u[7])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -341,12 +360,12 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// psi: ELU+1 (x + 1 for x > 0, e^x otherwise; the fast exponential, about 2^-21 relative,
-// far below the 2^-16 of the split bf16 operands) or the identity.
+// psi: ELU+1 (x + 1 for x > 0, e^x = 2^(x log2 e) otherwise, by the hardware exponential:
+// about 2^-21 relative, far below the 2^-16 of the split bf16 operands) or the identity.
 template <int FM>
 __device__ __forceinline__ float feature(float x) {
   if constexpr (FM == 1) {
-    return x > 0.f ? x + 1.f : __expf(x);
+    return x > 0.f ? x + 1.f : exp2_approx(x * 1.4426950408889634f);
   } else {
     return x;
   }

@@ -496,29 +496,85 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
   const bool tf32x = kTf32X && sp.tf32_prefix && (!DECAY || renorm);
 
+  // The prefix operand of the X MMA is prepared by the transform warps for the tf32 product
+  // (a float32 copy of Q) and by the epilogue warps otherwise (P split into bf16 hi / lo in
+  // TMEM), which leaves the transform warps, whose psi pass sets the pace of the feature-
+  // mapped forms, the chunk's operands alone.  Either role covers the 128 TMEM lanes with
+  // its 8 warps: lanes 32 (warp % 4) .. + 31, key features kHalf (warp / 4 % 2) .. + kHalf - 1.
+  constexpr int kHalf = DK / 2;
+  const uint32_t pcol = static_cast<uint32_t>((warp >> 2) & 1) * kHalf;
+  // The segment's exclusive prefix into TMEM: row (lane) of P^T, this thread's half.
+  auto load_prefix = [&]() {
+    const int row = (warp & 3) * 32 + lane;
+    const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
+#pragma unroll
+    for (int q4 = 0; q4 < kHalf / 32; ++q4) {
+      uint32_t u[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 f = row < DVR ? src[q4 * 8 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        u[4 * e] = __float_as_uint(f.x);
+        u[4 * e + 1] = __float_as_uint(f.y);
+        u[4 * e + 2] = __float_as_uint(f.z);
+        u[4 * e + 3] = __float_as_uint(f.w);
+      }
+      tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
+    }
+    tmem_st_wait();
+  };
+  // Prefix operand for chunk i (the state after chunk i - 1, in TMEM once statedone(i - 1)
+  // completed), this thread's half of the key features: a window's first chunk turns P~
+  // back into P (c = gamma^(64 W) since the last one), then P goes to bf16 hi / lo, and a
+  // head without a window pre-decays P by gamma^L for the state update of chunk i.
+  auto split_prefix = [&](int i) {
+    const bool rescale = renorm && i > 0 && i % W == 0;
+    const float c_w = rescale ? sCw[W] : 1.f;
+    const int L = chunk_len(sp, cb + i);
+    const float a_c = DECAY ? (L == kC ? g64 : powf(g, static_cast<float>(L))) : 1.f;
+    const bool decay_now = DECAY && !renorm && i != n - 1;
+    // 16 columns at a time: this runs in the epilogue warps between the score and output
+    // phases, inside their register budget.
+#pragma unroll 2
+    for (int q = 0; q < kHalf / 16; ++q) {
+      const uint32_t col = pcol + q * 16;
+      float rr[16];
+      tmem_ld16(tmem + lane_base + kColP + col, rr);
+      tmem_ld_wait();
+      if (rescale) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          rr[e] *= c_w;
+          u[e] = __float_as_uint(rr[e]);
+        }
+        tmem_st16(tmem + lane_base + kColP + col, u);
+      }
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(rr[2 * e], rr[2 * e + 1]);
+        const float2 hf = __bfloat1622float2(h);
+        hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
+      }
+      tmem_st8(tmem + lane_base + kColPH + col / 2, hi);
+      tmem_st8(tmem + lane_base + kColPL + col / 2, lo);
+      if (decay_now) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(rr[e] * a_c);
+        tmem_st16(tmem + lane_base + kColP + col, u);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(pready);
+  };
+
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
     const int tw = tid;
-    constexpr int kHalf = DK / 2;  // key features of P handled by this thread
-    const uint32_t pcol = static_cast<uint32_t>(warp >> 2) * kHalf;
-    {  // the segment's exclusive prefix: row (lane) of P^T, this thread's half
-      const int row = (warp & 3) * 32 + lane;
-      const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
-#pragma unroll
-      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
-        uint32_t u[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 f = row < DVR ? src[q4 * 8 + e] : make_float4(0.f, 0.f, 0.f, 0.f);
-          u[4 * e] = __float_as_uint(f.x);
-          u[4 * e + 1] = __float_as_uint(f.y);
-          u[4 * e + 2] = __float_as_uint(f.z);
-          u[4 * e + 3] = __float_as_uint(f.w);
-        }
-        tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
-      }
-      tmem_st_wait();
-    }
+    if (tf32x) load_prefix();
     constexpr int NCC = DK / 8;
     constexpr int RG = kXfThreads / NCC;
     constexpr int kRows = kC / RG;
@@ -526,7 +582,6 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       const int L = chunk_len(sp, cb + i);
-      const bool last = i == n - 1;
       uint8_t* sQ = base + s * L_::kStage;
       uint8_t* sK = sQ + L_::kQ;
       uint8_t* sQl = sLo + s * L_::kLo;
@@ -670,58 +725,17 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(pready);
-        continue;
       }
-      // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of
-      // the key features.
-      if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
-      tc_fence_after();
-      // A window's first chunk turns P~ back into P (c = gamma^(64 W) since the last one).
-      const bool rescale = renorm && i > 0 && i % W == 0;
-      const float c_w = rescale ? sCw[W] : 1.f;
-#pragma unroll
-      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
-        const uint32_t col = pcol + q4 * 32;
-        float rr[32];
-        tmem_ld32(tmem + lane_base + kColP + col, rr);
-        tmem_ld_wait();
-        if (rescale) {
-          uint32_t u[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            rr[e] *= c_w;
-            u[e] = __float_as_uint(rr[e]);
-          }
-          tmem_st32(tmem + lane_base + kColP + col, u);
-        }
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(rr[2 * e], rr[2 * e + 1]);
-          const float2 hf = __bfloat1622float2(h);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
-        }
-        tmem_st16(tmem + lane_base + kColPH + col / 2, hi);
-        tmem_st16(tmem + lane_base + kColPL + col / 2, lo);
-        if constexpr (DECAY) {
-          if (!renorm && !last) {
-            uint32_t u[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * a_c);
-            tmem_st32(tmem + lane_base + kColP + col, u);
-          }
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(pready);
     }
   } else if (warp < 16) {
     // ------------------------------------------------------------------ epilogue
     const int tw = tid - kXfThreads;
     const int quarter = warp & 3, half = (warp - 8) >> 2;
     const int j = quarter * 32 + lane;  // value feature of this thread's output column
+    if (!tf32x) {
+      load_prefix();
+      split_prefix(0);
+    }
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       const long long t0 = rev ? sp.T - static_cast<long long>(cb + i + 1) * kC
@@ -778,6 +792,14 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         }
       }
       mbar_arrive(aready);
+
+      // The next chunk's prefix operand, while N(i) runs: X(i) and the state update with
+      // chunk i are done once statedone(i) completes.
+      if (!tf32x && i + 1 < n) {
+        wait(statedone, i & 1, kErrMmaTimeout);
+        tc_fence_after();
+        split_prefix(i + 1);
+      }
 
       wait(ndone, i & 1, kErrMmaTimeout);
       tc_fence_after();
