@@ -365,7 +365,11 @@ __device__ __forceinline__ float exp2_approx(float x) {
 template <int FM>
 __device__ __forceinline__ float feature(float x) {
   if constexpr (FM == 1) {
-    return x > 0.f ? x + 1.f : exp2_approx(x * 1.4426950408889634f);
+    // The exponential is taken unconditionally (of min(x, 0), so it never overflows) and
+    // the result selected: no branch, so the scheduler can overlap the exponentials of
+    // independent elements instead of paying each one's latency in turn.
+    const float e = exp2_approx(fminf(x, 0.f) * 1.4426950408889634f);
+    return x > 0.f ? x + 1.f : e;
   } else {
     return x;
   }
