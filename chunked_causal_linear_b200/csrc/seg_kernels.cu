@@ -316,8 +316,9 @@ k1_seg(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtenso
 //               built once per stage; each k-step only adds a constant offset, so the
 //               tensor pipe, not the issuing thread, sets the pace.
 // Warp w reads TMEM lanes 32 (w % 4) .. + 31.  Accumulators (TMEM columns): scores
-// [0, 64), X (two buffers) [64, 128) and [448, 512), N [128, 192), P [192, 192 + dk),
-// P hi / lo after it.  Each is released by an mbarrier once its readers are done.
+// [0, 64) ([0, 128) for psi = ELU+1: the hi-key and lo-key halves side by side), then X,
+// N (64 each), P (dk) and P hi / lo; a second X buffer at [448, 512) where that is free.
+// Each is released by an mbarrier once its readers are done.
 
 constexpr int kThreads3 = 576;
 constexpr int kXfThreads = 256;  // transform warps 0-7
@@ -328,9 +329,14 @@ struct K3sSmem {
   static constexpr int DV = 128;
   static constexpr uint32_t kQ = DK * kC * 2;
   static constexpr uint32_t kK = DK * kC * 2;
+  // A stage's K region: for psi = ELU+1 the hi and lo tiles of psi(K) interleaved per
+  // 64-feature block (hi block b, then its lo block), so that [hi; lo] is one 128-row
+  // operand of the scores MMA.
+  static constexpr uint32_t kKBlk = FM == 1 ? 2 * kC * 128 : kC * 128;
+  static constexpr uint32_t kKs = FM == 1 ? 2 * kK : kK;
   static constexpr uint32_t kV = DV * kC * 2;
-  static constexpr uint32_t kStage = kQ + kK + kV;
-  static constexpr uint32_t kLo = FM == 1 ? kQ + kK : 0;  // lo tiles of psi(Q), psi(K)
+  static constexpr uint32_t kStage = kQ + kKs + kV;
+  static constexpr uint32_t kLo = FM == 1 ? kQ : 0;  // lo tile of psi(Q)
   static constexpr uint32_t kKpp = DECAY ? 2 * kK : 0;    // Xi .* psi(K), hi + lo
   static constexpr uint32_t kA = kC * kC * 2;
   static constexpr uint32_t kQf = FM == 0 ? kC * DK * 4 : 0;  // float32 copy of Q (tf32 X)
@@ -362,15 +368,15 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
   // heads decaying faster than gamma ~ 0.52 (no renormalised window).
   constexpr bool kTf32X = FM == 0 && !NORM && !REV;
   constexpr uint32_t kTmemCols = 512;
-  constexpr uint32_t kColS = 0, kColN = 128, kColP = 192;
+  constexpr uint32_t kSCols = kSplitQK ? 128 : 64;
+  constexpr uint32_t kColS = 0, kColX0 = kSCols, kColN = kColX0 + 64, kColP = kColN + 64;
   constexpr uint32_t kColPH = kColP + DK, kColPL = kColPH + DK / 2;
-  constexpr uint32_t kColX[2] = {64, 448};
-  static_assert(kColPL + DK / 2 <= 448, "TMEM budget");
+  static_assert(kColPL + DK / 2 <= kTmemCols, "TMEM budget");
   static_assert(L_::kTotal <= 232448, "shared memory budget");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
-  uint8_t* sLo = base + 2 * L_::kStage;      // [2] x (Q lo, K lo)
+  uint8_t* sLo = base + 2 * L_::kStage;      // [2] x Q lo
   uint8_t* sKpp = sLo + 2 * L_::kLo;         // [2] x (hi, lo)
   uint8_t* sAh = sKpp + 2 * L_::kKpp;
   uint8_t* sAl = sAh + L_::kA;
@@ -469,7 +475,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     // The V tiles' upper 64 value features: zero once, never loaded.
     for (int e = tid; e < 2 * (kC * 128 / 16); e += kThreads3) {
       const int st = e / (kC * 128 / 16), o = e % (kC * 128 / 16);
-      reinterpret_cast<uint4*>(base + st * L_::kStage + L_::kQ + L_::kK + kC * 128)[o] =
+      reinterpret_cast<uint4*>(base + st * L_::kStage + L_::kQ + L_::kKs + kC * 128)[o] =
           make_uint4(0u, 0u, 0u, 0u);
     }
     fence_async_smem();
@@ -495,6 +501,11 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 
   // The tf32 prefix product (see kTf32X) where the state needs no per-chunk pass.
   const bool tf32x = kTf32X && sp.tf32_prefix && (!DECAY || renorm);
+  // X is double-buffered where [448, 512) is free of P hi / lo (the tf32 product does not
+  // use them); otherwise X(i) waits until the epilogue has read X(i - 1).
+  const bool x2 = tf32x || kColPL + DK / 2 <= 448;
+  const uint32_t col_x1 = x2 ? 448u : kColX0;
+  auto col_x = [&](int st) -> uint32_t { return st ? col_x1 : kColX0; };
 
   // The prefix operand of the X MMA is prepared by the transform warps for the tf32 product
   // (a float32 copy of Q) and by the epilogue warps otherwise (P split into bf16 hi / lo in
@@ -585,7 +596,6 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       uint8_t* sQ = base + s * L_::kStage;
       uint8_t* sK = sQ + L_::kQ;
       uint8_t* sQl = sLo + s * L_::kLo;
-      uint8_t* sKl = sQl + L_::kQ;
       uint8_t* sKph = sKpp + s * L_::kKpp;
       uint8_t* sKpl = sKph + L_::kK;
       float* xi = sXi + s * kC;
@@ -601,6 +611,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
       for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
       const uint32_t boff = (cc / 8) * (kC * 128);
+      const uint32_t boffK = (cc / 8) * L_::kKBlk;
       float zp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) zp[e] = NORM ? sZP[cc * 8 + e] : 0.f;
@@ -613,7 +624,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         const int r = rg + k * RG;
         const uint32_t off = boff + sw128_offset(r, cc % 8);
         if constexpr (kSplitQK || DECAY || NORM) {
-          kraw[k] = *reinterpret_cast<const uint4*>(sK + off);
+          kraw[k] = *reinterpret_cast<const uint4*>(sK + boffK + sw128_offset(r, cc % 8));
           wr[k] = xi[r];
         }
         if constexpr (kSplitQK || NORM) qraw[k] = *reinterpret_cast<const uint4*>(sQ + off);
@@ -630,8 +641,9 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
           if constexpr (kSplitQK) {
             uint4 hi, lo;
             split8(x, hi, lo);
-            *reinterpret_cast<uint4*>(sK + off) = hi;
-            *reinterpret_cast<uint4*>(sKl + off) = lo;
+            const uint32_t offK = boffK + sw128_offset(r, cc % 8);
+            *reinterpret_cast<uint4*>(sK + offK) = hi;
+            *reinterpret_cast<uint4*>(sK + offK + kC * 128) = lo;
           }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -753,6 +765,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         const int kb = 32 * half + 16 * (lane >> 4);
         float sc[16];
         tmem_ld16x2_x16(tmem + lane_base + kColS + 32 * half, sc);
+        if constexpr (kSplitQK) {  // the lo-key half
+          float sl[16];
+          tmem_ld16x2_x16(tmem + lane_base + kColS + 64 + 32 * half, sl);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) sc[e] += sl[e];
+        }
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(sfree);
@@ -805,7 +824,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
       tc_fence_after();
       // Column j (value feature), tokens 32 half .. + 31.
       float xo[32], no[32];
-      if (has_prefix) tmem_ld32(tmem + lane_base + kColX[s] + 32 * half, xo);
+      if (has_prefix) tmem_ld32(tmem + lane_base + col_x(s) + 32 * half, xo);
       tmem_ld32(tmem + lane_base + kColN + 32 * half, no);
       tmem_ld_wait();
       tc_fence_before();
@@ -859,13 +878,13 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         if (i >= 2 && !wait(&empty[i & 1], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
         uint8_t* sQ = base + (i & 1) * L_::kStage;
         uint8_t* sK = sQ + L_::kQ;
-        uint8_t* sV = sK + L_::kK;
+        uint8_t* sV = sK + L_::kKs;
         const int t0 = rev ? static_cast<int>(sp.T) - (cb + i + 1) * kC : (cb + i) * kC;
         mbar_arrive_expect_tx(&full[i & 1], L_::kQ + L_::kK + DVR * kC * 2);
 #pragma unroll
         for (int b = 0; b < DK / 64; ++b) {
           tma_load_3d(sQ + b * kC * 128, &tm_q, &full[i & 1], b * 64, t0, bh);
-          tma_load_3d(sK + b * kC * 128, &tm_k, &full[i & 1], b * 64, t0, bh);
+          tma_load_3d(sK + b * L_::kKBlk, &tm_k, &full[i & 1], b * 64, t0, bh);
         }
 #pragma unroll
         for (int b = 0; b < DVR / 64; ++b)
@@ -882,13 +901,12 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     // 128-byte atoms, kC * 128 bytes apart); stage 1 is kStage bytes further on.
     const uint32_t a0 = smem_u32(base);
     const uint64_t dQk = smem_desc_sw128(a0, 16, 1024);                       // Q, K-major
-    const uint64_t dKk = smem_desc_sw128(a0 + L_::kQ, 16, 1024);              // K, K-major
-    const uint64_t dKm = smem_desc_sw128(a0 + L_::kQ, kC * 128, 1024);        // K, MN-major
-    const uint64_t dVm = smem_desc_sw128(a0 + L_::kQ + L_::kK, kC * 128, 1024);  // V, MN-major
+    const uint64_t dKk = smem_desc_sw128(a0 + L_::kQ, 16, 1024);                // K, K-major
+    const uint64_t dKm = smem_desc_sw128(a0 + L_::kQ, L_::kKBlk, 1024);         // K, MN-major
+    const uint64_t dKlm = smem_desc_sw128(a0 + L_::kQ + kC * 128, L_::kKBlk, 1024);  // K lo
+    const uint64_t dVm = smem_desc_sw128(a0 + L_::kQ + L_::kKs, kC * 128, 1024);  // V, MN-major
     const uint32_t lo0 = smem_u32(sLo), kp0 = smem_u32(sKpp);
     const uint64_t dQlk = smem_desc_sw128(lo0, 16, 1024);
-    const uint64_t dKlk = smem_desc_sw128(lo0 + L_::kQ, 16, 1024);
-    const uint64_t dKlm = smem_desc_sw128(lo0 + L_::kQ, kC * 128, 1024);
     const uint64_t dKhm = smem_desc_sw128(kp0, kC * 128, 1024);
     const uint64_t dKpm = smem_desc_sw128(kp0 + L_::kK, kC * 128, 1024);
     const uint64_t dAh = smem_desc_sw128(smem_u32(sAh), 16, 1024);
@@ -899,18 +917,25 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
     auto issue_scores = [&](int i) -> bool {
       const int s = i & 1;
       const uint64_t q = dQk + s * kStageD, k = dKk + s * kStageD;
-      const uint64_t ql = dQlk + s * kLoD, kl = dKlk + s * kLoD;
+      const uint64_t ql = dQlk + s * kLoD;
       if (!wait(&ops[s], (i >> 1) & 1, kErrMmaTimeout)) return false;
       if (i > 0 && !wait(sfree, (i - 1) & 1, kErrMmaTimeout)) return false;
       tc_fence_after();
       constexpr uint32_t ids = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 64, 64);
+      // psi = ELU+1: psi(Q)_hi [psi(K)_hi; psi(K)_lo]^T as one N = 128 MMA (the hi-key
+      // and lo-key scores side by side, summed by the epilogue), plus psi(Q)_lo psi(K)_hi^T
+      // into the hi-key half: two MMAs per 16 features instead of three (an MMA costs
+      // about as much at N = 128 as at N = 64).
+      constexpr uint32_t ids2 = instr_desc(kFmtBF16, kFmtBF16, kKMajor, kKMajor, 64, 128);
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk) {
         const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
-        mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(k, off), ids, kk > 0 ? 1u : 0u);
+        const uint32_t offk = (kk / 4) * L_::kKBlk + (kk % 4) * 32;
         if constexpr (kSplitQK) {
-          mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(kl, off), ids, 1u);
-          mma_bf16_ss(tmem + kColS, desc_at(ql, off), desc_at(k, off), ids, 1u);
+          mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(k, offk), ids2, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + kColS, desc_at(ql, off), desc_at(k, offk), ids, 1u);
+        } else {
+          mma_bf16_ss(tmem + kColS, desc_at(q, off), desc_at(k, offk), ids, kk > 0 ? 1u : 0u);
         }
       }
       mma_commit(sdone);
@@ -926,7 +951,11 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 
       // X(i) = P^T psi(Q)^T and the prefix update with chunk i.
       if (!wait(pready, i & 1, kErrMmaTimeout)) break;
-      if (i > 1 && !wait(&xfree[s], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
+      if (x2) {
+        if (i > 1 && !wait(&xfree[s], ((i - 2) >> 1) & 1, kErrMmaTimeout)) break;
+      } else if (i > 0 && !wait(&xfree[s ^ 1], ((i - 1) >> 1) & 1, kErrMmaTimeout)) {
+        break;
+      }
       tc_fence_after();
       if (tf32x) {
         if (has_prefix) {
@@ -934,7 +963,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
           for (int kk = 0; kk < DK / 8; ++kk) {
             const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
-            mma_tf32_ts(tmem + kColX[s], tmem + kColP + kk * 8, desc_at(dQf, off), idt,
+            mma_tf32_ts(tmem + col_x(s), tmem + kColP + kk * 8, desc_at(dQf, off), idt,
                         kk > 0 ? 1u : 0u);
           }
         }
@@ -943,17 +972,17 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kC * 128) + (kk % 4) * 32;
-          mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, desc_at(q, off), idx,
+          mma_bf16_ts(tmem + col_x(s), tmem + kColPH + kk * 8, desc_at(q, off), idx,
                       kk > 0 ? 1u : 0u);
-          mma_bf16_ts(tmem + kColX[s], tmem + kColPL + kk * 8, desc_at(q, off), idx, 1u);
+          mma_bf16_ts(tmem + col_x(s), tmem + kColPL + kk * 8, desc_at(q, off), idx, 1u);
           if constexpr (kSplitQK)
-            mma_bf16_ts(tmem + kColX[s], tmem + kColPH + kk * 8, desc_at(ql, off), idx, 1u);
+            mma_bf16_ts(tmem + col_x(s), tmem + kColPH + kk * 8, desc_at(ql, off), idx, 1u);
         }
       }
       if (!last) {
         constexpr uint32_t idp = instr_desc(kFmtBF16, kFmtBF16, kMNMajor, kMNMajor, 128, DK);
         const uint64_t bh_ = DECAY ? dKhm + s * kKppD : dKm + s * kStageD;
-        const uint64_t bl_ = DECAY ? dKpm + s * kKppD : dKlm + s * kLoD;
+        const uint64_t bl_ = DECAY ? dKpm + s * kKppD : dKlm + s * kStageD;
 #pragma unroll
         for (int kk = 0; kk < kC / 16; ++kk) {
           mma_bf16_ss(tmem + kColP, desc_at(v, kk * 2048), desc_at(bh_, kk * 2048), idp, 1u);
