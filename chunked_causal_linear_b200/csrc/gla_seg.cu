@@ -62,12 +62,22 @@ __device__ __forceinline__ void chunk_cumlog(float* sA, float* sTot, float* sLc,
   constexpr int NP = kXf / DK;  // parts per feature
   constexpr int RP = kC / NP;   // rows per part
   const int f = tw % DK, part = tw / DK;
+  // All of the part's gates first, then their logarithms (independent, so they overlap;
+  // taken unconditionally and selected: a padding row reads as zero), then the running
+  // sum in registers; the tile is written once, with the earlier parts' total added.
+  float l[RP];
+#pragma unroll
+  for (int j = 0; j < RP; ++j) l[j] = sA[(part * RP + j) * DK + f];
+#pragma unroll
+  for (int j = 0; j < RP; ++j) {
+    const float lg = __log2f(l[j]);
+    l[j] = part * RP + j < L ? fmaxf(lg, -126.f) : 0.f;
+  }
   float acc = 0.f;
-#pragma unroll 4
-  for (int r = part * RP; r < part * RP + RP; ++r) {
-    const float l = r < L ? fmaxf(__log2f(sA[r * DK + f]), -126.f) : 0.f;
-    acc += l;
-    sA[r * DK + f] = acc;
+#pragma unroll
+  for (int j = 0; j < RP; ++j) {
+    acc += l[j];
+    l[j] = acc;
   }
   sTot[part * DK + f] = acc;
   named_barrier(1, kXf);
@@ -75,10 +85,8 @@ __device__ __forceinline__ void chunk_cumlog(float* sA, float* sTot, float* sLc,
 #pragma unroll
   for (int p = 0; p < NP; ++p)
     if (p < part) off += sTot[p * DK + f];
-  if (part > 0) {
-#pragma unroll 4
-    for (int r = part * RP; r < part * RP + RP; ++r) sA[r * DK + f] += off;
-  }
+#pragma unroll
+  for (int j = 0; j < RP; ++j) sA[(part * RP + j) * DK + f] = l[j] + off;
   if (part == NP - 1) sLc[f] = acc + off;
   named_barrier(1, kXf);
 }
@@ -456,7 +464,7 @@ struct GK3Smem {
   static constexpr uint32_t kStage = kQ + kK + kV + kG;
   static_assert(kG == kQ + kK, "the lo tiles fill the gate tile");
   static constexpr uint32_t kA = kC * kC * 2;
-  static constexpr uint32_t kSmallFloats = 6 * DK + kXf + 16 + 4;
+  static constexpr uint32_t kSmallFloats = 8 * DK + kXf + 16 + 4;
   static constexpr uint32_t kBars = 15;
   static constexpr uint32_t kTotal = 2 * kStage + 2 * kA + kSmallFloats * 4 + (kBars + 1) * 8 + 1024;
 };
@@ -483,9 +491,9 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
   float* sLc = sW + DK;
   float* sBq = sLc + DK;
   float* sBk = sBq + DK;
-  float* sScale = sBk + DK;
-  float* sScale2 = sScale + DK;
-  float* sTot = sScale2 + DK;  // [kXf]: the cumulative-log parts
+  float* sScale = sBk + DK;         // [2][DK], by stage: read by the epilogue's prefix split
+  float* sScale2 = sScale + 2 * DK;  // [2][DK]
+  float* sTot = sScale2 + 2 * DK;    // [kXf]: the cumulative-log parts
   float* sRed = sTot + kXf;     // [16]
   int* sMode = reinterpret_cast<int*>(sRed + 16);  // [2], per stage
   uint64_t* bars = reinterpret_cast<uint64_t*>(sMode + 4);
@@ -550,33 +558,78 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
     return false;
   };
 
+  // The prefix operand of the X MMA, prepared by the epilogue warps between their score and
+  // output phases (the transform warps, whose gate pass sets the pace, keep only the chunk's
+  // operands): warp w covers TMEM lanes 32 (w % 4) .. + 31 and key features
+  // kHalf (w / 4 % 2) .. + kHalf - 1.
+  constexpr int kHalf = DK / 2;
+  const uint32_t pcol = static_cast<uint32_t>((warp >> 2) & 1) * kHalf;
+  auto load_prefix = [&]() {  // the segment's exclusive prefix: row (lane) of P^T
+    const int row = (warp & 3) * 32 + lane;
+    const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
+#pragma unroll
+    for (int q4 = 0; q4 < kHalf / 32; ++q4) {
+      uint32_t u[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 f = src[q4 * 8 + e];
+        u[4 * e] = __float_as_uint(f.x);
+        u[4 * e + 1] = __float_as_uint(f.y);
+        u[4 * e + 2] = __float_as_uint(f.z);
+        u[4 * e + 3] = __float_as_uint(f.w);
+      }
+      tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
+    }
+    tmem_st_wait();
+  };
+  // Prefix operand for chunk i (the state after chunk i - 1, final once statedone(i - 1)
+  // completed; the chunk's mode and scales are set once ops of its stage completed):
+  // P = P~ 2^W on a rebase (and, for the chunk's update, times 2^(L_last) in a steep chunk);
+  // P~ itself inside a window.  16 columns at a time, inside the epilogue's register budget.
+  auto split_prefix = [&](int i) {
+    const int st = i & 1;
+    const bool last = i == n - 1;
+    const bool rebase = sMode[st] != kModeWindow;
+    const float* scale = sScale + st * DK;
+    const float* scale2 = sScale2 + st * DK;
+#pragma unroll 2
+    for (int q = 0; q < kHalf / 16; ++q) {
+      const uint32_t col = pcol + q * 16;
+      float rr[16];
+      tmem_ld16(tmem + lane_base + kColP + col, rr);
+      tmem_ld_wait();
+      if (rebase) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) rr[e] *= scale[col + e];
+      }
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(rr[2 * e], rr[2 * e + 1]);
+        const float2 hf = __bfloat1622float2(h);
+        hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+        lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
+      }
+      tmem_st8(tmem + lane_base + kColPH + col / 2, hi);
+      tmem_st8(tmem + lane_base + kColPL + col / 2, lo);
+      if (rebase && !last) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(rr[e] * scale2[col + e]);
+        tmem_st16(tmem + lane_base + kColP + col, u);
+      }
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(pready);
+  };
+
   if (warp < 8) {
     // ------------------------------------------------------------------ transform
     const int tw = tid;
-    constexpr int kHalf = DK / 2;
-    const uint32_t pcol = static_cast<uint32_t>(warp >> 2) * kHalf;
-    {  // the segment's exclusive prefix: row (lane) of P^T, this thread's half
-      const int row = (warp & 3) * 32 + lane;
-      const float4* src = reinterpret_cast<const float4*>(srec + static_cast<long long>(row) * DK + pcol);
-#pragma unroll
-      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
-        uint32_t u[32];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 f = src[q4 * 8 + e];
-          u[4 * e] = __float_as_uint(f.x);
-          u[4 * e + 1] = __float_as_uint(f.y);
-          u[4 * e + 2] = __float_as_uint(f.z);
-          u[4 * e + 3] = __float_as_uint(f.w);
-        }
-        tmem_st32(tmem + lane_base + kColP + pcol + q4 * 32, u);
-      }
-      tmem_st_wait();
-    }
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       const int L = chunk_len(sp, cb + i);
-      const bool last = i == n - 1;
       uint8_t* sQ = base + s * L_::kStage;
       uint8_t* sK = sQ + L_::kQ;
       uint8_t* sQl = sK + L_::kK + L_::kV;  // the gate tile, reused for the lo halves
@@ -584,7 +637,8 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       float* sA = reinterpret_cast<float*>(sQl);
       wait(&full[s], (i >> 1) & 1, kErrTmaTimeout);
       chunk_cumlog<DK>(sA, sTot, sLc, tw, L, false);
-      const int mode = chunk_mode<DK>(sW, sLc, sBq, sBk, sScale, sScale2, sRed, tw, warp, lane);
+      const int mode = chunk_mode<DK>(sW, sLc, sBq, sBk, sScale + s * DK, sScale2 + s * DK, sRed,
+                                      tw, warp, lane);
       if (tw == 0) sMode[s] = mode;
       {
         uint4 qlo[FactorShape<DK>::kRows], klo[FactorShape<DK>::kRows];
@@ -596,50 +650,15 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       }
       fence_async_smem();
       mbar_arrive(&ops[s]);
-      // The state is final before the prefix pass (the previous chunk's MMAs are done).
-      if (i > 0) wait(statedone, (i - 1) & 1, kErrMmaTimeout);
-
-      // Prefix operand for chunk i (the state after chunk i - 1), this thread's half of the
-      // key features: P = P~ 2^W on a rebase (and, for the chunk's update, times 2^(L_last)
-      // in a steep chunk); P~ itself inside a window.
-      tc_fence_after();
-      const bool rebase = mode != kModeWindow;
-#pragma unroll
-      for (int q4 = 0; q4 < kHalf / 32; ++q4) {
-        const uint32_t col = pcol + q4 * 32;
-        float rr[32];
-        tmem_ld32(tmem + lane_base + kColP + col, rr);
-        tmem_ld_wait();
-        if (rebase) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] *= sScale[col + e];
-        }
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const __nv_bfloat162 h = __floats2bfloat162_rn(rr[2 * e], rr[2 * e + 1]);
-          const float2 hf = __bfloat1622float2(h);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[e] = pack2(rr[2 * e] - hf.x, rr[2 * e + 1] - hf.y);
-        }
-        tmem_st16(tmem + lane_base + kColPH + col / 2, hi);
-        tmem_st16(tmem + lane_base + kColPL + col / 2, lo);
-        if (rebase && !last) {
-          uint32_t u[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(rr[e] * sScale2[col + e]);
-          tmem_st32(tmem + lane_base + kColP + col, u);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(pready);
     }
   } else if (warp < 16) {
     // ------------------------------------------------------------------ epilogue
     const int tw = tid - kXf;
     const int quarter = warp & 3, half = (warp - 8) >> 2;
     const int j = quarter * 32 + lane;  // value feature of this thread's output column
+    load_prefix();
+    wait(&ops[0], 0, kErrMmaTimeout);  // chunk 0's mode and scales
+    split_prefix(0);
     for (int i = 0; i < n; ++i) {
       const int s = i & 1;
       const long long t0 = static_cast<long long>(cb + i) * kC;
@@ -678,6 +697,14 @@ gla_k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUt
       fence_async_smem();
       mbar_arrive(aready);
       if (tw == 0) sp.steep[static_cast<long long>(bh) * sp.NC + cb + i] = mode == kModeSteep ? 1 : 0;
+
+      // The next chunk's prefix operand, while N(i) runs.
+      if (i + 1 < n) {
+        wait(statedone, i & 1, kErrMmaTimeout);
+        wait(&ops[(i + 1) & 1], ((i + 1) >> 1) & 1, kErrMmaTimeout);
+        tc_fence_after();
+        split_prefix(i + 1);
+      }
 
       wait(ndone, i & 1, kErrMmaTimeout);
       tc_fence_after();
