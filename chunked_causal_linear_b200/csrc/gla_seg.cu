@@ -70,7 +70,8 @@ __device__ __forceinline__ void chunk_cumlog(float* sA, float* sTot, float* sLc,
   for (int j = 0; j < RP; ++j) l[j] = sA[(part * RP + j) * DK + f];
 #pragma unroll
   for (int j = 0; j < RP; ++j) {
-    const float lg = __log2f(l[j]);
+    // Gates below 2^-126 read as zero and clamp to -126, as they would unflushed.
+    const float lg = log2_approx(l[j]);
     l[j] = part * RP + j < L ? fmaxf(lg, -126.f) : 0.f;
   }
   float acc = 0.f;

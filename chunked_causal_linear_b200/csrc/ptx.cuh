@@ -360,6 +360,14 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// log2 x by the hardware's approximate base-2 logarithm (PTX lg2.approx.ftz.f32: about 2^-22
+// absolute; subnormal inputs flush to zero and give -inf).
+__device__ __forceinline__ float log2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // psi: ELU+1 (x + 1 for x > 0, e^x = 2^(x log2 e) otherwise, by the hardware exponential:
 // about 2^-21 relative, far below the 2^-16 of the split bf16 operands) or the identity.
 template <int FM>
