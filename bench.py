@@ -52,9 +52,10 @@ BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 K2_NAMES = {"logdepth": ["k2_reduce", "k2_block_scan", "k2_downsweep"],
             "sequential": ["k2_sequential"]}
 SCAN_BLOCK_ELEMS = 2048  # the log-depth scan's one-level limit (lin_attn_scan_plan)
+SCAN_WARP_ELEMS = 32     # up to this many elements the block level runs as k2_warp_scan
 KERNEL_SOURCES = {"k1_tc": "tc_kernels.cu", "k3_tc": "tc_kernels.cu", "k1_fma": "fma_kernels.cu",
                   "k3_fma": "fma_kernels.cu", "k2_reduce": "scan.cu",
-                  "k2_block_scan": "scan.cu", "k2_downsweep": "scan.cu",
+                  "k2_block_scan": "scan.cu", "k2_warp_scan": "scan.cu", "k2_downsweep": "scan.cu",
                   "k2_sequential": "scan.cu", "k1_seg": "seg_kernels.cu",
                   "k3_seg": "seg_kernels.cu"}
 
@@ -80,8 +81,13 @@ def kernel_names(w, algo: str, scan: str, lseg: int = 0) -> list[str]:
     k1, k3 = ("k1_seg", "k3_seg") if algo == "segmented" else ("k1_tc", "k3_tc")
     if kernel_path_for(w) == "fma":
         k1, k3 = "k1_fma", "k3_fma"
-    n, _, _ = layout(w, algo, lseg)
-    k2 = ["k2_block_scan"] if scan == "logdepth" and n <= SCAN_BLOCK_ELEMS else K2_NAMES[scan]
+    n, G, _ = layout(w, algo, lseg)
+    k2 = ["k2_block_scan"] if scan == "logdepth" and n <= SCAN_BLOCK_ELEMS else list(K2_NAMES[scan])
+    if scan == "logdepth":
+        # The block level over at most 32 elements (n one level, G two) is the warp scan.
+        m = n if n <= SCAN_BLOCK_ELEMS else G
+        if m <= SCAN_WARP_ELEMS:
+            k2 = ["k2_warp_scan" if x == "k2_block_scan" else x for x in k2]
     return [k1, *k2, k3]
 
 
@@ -121,7 +127,7 @@ def kernel_bytes(w, name: str, out_elem: int, algo: str = "chunked", lseg: int =
         return BH * w.T * (w.dk + w.dv) * e_in + rec
     if name == "k2_reduce":
         return rec + BH * G * R * 4
-    if name == "k2_block_scan":
+    if name in ("k2_block_scan", "k2_warp_scan"):
         # One level: the records read once (the second read of a CTA's slab comes from L2)
         # and written once; two levels: the same over the segment folds.  Plus the final
         # states.

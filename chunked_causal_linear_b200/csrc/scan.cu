@@ -256,6 +256,71 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   if (e1 == p.NC) write_final(p, bh, col4 * 4, carry);
 }
 
+// The blocked scan for at most 32 elements (the segmented arrangement's usual case): one
+// warp per (b*h, kWarpScanCols float4 columns), lane e holding element e, Hillis-Steele over
+// the lanes by shuffles (5 rounds, as the blocked scan's group rounds at 32 groups of one
+// element) and no CTA-wide barrier, so every warp keeps its loads in flight on its own.
+// Lanes past the last element hold the identity (decay 1, state 0).
+constexpr int kWarpScanCols = 4;
+constexpr int kWarpScanThreads = 256;
+
+template <bool DECAY>
+__global__ void __launch_bounds__(kWarpScanThreads) k2_warp_scan(PrefillParams p, GammaTable gt) {
+  const int lane = threadIdx.x & 31;
+  const long long wid = (static_cast<long long>(blockIdx.x) * kWarpScanThreads + threadIdx.x) >> 5;
+  const int R4 = p.R / 4;
+  const int nblk = (R4 + kWarpScanCols - 1) / kWarpScanCols;
+  if (wid >= static_cast<long long>(nblk) * p.BH) return;  // (whole warps)
+  const int bh = static_cast<int>(wid / nblk);
+  const int c0 = static_cast<int>(wid % nblk) * kWarpScanCols;
+  float gC = 1.f, aL = 1.f;
+  if (DECAY) {
+    const float g = gt.g[bh % p.H];
+    gC = powf(g, static_cast<float>(p.C));
+    aL = powf(g, static_cast<float>(p.L_last));
+  }
+  const bool el = lane < p.NC;
+  float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) +
+                 static_cast<long long>(lane) * R4 + c0;
+  float4 x[kWarpScanCols];
+#pragma unroll
+  for (int u = 0; u < kWarpScanCols; ++u)
+    x[u] = el && c0 + u < R4 ? base[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+  float A = el && DECAY ? (lane == p.NC - 1 ? aL : gC) : 1.f;
+  // Inclusive: (A, x) of elements 0..lane under (a1, x1) (+) (a2, x2) = (a1 a2, a2 x1 + x2).
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const float Ap = __shfl_up_sync(0xffffffffu, A, d);
+#pragma unroll
+    for (int u = 0; u < kWarpScanCols; ++u) {
+      float4 xp;
+      xp.x = __shfl_up_sync(0xffffffffu, x[u].x, d);
+      xp.y = __shfl_up_sync(0xffffffffu, x[u].y, d);
+      xp.z = __shfl_up_sync(0xffffffffu, x[u].z, d);
+      xp.w = __shfl_up_sync(0xffffffffu, x[u].w, d);
+      if (lane >= d) x[u] = axpy4(A, xp, x[u]);
+    }
+    if (lane >= d) A *= Ap;
+  }
+  // Exclusive: element e's prefix is (A, x) of elements 0..e-1 applied to the initial state.
+  const float Ae = __shfl_up_sync(0xffffffffu, A, 1);
+#pragma unroll
+  for (int u = 0; u < kWarpScanCols; ++u) {
+    const bool live = c0 + u < R4;
+    const float4 init = live && p.has_init ? read_init(p, bh, (c0 + u) * 4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 xe;
+    xe.x = __shfl_up_sync(0xffffffffu, x[u].x, 1);
+    xe.y = __shfl_up_sync(0xffffffffu, x[u].y, 1);
+    xe.z = __shfl_up_sync(0xffffffffu, x[u].z, 1);
+    xe.w = __shfl_up_sync(0xffffffffu, x[u].w, 1);
+    if (el && live) {
+      base[u] = lane == 0 ? init : axpy4(Ae, init, xe);
+      if (lane == p.NC - 1) write_final(p, bh, (c0 + u) * 4, axpy4(A, init, x[u]));
+    }
+  }
+}
+
 // Second pass: each segment writes its chunks' exclusive prefixes in place.
 template <bool DECAY>
 __global__ void __launch_bounds__(kScanThreads) k2_downsweep(PrefillParams p, GammaTable gt) {
@@ -278,7 +343,16 @@ __global__ void __launch_bounds__(kScanThreads) k2_downsweep(PrefillParams p, Ga
 }
 
 template <bool DECAY>
-cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_t s) {
+cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_t s,
+                       Recorder* rec) {
+  if (p.NC <= 32) {
+    if (rec) rec->mark(s, "k2_warp_scan");
+    const long long warps = static_cast<long long>((p.R / 4 + kWarpScanCols - 1) / kWarpScanCols) * p.BH;
+    const long long blocks = (warps * 32 + kWarpScanThreads - 1) / kWarpScanThreads;
+    k2_warp_scan<DECAY><<<static_cast<unsigned>(blocks), kWarpScanThreads, 0, s>>>(p, gt);
+    return cudaGetLastError();
+  }
+  if (rec) rec->mark(s, "k2_block_scan");
   const ScanPlan bp = scan_plan(p.NC);  // p.NC <= kScanBlockElems: a single block level
   const int R4 = p.R / 4;
   const int W = kBlockThreads / bp.NG;
@@ -303,8 +377,7 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
   }
   if (p.NC <= kScanBlockElems) {
     // One block level: the blocked scan alone, in place on the records.
-    if (rec) rec->mark(s, "k2_block_scan");
-    return block_scan<DECAY>(p, gt, s);
+    return block_scan<DECAY>(p, gt, s, rec);
   }
   // Two levels: segment folds, the blocked scan over them, the per-segment sweep.
   const ScanPlan plan = scan_plan(p.NC);
@@ -321,8 +394,7 @@ cudaError_t go(const PrefillParams& p, const GammaTable& gt, int mode, cudaStrea
   q.NC = p.G;
   q.C = p.C * p.Ls;
   q.L_last = static_cast<int>(p.T - static_cast<long long>(p.G - 1) * p.Ls * p.C);
-  if (rec) rec->mark(s, "k2_block_scan");
-  e = block_scan<DECAY>(q, gt, s);
+  e = block_scan<DECAY>(q, gt, s, rec);
   if (e != cudaSuccess) return e;
   if (rec) rec->mark(s, "k2_downsweep");
   k2_downsweep<DECAY><<<static_cast<unsigned>(grid), kScanThreads, 0, s>>>(p, gt);

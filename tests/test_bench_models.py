@@ -36,8 +36,9 @@ def test_backward_bytes_are_three_prefills_on_the_retention_workload():
     w = WORKLOADS["retention_128k"]
     ops = bench.backward_bytes(w, 4, "auto")
     names = [n for n, _ in ops]
-    # reverse-mode passes: no element-wise kernel, three (k1_seg, k2_block_scan, k3_seg)
-    assert names == ["k1_seg", "k2_block_scan", "k3_seg"] * 3
+    # reverse-mode passes: no element-wise kernel, three (k1_seg, the scan, k3_seg); 32
+    # segments per head, so the scan's block level is the warp scan
+    assert names == ["k1_seg", "k2_warp_scan", "k3_seg"] * 3
     k3 = [b for n, b in ops if n == "k3_seg"]
     assert len(set(k3)) == 1 and k3[0] == bench.kernel_bytes(w, "k3_seg", 4, "segmented")
 
@@ -63,3 +64,17 @@ def test_oracle_backward_and_gla_do_not_depend_on_the_thread_count():
     g1 = o.gla_forward(q, k, v, a, nthreads=1)
     g4 = o.gla_forward(q, k, v, a, nthreads=4)
     assert all(np.array_equal(x, y) for x, y in zip(g1, g4))
+
+
+def test_scan_kernel_names_follow_the_element_count():
+    """Up to 32 scan elements the block level is k2_warp_scan, beyond it k2_block_scan; two
+    levels put the block level between k2_reduce and k2_downsweep."""
+    base = WORKLOADS["retention_128k"]
+    assert bench.kernel_names(base, "segmented", "logdepth") == ["k1_seg", "k2_warp_scan", "k3_seg"]
+    assert bench.kernel_names(base, "chunked", "logdepth") == ["k1_tc", "k2_block_scan", "k3_tc"]
+    assert bench.kernel_names(base, "chunked", "sequential") == ["k1_tc", "k2_sequential", "k3_tc"]
+    long = base.with_(T=64 * 16384)  # 16384 chunks: two levels over 1024 segments of 16
+    assert bench.kernel_names(long, "chunked", "logdepth") == \
+        ["k1_tc", "k2_reduce", "k2_block_scan", "k2_downsweep", "k3_tc"]
+    assert bench.kernel_bytes(base, "k2_warp_scan", 4, "segmented") == \
+        bench.kernel_bytes(base, "k2_block_scan", 4, "segmented")
