@@ -7,7 +7,8 @@ scan at once: a per-head decay, an initial state (the scan's first element), a r
 chunk and the final states, in the chunked arrangement (elements = chunks) and in the
 segmented one with one chunk per segment (elements = segments).  Tolerance 2e-2 rms
 (bf16 inputs, float32 outputs), both scan modes; the number of kernels each run launches
-matches the plan.
+matches the plan.  A last group covers the boundary between the block level's two forms:
+k2_warp_scan up to 32 elements, k2_block_scan beyond.
 """
 
 from __future__ import annotations
@@ -80,3 +81,24 @@ def test_scan_plan_shapes_the_launches():
                                          algorithm="chunked", out_dtype="f32")
         assert len(times) == 2 + (1 if levels == 1 else 3)
         assert np.all(np.isfinite(to_np(out)))
+
+
+@pytest.mark.parametrize("scan_elems", [1, 2, 31, 32, 33, 64])
+@pytest.mark.parametrize("fm,decay,norm", [("identity", True, False), ("elu1", True, True)])
+def test_warp_and_block_scan_boundary(scan_elems, fm, decay, norm):
+    """The block level runs as k2_warp_scan up to 32 elements and as k2_block_scan beyond:
+    both against the oracle at the boundary, chunked (elements = chunks) with a ragged last
+    chunk, a per-head decay and an initial state."""
+    T = 64 * (scan_elems - 1) + 23
+    w, q, k, v, S0, Z0, gamma = _case(T, fm, decay, norm, seed=11 + scan_elems)
+    kw = dict(chunk=64, feature_map=fm, gamma=gamma, normalize=norm, scan="logdepth",
+              kernel_path="tensor_core", algorithm="chunked", out_dtype="f32")
+    out, S, Z = B.lin_attn_prefill(q, k, v, S_init=S0, Z_init=Z0, **kw)
+    torch.cuda.synchronize()
+    assert B.lin_attn_device_error() == 0
+    o_ref, S_ref, Z_ref = oracle_prefill(q, k, v, feature_map=fm, gamma=gamma, normalize=norm,
+                                         S_init=S0, Z_init=Z0)
+    assert_close(to_np(out), o_ref, TOL_BF16, "out")
+    assert_close(to_np(S), S_ref, TOL_BF16, "S_final")
+    if norm:
+        assert_close(to_np(Z), Z_ref, TOL_BF16, "Z_final")
