@@ -97,11 +97,21 @@ def kernel_names(w, algo: str, scan: str, lseg: int = 0) -> list[str]:
 
 def segment_length(w, lseg: int = 0) -> int:
     """Chunks per segment of the segmented algorithm: the requested count, else the
-    library's automatic choice (about four segments per SM, at most 64 chunks)."""
+    library's automatic choice (about four segments per SM, at most 64 chunks, unless the
+    model waves x (4 + chunks per segment) predicts at least 25 % less time for a longer
+    segment)."""
     NC = -(-w.T // w.C)
     if lseg > 0:
         return min(lseg, NC)
-    return max(1, min(64, (w.B * w.H * NC) // (4 * 148)))
+    BH = w.B * w.H
+    cap = min(64, max(1, NC))
+    l0 = max(1, min(cap, (BH * NC) // (4 * 148)))
+
+    def cost(l):
+        return -(-BH * -(-NC // l) // 148) * (4.0 + l)
+
+    best = min(range(1, cap + 1), key=lambda l: (cost(l), l != l0, l))
+    return best if cost(best) <= 0.75 * cost(l0) else l0
 
 
 def layout(w, algo: str = "chunked", lseg: int = 0):

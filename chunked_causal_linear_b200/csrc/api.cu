@@ -211,13 +211,34 @@ int validate(const la_prefill_args& a, Path* path) {
   return LA_OK;
 }
 
-// Chunks per segment for the segmented algorithm: enough segments to give every SM a
-// few, at most 64 chunks each.
+// Chunks per segment for the segmented algorithm.  The base choice gives every SM about four
+// segments of at most 64 chunks.  A segment's CTA pays a pipeline fill and drain of about
+// four chunks' work (~12 us against ~2.4 us per chunk on retention_128k), and CTAs run in
+// waves of one per SM, so the time goes roughly as waves x (4 + chunks per segment).  The
+// model overstates partial last waves, so a longer segment is taken only where it predicts
+// at least 25 % less time than the base choice: small problems, where the base choice leaves
+// many short segments in many waves (norm_b4h16: 6 -> 32 chunks, k3_seg 0.099 -> 0.088 ms
+// measured; ragged_b2h32 keeps 27, which measured best among 27-64).
 int segment_chunks(long long BH, int NC) {
-  long long l = BH * NC / (4LL * 148);
-  if (l < 1) l = 1;
-  if (l > 64) l = 64;
-  return static_cast<int>(l);
+  const int cap = NC < 64 ? (NC < 1 ? 1 : NC) : 64;
+  long long l0 = BH * NC / (4LL * 148);
+  if (l0 < 1) l0 = 1;
+  if (l0 > cap) l0 = cap;
+  auto cost = [&](long long l) {
+    const long long ctas = BH * ((NC + l - 1) / l);
+    return static_cast<double>((ctas + 147) / 148) * (4.0 + static_cast<double>(l));
+  };
+  const double c0 = cost(l0);
+  long long best = l0;
+  double cb = c0;
+  for (long long l = 1; l <= cap; ++l) {
+    const double c = cost(l);
+    if (c < cb) {
+      cb = c;
+      best = l;
+    }
+  }
+  return static_cast<int>(cb <= 0.75 * c0 ? best : l0);
 }
 
 int to_status(cudaError_t e) {

@@ -256,67 +256,72 @@ k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
   if (e1 == p.NC) write_final(p, bh, col4 * 4, carry);
 }
 
-// The blocked scan for at most 32 elements (the segmented arrangement's usual case): one
-// warp per (b*h, kWarpScanCols float4 columns), lane e holding element e, Hillis-Steele over
-// the lanes by shuffles (5 rounds, as the blocked scan's group rounds at 32 groups of one
-// element) and no CTA-wide barrier, so every warp keeps its loads in flight on its own.
+// The blocked scan for at most 32 elements (the segmented arrangement's usual case): lanes
+// in runs of `seg` (the element count rounded up to a power of two), one run per (b*h,
+// kWarpScanCols float4 columns), lane e of a run holding element e; Hillis-Steele over the
+// run by shuffles (log2 seg rounds, as the blocked scan's group rounds at one element per
+// group) and no CTA-wide barrier, so every warp keeps its loads in flight on its own.
 // Lanes past the last element hold the identity (decay 1, state 0).
 constexpr int kWarpScanCols = 4;
 constexpr int kWarpScanThreads = 256;
 
 template <bool DECAY>
-__global__ void __launch_bounds__(kWarpScanThreads) k2_warp_scan(PrefillParams p, GammaTable gt) {
+__global__ void __launch_bounds__(kWarpScanThreads) k2_warp_scan(PrefillParams p, GammaTable gt,
+                                                                 int seg) {
   const int lane = threadIdx.x & 31;
+  const int e = lane & (seg - 1);
+  const int runs = 32 / seg;
   const long long wid = (static_cast<long long>(blockIdx.x) * kWarpScanThreads + threadIdx.x) >> 5;
   const int R4 = p.R / 4;
-  const int nblk = (R4 + kWarpScanCols - 1) / kWarpScanCols;
-  if (wid >= static_cast<long long>(nblk) * p.BH) return;  // (whole warps)
-  const int bh = static_cast<int>(wid / nblk);
-  const int c0 = static_cast<int>(wid % nblk) * kWarpScanCols;
+  const long long nblk = (R4 + kWarpScanCols - 1) / kWarpScanCols;
+  if (wid * runs >= nblk * p.BH) return;  // (whole warps)
+  const long long blk = wid * runs + lane / seg;
+  const bool in = blk < nblk * p.BH;
+  const int bh = in ? static_cast<int>(blk / nblk) : 0;
+  const int c0 = in ? static_cast<int>(blk % nblk) * kWarpScanCols : 0;
   float gC = 1.f, aL = 1.f;
   if (DECAY) {
     const float g = gt.g[bh % p.H];
     gC = powf(g, static_cast<float>(p.C));
     aL = powf(g, static_cast<float>(p.L_last));
   }
-  const bool el = lane < p.NC;
+  const bool el = in && e < p.NC;
   float4* base = reinterpret_cast<float4*>(p.rec + static_cast<long long>(bh) * p.NC * p.R) +
-                 static_cast<long long>(lane) * R4 + c0;
+                 static_cast<long long>(e) * R4 + c0;
   float4 x[kWarpScanCols];
 #pragma unroll
   for (int u = 0; u < kWarpScanCols; ++u)
     x[u] = el && c0 + u < R4 ? base[u] : make_float4(0.f, 0.f, 0.f, 0.f);
-  float A = el && DECAY ? (lane == p.NC - 1 ? aL : gC) : 1.f;
-  // Inclusive: (A, x) of elements 0..lane under (a1, x1) (+) (a2, x2) = (a1 a2, a2 x1 + x2).
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const float Ap = __shfl_up_sync(0xffffffffu, A, d);
+  float A = el && DECAY ? (e == p.NC - 1 ? aL : gC) : 1.f;
+  // Inclusive: (A, x) of elements 0..e under (a1, x1) (+) (a2, x2) = (a1 a2, a2 x1 + x2).
+  for (int d = 1; d < seg; d <<= 1) {
+    const float Ap = __shfl_up_sync(0xffffffffu, A, d, seg);
 #pragma unroll
     for (int u = 0; u < kWarpScanCols; ++u) {
       float4 xp;
-      xp.x = __shfl_up_sync(0xffffffffu, x[u].x, d);
-      xp.y = __shfl_up_sync(0xffffffffu, x[u].y, d);
-      xp.z = __shfl_up_sync(0xffffffffu, x[u].z, d);
-      xp.w = __shfl_up_sync(0xffffffffu, x[u].w, d);
-      if (lane >= d) x[u] = axpy4(A, xp, x[u]);
+      xp.x = __shfl_up_sync(0xffffffffu, x[u].x, d, seg);
+      xp.y = __shfl_up_sync(0xffffffffu, x[u].y, d, seg);
+      xp.z = __shfl_up_sync(0xffffffffu, x[u].z, d, seg);
+      xp.w = __shfl_up_sync(0xffffffffu, x[u].w, d, seg);
+      if (e >= d) x[u] = axpy4(A, xp, x[u]);
     }
-    if (lane >= d) A *= Ap;
+    if (e >= d) A *= Ap;
   }
   // Exclusive: element e's prefix is (A, x) of elements 0..e-1 applied to the initial state.
-  const float Ae = __shfl_up_sync(0xffffffffu, A, 1);
+  const float Ae = __shfl_up_sync(0xffffffffu, A, 1, seg);
 #pragma unroll
   for (int u = 0; u < kWarpScanCols; ++u) {
     const bool live = c0 + u < R4;
-    const float4 init = live && p.has_init ? read_init(p, bh, (c0 + u) * 4)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 init = el && live && p.has_init ? read_init(p, bh, (c0 + u) * 4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 xe;
-    xe.x = __shfl_up_sync(0xffffffffu, x[u].x, 1);
-    xe.y = __shfl_up_sync(0xffffffffu, x[u].y, 1);
-    xe.z = __shfl_up_sync(0xffffffffu, x[u].z, 1);
-    xe.w = __shfl_up_sync(0xffffffffu, x[u].w, 1);
+    xe.x = __shfl_up_sync(0xffffffffu, x[u].x, 1, seg);
+    xe.y = __shfl_up_sync(0xffffffffu, x[u].y, 1, seg);
+    xe.z = __shfl_up_sync(0xffffffffu, x[u].z, 1, seg);
+    xe.w = __shfl_up_sync(0xffffffffu, x[u].w, 1, seg);
     if (el && live) {
-      base[u] = lane == 0 ? init : axpy4(Ae, init, xe);
-      if (lane == p.NC - 1) write_final(p, bh, (c0 + u) * 4, axpy4(A, init, x[u]));
+      base[u] = e == 0 ? init : axpy4(Ae, init, xe);
+      if (e == p.NC - 1) write_final(p, bh, (c0 + u) * 4, axpy4(A, init, x[u]));
     }
   }
 }
@@ -347,9 +352,13 @@ cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_
                        Recorder* rec) {
   if (p.NC <= 32) {
     if (rec) rec->mark(s, "k2_warp_scan");
-    const long long warps = static_cast<long long>((p.R / 4 + kWarpScanCols - 1) / kWarpScanCols) * p.BH;
+    int seg = 1;
+    while (seg < p.NC) seg <<= 1;
+    const long long runs =
+        static_cast<long long>((p.R / 4 + kWarpScanCols - 1) / kWarpScanCols) * p.BH;
+    const long long warps = (runs + 32 / seg - 1) / (32 / seg);
     const long long blocks = (warps * 32 + kWarpScanThreads - 1) / kWarpScanThreads;
-    k2_warp_scan<DECAY><<<static_cast<unsigned>(blocks), kWarpScanThreads, 0, s>>>(p, gt);
+    k2_warp_scan<DECAY><<<static_cast<unsigned>(blocks), kWarpScanThreads, 0, s>>>(p, gt, seg);
     return cudaGetLastError();
   }
   if (rec) rec->mark(s, "k2_block_scan");
