@@ -784,7 +784,7 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int d = rev ? kb + q * 8 + e - row : row - kb - q * 8 - e;
-            a[e] = d >= 0 ? sc[q * 8 + e] * sPow[d] : 0.f;
+            a[e] = d >= 0 ? (DECAY ? sc[q * 8 + e] * sPow[d] : sc[q * 8 + e]) : 0.f;
             den_loc += a[e];
           }
           split8(a, hi[q], lo[q]);
@@ -807,7 +807,9 @@ k3_seg(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtenso
         if (tw < kC) {
           const float den_loc = sDenPart[tw] + sDenPart[kC + tw];
           // The reciprocal, so that the 32 outputs of a thread take multiplications.
-          sDen[tw] = 1.f / ((has_prefix ? fmaf(sTh[tw], sDenX[s * kC + tw], den_loc) : den_loc) + sp.eps);
+          // (The fast reciprocal: ~2 ulp, far below the split operands' 2^-16; the
+          // denominator is a positive sum of bounded scores, never near 2^126.)
+          sDen[tw] = __fdividef(1.f, (has_prefix ? fmaf(sTh[tw], sDenX[s * kC + tw], den_loc) : den_loc) + sp.eps);
         }
       }
       mbar_arrive(aready);
