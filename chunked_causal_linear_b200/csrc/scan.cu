@@ -43,8 +43,9 @@ namespace {
 
 constexpr int kScanThreads = 128;
 constexpr int kUnroll = 8;
-constexpr int kBlockThreads = 1024;  // block-scan CTA: groups x slab columns
-constexpr int kMaxGroups = 128;      // groups per block-scan CTA (slab of at least 8 float4)
+constexpr int kBlockThreads = 1024;  // block-scan CTA, groups of one element
+constexpr int kBlockThreadsU = 512;  // block-scan CTA, longer groups (two per SM)
+constexpr int kMaxGroups = 128;      // groups per block-scan CTA (slab of at least 4 float4)
 
 __device__ __forceinline__ float4 axpy4(float a, float4 x, float4 y) {
   return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
@@ -163,19 +164,20 @@ __global__ void __launch_bounds__(kScanThreads) k2_reduce(PrefillParams p, Gamma
   reinterpret_cast<float4*>(p.tot + (static_cast<long long>(bh) * p.G + s) * p.R)[col4] = agg;
 }
 
-// Blocked scan of N = p.NC elements, in place, one CTA per (b*H + h, slab of W = 1024 / NG
-// float4 columns: at least 128 contiguous bytes of every record); NG groups of E consecutive
-// elements (NG a power of two, NG * E >= N).
-// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 8 for longer groups (64
-// registers, one CTA per SM; two CTAs of 32 registers measured slower), 1 for groups of one
-// element (32 registers, two CTAs per SM).
-template <bool DECAY, int U>
-__global__ void __launch_bounds__(kBlockThreads, U == 1 ? 2 : 1)
+// Blocked scan of N = p.NC elements, in place, one CTA of NT threads per (b*H + h, slab of
+// W = NT / NG float4 columns); NG groups of E consecutive elements (NG a power of two,
+// NG * E >= N).
+// U: loads in flight per thread (pass 1 U, pass 2 U / 2): 8 for longer groups (NT = 512,
+// 64 registers, two CTAs per SM, so that one CTA's loads overlap the other's barrier rounds
+// and second pass; one CTA of 1024 threads per SM left HBM idle during them), 1 for groups
+// of one element (NT = 1024, 32 registers, two CTAs per SM).
+template <bool DECAY, int U, int NT>
+__global__ void __launch_bounds__(NT, 2)
 k2_block_scan(PrefillParams p, GammaTable gt, int NG, int E) {
-  __shared__ float4 sX[kBlockThreads];
-  __shared__ float sA[kBlockThreads];
+  __shared__ float4 sX[NT];
+  __shared__ float sA[NT];
   __shared__ float sG[2];
-  const int kSlab = kBlockThreads / NG;  // W
+  const int kSlab = NT / NG;  // W
   const int R4 = p.R / 4;
   const int nslab = (R4 + kSlab - 1) / kSlab;
   const int bh = blockIdx.x / nslab;
@@ -364,13 +366,14 @@ cudaError_t block_scan(const PrefillParams& p, const GammaTable& gt, cudaStream_
   if (rec) rec->mark(s, "k2_block_scan");
   const ScanPlan bp = scan_plan(p.NC);  // p.NC <= kScanBlockElems: a single block level
   const int R4 = p.R / 4;
-  const int W = kBlockThreads / bp.NG;
+  const int nt = bp.E == 1 ? kBlockThreads : kBlockThreadsU;
+  const int W = nt / bp.NG;
   const long long nslab = (R4 + W - 1) / W;
   const unsigned grid = static_cast<unsigned>(nslab * p.BH);
   if (bp.E == 1)
-    k2_block_scan<DECAY, 1><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
+    k2_block_scan<DECAY, 1, kBlockThreads><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
   else
-    k2_block_scan<DECAY, kUnroll><<<grid, kBlockThreads, 0, s>>>(p, gt, bp.NG, bp.E);
+    k2_block_scan<DECAY, kUnroll, kBlockThreadsU><<<grid, kBlockThreadsU, 0, s>>>(p, gt, bp.NG, bp.E);
   return cudaGetLastError();
 }
 
