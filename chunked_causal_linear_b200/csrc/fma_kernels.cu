@@ -95,13 +95,17 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
        Tout* __restrict__ out, PrefillParams p, GammaTable gt) {
   extern __shared__ float smem[];
   const int dk = p.dk, dv = p.dv, C = p.C;
-  float* sQ = smem;             // [C][dk] psi(q)
-  float* sK = sQ + C * dk;      // [C][dk] psi(k), zero past the chunk end
-  float* sV = sK + C * dk;      // [C][dv]
-  float* sP = sV + C * dv;      // [dv][dk] exclusive prefix state, transposed as stored
-  float* sZP = sP + dk * dv;    // [dk]
-  float* sA = sZP + dk;         // [C][C] masked, decayed scores
-  float* sDen = sA + C * C;     // [C]
+  // Rows of dk + 1 and C + 1 floats: the loops below read one row per lane (sK, sP, and sQ,
+  // sA in the denominators), and a stride of a multiple of 32 words would put every lane
+  // on the same bank.
+  const int ldk = dk + 1, lc = C + 1;
+  float* sQ = smem;             // [C][ldk] psi(q)
+  float* sK = sQ + C * ldk;     // [C][ldk] psi(k), zero past the chunk end
+  float* sV = sK + C * ldk;     // [C][dv]
+  float* sP = sV + C * dv;      // [dv][ldk] exclusive prefix state, transposed as stored
+  float* sZP = sP + dv * ldk;   // [dk]
+  float* sA = sZP + dk;         // [C][lc] masked, decayed scores
+  float* sDen = sA + C * lc;    // [C]
   float* sTh = sDen + C;        // [C] Theta_i
 
   const long long item = blockIdx.x;
@@ -117,13 +121,15 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
   const Tin* kb = k + (static_cast<long long>(bh) * p.T + t0) * dk;
   const Tin* vb = v + (static_cast<long long>(bh) * p.T + t0) * dv;
   for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
-    const bool ok = e / dk < L;
-    sQ[e] = ok ? feature<FM>(to_f(qb[e])) : 0.f;
-    sK[e] = ok ? feature<FM>(to_f(kb[e])) : 0.f;
+    const int t = e / dk, col = e % dk;
+    const bool ok = t < L;
+    sQ[t * ldk + col] = ok ? feature<FM>(to_f(qb[e])) : 0.f;
+    sK[t * ldk + col] = ok ? feature<FM>(to_f(kb[e])) : 0.f;
   }
   for (int e = threadIdx.x; e < C * dv; e += blockDim.x) sV[e] = e / dv < L ? to_f(vb[e]) : 0.f;
   const float* rec = p.rec + (static_cast<long long>(bh) * p.NC + c) * p.R;
-  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) sP[e] = pre ? rec[e] : 0.f;
+  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
+    sP[(e / dk) * ldk + e % dk] = pre ? rec[e] : 0.f;
   if (NORM)
     for (int i = threadIdx.x; i < dk; i += blockDim.x) sZP[i] = pre ? rec[dk * dv + i] : 0.f;
   for (int i = threadIdx.x; i < C; i += blockDim.x)
@@ -134,17 +140,18 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
     const int i = e / C, j = e % C;
     float a = 0.f;
     if (j <= i && i < L) {
-      for (int kk = 0; kk < dk; ++kk) a = fmaf(sQ[i * dk + kk], sK[j * dk + kk], a);
-      if (DECAY) a *= powf(g, static_cast<float>(i - j));
+      for (int kk = 0; kk < dk; ++kk) a = fmaf(sQ[i * ldk + kk], sK[j * ldk + kk], a);
+      // gamma^(i-j) from the Theta table: sTh[d - 1] = gamma^d, and gamma^0 = 1.
+      if (DECAY && j < i) a *= sTh[i - j - 1];
     }
-    sA[e] = a;
+    sA[i * lc + j] = a;
   }
   __syncthreads();
   if (NORM) {
     for (int i = threadIdx.x; i < C; i += blockDim.x) {
       float inter = 0.f, loc = 0.f;
-      for (int kk = 0; kk < dk; ++kk) inter = fmaf(sQ[i * dk + kk], sZP[kk], inter);
-      for (int j = 0; j <= i; ++j) loc += sA[i * C + j];
+      for (int kk = 0; kk < dk; ++kk) inter = fmaf(sQ[i * ldk + kk], sZP[kk], inter);
+      for (int j = 0; j <= i; ++j) loc += sA[i * lc + j];
       sDen[i] = fmaf(sTh[i], inter, loc) + p.eps;
     }
     __syncthreads();
@@ -155,8 +162,8 @@ k3_fma(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restri
     if (i >= L) continue;
     float inter = 0.f, loc = 0.f;
     if (pre)
-      for (int kk = 0; kk < dk; ++kk) inter = fmaf(sQ[i * dk + kk], sP[j * dk + kk], inter);
-    for (int t = 0; t <= i; ++t) loc = fmaf(sA[i * C + t], sV[t * dv + j], loc);
+      for (int kk = 0; kk < dk; ++kk) inter = fmaf(sQ[i * ldk + kk], sP[j * ldk + kk], inter);
+    for (int t = 0; t <= i; ++t) loc = fmaf(sA[i * lc + t], sV[t * dv + j], loc);
     float o = fmaf(sTh[i], inter, loc);
     if (NORM) o = o / sDen[i];
     ob[e] = from_f<Tout>(o);
@@ -168,7 +175,7 @@ size_t k1_fma_smem(const PrefillParams& p) {
 }
 size_t k3_fma_smem(const PrefillParams& p) {
   const size_t C = p.C, dk = p.dk, dv = p.dv;
-  return sizeof(float) * (2 * C * dk + C * dv + dk * dv + dk + C * C + 2 * C);
+  return sizeof(float) * (2 * C * (dk + 1) + C * dv + dv * (dk + 1) + dk + C * (C + 1) + 2 * C);
 }
 
 template <typename Kern>
