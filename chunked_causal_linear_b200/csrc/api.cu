@@ -71,19 +71,15 @@ bool dim_ok_fma(int d) { return d >= 4 && d <= 128 && d % 4 == 0; }
 bool chunk_ok_fma(int C) { return C == 16 || C == 32 || C == 64; }
 bool dim_ok_tc(int d) { return d == 64 || d == 128; }
 
-// Address of the device error word on the current device (cached per device).
+// Address of the device error word on the current device.  Looked up on every call and
+// not cached: after cudaDeviceReset the module is loaded again and the word may move.
 int* error_word_ptr() {
-  static std::mutex mu;
-  static int* cache[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int*>(ptr);
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return cache[dev];
+  return static_cast<int*>(ptr);
 }
 
 bool device_is_sm100() {

@@ -17,8 +17,6 @@
 
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/linattn.h"
 #include "launch.h"
 
@@ -26,25 +24,17 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of the array for the current device.  In host code the array's name
-// is only a host-side stand-in, so the address is looked up once per device, with that
-// device current, and cached.
+// Device address of the array on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address is looked up, on every call: a cached address
+// would go stale after cudaDeviceReset, which loads the module again.
 int scratch_address(void** out) {
-  static std::mutex mu;
-  static void* cache[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) {
-    void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || ptr == nullptr) {
-      cudaGetLastError();
-      return LA_ERR_CUDA;
-    }
-    cache[dev] = ptr;
+  void* ptr = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess || ptr == nullptr) {
+    cudaGetLastError();
+    return LA_ERR_CUDA;
   }
-  *out = cache[dev];
+  *out = ptr;
   return LA_OK;
 }
 
