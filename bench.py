@@ -193,6 +193,31 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def copy_bound_ms(h2d_pairs, d2h_pairs, reps=2):
+    """Device time of the end-to-end step's copies alone: every (device, pinned host) pair of
+    h2d_pairs copied in on one stream while every (pinned host, device) pair of d2h_pairs is
+    copied out on another, from one event to the join of both (best of reps, after one
+    warm-up).  The host-buffer prefill cannot finish faster than this."""
+    dev = h2d_pairs[0][0].device
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    cur = torch.cuda.current_stream(dev)
+    best = float("inf")
+    for r in range(reps + 1):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for st, pairs in ((s_in, h2d_pairs), (s_out, d2h_pairs)):
+            st.wait_event(e0)
+            with torch.cuda.stream(st):
+                for dst, src in pairs:
+                    dst.copy_(src, non_blocking=True)
+            cur.wait_stream(st)
+        e1.record(cur)
+        torch.cuda.synchronize(dev)
+        if r > 0:
+            best = min(best, e0.elapsed_time(e1))
+    return best
+
+
 def source_hash(fname: str) -> str:
     csrc = ROOT / "chunked_causal_linear_b200" / "csrc"
     h = hashlib.sha256()
@@ -1135,9 +1160,14 @@ def main():
         e_ms = ranks.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, info, dev)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
         d2h = oh.numel() * oh.element_size() + Sh.numel() * 4 + (Zh.numel() * 4 if Zh is not None else 0)
+        copy_ms = copy_bound_ms([(q, qh), (k, kh), (v, vh)],
+                                [(oh, out), (Sh, S)] + ([(Zh, Z)] if Zh is not None else []))
         e2e = {"value": info.world * w.tokens_heads / (e_ms / 1000.0), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "lin_attn_prefill_host (pinned host buffers; copies in, kernels and copies out overlapped across groups of heads; synchronous)"}
+               "api": "lin_attn_prefill_host (pinned host buffers; copies in, kernels and copies out overlapped across groups of heads; synchronous)",
+               "copy_bound_ms": copy_ms, "frac_of_copy_bound": copy_ms / e_ms,
+               "copy_bound": "the same bytes as plain copies between the same pinned buffers and "
+                             "device memory, both directions at once on two streams, no kernels"}
         del qh, kh, vh, oh, Sh, Zh, dbuf
 
     cpu = None
