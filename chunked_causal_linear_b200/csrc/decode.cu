@@ -121,7 +121,10 @@ __device__ __forceinline__ void st4(__nv_bfloat16* p, long long i, float4 x) {
   *reinterpret_cast<uint2*>(p + i) = u;
 }
 
-template <typename T, int FM, bool DECAY, bool NORM, int TR>
+// RPT: rows per thread, at least ceil(TR / row lanes).  It is a template argument so that
+// the state registers are only the rows a thread really holds (at TR = 64 and dv = 128, 8
+// float4 instead of 16: about 60 registers instead of 110, four CTAs per SM instead of two).
+template <typename T, int FM, bool DECAY, bool NORM, int TR, int RPT>
 __global__ void __launch_bounds__(kTileThreads)
 decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
              T* __restrict__ out, float* __restrict__ S, float* __restrict__ Z, int H, int dk,
@@ -145,7 +148,7 @@ decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restri
   const int lanes = kTileThreads / dv4;  // row lanes (>= 4)
   const int c4 = tid % dv4, rl = tid / dv4;
   const bool active = rl < lanes && rl < TR;
-  constexpr int kMax = TR / 4;  // rows per thread (lanes >= 4)
+  constexpr int kMax = RPT;  // rows per thread: RPT * lanes >= TR
   float* Sb = S + (static_cast<long long>(bh) * dk + i0) * dv + 4 * c4;
   float4 s[kMax];
   if (active) {
@@ -259,7 +262,7 @@ bool tiles_ok(const void* q, const void* k, const void* v, const void* out, cons
          a16(k) && a16(v) && a16(out) && a16(S) && a16(Z);
 }
 
-template <typename T, int FM, bool DECAY, bool NORM, int TR>
+template <typename T, int FM, bool DECAY, bool NORM, int TR, int RPT>
 cudaError_t go_tiles_r(const void* q, const void* k, const void* v, void* out, float* S,
                        float* Z, int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
                        cudaStream_t s) {
@@ -276,7 +279,7 @@ cudaError_t go_tiles_r(const void* q, const void* k, const void* v, void* out, f
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tiles<T, FM, DECAY, NORM, TR>, static_cast<const T*>(q),
+  return cudaLaunchKernelEx(&cfg, decode_tiles<T, FM, DECAY, NORM, TR, RPT>, static_cast<const T*>(q),
                             static_cast<const T*>(k), static_cast<const T*>(v),
                             static_cast<T*>(out), S, Z, H, dk, dv, eps, gt);
 }
@@ -285,9 +288,17 @@ template <typename T, int FM, bool DECAY, bool NORM>
 cudaError_t go_tiles(const void* q, const void* k, const void* v, void* out, float* S, float* Z,
                      int BH, int H, int dk, int dv, float eps, const GammaTable& gt,
                      cudaStream_t s) {
-  if (tile_rows(BH, dk) == 64)
-    return go_tiles_r<T, FM, DECAY, NORM, 64>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
-  return go_tiles_r<T, FM, DECAY, NORM, 16>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
+  // Row lanes = threads / (dv / 4) >= 4 (dv <= 256); each thread takes ceil(TR / lanes) rows.
+  const int lanes = kTileThreads / (dv / 4);
+  if (tile_rows(BH, dk) == 64) {
+    const int rpt = (64 + lanes - 1) / lanes;
+    if (rpt <= 4)
+      return go_tiles_r<T, FM, DECAY, NORM, 64, 4>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
+    if (rpt <= 8)
+      return go_tiles_r<T, FM, DECAY, NORM, 64, 8>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
+    return go_tiles_r<T, FM, DECAY, NORM, 64, 16>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
+  }
+  return go_tiles_r<T, FM, DECAY, NORM, 16, 4>(q, k, v, out, S, Z, BH, H, dk, dv, eps, gt, s);
 }
 
 template <typename T, int FM, bool DECAY, bool NORM>
