@@ -63,6 +63,35 @@ def test_decode_from_a_given_state(dk, dv, fm, norm, decay, dtype):
     assert_close(to_np(Z), Z_ref, tol, "Z")
 
 
+@pytest.mark.parametrize("dk,dv", [(128, 256), (128, 100), (128, 64), (64, 48), (128, 128)])
+@pytest.mark.parametrize("fm,norm,decay", [("elu1", True, False), ("identity", False, True)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_64_row_tiles_every_rows_per_thread(dk, dv, fm, norm, decay, dtype):
+    """Enough heads for the 64-row tiles (B.H.dk / 64 >= 2 x 148), at value widths that give a
+    thread 4, 8 and 16 state rows (dv <= 64, 100 or 128, 256)."""
+    Bn, H = (4, 40) if dk == 128 else (8, 40)
+    S0, Z0, (q, k, v) = _case(Bn, H, dk, dv, dtype, seed=7 * dk + dv)
+    gamma = gammas_for(H, 5) if decay else None
+    S = torch.tensor(S0, device="cuda")
+    Z = torch.tensor(Z0, device="cuda")
+    out = B.lin_attn_decode_step(q.cuda(), k.cuda(), v.cuda(), S, Z, feature_map=fm,
+                                 gamma=gamma, normalize=norm)
+    torch.cuda.synchronize()
+    f = lambda t: t.float().numpy()[:, :, None]
+    o_ref, S_ref, Z_ref = default_oracle().forward(
+        f(q), f(k), f(v), feature_map=fm, normalize=norm,
+        gamma=None if gamma is None else np.asarray(gamma, dtype=np.float64),
+        S_init=S0, Z_init=Z0)
+    if dtype == "f32":
+        assert_close(to_np(out), o_ref[:, :, 0], TOL_F32, "out")
+        tol = TOL_F32
+    else:
+        assert_close_rounded_out(to_np(out), o_ref[:, :, 0], TOL_BF16, "out")
+        tol = TOL_BF16
+    assert_close(to_np(S), S_ref, tol, "S")
+    assert_close(to_np(Z), Z_ref, tol, "Z")
+
+
 def test_decode_many_heads_and_repeated_steps():
     """B.H = 256 (the size the decode benchmark starts at), eight steps in a row, each step's
     output against the oracle's token loop over the same eight tokens."""
