@@ -123,7 +123,7 @@ __device__ __forceinline__ void st4(__nv_bfloat16* p, long long i, float4 x) {
 
 // RPT: rows per thread, at least ceil(TR / row lanes).  It is a template argument so that
 // the state registers are only the rows a thread really holds (at TR = 64 and dv = 128, 8
-// float4 instead of 16: about 60 registers instead of 110, four CTAs per SM instead of two).
+// float4 instead of 16: 64 registers instead of ~110, four CTAs per SM instead of two).
 template <typename T, int FM, bool DECAY, bool NORM, int TR, int RPT>
 __global__ void __launch_bounds__(kTileThreads)
 decode_tiles(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
